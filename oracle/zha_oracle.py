@@ -1,0 +1,363 @@
+"""CPU oracle of the Zyphra Hierarchical Attention (ZHA) hot path.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path imports, calls or runs
+this module: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it.  It shares no code with the CUDA library.
+
+Plain numpy in float64, written step by step from the method's definitions:
+
+* "ZHA summary" page (picx.dev), Methodology -> Tree Construction: chunk LSE
+  F_C(q), tangent at a reference query (k_hat_r, b_hat_r), node score
+  max_r t_r(q), recursive parents.
+* "Subquadratic Attention with a Hierarchical Tree-Structured Indexer"
+  (arXiv 2610.42112), §III-A (tree construction, b_hat is the entropy of the
+  reference attention weights), §III-B (shared reference queries, estimated log
+  attention mass of a child), §III-C (top-down top-p routing), App. D-B2
+  (stable-state merge of the children's per-reference state, without
+  Taylor/RoPE re-anchoring), App. E-E (nodes without complete parents join the
+  frontier; the first key and the partial chunk are always read).
+* "ZHA summary" page, Methodology -> Routing: m_l(q), the final index set
+  I(q) = {0} u (union of selected leaf chunks) u C_cur(q), o(q) = Attn(q, K_I, V_I).
+
+Readings where the pages are silent (each is listed in the design doc):
+  * Tree nodes are stateless functions of the keys: a level-l node i spans
+    keys [i*S_l, (i+1)*S_l), S_l = leaf * branch**(l-1); it exists once all its
+    keys are in the cache.
+  * A node is visible to a query at position t iff its span ends at or before
+    V(t) = leaf * floor(t / leaf), the start of the query's own chunk.
+  * Parents merge their children's per-reference state (LSE F and normalised
+    k_hat) exactly; with no RoPE the re-anchoring term is zero, so in exact
+    arithmetic the parent equals the leaf formula over its whole span.
+  * Storage precision: the merge state (F, k_hat) is stored as fp32, the routing
+    copy of k_hat in the KV dtype (bf16 or fp32), b_hat as fp32.  The oracle
+    models these stores by rounding (round-to-nearest-even) exactly where they
+    happen; ``storage="f64"`` switches the rounding off.
+  * Top-p: candidates are ordered by (score desc, node index asc); m is the
+    smallest prefix whose softmax mass reaches p, or all candidates if the
+    rounded cumulative mass never does; p >= 1 keeps every candidate.
+  * Scores, softmax and cumulative sums are float64 (the routing decision is
+    made in float64 on both sides).
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+# ---------------------------------------------------------------------------
+# storage rounding
+# ---------------------------------------------------------------------------
+
+
+def round_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bfloat16 (ties to even), as float64.
+
+    Direct rounding of the float64 value to 8 significant bits (no detour via
+    float32, which could round twice).  Values are finite; bf16 shares fp32's
+    exponent range, and the subnormal range is treated like the normal range
+    (never reached by the data here).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)               # x = m * 2**e, 0.5 <= |m| < 1
+    r = np.rint(m * 256.0) / 256.0   # 8 significant bits, ties to even
+    return np.ldexp(r, e)
+
+
+def round_f32(x: np.ndarray) -> np.ndarray:
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def round_to(x: np.ndarray, storage: str) -> np.ndarray:
+    if storage == "bf16":
+        return round_bf16(x)
+    if storage == "f32":
+        return round_f32(x)
+    if storage == "f64":
+        return np.asarray(x, dtype=np.float64)
+    raise ValueError(storage)
+
+
+# ---------------------------------------------------------------------------
+# chunk log-mass and its tangent (summary page, Tree Construction; paper §III-A)
+# ---------------------------------------------------------------------------
+
+
+def lse(x: np.ndarray, axis=-1) -> np.ndarray:
+    """log(sum(exp(x))) along ``axis``, shifted by the maximum."""
+    m = np.max(x, axis=axis, keepdims=True)
+    return np.squeeze(m, axis) + np.log(np.sum(np.exp(x - m), axis=axis))
+
+
+def chunk_lse(q: np.ndarray, Kc: np.ndarray, scale: float) -> np.ndarray:
+    """F_C(q) = log sum_j exp(q . k_j * scale).  q: [..., d], Kc: [C, d]."""
+    return lse(q @ Kc.T * scale, axis=-1)
+
+
+def leaf_summary(Kc: np.ndarray, qref: np.ndarray, scale: float):
+    """Tangent-plane summary of one chunk for every reference query.
+
+    k_hat_r = sum_j softmax_j(q_hat_r . k_j * scale) k_j
+    F_r     = F_C(q_hat_r)
+    b_hat_r = F_r - q_hat_r . k_hat_r * scale
+    Kc: [C, d] keys, qref: [R, d].  Returns (k_hat [R, d], F [R], b_hat [R]).
+    """
+    s = qref @ Kc.T * scale                      # [R, C]
+    F = lse(s, axis=-1)                          # [R]
+    a = np.exp(s - F[:, None])                   # attention weights at q_hat_r
+    k_hat = a @ Kc                               # [R, d]
+    b_hat = F - np.sum(qref * k_hat, axis=-1) * scale
+    return k_hat, F, b_hat
+
+
+def merge_summaries(F_c: np.ndarray, k_hat_c: np.ndarray, qref: np.ndarray, scale: float):
+    """Parent summary from its children's per-reference state.
+
+    For each reference r independently (stable-state merge):
+      F_P   = LSE_c F_c
+      w_c   = exp(F_c - F_P)            (share of the parent's mass in child c)
+      k_hat = sum_c w_c k_hat_c
+      b_hat = F_P - q_hat_r . k_hat * scale
+    F_c: [C, R], k_hat_c: [C, R, d].  Returns (k_hat [R, d], F [R], b_hat [R]).
+    """
+    F = lse(F_c, axis=0)                         # [R]
+    w = np.exp(F_c - F[None, :])                 # [C, R]
+    k_hat = np.einsum("cr,crd->rd", w, k_hat_c)
+    b_hat = F - np.sum(qref * k_hat, axis=-1) * scale
+    return k_hat, F, b_hat
+
+
+# ---------------------------------------------------------------------------
+# the tree of one (batch, KV head) unit
+# ---------------------------------------------------------------------------
+
+
+@dataclass
+class Level:
+    span: int                      # keys per node
+    k_route: np.ndarray            # [n, R, d] routing copy of k_hat (stored precision)
+    b_hat: np.ndarray              # [n, R]    (stored precision)
+    F: np.ndarray                  # [n, R]    merge state (stored precision)
+    k_state: np.ndarray            # [n, R, d] merge state (stored precision)
+
+    @property
+    def n(self) -> int:
+        return self.k_route.shape[0]
+
+
+@dataclass
+class Tree:
+    leaf: int
+    branch: int
+    depth: int
+    levels: List[Level] = field(default_factory=list)   # levels[l-1] is level l
+
+    def span(self, level: int) -> int:
+        return self.leaf * self.branch ** (level - 1)
+
+
+def _store_level(span, k_hat, F, b_hat, route_storage, state_storage):
+    return Level(span=span,
+                 k_route=round_to(k_hat, route_storage),
+                 b_hat=round_to(b_hat, "f32" if state_storage != "f64" else "f64"),
+                 F=round_to(F, state_storage),
+                 k_state=round_to(k_hat, state_storage))
+
+
+def build_tree(K: np.ndarray, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
+               branch: int = 16, route_storage: str = "bf16", state_storage: str = "f32",
+               block: int = 4096) -> Tree:
+    """All full nodes over keys [0, T) of one unit.
+
+    K: [>=T, d] keys (float64 values of the stored keys), qref: [R, d].
+    Level 1 summarises raw keys (``leaf_summary``); level l >= 2 merges the
+    stored state of ``branch`` consecutive level-(l-1) nodes (``merge_summaries``).
+    ``block`` only bounds the temporary memory of the vectorised leaf pass.
+    """
+    d = K.shape[1]
+    scale = 1.0 / math.sqrt(d)
+    R = qref.shape[0]
+    tree = Tree(leaf=leaf, branch=branch, depth=depth)
+    n1 = T // leaf
+    k1 = np.zeros((n1, R, d))
+    F1 = np.zeros((n1, R))
+    b1 = np.zeros((n1, R))
+    for i0 in range(0, n1, block):
+        i1 = min(n1, i0 + block)
+        Kc = K[i0 * leaf:i1 * leaf].reshape(i1 - i0, leaf, d)
+        s = np.einsum("rd,ncd->nrc", qref, Kc) * scale
+        F = lse(s, axis=-1)
+        a = np.exp(s - F[..., None])
+        kh = np.einsum("nrc,ncd->nrd", a, Kc)
+        k1[i0:i1] = kh
+        F1[i0:i1] = F
+        b1[i0:i1] = F - np.einsum("rd,nrd->nr", qref, kh) * scale
+    tree.levels.append(_store_level(leaf, k1, F1, b1, route_storage, state_storage))
+    for lvl in range(2, depth + 1):
+        child = tree.levels[-1]
+        n = child.n // branch
+        Fc = child.F[:n * branch].reshape(n, branch, R)
+        kc = child.k_state[:n * branch].reshape(n, branch, R, d)
+        F = lse(Fc, axis=1)                                     # [n, R]
+        w = np.exp(Fc - F[:, None, :])                          # [n, C, R]
+        kh = np.einsum("ncr,ncrd->nrd", w, kc)
+        bh = F - np.einsum("rd,nrd->nr", qref, kh) * scale
+        tree.levels.append(_store_level(tree.span(lvl), kh, F, bh, route_storage, state_storage))
+    return tree
+
+
+# ---------------------------------------------------------------------------
+# routing (summary page, Routing; paper §III-B normaliser over candidates, §III-C)
+# ---------------------------------------------------------------------------
+
+
+def node_scores(q: np.ndarray, level: Level, ids: np.ndarray, scale: float) -> np.ndarray:
+    """s(q) = max_r [ q . k_hat_r * scale + b_hat_r ] for the nodes ``ids``."""
+    t = np.einsum("d,nrd->nr", q, level.k_route[ids]) * scale + level.b_hat[ids]
+    return np.max(t, axis=-1)
+
+
+@dataclass
+class Selection:
+    ids: np.ndarray        # selected node ids, ascending
+    m: int                 # number selected
+    n: int                 # number of candidates
+    margin: float          # min(cum_m - p, p - cum_{m-1}); inf when p >= 1 or m == n without reaching p
+    gap: float             # pi_(m) - pi_(m+1) (inf if m == n)
+
+
+def top_p(scores: np.ndarray, ids: np.ndarray, p: float) -> Selection:
+    """Smallest prefix (scores desc, ids asc) whose softmax mass reaches p."""
+    n = len(ids)
+    if n == 0:
+        return Selection(np.zeros(0, np.int64), 0, 0, math.inf, math.inf)
+    order = np.lexsort((ids, -scores))
+    s = scores[order]
+    e = np.exp(s - s[0])
+    pi = e / np.sum(e)
+    cum = np.cumsum(pi)
+    if p >= 1.0:
+        m = n
+        margin = math.inf
+    else:
+        hit = np.nonzero(cum >= p)[0]
+        m = int(hit[0]) + 1 if len(hit) else n
+        before = cum[m - 2] if m >= 2 else 0.0
+        margin = min(cum[m - 1] - p, p - before) if len(hit) else abs(p - cum[-1])
+    gap = pi[m - 1] - pi[m] if m < n else math.inf
+    return Selection(np.sort(ids[order[:m]]), m, n, float(margin), float(gap))
+
+
+def visible_count(t: int, span: int, leaf: int) -> int:
+    """Full nodes of size ``span`` that end at or before the query's own chunk."""
+    return (leaf * (t // leaf)) // span
+
+
+@dataclass
+class Route:
+    top: int                                  # top level routed (0: nothing visible)
+    cand: Dict[int, np.ndarray]               # level -> candidate ids (ascending)
+    sel: Dict[int, Selection]                 # level -> selection
+    leaves: np.ndarray                        # S_1(q), ascending chunk ids
+
+
+def route(q: np.ndarray, t: int, tree: Tree, p: float) -> Route:
+    """Top-down top-p routing of one query head at position ``t``.
+
+    The top level is the highest level with a visible node; all its visible
+    nodes are candidates.  Below it, the candidates are the children of the
+    selected nodes plus the visible nodes whose parent is not visible.
+    """
+    d = q.shape[0]
+    scale = 1.0 / math.sqrt(d)
+    nvis = {l: visible_count(t, tree.span(l), tree.leaf) for l in range(1, tree.depth + 1)}
+    for l in nvis:
+        if l <= len(tree.levels) and nvis[l] > tree.levels[l - 1].n:
+            raise ValueError(f"level {l}: {nvis[l]} nodes visible at t={t} but only "
+                             f"{tree.levels[l - 1].n} built")
+    top = max([l for l in nvis if nvis[l] >= 1], default=0)
+    out = Route(top=top, cand={}, sel={}, leaves=np.zeros(0, np.int64))
+    if top == 0:
+        return out
+    cand = np.arange(nvis[top], dtype=np.int64)
+    for l in range(top, 0, -1):
+        s = node_scores(q, tree.levels[l - 1], cand, scale)
+        sel = top_p(s, cand, p)
+        out.cand[l] = cand
+        out.sel[l] = sel
+        if l > 1:
+            children = (sel.ids[:, None] * tree.branch + np.arange(tree.branch)[None, :]).ravel()
+            orphans = np.arange(nvis[l] * tree.branch, nvis[l - 1], dtype=np.int64)
+            cand = np.concatenate([children, orphans]).astype(np.int64)
+    out.leaves = out.sel[1].ids
+    return out
+
+
+def index_set(leaves: Sequence[int], t: int, leaf: int = 64) -> np.ndarray:
+    """I(q) = {0} u (keys of the selected leaf chunks) u C_cur(q), ascending.
+
+    C_cur(q) holds the keys of the query's own chunk up to and including t.
+    """
+    v = leaf * (t // leaf)
+    parts = [np.array([0], np.int64), np.arange(v, t + 1, dtype=np.int64)]
+    for c in leaves:
+        parts.append(np.arange(c * leaf, (c + 1) * leaf, dtype=np.int64))
+    return np.unique(np.concatenate(parts))
+
+
+# ---------------------------------------------------------------------------
+# attention (summary page, Routing: o(q) = Attn(q, K_I, V_I))
+# ---------------------------------------------------------------------------
+
+
+def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray):
+    """Softmax attention of q over the keys ``idx``.  Returns (o [d], lse)."""
+    scale = 1.0 / math.sqrt(q.shape[0])
+    z = K[idx] @ q * scale
+    m = np.max(z)
+    e = np.exp(z - m)
+    return (e @ V[idx]) / np.sum(e), float(m + np.log(np.sum(e)))
+
+
+def dense_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int):
+    """Causal dense attention over keys [0, t]."""
+    return attention(q, K, V, np.arange(t + 1))
+
+
+def flat_scores(q: np.ndarray, K: np.ndarray, t: int, leaf: int = 64) -> np.ndarray:
+    """Exact chunk log-mass F_C(q) of every visible leaf chunk (flat indexer)."""
+    d = q.shape[0]
+    n = visible_count(t, leaf, leaf)
+    if n == 0:
+        return np.zeros(0)
+    z = (K[:n * leaf] @ q) / math.sqrt(d)
+    return lse(z.reshape(n, leaf), axis=-1)
+
+
+def flat_select(q: np.ndarray, K: np.ndarray, t: int, p: float, leaf: int = 64) -> Selection:
+    """Top-p over all visible leaf chunks scored by their exact log-mass."""
+    s = flat_scores(q, K, t, leaf)
+    return top_p(s, np.arange(len(s), dtype=np.int64), p)
+
+
+# ---------------------------------------------------------------------------
+# whole-path helpers over [B, Hkv, t, d] caches
+# ---------------------------------------------------------------------------
+
+
+def build_unit_trees(K: np.ndarray, T: int, qref: np.ndarray, depth: int,
+                     route_storage: str, units: Optional[Sequence[tuple]] = None,
+                     leaf: int = 64, branch: int = 16, state_storage: str = "f32"):
+    """Trees of the (b, h_kv) ``units`` (all when None).  K: [B, Hkv, >=T, d]."""
+    B, Hkv = K.shape[:2]
+    units = units if units is not None else [(b, h) for b in range(B) for h in range(Hkv)]
+    return {u: build_tree(np.asarray(K[u[0], u[1]], np.float64), T, np.asarray(qref[u[1]], np.float64),
+                          depth, leaf, branch, route_storage, state_storage) for u in units}
+
+
+def decode_head(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int, tree: Tree, p: float):
+    """Route one query head and attend over its index set.  Returns (route, o, lse)."""
+    r = route(q, t, tree, p)
+    o, l = attention(q, K, V, index_set(r.leaves, t, tree.leaf))
+    return r, o, l
