@@ -1,0 +1,406 @@
+"""Benchmark of the ZHA decode hot path on B200.
+
+One step = one decode token for every sequence of the workload: append the new key/value
+(and summarise any node it completes), route every query head top-down with top-p, and
+attend over the selected index set (zha_decode: all kernels of the hot path).  Inputs are
+seeded synthetic clustered keys; the KV cache (8 GiB for the default workload) is larger
+than L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zha|reference]
+                    [--workload NAME] [--p P]
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own independent replica of
+the workload (the path shards over (sequence, KV head) units with no exchange), so the
+scaling is weak and the reported value is the sum over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+import zha_synth as S  # noqa: E402
+
+DEFAULT_WORKLOAD = "batched-decode-128k"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="zha", choices=["zha", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(S.WORKLOADS))
+    ap.add_argument("--p", type=float, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    return ap.parse_args()
+
+
+# ---------------------------------------------------------------------------
+# process group
+# ---------------------------------------------------------------------------
+
+
+def dist_setup(n):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, ws: int) -> float:
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.path = tempfile.mktemp(suffix=".csv")
+        self.proc = None
+        sel = []
+        try:
+            bus = torch.cuda.get_device_properties(device).pci_bus_id
+            sel = ["-i", bus]
+        except Exception:
+            sel = ["-i", str(device)]
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        self.t_start = self.t_end = None
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9], parts[4]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        # keep the samples taken while the GPU was busy (highest-clock half if the tail idles)
+        sm = [r[0] for r in rows]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[2]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host cores (CPU baseline and reference arm)
+# ---------------------------------------------------------------------------
+
+
+def oracle_rate(w: S.Workload, p: float, seconds: float, device: str):
+    """Query-heads/s of the CPU oracle on a bounded sample of the decode step.
+
+    The sample: whole KV groups (G query heads of one (sequence, KV head) unit) of the
+    same seeded workload, routed and attended by the oracle one head at a time until
+    ``seconds`` of CPU time have been spent (at least one group).  The oracle's tree of
+    each sampled unit is built first, untimed (it is the decode step's prior state).
+    """
+    from oracle import zha_oracle as zo
+    try:
+        from threadpoolctl import threadpool_limits
+        limiter = threadpool_limits(1)
+    except Exception:  # pragma: no cover
+        limiter = None
+    one = S.scaled(w, T=w.T, B=1)
+    C, K, V = S.clustered_kv(one, device)
+    qref = S.reference_queries(one, device)
+    kn, vn = S.new_tokens(one, C, 1, device)
+    q = S.queries(one, C, 1, device)
+    K[:, :, w.T] = kn[:, 0]
+    V[:, :, w.T] = vn[:, 0]
+    Kc, Vc = K.cpu(), V.cpu()
+    qc = q.double().cpu().numpy()
+    qr = qref.double().cpu().numpy()
+    heads, spent = 0, 0.0
+    for hk in range(w.Hkv):
+        tree = zo.build_tree(Kc[0, hk], w.T + 1, qr[hk], w.depth,
+                             route_storage="bf16" if w.dtype == "bf16" else "f32")
+        t0 = time.process_time()
+        for h in range(hk * w.G, (hk + 1) * w.G):
+            zo.decode_head(qc[0, 0, h], Kc[0, hk], Vc[0, hk], w.T, tree, p)
+            heads += 1
+        spent += time.process_time() - t0
+        if spent >= seconds:
+            break
+    if limiter is not None:
+        limiter.unregister() if hasattr(limiter, "unregister") else None
+    return heads / spent, heads, spent
+
+
+def run_reference(args, w, p, ws, rank):
+    if rank != 0:
+        return
+    K, W = args.steps, args.warmup
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    per_step = max(1.0, 150.0 / max(1, K + W))
+    rates = []
+    for i in range(W + K):
+        r, heads, spent = oracle_rate(w, p, min(per_step, args.cpu_seconds), dev)
+        if i >= W:
+            rates.append((r, heads, spent))
+    value = statistics.median(r[0] for r in rates)
+    ms = 1e3 * w.B * w.Hq / value
+    line = {
+        "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": 1,
+        "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, p), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{rates[0][1]} query heads (whole KV groups) per step, fp64 numpy, 1 thread"},
+        "e2e": {"value": value, "unit": "query-heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, p):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "depth": w.depth,
+            "leaf": w.leaf, "branch": w.branch, "R": w.R, "p": p, "n_centres": w.n_centres,
+            "kv_bytes": 2 * w.B * w.Hkv * w.T * w.d * (2 if w.dtype == "bf16" else 4),
+            "l2": "no flush: the KV cache read per step is larger than the 126 MB L2"}
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+
+
+def main():
+    args = parse()
+    w = S.workload(args.workload)
+    p = args.p if args.p is not None else w.p[0]
+    ws, rank, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        run_reference(args, w, p, ws, rank)
+        barrier(ws)
+        return
+
+    import hierarchical_sparse_attention_02_b200 as Z
+    from hierarchical_sparse_attention_02_b200 import _lib
+    Z.load_library()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    wr = S.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
+    g = Z.Geometry(B=w.B, Hq=w.Hq, Hkv=w.Hkv, t_cap=w.t_cap, depth=w.depth, R=w.R, d=w.d,
+                   dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+    C, K, V = S.clustered_kv(wr, dev)
+    qref = S.reference_queries(wr, dev)
+    k_new, v_new = S.new_tokens(wr, C, 1, dev)
+    q = S.queries(wr, C, 1, dev)
+    del C
+    tree = Z.empty_tree(g, dev)
+    wsb = Z.empty_workspace(g, 1, Z.ZHA_OP_DECODE, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    cap = Z.leaf_cap(g)
+    ids = torch.empty(w.B, 1, w.Hq, cap, dtype=torch.int32, device=dev)
+    cnt = torch.empty(w.B, 1, w.Hq, dtype=torch.int32, device=dev)
+    O = torch.empty(w.B, 1, w.Hq, w.d, dtype=g.dtype, device=dev)
+    stream = torch.cuda.current_stream()
+
+    # tree build (prefill of the summaries), timed once
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Z.zha_build_tree(g, K, w.T, qref, tree, st)          # warm
+    torch.cuda.synchronize()
+    e0.record(); Z.zha_build_tree(g, K, w.T, qref, tree, st); e1.record()
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    k_bytes = w.B * w.Hkv * w.T * w.d * (2 if w.dtype == "bf16" else 4)
+
+    def step():
+        Z.zha_decode(g, q, k_new, v_new, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if st.item() != 0:
+        raise RuntimeError(f"device status {st.item()} after warm-up")
+
+    Ksteps = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(Ksteps)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(Ksteps)]
+    arr_s = (ctypes.c_void_p * Ksteps)(*[ctypes.c_void_p(e.cuda_event) for e in starts])
+    arr_e = (ctypes.c_void_p * Ksteps)(*[ctypes.c_void_p(e.cuda_event) for e in stops])
+    lib = _lib.load()
+    clocks = ClockSampler(torch.cuda.current_device())
+    time.sleep(0.3)
+    barrier(ws)
+    torch.cuda.synchronize()
+    lib.zha_trace(_lib.ZHA_TRACE_ATTN, arr_s, arr_e, Ksteps)
+    n_launch0 = Z.launch_count()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
+    t_start.record(stream)
+    for _ in range(Ksteps):
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark_end()
+    barrier(ws)
+    launches = Z.launch_count() - n_launch0
+    traced = lib.zha_trace_count(_lib.ZHA_TRACE_ATTN)
+    lib.zha_trace(_lib.ZHA_TRACE_ATTN, None, None, 0)
+    ms_local = t_start.elapsed_time(t_end) / Ksteps
+    attn_ms = sum(a.elapsed_time(b) for a, b in zip(starts[:traced], stops[:traced])) / max(1, traced)
+    if st.item() != 0:
+        raise RuntimeError(f"device status {st.item()} in the timed region")
+    ms = max_over_ranks(ms_local, ws)
+
+    # end to end through the public API with host buffers
+    pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
+    hq, hk, hv, hO = pin(q), pin(k_new), pin(v_new), pin(O)
+    hq.copy_(q); hk.copy_(k_new); hv.copy_(v_new)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k_new), torch.empty_like(v_new)
+
+    def e2e_step():
+        dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
+        Z.zha_decode(g, dq, dk, dv, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st)
+        hO.copy_(O, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(Ksteps):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / Ksteps, ws)
+    barrier(ws)
+    clk = clocks.stop()
+
+    # workload statistics (untimed): index-set sizes, KV-group unions, frontiers
+    es = 2 if w.dtype == "bf16" else 4
+    T1 = w.T + 1
+    vstart = (w.T // 64) * 64
+    partial = w.T - vstart + 1
+    ids_c, cnt_c = ids.cpu().numpy(), cnt.cpu().numpy()
+    per_head, union_rows, entries = [], 0, 0
+    for bb in range(w.B):
+        for hkv in range(w.Hkv):
+            lists = [ids_c[bb, 0, h, :cnt_c[bb, 0, h]] for h in range(hkv * w.G, (hkv + 1) * w.G)]
+            for lst in lists:
+                has0 = len(lst) and lst[0] == 0
+                per_head.append((len(lst) * 64 + (0 if has0 else 1) + partial) / T1)
+            u = np.unique(np.concatenate(lists)) if lists else np.zeros(0)
+            sink = any(not (len(l) and l[0] == 0) for l in lists) and vstart >= 64
+            union_rows += len(u) * 64 + (1 if sink else 0) + partial
+            entries += len(u) + (1 if sink else 0) + 1
+    units = w.B * w.Hkv
+    c1 = w.t_cap // 64
+    cps = max(16, -(-units * (c1 + 2) // 16384))
+    items = -(-entries // cps)                                        # ranges: one per unit here
+    gathered = union_rows * 2 * w.d * es
+    partial_bytes = items * w.G * (w.d + 2) * 4
+    attn_bytes = gathered + partial_bytes
+    peak, peak_kind = hbm_peak()
+    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+    value = ws * w.B * w.Hq / (ms * 1e-3)
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda")
+        cpu = {"value": r, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
+               "sample": f"{heads} query heads (whole KV groups of sequence 0) of {w.name}, "
+                         f"route + attention, fp64 numpy, 1 thread, {spent:.1f} s CPU"}
+    line = {
+        "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": ws,
+        "steps": Ksteps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": config_of(w, p),
+        "roofline": {"bound": "hbm", "kernel": "attn_split_kernel", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "algorithmic_bytes_per_launch": attn_bytes, "kernel_ms": attn_ms},
+        "step_hbm_gbs": attn_bytes / (ms * 1e-3) / 1e9,
+        "kv_touched": {"mean": float(np.mean(per_head)), "p50": float(np.median(per_head)),
+                       "p99": float(np.percentile(per_head, 99)),
+                       "group_union": union_rows / (units * T1)},
+        "tree_build": {"ms": build_ms, "gbs": k_bytes / (build_ms * 1e-3) / 1e9},
+        "e2e": {"value": ws * w.B * w.Hq / (e2e_ms * 1e-3), "unit": "query-heads/s",
+                "h2d_bytes_per_step": (q.numel() + k_new.numel() + v_new.numel()) * es,
+                "d2h_bytes_per_step": O.numel() * es},
+        "gpu_launches": launches,
+        "clocks": clk,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

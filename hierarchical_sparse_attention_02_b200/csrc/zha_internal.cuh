@@ -1,0 +1,244 @@
+// Internal helpers shared by the ZHA kernels: geometry arithmetic, buffer layouts,
+// exact number conversions, block reductions and the device status word.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <atomic>
+
+#include "zha.h"
+
+namespace zha {
+
+constexpr int kD = 128;          // head dimension supported by this build
+constexpr int kLeaf = 64;        // keys per leaf chunk
+constexpr int kMaxR = 16;        // reference queries per KV head
+constexpr int kMaxG = 8;         // query heads per KV head
+constexpr int kMaxDepth = 8;
+constexpr int kRange = 4096;     // chunk ids per union-building block
+constexpr size_t kAlign = 256;
+
+inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
+
+// ---------------------------------------------------------------------------
+// geometry (host)
+// ---------------------------------------------------------------------------
+
+inline int64_t span_of(const zha_geom& g, int level) {
+  int64_t s = g.leaf;
+  for (int l = 1; l < level; ++l) s *= g.branch;
+  return s;
+}
+
+inline int64_t ncap_of(const zha_geom& g, int level) { return g.t_cap / span_of(g, level); }
+
+inline int elem_bytes(const zha_geom& g) { return g.dtype == ZHA_BF16 ? 2 : 4; }
+
+struct TreeLayout {
+  zha_level_layout lv[kMaxDepth + 1];  // index = level (1..depth)
+  size_t bytes;
+};
+
+inline TreeLayout tree_layout(const zha_geom& g) {
+  TreeLayout t{};
+  size_t off = 0;
+  for (int l = 1; l <= g.depth; ++l) {
+    zha_level_layout& L = t.lv[l];
+    L.span = span_of(g, l);
+    L.n_cap = g.t_cap / L.span;
+    const size_t nodes = (size_t)g.B * g.Hkv * (size_t)L.n_cap;
+    L.k_route_off = off;
+    off = align_up(off + nodes * g.R * g.d * elem_bytes(g));
+    L.b_hat_off = off;
+    off = align_up(off + nodes * g.R * sizeof(float));
+    L.F_off = off;
+    off = align_up(off + nodes * g.R * sizeof(float));
+    L.k_state_off = off;
+    off = align_up(off + nodes * g.R * g.d * sizeof(float));
+  }
+  t.bytes = off;
+  return t;
+}
+
+// Split size (chunks per attention work item) chosen from the geometry only, so that
+// the workspace bound is known on the host: about 16K items per call, >= 16 chunks each.
+inline int64_t chunks_per_split(int64_t units, int64_t c1) {
+  const int64_t total = units * (c1 + 2);
+  int64_t cps = (total + 16383) / 16384;
+  return cps < 16 ? 16 : cps;
+}
+
+struct RouteWs {
+  size_t cand_ids, cand_score, cand_mass, selA, selB, cand_cnt, selA_cnt, selB_cnt, pos, bytes;
+  int64_t C1, C2;
+};
+
+inline RouteWs route_ws(const zha_geom& g, int nq, size_t base = 0) {
+  RouteWs w{};
+  const int64_t nqh = (int64_t)g.B * nq * g.Hq;
+  w.C1 = ncap_of(g, 1);
+  w.C2 = g.depth >= 2 ? ncap_of(g, 2) : 1;
+  if (w.C2 < 1) w.C2 = 1;
+  size_t off = base;
+  w.cand_ids = off;   off = align_up(off + (size_t)nqh * w.C1 * 4);
+  w.cand_score = off; off = align_up(off + (size_t)nqh * w.C1 * 8);
+  w.cand_mass = off;  off = align_up(off + (size_t)nqh * w.C1 * 8);
+  w.selA = off;       off = align_up(off + (size_t)nqh * w.C2 * 4);
+  w.selB = off;       off = align_up(off + (size_t)nqh * w.C2 * 4);
+  w.cand_cnt = off;   off = align_up(off + (size_t)nqh * 4);
+  w.selA_cnt = off;   off = align_up(off + (size_t)nqh * 4);
+  w.selB_cnt = off;   off = align_up(off + (size_t)nqh * 4);
+  w.pos = off;        off = align_up(off + (size_t)g.B * nq * 8);
+  w.bytes = off;
+  return w;
+}
+
+struct AttnWs {
+  size_t stage_ids, stage_mask, stage_cnt, pair_off, partials, pos, bytes;
+  int64_t units, nr, pairs, cps, items_max, C1;
+};
+
+inline AttnWs attn_ws(const zha_geom& g, int nq, size_t base = 0) {
+  AttnWs w{};
+  const int G = g.Hq / g.Hkv;
+  w.units = (int64_t)g.B * nq * g.Hkv;
+  w.C1 = ncap_of(g, 1);
+  w.nr = (w.C1 + 1 + kRange - 1) / kRange;
+  w.pairs = w.units * w.nr;
+  w.cps = chunks_per_split(w.units, w.C1);
+  w.items_max = w.pairs + (w.units * (w.C1 + 2) + w.cps - 1) / w.cps;
+  size_t off = base;
+  w.stage_ids = off;  off = align_up(off + (size_t)w.pairs * (kRange + 2) * 4);
+  w.stage_mask = off; off = align_up(off + (size_t)w.pairs * (kRange + 2) * 4);
+  w.stage_cnt = off;  off = align_up(off + (size_t)w.pairs * 4);
+  w.pair_off = off;   off = align_up(off + (size_t)(w.pairs + 1) * 4);
+  w.partials = off;   off = align_up(off + (size_t)w.items_max * G * (g.d + 2) * 4);
+  w.pos = off;        off = align_up(off + (size_t)g.B * nq * 8);
+  w.bytes = off;
+  return w;
+}
+
+// Host-side launch counter (exported as zha_launch_count).
+extern std::atomic<int64_t> g_launches;
+inline void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Event tracing around chosen kernels (zha_trace): record before / after one launch.
+struct Tracer {
+  void* const* start = nullptr;
+  void* const* stop = nullptr;
+  int n = 0, done = 0;
+};
+extern Tracer g_trace[4];
+inline void trace_begin(int which, cudaStream_t s) {
+  Tracer& t = g_trace[which];
+  if (t.done < t.n) cudaEventRecord((cudaEvent_t)t.start[t.done], s);
+}
+inline void trace_end(int which, cudaStream_t s) {
+  Tracer& t = g_trace[which];
+  if (t.done < t.n) { cudaEventRecord((cudaEvent_t)t.stop[t.done], s); ++t.done; }
+}
+
+// ---------------------------------------------------------------------------
+// device helpers
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ void set_status(int32_t* st, int32_t code) {
+  if (st) atomicCAS(st, 0, code);
+}
+
+// bf16 -> fp64 exactly, with integer operations: a normal bf16 value maps to the double
+// with the same sign, the exponent rebased from 127 to 1023, the 7 mantissa bits on top
+// of the 52-bit mantissa.  Zero and subnormals take the (exact) float path.
+__device__ __forceinline__ double bf16_bits_to_f64(uint32_t h) {
+  const uint32_t mag = h & 0x7fffu;
+  if ((mag & 0x7f80u) == 0u || (mag & 0x7f80u) == 0x7f80u) {
+    return (double)__uint_as_float(h << 16);
+  }
+  const uint32_t hi = ((h & 0x8000u) << 16) | ((mag + ((1023u - 127u) << 7)) << 13);
+  return __hiloint2double((int)hi, 0);
+}
+
+__device__ __forceinline__ double to_f64(float x) { return (double)x; }
+__device__ __forceinline__ double to_f64(__nv_bfloat16 x) {
+  return bf16_bits_to_f64((uint32_t)__bfloat16_as_ushort(x));
+}
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// fp64 -> storage type, a single round-to-nearest-even.
+__device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rn(double x) {
+  unsigned short r;
+  asm("cvt.rn.bf16.f64 %0, %1;" : "=h"(r) : "d"(x));
+  return __ushort_as_bfloat16(r);
+}
+template <typename T> __device__ __forceinline__ T from_f64(double x);
+template <> __device__ __forceinline__ float from_f64<float>(double x) { return __double2float_rn(x); }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f64<__nv_bfloat16>(double x) { return f64_to_bf16_rn(x); }
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
+
+__device__ __forceinline__ double shfl_xor_f64(double v, int m) { return __shfl_xor_sync(0xffffffffu, v, m); }
+
+// Position of the query of (b, qi): from q_pos, or the uniform position when q_pos is null.
+__device__ __forceinline__ int64_t query_pos(const int64_t* q_pos, int64_t uniform, int64_t bq) {
+  return q_pos ? q_pos[bq] : uniform;
+}
+
+// Visible full nodes of size `span` for a query at position t.
+__device__ __forceinline__ int64_t visible_nodes(int64_t t, int64_t span) {
+  return ((t / kLeaf) * kLeaf) / span;
+}
+
+// ---------------------------------------------------------------------------
+// internal calls composed by the C ABI
+// ---------------------------------------------------------------------------
+
+struct RouteCall {
+  const zha_geom* g;
+  int nq;
+  const void* Q;
+  const int64_t* q_pos;          // [B, nq] device, or null: every query at pos_uniform
+  int64_t pos_uniform;
+  double p;
+  void* tree;                    // tree buffer (route_all) or the K cache (flat_select)
+  int* leaf_ids;
+  int* leaf_cnt;
+  int leaf_cap;
+  int* level_cnt;
+  int* level_ids;
+  char* ws;                      // workspace base, layout route_ws(g, nq, 0)
+  int32_t* dev_status;
+  cudaStream_t stream;
+};
+
+struct AttnCall {
+  const zha_geom* g;
+  int nq;
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int64_t* q_pos;
+  int64_t pos_uniform;
+  int dense;                     // 1: every key [0, t] (baseline), 0: the routed index set
+  const int* leaf_ids;
+  const int* leaf_cnt;
+  int leaf_cap;
+  void* O;
+  float* lse;
+  char* ws;                      // workspace base, layout attn_ws(g, nq, 0)
+  int32_t* dev_status;
+  cudaStream_t stream;
+};
+
+cudaError_t tree_extend(const zha_geom& g, const void* K, const float* qref, void* tree,
+                        int64_t t_old, int64_t t_new, cudaStream_t s);
+cudaError_t append_tokens(const zha_geom& g, void* K, void* V, const void* k_new,
+                          const void* v_new, int64_t t_old, int n_new, cudaStream_t s);
+cudaError_t route_all(const RouteCall& c);
+cudaError_t flat_select(const RouteCall& c);
+cudaError_t attention(const AttnCall& c);
+
+}  // namespace zha

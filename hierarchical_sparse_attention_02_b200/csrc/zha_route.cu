@@ -1,0 +1,588 @@
+// Top-down adaptive top-p routing ("ZHA summary" page, Routing; arXiv 2610.42112 §III-C,
+// App. E-E) and the flat exact-log-mass indexer used as a baseline.
+//
+// One level is two kernels over all (query, query head) pairs:
+//   score : candidate ids of the level (top level: every visible node; below: the
+//           children of the kept parents, then the visible nodes whose parent is not
+//           visible) and their scores s = max_r [q . k_hat_r / sqrt(d) + b_hat_r], in fp64.
+//   select: per query head, the smallest prefix of the candidates ordered by
+//           (score desc, id asc) whose softmax mass reaches p.  Masses are fixed-point
+//           integers 2^S * exp(s - max), so the sums are exact and order-free; the cutoff
+//           is found by a radix select over the order-preserving 64-bit key of s, and
+//           the kept ids are compacted in ascending order with a block scan.
+#include "zha_internal.cuh"
+
+namespace zha {
+
+struct RouteGeom {
+  int B, nq, Hq, Hkv, G, R, branch, depth;
+  int64_t span[kMaxDepth + 2];   // span[l], l = 1..depth (span[depth+1] unused)
+  int64_t ncap[kMaxDepth + 2];
+  const int64_t* q_pos;          // [B, nq] or null
+  int64_t pos_uniform;
+  int64_t t_cap;
+};
+
+// Positions outside [0, t_cap) are rejected on the device: the query routes nothing.
+__device__ __forceinline__ bool pos_ok(const RouteGeom& g, int64_t t) { return t >= 0 && t < g.t_cap; }
+
+// Highest level with a visible node for a query at position t (0 if none).
+__device__ __forceinline__ int top_level(const RouteGeom& g, int64_t t) {
+  for (int l = g.depth; l >= 1; --l)
+    if (visible_nodes(t, g.span[l]) >= 1) return l;
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
+// score kernel: 128 threads, one candidate per thread; persistent over (qh, block)
+// ---------------------------------------------------------------------------
+
+struct ScoreArgs {
+  RouteGeom g;
+  int level;
+  const void* Q;                 // [B, nq, Hq, d]
+  const void* k_route;           // level's routing k_hat [B, Hkv, ncap, R, d]
+  const float* b_hat;            // [B, Hkv, ncap, R]
+  const int* parents;            // kept ids of level+1, [nqh, C2]
+  const int* parents_cnt;        // [nqh]
+  int64_t C1, C2;
+  int* cand_ids;                 // [nqh, C1]
+  double* cand_score;            // [nqh, C1]
+  int* cand_cnt;                 // [nqh]
+  int64_t nblk;                  // candidate blocks per query head
+  int32_t* dev_status;
+};
+
+template <typename KT>
+__global__ void __launch_bounds__(128) route_score_kernel(ScoreArgs a) {
+  __shared__ double qs[kD];
+  const RouteGeom& g = a.g;
+  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
+  const double scale = 1.0 / sqrt((double)kD);
+  for (int64_t w = blockIdx.x; w < nqh * a.nblk; w += gridDim.x) {
+    const int64_t qh = w / a.nblk;
+    const int64_t blk = w % a.nblk;
+    const int64_t bq = qh / g.Hq;
+    const int hq = (int)(qh % g.Hq);
+    const int64_t b = bq / g.nq;
+    const int hk = hq / g.G;
+    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
+    if (!pos_ok(g, t)) {
+      if (blk == 0 && threadIdx.x == 0) set_status(a.dev_status, ZHA_ERR_INVALID_ARG);
+      continue;
+    }
+    const int top = top_level(g, t);
+    if (a.level > top) continue;                       // uniform over the CTA
+    const int64_t nvis = visible_nodes(t, g.span[a.level]);
+    int64_t n, nchild = 0, orph_lo = 0;
+    const int* par = a.parents + qh * a.C2;
+    if (a.level == top) {
+      n = nvis;
+    } else {
+      nchild = (int64_t)a.parents_cnt[qh] * g.branch;
+      orph_lo = visible_nodes(t, g.span[a.level + 1]) * g.branch;
+      n = nchild + (nvis - orph_lo);
+    }
+    if (blk == 0 && threadIdx.x == 0) a.cand_cnt[qh] = (int)n;
+    const int64_t k = blk * 128 + threadIdx.x;
+    if (blk * 128 >= n) continue;                      // uniform over the CTA
+    __syncthreads();
+    const KT* q = reinterpret_cast<const KT*>(a.Q) + qh * kD;
+    qs[threadIdx.x] = to_f64(q[threadIdx.x]);
+    __syncthreads();
+    if (k >= n) continue;
+    int64_t id;
+    if (a.level == top) id = k;
+    else if (k < nchild) id = (int64_t)par[k / g.branch] * g.branch + k % g.branch;
+    else id = orph_lo + (k - nchild);
+    const int64_t node = ((b * g.Hkv + hk) * g.ncap[a.level] + id);
+    const KT* kr = reinterpret_cast<const KT*>(a.k_route) + node * g.R * kD;
+    const float* bh = a.b_hat + node * g.R;
+    double best = -INFINITY;
+    for (int r = 0; r < g.R; ++r) {
+      double acc = 0.0;
+      const KT* row = kr + r * kD;
+      constexpr int kVec = 16 / sizeof(KT);
+#pragma unroll 4
+      for (int c = 0; c < kD; c += kVec) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + c);
+        const KT* e = reinterpret_cast<const KT*>(&v);
+#pragma unroll
+        for (int u = 0; u < kVec; ++u) acc = fma(qs[c + u], to_f64(e[u]), acc);
+      }
+      const double s = fma(acc, scale, (double)bh[r]);
+      best = fmax(best, s);
+    }
+    if (best == 0.0) best = 0.0;                       // one zero (no -0.0) for the key order
+    a.cand_ids[qh * a.C1 + k] = (int)id;
+    a.cand_score[qh * a.C1 + k] = best;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// flat indexer scores: F_C(q) of every visible chunk, all G heads of a KV head per CTA
+// ---------------------------------------------------------------------------
+
+struct FlatArgs {
+  RouteGeom g;
+  const void* Q;
+  const void* K;                 // [B, Hkv, t_cap, d]
+  int64_t t_cap;
+  int64_t C1;
+  int* cand_ids;
+  double* cand_score;
+  int* cand_cnt;
+  int64_t nblk;                  // chunk blocks (of 8 chunks) per unit
+};
+
+template <typename KT>
+__global__ void __launch_bounds__(256) flat_score_kernel(FlatArgs a) {
+  // 8 warps; warp w handles chunk (blk*8 + w) for every head of the unit
+  __shared__ float qs[kMaxG][kD];
+  const RouteGeom& g = a.g;
+  const int64_t units = (int64_t)g.B * g.nq * g.Hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const float scale = 1.0f / sqrtf((float)kD);
+  for (int64_t w = blockIdx.x; w < units * a.nblk; w += gridDim.x) {
+    const int64_t u = w / a.nblk, blk = w % a.nblk;
+    const int64_t bq = u / g.Hkv;
+    const int hk = (int)(u % g.Hkv);
+    const int64_t b = bq / g.nq;
+    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
+    const int64_t nvis = pos_ok(g, t) ? visible_nodes(t, kLeaf) : 0;
+    if (blk == 0 && threadIdx.x < g.G) a.cand_cnt[bq * g.Hq + hk * g.G + threadIdx.x] = (int)nvis;
+    if (blk * 8 >= nvis) continue;
+    __syncthreads();
+    for (int i = threadIdx.x; i < g.G * kD; i += blockDim.x) {
+      const KT* q = reinterpret_cast<const KT*>(a.Q) + (bq * g.Hq + hk * g.G) * kD;
+      qs[i / kD][i % kD] = to_f32(q[i]);
+    }
+    __syncthreads();
+    const int64_t c = blk * 8 + warp;
+    if (c >= nvis) continue;
+    // lane handles keys lane and lane + 32 of the chunk
+    const KT* k0 = reinterpret_cast<const KT*>(a.K) + ((b * g.Hkv + hk) * a.t_cap + c * kLeaf) * kD;
+    float s0[kMaxG], s1[kMaxG];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) s0[h] = s1[h] = 0.f;
+    const KT* ra = k0 + lane * kD;
+    const KT* rb = k0 + (lane + 32) * kD;
+    constexpr int kVec = 16 / sizeof(KT);
+    for (int cc = 0; cc < kD; cc += kVec) {
+      const uint4 va = *reinterpret_cast<const uint4*>(ra + cc);
+      const uint4 vb = *reinterpret_cast<const uint4*>(rb + cc);
+      const KT* ea = reinterpret_cast<const KT*>(&va);
+      const KT* eb = reinterpret_cast<const KT*>(&vb);
+#pragma unroll
+      for (int uu = 0; uu < kVec; ++uu) {
+        const float xa = to_f32(ea[uu]), xb = to_f32(eb[uu]);
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+          if (h < g.G) {
+            s0[h] = fmaf(qs[h][cc + uu], xa, s0[h]);
+            s1[h] = fmaf(qs[h][cc + uu], xb, s1[h]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h >= g.G) break;
+      const float x0 = s0[h] * scale, x1 = s1[h] * scale;
+      float m = fmaxf(x0, x1);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      float z = expf(x0 - m) + expf(x1 - m);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+      if (lane == 0) {
+        const int64_t qh = bq * g.Hq + hk * g.G + h;
+        double F = (double)m + log((double)z);
+        if (F == 0.0) F = 0.0;
+        a.cand_ids[qh * a.C1 + c] = (int)c;
+        a.cand_score[qh * a.C1 + c] = F;
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// select kernel: one CTA of 512 threads per query head (persistent)
+// ---------------------------------------------------------------------------
+
+constexpr int kSelThreads = 512;
+constexpr int kDigit = 11;
+constexpr int kBuckets = 1 << kDigit;
+
+struct SelectArgs {
+  RouteGeom g;
+  int level;
+  int flat;                      // 1: a single level over all visible leaves
+  double p;
+  int mass_shift;                // fixed-point scale 2^mass_shift
+  const int* cand_ids;
+  const double* cand_score;
+  unsigned long long* cand_mass;
+  const int* cand_cnt;
+  int64_t C1;
+  int* out_ids;                  // [nqh, out_stride]
+  int* out_cnt;                  // [nqh]
+  int64_t out_stride;
+  int out_cap;
+  int* level_cnt;                // nullable [nqh, depth, 2]
+  int* level_ids;                // nullable [nqh, level_ids_stride]
+  int64_t level_ids_stride, level_ids_off, level_ids_cap;
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ unsigned long long order_key(double s) {
+  const unsigned long long b = (unsigned long long)__double_as_longlong(s);
+  return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
+}
+
+struct SelSmem {
+  unsigned int cnt[kBuckets];
+  unsigned long long mass[kBuckets];
+  unsigned long long wsum[kSelThreads / 32];
+  double wd[kSelThreads / 32];
+  unsigned int wcnt[kSelThreads / 32];
+  unsigned long long bc_u64[4];
+  double bc_f64[2];
+  int bc_int[4];
+};
+
+__device__ __forceinline__ double block_max_f64(double v, SelSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, shfl_xor_f64(v, o));
+  __syncthreads();
+  if (lane == 0) sm.wd[warp] = v;
+  __syncthreads();
+  double r = sm.wd[0];
+  for (int i = 1; i < kSelThreads / 32; ++i) r = fmax(r, sm.wd[i]);
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v, SelSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) sm.wsum[warp] = v;
+  __syncthreads();
+  unsigned long long r = 0;
+  for (int i = 0; i < kSelThreads / 32; ++i) r += sm.wsum[i];
+  return r;
+}
+
+// Exclusive block scan of small counts in thread order; returns the block total in *total.
+__device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, SelSmem& sm, unsigned int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) sm.wcnt[warp] = x;
+  __syncthreads();
+  unsigned int before = 0, all = 0;
+  for (int i = 0; i < kSelThreads / 32; ++i) {
+    if (i < warp) before += sm.wcnt[i];
+    all += sm.wcnt[i];
+  }
+  *total = all;
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(kSelThreads) route_select_kernel(SelectArgs a) {
+  __shared__ SelSmem sm;
+  const RouteGeom& g = a.g;
+  const int tid = threadIdx.x;
+  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
+  for (int64_t qh = blockIdx.x; qh < nqh; qh += gridDim.x) {
+    const int64_t bq = qh / g.Hq;
+    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
+    const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
+    int* lc = a.level_cnt ? a.level_cnt + (qh * g.depth + (a.level - 1)) * 2 : nullptr;
+    if (a.level > top) {
+      if (tid == 0) {
+        if (lc) { lc[0] = 0; lc[1] = 0; }
+        if (a.level == 1) a.out_cnt[qh] = 0;
+      }
+      continue;
+    }
+    const int n = a.cand_cnt[qh];
+    const double* s = a.cand_score + qh * a.C1;
+    const int* ids = a.cand_ids + qh * a.C1;
+    unsigned long long* E = a.cand_mass + qh * a.C1;
+
+    // 1. maximum and minimum score
+    double mx = -INFINITY, mn = INFINITY;
+    for (int i = tid; i < n; i += kSelThreads) { mx = fmax(mx, s[i]); mn = fmin(mn, s[i]); }
+    const double M = block_max_f64(mx, sm);
+    const double Mn = -block_max_f64(-mn, sm);
+    // 2. fixed-point masses and their exact total
+    unsigned long long z = 0;
+    for (int i = tid; i < n; i += kSelThreads) {
+      const unsigned long long e = __double2ull_rn(ldexp(exp(s[i] - M), a.mass_shift));
+      E[i] = e;
+      z += e;
+    }
+    const unsigned long long Z = block_sum_u64(z, sm);
+    __syncthreads();   // E[] written by this block is visible to all its threads
+
+    // 3. cutoff: key threshold and the number of tied elements to keep
+    bool keep_all = a.p >= 1.0 || n == 0;
+    unsigned long long pfx = 0, need = 0;
+    int shift = 0;
+    if (!keep_all) {
+      double tg = ceil(a.p * (double)Z);
+      unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
+      if (tgt > Z) tgt = Z;
+      const unsigned long long kmax = order_key(M), kmin = order_key(Mn);
+      unsigned long long above = 0;
+      unsigned int cnt_b = (unsigned int)n;
+      unsigned long long mass_b = Z;
+      if (kmax == kmin) {
+        shift = 0;
+        pfx = kmax;
+      } else {
+        int hi = 63 - __clzll((long long)(kmax ^ kmin));
+        pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
+        while (true) {
+          const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
+          const int lo = hi + 1 - width;
+          for (int i = tid; i < kBuckets; i += kSelThreads) { sm.cnt[i] = 0; sm.mass[i] = 0; }
+          if (tid == 0) { sm.bc_int[0] = 0; sm.bc_u64[0] = above; }
+          __syncthreads();
+          for (int i = tid; i < n; i += kSelThreads) {
+            const unsigned long long key = order_key(s[i]);
+            if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+              const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+              atomicAdd(&sm.cnt[bkt], 1u);
+              atomicAdd(&sm.mass[bkt], E[i]);
+            }
+          }
+          __syncthreads();
+          // thread j owns the 4 buckets [kBuckets-4(j+1), kBuckets-4j), scanned from the top
+          constexpr int kPer = kBuckets / kSelThreads;
+          unsigned long long local = 0;
+          for (int q = 0; q < kPer; ++q) local += sm.mass[kBuckets - 1 - (tid * kPer + q)];
+          // exclusive scan of the u64 partials in thread order
+          unsigned long long x = local;
+          const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+          if (lane == 31) sm.wsum[warp] = x;
+          __syncthreads();
+          unsigned long long before = above;
+          for (int i = 0; i < warp; ++i) before += sm.wsum[i];
+          before += x - local;
+          if (before < tgt && before + local >= tgt) {
+            unsigned long long acc = before;
+            unsigned int cacc = 0;
+            for (int q = 0; q < kPer; ++q) {
+              const int bkt = kBuckets - 1 - (tid * kPer + q);
+              if (acc + sm.mass[bkt] >= tgt) {
+                sm.bc_int[0] = bkt;
+                sm.bc_u64[0] = acc;       // mass strictly above the boundary bucket
+                break;
+              }
+              acc += sm.mass[bkt];
+              cacc += sm.cnt[bkt];
+            }
+          }
+          __syncthreads();
+          const int bstar = sm.bc_int[0];
+          above = sm.bc_u64[0];
+          cnt_b = sm.cnt[bstar];
+          mass_b = sm.mass[bstar];
+          pfx = (pfx << width) | (unsigned long long)bstar;
+          __syncthreads();
+          if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
+          hi = lo - 1;
+        }
+      }
+      // number of boundary-group elements to keep (exact ties share one mass value)
+      if (cnt_b <= 1) {
+        need = 1;
+      } else {
+        const unsigned long long e1 = mass_b / cnt_b;
+        need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
+        if (need < 1) need = 1;
+        if (need > cnt_b) need = cnt_b;
+      }
+    }
+
+    // 4. ordered compaction of the kept ids
+    int* outp = a.out_ids + qh * a.out_stride;
+    unsigned int written = 0, ties_seen = 0;
+    bool overflow = false;
+    for (int base = 0; base < n; base += kSelThreads) {
+      const int i = base + tid;
+      bool keep = false, tie = false;
+      if (i < n) {
+        if (keep_all) keep = true;
+        else {
+          const unsigned long long kk = order_key(s[i]) >> shift;
+          if (kk > pfx) keep = true;
+          else if (kk == pfx) tie = true;
+        }
+      }
+      unsigned int tie_total;
+      const unsigned int tie_rank = block_excl_scan(tie ? 1u : 0u, sm, &tie_total) + ties_seen;
+      if (tie && tie_rank < need) keep = true;
+      unsigned int keep_total;
+      const unsigned int pos = block_excl_scan(keep ? 1u : 0u, sm, &keep_total) + written;
+      if (keep) {
+        if ((int64_t)pos < a.out_cap) outp[pos] = ids[i];
+        else overflow = true;
+        if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
+          a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = ids[i];
+      }
+      written += keep_total;
+      ties_seen += tie_total;
+    }
+    if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
+    if (tid == 0) {
+      a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
+      if (lc) { lc[0] = n; lc[1] = (int)written; }
+    }
+    __syncthreads();
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host driver
+// ---------------------------------------------------------------------------
+
+
+
+static RouteGeom make_route_geom(const zha_geom& g, int nq, const int64_t* q_pos, int64_t pu) {
+  RouteGeom r{};
+  r.B = g.B; r.nq = nq; r.Hq = g.Hq; r.Hkv = g.Hkv; r.G = g.Hq / g.Hkv; r.R = g.R;
+  r.branch = g.branch; r.depth = g.depth; r.q_pos = q_pos; r.pos_uniform = pu; r.t_cap = g.t_cap;
+  for (int l = 1; l <= g.depth; ++l) { r.span[l] = span_of(g, l); r.ncap[l] = ncap_of(g, l); }
+  r.span[g.depth + 1] = r.span[g.depth] * g.branch;
+  r.ncap[g.depth + 1] = 0;
+  return r;
+}
+
+static int mass_shift_for(int64_t n) {
+  int bits = 0;
+  while ((1ll << bits) <= n) ++bits;     // bits to hold n
+  return 62 - bits;
+}
+
+static int grid_for(int64_t work, int per_sm) {
+  int64_t cap = 148ll * per_sm;
+  return (int)(work < cap ? (work < 1 ? 1 : work) : cap);
+}
+
+template <typename KT>
+static cudaError_t route_levels(const RouteCall& c) {
+  const zha_geom& g = *c.g;
+  const TreeLayout L = tree_layout(g);
+  const RouteWs w = route_ws(g, c.nq, 0);
+  const RouteGeom rg = make_route_geom(g, c.nq, c.q_pos, c.pos_uniform);
+  const int64_t nqh = (int64_t)g.B * c.nq * g.Hq;
+  int* selbuf[2] = {(int*)(c.ws + w.selA), (int*)(c.ws + w.selB)};
+  int* selcnt[2] = {(int*)(c.ws + w.selA_cnt), (int*)(c.ws + w.selB_cnt)};
+  int64_t level_ids_stride = 0;
+  for (int l = 2; l <= g.depth; ++l) level_ids_stride += ncap_of(g, l);
+  int64_t level_off = level_ids_stride;
+  for (int l = g.depth; l >= 1; --l) {
+    const int cur = l & 1, prev = (l + 1) & 1;
+    ScoreArgs sa{};
+    sa.g = rg; sa.level = l; sa.Q = c.Q;
+    sa.k_route = (char*)c.tree + L.lv[l].k_route_off;
+    sa.b_hat = (const float*)((char*)c.tree + L.lv[l].b_hat_off);
+    sa.parents = selbuf[prev]; sa.parents_cnt = selcnt[prev];
+    sa.C1 = w.C1; sa.C2 = w.C2;
+    sa.cand_ids = (int*)(c.ws + w.cand_ids);
+    sa.cand_score = (double*)(c.ws + w.cand_score);
+    sa.cand_cnt = (int*)(c.ws + w.cand_cnt);
+    sa.dev_status = c.dev_status;
+    sa.nblk = (L.lv[l].n_cap + 127) / 128;
+    if (sa.nblk < 1) sa.nblk = 1;
+    trace_begin(ZHA_TRACE_ROUTE_SCORE, c.stream);
+    route_score_kernel<KT><<<grid_for(nqh * sa.nblk, 16), 128, 0, c.stream>>>(sa);
+    trace_end(ZHA_TRACE_ROUTE_SCORE, c.stream);
+    count_launch();
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    SelectArgs se{};
+    se.g = rg; se.level = l; se.flat = 0; se.p = c.p;
+    se.mass_shift = mass_shift_for(w.C1);
+    se.cand_ids = sa.cand_ids; se.cand_score = sa.cand_score;
+    se.cand_mass = (unsigned long long*)(c.ws + w.cand_mass);
+    se.cand_cnt = sa.cand_cnt; se.C1 = w.C1;
+    if (l == 1) {
+      se.out_ids = c.leaf_ids; se.out_cnt = c.leaf_cnt; se.out_stride = c.leaf_cap; se.out_cap = c.leaf_cap;
+    } else {
+      se.out_ids = selbuf[cur]; se.out_cnt = selcnt[cur]; se.out_stride = w.C2; se.out_cap = (int)w.C2;
+    }
+    se.level_cnt = c.level_cnt;
+    se.level_ids = c.level_ids;
+    se.level_ids_stride = level_ids_stride;
+    if (l >= 2) level_off -= ncap_of(g, l);
+    se.level_ids_off = l >= 2 ? level_off : 0;
+    se.level_ids_cap = l >= 2 ? ncap_of(g, l) : 0;
+    se.dev_status = c.dev_status;
+    trace_begin(ZHA_TRACE_ROUTE_SELECT, c.stream);
+    route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+    trace_end(ZHA_TRACE_ROUTE_SELECT, c.stream);
+    count_launch();
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+cudaError_t route_all(const RouteCall& c) {
+  return c.g->dtype == ZHA_BF16 ? route_levels<__nv_bfloat16>(c) : route_levels<float>(c);
+}
+
+template <typename KT>
+static cudaError_t flat_select_t(const RouteCall& c) {
+  const zha_geom& g = *c.g;
+  const RouteWs w = route_ws(g, c.nq, 0);
+  const RouteGeom rg = make_route_geom(g, c.nq, c.q_pos, c.pos_uniform);
+  const int64_t units = (int64_t)g.B * c.nq * g.Hkv;
+  const int64_t nqh = (int64_t)g.B * c.nq * g.Hq;
+  FlatArgs fa{};
+  fa.g = rg; fa.Q = c.Q; fa.K = c.tree; fa.t_cap = g.t_cap; fa.C1 = w.C1;
+  fa.cand_ids = (int*)(c.ws + w.cand_ids);
+  fa.cand_score = (double*)(c.ws + w.cand_score);
+  fa.cand_cnt = (int*)(c.ws + w.cand_cnt);
+  fa.nblk = (w.C1 + 7) / 8;
+  if (fa.nblk < 1) fa.nblk = 1;
+  flat_score_kernel<KT><<<grid_for(units * fa.nblk, 8), 256, 0, c.stream>>>(fa);
+  count_launch();
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  SelectArgs se{};
+  se.g = rg; se.level = 1; se.flat = 1; se.p = c.p;
+  se.mass_shift = mass_shift_for(w.C1);
+  se.cand_ids = fa.cand_ids; se.cand_score = fa.cand_score;
+  se.cand_mass = (unsigned long long*)(c.ws + w.cand_mass);
+  se.cand_cnt = fa.cand_cnt; se.C1 = w.C1;
+  se.out_ids = c.leaf_ids; se.out_cnt = c.leaf_cnt; se.out_stride = c.leaf_cap; se.out_cap = c.leaf_cap;
+  se.dev_status = c.dev_status;
+  route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+  count_launch();
+  return cudaGetLastError();
+}
+
+// Flat indexer: `c.tree` carries the K cache pointer.
+cudaError_t flat_select(const RouteCall& c) {
+  return c.g->dtype == ZHA_BF16 ? flat_select_t<__nv_bfloat16>(c) : flat_select_t<float>(c);
+}
+
+}  // namespace zha

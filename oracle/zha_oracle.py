@@ -165,12 +165,21 @@ def _store_level(span, k_hat, F, b_hat, route_storage, state_storage):
                  k_state=round_to(k_hat, state_storage))
 
 
-def build_tree(K: np.ndarray, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
+def rows_f64(K, a: int, b: int) -> np.ndarray:
+    """Rows [a, b) of a key/value array as float64 (numpy or a CPU torch tensor)."""
+    x = K[a:b]
+    if hasattr(x, "double"):          # torch tensor: convert only this block
+        return x.double().numpy()
+    return np.asarray(x, dtype=np.float64)
+
+
+def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
                branch: int = 16, route_storage: str = "bf16", state_storage: str = "f32",
                block: int = 4096) -> Tree:
     """All full nodes over keys [0, T) of one unit.
 
-    K: [>=T, d] keys (float64 values of the stored keys), qref: [R, d].
+    K: [>=T, d] keys (float64 values of the stored keys, or a CPU torch tensor
+    read block by block), qref: [R, d].
     Level 1 summarises raw keys (``leaf_summary``); level l >= 2 merges the
     stored state of ``branch`` consecutive level-(l-1) nodes (``merge_summaries``).
     ``block`` only bounds the temporary memory of the vectorised leaf pass.
@@ -185,7 +194,7 @@ def build_tree(K: np.ndarray, T: int, qref: np.ndarray, depth: int, leaf: int = 
     b1 = np.zeros((n1, R))
     for i0 in range(0, n1, block):
         i1 = min(n1, i0 + block)
-        Kc = K[i0 * leaf:i1 * leaf].reshape(i1 - i0, leaf, d)
+        Kc = rows_f64(K, i0 * leaf, i1 * leaf).reshape(i1 - i0, leaf, d)
         s = np.einsum("rd,ncd->nrc", qref, Kc) * scale
         F = lse(s, axis=-1)
         a = np.exp(s - F[..., None])
@@ -311,13 +320,29 @@ def index_set(leaves: Sequence[int], t: int, leaf: int = 64) -> np.ndarray:
 # ---------------------------------------------------------------------------
 
 
-def attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, idx: np.ndarray):
-    """Softmax attention of q over the keys ``idx``.  Returns (o [d], lse)."""
+def attention(q: np.ndarray, K, V, idx: np.ndarray, block: int = 1 << 20):
+    """Softmax attention of q over the keys ``idx``.  Returns (o [d], lse).
+
+    K, V: float64 arrays or CPU torch tensors.  The logits and the weighted sum
+    of values are accumulated over ``block`` keys at a time only to bound the
+    float64 temporaries of very long index sets.
+    """
     scale = 1.0 / math.sqrt(q.shape[0])
-    z = K[idx] @ q * scale
+    idx = np.asarray(idx)
+    z = np.concatenate([_take_f64(K, idx[i:i + block]) @ q * scale for i in range(0, len(idx), block)])
     m = np.max(z)
     e = np.exp(z - m)
-    return (e @ V[idx]) / np.sum(e), float(m + np.log(np.sum(e)))
+    o = np.zeros(q.shape[0])
+    for i in range(0, len(idx), block):
+        o += e[i:i + block] @ _take_f64(V, idx[i:i + block])
+    return o / np.sum(e), float(m + np.log(np.sum(e)))
+
+
+def _take_f64(X, idx: np.ndarray) -> np.ndarray:
+    if hasattr(X, "double"):
+        import torch
+        return X[torch.from_numpy(np.ascontiguousarray(idx))].double().numpy()
+    return np.asarray(X[idx], dtype=np.float64)
 
 
 def dense_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, t: int):
@@ -331,8 +356,13 @@ def flat_scores(q: np.ndarray, K: np.ndarray, t: int, leaf: int = 64) -> np.ndar
     n = visible_count(t, leaf, leaf)
     if n == 0:
         return np.zeros(0)
-    z = (K[:n * leaf] @ q) / math.sqrt(d)
-    return lse(z.reshape(n, leaf), axis=-1)
+    out = np.empty(n)
+    step = 1 << 14
+    for c0 in range(0, n, step):
+        c1 = min(n, c0 + step)
+        z = (rows_f64(K, c0 * leaf, c1 * leaf) @ q) / math.sqrt(d)
+        out[c0:c1] = lse(z.reshape(c1 - c0, leaf), axis=-1)
+    return out
 
 
 def flat_select(q: np.ndarray, K: np.ndarray, t: int, p: float, leaf: int = 64) -> Selection:

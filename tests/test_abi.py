@@ -1,0 +1,104 @@
+"""The C-ABI library on the host: it loads, exports every symbol include/zha.h declares,
+and rejects bad arguments before it enqueues anything (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hierarchical_sparse_attention_02_b200 import _lib
+from hierarchical_sparse_attention_02_b200 import build as zbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    zbuild.build()
+    return _lib.load()
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "zha.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s+(zha_[a-z_]+)\s*\(", src, flags=re.M)
+
+
+def test_exports_every_declared_symbol(lib):
+    decl = declared_symbols()
+    assert len(decl) == 16
+    assert sorted(decl) == sorted(_lib.EXPORTS)
+    for name in decl:
+        assert hasattr(lib, name), name
+
+
+def geom(**kw):
+    base = dict(B=2, Hq=16, Hkv=2, d=128, leaf=64, branch=16, depth=3, R=4, t_cap=65536, dtype=1, reserved=0)
+    base.update(kw)
+    return _lib.Geom(**base)
+
+
+def test_status_strings(lib):
+    assert lib.zha_status_str(0) == b"ok"
+    assert lib.zha_status_str(3) == b"capacity exceeded"
+    assert lib.zha_status_str(99) == b"unknown status"
+
+
+@pytest.mark.parametrize("kw,code", [
+    ({}, 0), ({"d": 64}, 2), ({"leaf": 32}, 2), ({"Hq": 15}, 1), ({"Hq": 64, "Hkv": 2}, 2),
+    ({"R": 17}, 2), ({"R": 0}, 1), ({"depth": 9}, 2), ({"branch": 1}, 2), ({"t_cap": 1000}, 1),
+    ({"dtype": 7}, 2), ({"reserved": 1}, 1), ({"B": 0}, 1),
+])
+def test_check_geom(lib, kw, code):
+    assert lib.zha_check_geom(ctypes.byref(geom(**kw))) == code
+
+
+def test_sizes(lib):
+    g = geom()
+    assert lib.zha_leaf_cap(ctypes.byref(g)) == 1024
+    tb = lib.zha_tree_bytes(ctypes.byref(g))
+    lv = _lib.LevelLayout()
+    total = 0
+    for level in (1, 2, 3):
+        assert lib.zha_tree_level(ctypes.byref(g), level, ctypes.byref(lv)) == 0
+        assert lv.span == 64 * 16 ** (level - 1)
+        assert lv.n_cap == 65536 // lv.span
+        assert lv.k_route_off % 256 == 0 and lv.k_state_off % 256 == 0
+        total = lv.k_state_off + 2 * 2 * lv.n_cap * 4 * 128 * 4
+    assert tb >= total
+    assert lib.zha_tree_level(ctypes.byref(g), 4, ctypes.byref(lv)) == 1
+    for op in (1, 2, 3, 4, 5):
+        assert lib.zha_workspace_bytes(ctypes.byref(g), 1, op) > 0
+    assert lib.zha_workspace_bytes(ctypes.byref(g), 0, 1) == 0
+    assert lib.zha_workspace_bytes(ctypes.byref(g), 1, 9) == 0
+    assert lib.zha_tree_bytes(ctypes.byref(geom(d=64))) == 0
+
+
+def test_host_side_rejections_enqueue_nothing(lib):
+    """Invalid calls return before any launch; the pointers are never dereferenced."""
+    g = geom()
+    fake = ctypes.c_void_p(0x1000)
+    buf = _lib.Buf(0x1000, 1 << 40)
+    small = _lib.Buf(0x1000, 16)
+    n0 = lib.zha_launch_count()
+    # p outside (0, 1]
+    for p in (0.0, -0.5, 1.5, float("nan")):
+        assert lib.zha_route(ctypes.byref(g), fake, fake, 1, p, buf, fake, fake, 8, None, None, buf, fake, None) == 1
+    # null pointers
+    assert lib.zha_route(ctypes.byref(g), None, fake, 1, 0.9, buf, fake, fake, 8, None, None, buf, fake, None) == 1
+    assert lib.zha_sparse_attn(ctypes.byref(g), fake, fake, fake, fake, 1, fake, fake, 8, fake, None, buf, None,
+                               None) == 1
+    # buffers too small
+    assert lib.zha_build_tree(ctypes.byref(g), fake, 100, fake, small, fake, None) == 3
+    assert lib.zha_route(ctypes.byref(g), fake, fake, 1, 0.9, buf, fake, fake, 8, None, None, small, fake,
+                         None) == 3
+    # positions beyond the cache
+    assert lib.zha_build_tree(ctypes.byref(g), fake, 65537, fake, buf, fake, None) == 1
+    assert lib.zha_decode(ctypes.byref(g), fake, fake, fake, fake, fake, 65536, fake, 0.9, buf, fake, fake, 8,
+                          fake, buf, fake, None) == 1
+    assert lib.zha_append(ctypes.byref(g), fake, fake, fake, fake, 65000, 600, fake, buf, fake, None) == 1
+    # bad geometry
+    bad = geom(d=256)
+    assert lib.zha_decode(ctypes.byref(bad), fake, fake, fake, fake, fake, 5, fake, 0.9, buf, fake, fake, 8,
+                          fake, buf, fake, None) == 2
+    assert lib.zha_launch_count() == n0

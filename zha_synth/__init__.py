@@ -64,8 +64,10 @@ class Workload:
 
     @property
     def t_cap(self) -> int:
-        """Cache capacity: the existing keys plus the appended ones."""
-        return self.T + self.n_new
+        """Cache capacity: the existing keys plus the appended ones, rounded up to a
+        whole leaf chunk."""
+        n = self.T + self.n_new
+        return (n + self.leaf - 1) // self.leaf * self.leaf
 
 
 # The five workloads of the long-context study.  Reference-query count R=4 for
