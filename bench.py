@@ -364,7 +364,7 @@ def main():
     cps = max(16, -(-units * (c1 + 2) // 16384))
     items = -(-entries // cps)                                        # ranges: one per unit here
     gathered = union_rows * 2 * w.d * es
-    partial_bytes = items * w.G * (w.d + 2) * 4
+    partial_bytes = items * w.G * (w.d + 2) * 4          # o[d], m, l written per head and split
     attn_bytes = gathered + partial_bytes
     peak, peak_kind = hbm_peak()
     achieved = attn_bytes / (attn_ms * 1e-3) / 1e9

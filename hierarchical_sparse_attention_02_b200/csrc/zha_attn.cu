@@ -158,7 +158,7 @@ struct AttnArgs {
   const int* stage_cnt;
   const int* pair_off;
   int64_t pairs;
-  float* partials;               // [items, G, d + 2]
+  float* partials;               // [items, G, kPartStride]: o[d], m, l
 };
 
 constexpr int kRowPad = kD + 4;   // fp32 smem row stride (16-byte aligned, bank-skewed)
@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(256) attn_split_kernel(AttnArgs a) {
       }
     }
     if (h < g.G) {
-      float* P = a.partials + ((int64_t)item * g.G + h) * (kD + 2);
+      float* P = a.partials + ((int64_t)item * g.G + h) * kPartStride;
       reinterpret_cast<float4*>(P)[lane] = o;
       if (lane == 0) { P[kD] = m; P[kD + 1] = l; }
     }
@@ -280,11 +280,11 @@ __global__ void __launch_bounds__(128) combine_kernel(AttnGeom g, const int* pai
   const int hk = (int)(u % g.Hkv);
   const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
   float M = -INFINITY;
-  for (int64_t i = i0; i < i1; ++i) M = fmaxf(M, partials[(i * g.G + h) * (kD + 2) + kD]);
+  for (int64_t i = i0; i < i1; ++i) M = fmaxf(M, partials[(i * g.G + h) * kPartStride + kD]);
   float L = 0.f, acc = 0.f;
   if (M != -INFINITY) {
     for (int64_t i = i0; i < i1; ++i) {
-      const float* P = partials + (i * g.G + h) * (kD + 2);
+      const float* P = partials + (i * g.G + h) * kPartStride;
       const float w = exp2f(P[kD] - M);       // -inf partials weigh 0
       L = fmaf(w, P[kD + 1], L);
       acc = fmaf(w, P[threadIdx.x], acc);

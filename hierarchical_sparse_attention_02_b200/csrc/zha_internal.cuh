@@ -19,6 +19,9 @@ constexpr int kMaxG = 8;         // query heads per KV head
 constexpr int kMaxDepth = 8;
 constexpr int kRange = 4096;     // chunk ids per union-building block
 constexpr size_t kAlign = 256;
+// Floats per split-KV partial: o[d], the running max m and sum l, padded so that every
+// partial starts on a 16-byte boundary (vector stores).
+constexpr int kPartStride = kD + 4;
 
 inline size_t align_up(size_t x, size_t a = kAlign) { return (x + a - 1) / a * a; }
 
@@ -114,7 +117,7 @@ inline AttnWs attn_ws(const zha_geom& g, int nq, size_t base = 0) {
   w.stage_mask = off; off = align_up(off + (size_t)w.pairs * (kRange + 2) * 4);
   w.stage_cnt = off;  off = align_up(off + (size_t)w.pairs * 4);
   w.pair_off = off;   off = align_up(off + (size_t)(w.pairs + 1) * 4);
-  w.partials = off;   off = align_up(off + (size_t)w.items_max * G * (g.d + 2) * 4);
+  w.partials = off;   off = align_up(off + (size_t)w.items_max * G * kPartStride * 4);
   w.pos = off;        off = align_up(off + (size_t)g.B * nq * 8);
   w.bytes = off;
   return w;
