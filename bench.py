@@ -290,6 +290,9 @@ def main():
     Ksteps = args.steps
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(Ksteps)]
     stops = [torch.cuda.Event(enable_timing=True) for _ in range(Ksteps)]
+    for e in starts + stops:          # torch creates the CUDA event at its first record
+        e.record(stream)
+    torch.cuda.synchronize()
     arr_s = (ctypes.c_void_p * Ksteps)(*[ctypes.c_void_p(e.cuda_event) for e in starts])
     arr_e = (ctypes.c_void_p * Ksteps)(*[ctypes.c_void_p(e.cuda_event) for e in stops])
     lib = _lib.load()

@@ -19,7 +19,10 @@ from . import _lib
 class ZhaError(RuntimeError):
     def __init__(self, fn: str, status: int):
         lib = _lib.load()
-        super().__init__(f"{fn}: {lib.zha_status_str(status).decode()} (status {status})")
+        msg = f"{fn}: {lib.zha_status_str(status).decode()} (status {status})"
+        if status == _lib.ZHA_ERR_CUDA:
+            msg += f": {lib.zha_last_error().decode()}"
+        super().__init__(msg)
         self.status = status
 
 

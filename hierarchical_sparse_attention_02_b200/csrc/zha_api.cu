@@ -1,6 +1,7 @@
 // The C ABI declared in include/zha.h: argument validation, buffer sizing and the
 // composition of the kernels into the calls of the hot path.
 #include <math.h>
+#include <stdio.h>
 
 #include "zha_internal.cuh"
 
@@ -8,6 +9,12 @@ namespace zha {
 
 std::atomic<int64_t> g_launches{0};
 Tracer g_trace[4];
+
+static char g_last_error[256] = "no error";
+
+void note_cuda_error(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
+}
 
 
 
@@ -86,6 +93,8 @@ size_t zha_workspace_bytes(const zha_geom* g, int32_t nq, int32_t op) {
 }
 
 int64_t zha_launch_count(void) { return g_launches.load(); }
+
+const char* zha_last_error(void) { return g_last_error; }
 
 void zha_trace(int32_t which, void* const* start, void* const* stop, int32_t n) {
   if (which < 1 || which > 3) return;

@@ -318,13 +318,13 @@ static cudaError_t attention_t(const AttnCall& c) {
   ua.dev_status = c.dev_status;
   union_kernel<<<(unsigned)w.pairs, 256, 0, c.stream>>>(ua);
   count_launch();
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_status("union_kernel");
   if (e != cudaSuccess) return e;
 
   int* pair_off = (int*)(c.ws + w.pair_off);
   plan_kernel<<<1, 1024, 0, c.stream>>>(ua.stage_cnt, w.pairs, w.cps, pair_off);
   count_launch();
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_status("plan_kernel")) != cudaSuccess) return e;
 
   AttnArgs aa{};
   aa.g = ag; aa.Q = c.Q; aa.K = c.K; aa.V = c.V;
@@ -338,12 +338,12 @@ static cudaError_t attention_t(const AttnCall& c) {
   attn_split_kernel<KT><<<(unsigned)grid, 256, smem, c.stream>>>(aa);
   trace_end(ZHA_TRACE_ATTN, c.stream);
   count_launch();
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if ((e = launch_status("attn_split_kernel")) != cudaSuccess) return e;
 
   combine_kernel<KT><<<(unsigned)(w.units * ag.G), 128, 0, c.stream>>>(
       ag, pair_off, aa.partials, (KT*)c.O, c.lse);
   count_launch();
-  return cudaGetLastError();
+  return launch_status("combine_kernel");
 }
 
 cudaError_t attention(const AttnCall& c) {

@@ -127,6 +127,14 @@ inline AttnWs attn_ws(const zha_geom& g, int nq, size_t base = 0) {
 extern std::atomic<int64_t> g_launches;
 inline void count_launch(int n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
+// The error of the last failing CUDA call, kept for zha_last_error().
+void note_cuda_error(cudaError_t e, const char* where);
+inline cudaError_t launch_status(const char* kernel) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) note_cuda_error(e, kernel);
+  return e;
+}
+
 // Event tracing around chosen kernels (zha_trace): record before / after one launch.
 struct Tracer {
   void* const* start = nullptr;

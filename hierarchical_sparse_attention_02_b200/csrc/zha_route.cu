@@ -514,7 +514,7 @@ static cudaError_t route_levels(const RouteCall& c) {
     route_score_kernel<KT><<<grid_for(nqh * sa.nblk, 16), 128, 0, c.stream>>>(sa);
     trace_end(ZHA_TRACE_ROUTE_SCORE, c.stream);
     count_launch();
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_status("route_score_kernel");
     if (e != cudaSuccess) return e;
 
     SelectArgs se{};
@@ -539,7 +539,7 @@ static cudaError_t route_levels(const RouteCall& c) {
     route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
     trace_end(ZHA_TRACE_ROUTE_SELECT, c.stream);
     count_launch();
-    e = cudaGetLastError();
+    e = launch_status("route_select_kernel");
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -565,7 +565,7 @@ static cudaError_t flat_select_t(const RouteCall& c) {
   if (fa.nblk < 1) fa.nblk = 1;
   flat_score_kernel<KT><<<grid_for(units * fa.nblk, 8), 256, 0, c.stream>>>(fa);
   count_launch();
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_status("flat_score_kernel");
   if (e != cudaSuccess) return e;
   SelectArgs se{};
   se.g = rg; se.level = 1; se.flat = 1; se.p = c.p;
@@ -577,7 +577,7 @@ static cudaError_t flat_select_t(const RouteCall& c) {
   se.dev_status = c.dev_status;
   route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
   count_launch();
-  return cudaGetLastError();
+  return launch_status("route_select_kernel(flat)");
 }
 
 // Flat indexer: `c.tree` carries the K cache pointer.

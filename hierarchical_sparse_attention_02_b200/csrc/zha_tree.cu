@@ -263,7 +263,7 @@ static cudaError_t launch_leaves(const zha_geom& g, const TreeLayout& L, const v
       (const KT*)K, qref, g.Hkv, g.R, g.t_cap, lo, n, level_ptrs(g, L, tree, 1),
       1.0 / sqrt((double)g.d));
   count_launch();
-  return cudaGetLastError();
+  return launch_status("leaf_summarize_kernel");
 }
 
 template <typename KT>
@@ -276,7 +276,7 @@ static cudaError_t launch_merge(const zha_geom& g, const TreeLayout& L, const fl
       qref, g.Hkv, g.R, g.branch, lo, n, level_ptrs(g, L, tree, level - 1),
       level_ptrs(g, L, tree, level), 1.0 / sqrt((double)g.d));
   count_launch();
-  return cudaGetLastError();
+  return launch_status("parent_merge_kernel");
 }
 
 // Summarise every node completed when the cache grows from t_old to t_new keys.
@@ -311,7 +311,7 @@ cudaError_t append_tokens(const zha_geom& g, void* K, void* V, const void* k_new
                                                         (const uint4*)v_new, g.Hkv, n_new, g.t_cap,
                                                         t_old, vec_per_row, total);
   count_launch();
-  return cudaGetLastError();
+  return launch_status("append_kv_kernel");
 }
 
 }  // namespace zha

@@ -227,6 +227,10 @@ zha_status zha_flat_index(const zha_geom* g, const void* Q, const void* K, const
 /* Number of kernels this library has enqueued since it was loaded (host counter). */
 int64_t zha_launch_count(void);
 
+/* The kernel and CUDA error behind the last ZHA_ERR_CUDA (static string, "no error"
+ * before any failure; overwritten by the next failure). */
+const char* zha_last_error(void);
+
 /* Measurement hook.  Kernel ids for zha_trace. */
 typedef enum zha_trace_kernel {
   ZHA_TRACE_ATTN = 1,        /* the split-KV gather kernel of the sparse / dense attention */
