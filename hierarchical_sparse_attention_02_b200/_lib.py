@@ -18,9 +18,10 @@ ZHA_OP_ROUTE, ZHA_OP_ATTN, ZHA_OP_DECODE, ZHA_OP_DENSE, ZHA_OP_FLAT = 1, 2, 3, 4
 EXPORTS = [
     "zha_status_str", "zha_check_geom", "zha_tree_bytes", "zha_tree_level", "zha_workspace_bytes",
     "zha_leaf_cap", "zha_build_tree", "zha_append", "zha_route", "zha_sparse_attn", "zha_decode",
-    "zha_dense_decode", "zha_flat_index", "zha_launch_count", "zha_last_error", "zha_trace",
-    "zha_trace_count",
+    "zha_dense_decode", "zha_flat_index", "zha_sparse_attn_noalloc", "zha_launch_count",
+    "zha_last_error", "zha_trace", "zha_trace_count",
 ]
+ZHA_NOALLOC_SCRATCH_BYTES = 16 << 20
 ZHA_TRACE_ATTN, ZHA_TRACE_ROUTE_SCORE, ZHA_TRACE_ROUTE_SELECT = 1, 2, 3
 
 
@@ -58,6 +59,7 @@ _SIGS = {
     "zha_decode": (_I32, [_G, _P, _P, _P, _P, _P, _I64, _P, _F64, Buf, _P, _P, _I32, _P, Buf, _P, _P]),
     "zha_dense_decode": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_flat_index": (_I32, [_G, _P, _P, _P, _P, _I32, _F64, _P, _P, _I32, _P, Buf, _P, _P]),
+    "zha_sparse_attn_noalloc": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _P, _P, _P]),
     "zha_launch_count": (_I64, []),
     "zha_last_error": (ctypes.c_char_p, []),
     "zha_trace": (None, [_I32, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p), _I32]),

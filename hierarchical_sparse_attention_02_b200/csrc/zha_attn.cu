@@ -304,7 +304,7 @@ __global__ void __launch_bounds__(128) combine_kernel(AttnGeom g, const int* pai
 template <typename KT>
 static cudaError_t attention_t(const AttnCall& c) {
   const zha_geom& g = *c.g;
-  const AttnWs w = attn_ws(g, c.nq, 0);
+  const AttnWs w = attn_ws(g, c.nq, 0, c.cps);
   AttnGeom ag{};
   ag.B = g.B; ag.nq = c.nq; ag.Hq = g.Hq; ag.Hkv = g.Hkv; ag.G = g.Hq / g.Hkv; ag.t_cap = g.t_cap;
   ag.q_pos = c.q_pos; ag.pos_uniform = c.pos_uniform; ag.nr = w.nr; ag.cps = w.cps;

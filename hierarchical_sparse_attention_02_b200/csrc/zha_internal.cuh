@@ -103,14 +103,15 @@ struct AttnWs {
   int64_t units, nr, pairs, cps, items_max, C1;
 };
 
-inline AttnWs attn_ws(const zha_geom& g, int nq, size_t base = 0) {
+// cps = 0: the default split size; otherwise that many chunks per work item.
+inline AttnWs attn_ws(const zha_geom& g, int nq, size_t base = 0, int64_t cps = 0) {
   AttnWs w{};
   const int G = g.Hq / g.Hkv;
   w.units = (int64_t)g.B * nq * g.Hkv;
   w.C1 = ncap_of(g, 1);
   w.nr = (w.C1 + 1 + kRange - 1) / kRange;
   w.pairs = w.units * w.nr;
-  w.cps = chunks_per_split(w.units, w.C1);
+  w.cps = cps > 0 ? cps : chunks_per_split(w.units, w.C1);
   w.items_max = w.pairs + (w.units * (w.C1 + 2) + w.cps - 1) / w.cps;
   size_t off = base;
   w.stage_ids = off;  off = align_up(off + (size_t)w.pairs * (kRange + 2) * 4);
@@ -239,9 +240,10 @@ struct AttnCall {
   int leaf_cap;
   void* O;
   float* lse;
-  char* ws;                      // workspace base, layout attn_ws(g, nq, 0)
+  char* ws;                      // workspace base, layout attn_ws(g, nq, 0, cps)
   int32_t* dev_status;
   cudaStream_t stream;
+  int64_t cps = 0;               // chunks per work item; 0: the default of attn_ws
 };
 
 cudaError_t tree_extend(const zha_geom& g, const void* K, const float* qref, void* tree,

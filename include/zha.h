@@ -224,6 +224,34 @@ zha_status zha_flat_index(const zha_geom* g, const void* Q, const void* K, const
                           int32_t* leaf_cnt, int32_t leaf_cap, void* O, zha_buf ws,
                           int32_t* dev_status, void* stream);
 
+/*
+ * zha_sparse_attn_noalloc - zha_sparse_attn without a caller workspace.
+ *
+ * The paper has no counterpart: this entry point exists for callers that can pass the
+ * library their inputs and outputs but cannot provide extra device memory (an engine's
+ * plugin interface that hands over only the operator's buffers, or a process whose device
+ * memory is wholly owned by another allocator).  The scratch lives in one file-scope
+ * device array of ZHA_NOALLOC_SCRATCH_BYTES (16 MiB) that every GPU loading the library
+ * holds until the process exits; the call allocates nothing.
+ *   Arguments and result as zha_sparse_attn (same kernels; the split size is enlarged
+ *   until the scratch fits, so values agree with zha_sparse_attn to fp32 rounding).
+ *   Sizes whose scratch cannot fit even with the largest split return
+ *   ZHA_ERR_CAPACITY before anything is enqueued: the array holds about 400
+ *   (sequence, query, KV head) units while t_cap < 256K tokens, and proportionally
+ *   fewer for longer caches (about 32 KiB of union lists per unit and 4096 leaf chunks).
+ *   The first call on a device resolves the array's device address (cudaGetSymbolAddress
+ *   with that device current); make that first call before any stream capture.
+ *   Every call shares the array, and it keeps the previous call's contents (nothing in
+ *   it needs to start at zero: every value read is written earlier in the same call).
+ *   Calls that overlap on the GPU race on the array: issue them on one stream, or order
+ *   them.
+ */
+#define ZHA_NOALLOC_SCRATCH_BYTES (16u << 20)
+zha_status zha_sparse_attn_noalloc(const zha_geom* g, const void* Q, const void* K, const void* V,
+                                   const int64_t* q_pos, int32_t nq, const int32_t* leaf_ids,
+                                   const int32_t* leaf_cnt, int32_t leaf_cap, void* O, float* lse,
+                                   int32_t* dev_status, void* stream);
+
 /* Number of kernels this library has enqueued since it was loaded (host counter). */
 int64_t zha_launch_count(void);
 
