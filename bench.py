@@ -48,6 +48,8 @@ def parse():
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiling)")
     return ap.parse_args()
 
 
@@ -241,6 +243,8 @@ def config_of(w, p):
 def main():
     args = parse()
     w = S.workload(args.workload)
+    if args.batch is not None:
+        w = S.scaled(w, T=w.T, B=args.batch)
     p = args.p if args.p is not None else w.p[0]
     ws, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":
