@@ -94,24 +94,28 @@ def max_over_ranks(x: float, ws: int) -> float:
 
 
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device: int):
         self.path = tempfile.mktemp(suffix=".csv")
         self.proc = None
-        sel = []
+        self.why = None
+        # the physical GPU: CUDA_VISIBLE_DEVICES may renumber devices, nvidia-smi does not
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        index = str(device)
+        if vis:
+            parts = [p.strip() for p in vis.split(",") if p.strip()]
+            if device < len(parts):
+                index = parts[device]
         try:
-            bus = torch.cuda.get_device_properties(device).pci_bus_id
-            sel = ["-i", bus]
-        except Exception:
-            sel = ["-i", str(device)]
-        try:
-            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
-        except Exception:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", index, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.PIPE)
+        except Exception as e:  # noqa: BLE001
             self.proc = None
+            self.why = f"nvidia-smi unavailable: {type(e).__name__}: {e}"
         self.t_start = self.t_end = None
 
     def mark_start(self):
@@ -122,25 +126,35 @@ class ClockSampler:
 
     def stop(self):
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.why], "samples": 0}
+        t_busy_end = time.time()
         time.sleep(0.25)
         self.proc.terminate()
+        err = b""
         try:
-            self.proc.wait(5)
-        except Exception:
+            _, err = self.proc.communicate(timeout=5)
+        except Exception:  # noqa: BLE001
             self.proc.kill()
+        import datetime
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts[5:9], parts[4]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9], parts[4], ts))
             except ValueError:
                 continue
+        # samples from the start of the timed region on (the end-to-end steps that follow it
+        # keep the GPU on the same work)
+        if self.t_start is not None:
+            busy = [r for r in rows if self.t_start - 0.05 <= r[4] <= t_busy_end]
+            rows = busy or rows
         os.unlink(self.path)
         if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+            msg = (err or b"").decode(errors="replace").strip()[:200]
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"no samples: {msg}"], "samples": 0}
         # keep the samples taken while the GPU was busy (highest-clock half if the tail idles)
         sm = [r[0] for r in rows]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]

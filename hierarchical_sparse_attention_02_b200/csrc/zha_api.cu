@@ -51,6 +51,7 @@ zha_status zha_check_geom(const zha_geom* g) {
   if (g->reserved != 0) return ZHA_ERR_INVALID_ARG;
   if (g->d != kD || g->leaf != kLeaf) return ZHA_ERR_UNSUPPORTED;
   if (g->Hq / g->Hkv > kMaxG || g->R > kMaxR || g->depth > kMaxDepth) return ZHA_ERR_UNSUPPORTED;
+  if (g->R & (g->R - 1)) return ZHA_ERR_UNSUPPORTED;     // R in {1, 2, 4, 8, 16}
   if (g->branch < 2 || g->branch > 64) return ZHA_ERR_UNSUPPORTED;
   if (g->dtype != ZHA_F32 && g->dtype != ZHA_BF16) return ZHA_ERR_UNSUPPORTED;
   if (g->t_cap % kLeaf != 0) return ZHA_ERR_INVALID_ARG;

@@ -8,6 +8,8 @@
 // persistent kernel walks the items: each item streams its K/V blocks once and keeps
 // an online softmax (m, l, o[d]) per head; a combine kernel merges the items' partials
 // by log-sum-exp (split-KV partials, arXiv 2610.42112 App. D-B1).
+#include <type_traits>
+
 #include "zha_internal.cuh"
 
 namespace zha {
@@ -331,14 +333,25 @@ static cudaError_t attention_t(const AttnCall& c) {
   aa.stage_ids = ua.stage_ids; aa.stage_mask = ua.stage_mask; aa.stage_cnt = ua.stage_cnt;
   aa.pair_off = pair_off; aa.pairs = w.pairs;
   aa.partials = (float*)(c.ws + w.partials);
-  const size_t smem = (size_t)(2 * kLeaf * kRowPad + kMaxG * kD) * sizeof(float);
-  cudaFuncSetAttribute(attn_split_kernel<KT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  int64_t grid = w.items_max < 148 * 3 ? w.items_max : 148 * 3;
-  trace_begin(ZHA_TRACE_ATTN, c.stream);
-  attn_split_kernel<KT><<<(unsigned)grid, 256, smem, c.stream>>>(aa);
-  trace_end(ZHA_TRACE_ATTN, c.stream);
-  count_launch();
-  if ((e = launch_status("attn_split_kernel")) != cudaSuccess) return e;
+  if (std::is_same<KT, __nv_bfloat16>::value) {
+    // bf16 caches: TMA-fed, tensor-core kernel (zha_attn_tc.cu)
+    trace_begin(ZHA_TRACE_ATTN, c.stream);
+    e = attn_tc_launch(c, w, aa.stage_ids, aa.stage_mask, aa.stage_cnt, pair_off, aa.partials);
+    trace_end(ZHA_TRACE_ATTN, c.stream);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    if ((e = launch_status("attn_tc_kernel")) != cudaSuccess) return e;
+  } else {
+    // fp32 caches: CUDA-core kernel (fp32 products keep fp32 accuracy)
+    const size_t smem = (size_t)(2 * kLeaf * kRowPad + kMaxG * kD) * sizeof(float);
+    cudaFuncSetAttribute(attn_split_kernel<KT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int64_t grid = w.items_max < 148 * 3 ? w.items_max : 148 * 3;
+    trace_begin(ZHA_TRACE_ATTN, c.stream);
+    attn_split_kernel<KT><<<(unsigned)grid, 256, smem, c.stream>>>(aa);
+    trace_end(ZHA_TRACE_ATTN, c.stream);
+    count_launch();
+    if ((e = launch_status("attn_split_kernel")) != cudaSuccess) return e;
+  }
 
   combine_kernel<KT><<<(unsigned)(w.units * ag.G), 128, 0, c.stream>>>(
       ag, pair_off, aa.partials, (KT*)c.O, c.lse);

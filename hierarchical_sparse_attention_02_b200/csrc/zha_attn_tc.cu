@@ -1,0 +1,429 @@
+// Split-KV gather attention for bf16 caches on sm_100a: TMA-fed, tensor-core scored.
+//
+// One persistent CTA per SM walks the work items (splits of the union-of-heads chunk
+// lists built by union_kernel / plan_kernel).  A producer warp streams every selected
+// 64-key block of K and V into a 6-stage shared-memory ring with 3-D TMA loads
+// (cp.async.bulk.tensor, 128-byte swizzle, completion on mbarriers; no multicast).  Four
+// consumer warps each own 16 keys of every block and run, for the G <= 8 query heads that
+// share the block (GQA),
+//     S^T[16 keys x 8 heads] = K_blk . Q^T          (mma.sync m16n8k16, bf16 in, fp32 acc)
+//     online softmax per head (fp32, base 2), heads outside the block's mask at -inf
+//     O^T[128 x 8]          += V_blk^T . P^T        (P rounded to bf16)
+// and at the end of an item the four warps' (m, l, O) are merged into one split partial
+// (arXiv 2610.42112 App. D-B1: d_v values and two softmax statistics per split).
+// The kernel is bound by HBM bandwidth: every selected block of a KV group crosses HBM once.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "zha_internal.cuh"
+
+namespace zha {
+
+namespace tc {
+
+constexpr int kStages = 6;
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+constexpr int kBoxBytes = 64 * 128;              // 64 rows x 64 bf16, one swizzled box
+constexpr int kStageBytes = 4 * kBoxBytes;       // K lo/hi, V lo/hi
+constexpr uint32_t kTxBytes = kStageBytes;
+constexpr long long kSpinLimit = 1ll << 22;      // mbarrier polls before giving up
+
+struct Smem {
+  unsigned char stage[kStages][kStageBytes];     // 1024-byte aligned (swizzle atoms)
+  float o[kConsumerWarps][kMaxG][kD];            // per-warp O^T for the item merge
+  float ml[kConsumerWarps][kMaxG][2];
+  int2 meta[kStages];                            // (key count, head mask) of each stage
+  unsigned long long full[kStages];
+  unsigned long long empty[kStages];
+  int abort;                                     // set once any wait of the CTA gave up
+  int zero;                                      // always 0
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(unsigned long long* b, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_arrive_tx(unsigned long long* b, uint32_t tx) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(tx)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(unsigned long long* b) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try(unsigned long long* b, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait: false after kSpinLimit polls, or at once when another thread of the CTA
+// has given up (`abort` set); the caller then reports and stops waiting for anything.
+__device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity, const int* abort) {
+  for (long long i = 0; i < kSpinLimit; ++i) {
+    if ((i & 255) == 0 && *(volatile const int*)abort) return false;
+    if (mbar_try(b, parity)) return true;
+  }
+  return false;
+}
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
+                                            unsigned long long* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"((unsigned long long)map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9},"
+      " {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128B-swizzled box.
+__device__ __forceinline__ uint32_t swz(int row, int chunk) {
+  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
+}
+
+struct Args {
+  int B, nq, Hq, Hkv, G;
+  int64_t t_cap;
+  const int64_t* q_pos;
+  int64_t pos_uniform;
+  int64_t nr, cps;
+  const __nv_bfloat16* Q;
+  const int* stage_ids;
+  const unsigned int* stage_mask;
+  const int* stage_cnt;
+  const int* pair_off;
+  int64_t pairs;
+  float* partials;
+  int32_t* dev_status;
+};
+
+struct ItemInfo {
+  int64_t pair, u, bq, unit_kv;   // unit_kv = b * Hkv + hk (tensor-map z coordinate)
+  int hk, e0, e1;
+  int64_t t, vstart, nvis;
+};
+
+__device__ __forceinline__ ItemInfo item_info(const Args& a, int64_t item) {
+  ItemInfo it;
+  int64_t lo = 0, hi = a.pairs;                  // last pair with pair_off[pair] <= item
+  while (hi - lo > 1) { const int64_t m = (lo + hi) >> 1; if (a.pair_off[m] <= item) lo = m; else hi = m; }
+  it.pair = lo;
+  const int64_t sub = item - a.pair_off[lo];
+  it.u = lo / a.nr;
+  it.bq = it.u / a.Hkv;
+  it.hk = (int)(it.u % a.Hkv);
+  it.unit_kv = (it.bq / a.nq) * a.Hkv + it.hk;
+  it.t = query_pos(a.q_pos, a.pos_uniform, it.bq);
+  it.vstart = (it.t / kLeaf) * kLeaf;
+  it.nvis = it.vstart / kLeaf;
+  const int cnt = a.stage_cnt[lo];
+  it.e0 = (int)(sub * a.cps);
+  it.e1 = (int)((sub + 1) * a.cps < cnt ? (sub + 1) * a.cps : cnt);
+  return it;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap, Args a) {
+  extern __shared__ unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t total_items = a.pair_off[a.pairs];
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], kConsumerWarps); }
+    sm.abort = 0;
+    sm.zero = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: one lane issues the TMA loads ----------------
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&kmap) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&vmap) : "memory");
+      long long it_count = 0;
+      long long issued[kStages];
+      for (int s = 0; s < kStages; ++s) issued[s] = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+        const ItemInfo info = item_info(a, item);
+        const int* ids = a.stage_ids + info.pair * (kRange + 2);
+        const unsigned int* msk = a.stage_mask + info.pair * (kRange + 2);
+        for (int e = info.e0; e < info.e1; ++e, ++it_count) {
+          const int s = (int)(it_count % kStages);
+          if (it_count >= kStages) {
+            if (!mbar_wait(&sm.empty[s], (uint32_t)(((it_count / kStages) - 1) & 1), &sm.abort)) {
+              set_status(a.dev_status, ZHA_ERR_DEVICE);
+              atomicExch(&sm.abort, 1);
+              ok = false;
+              break;
+            }
+          }
+          if (*(volatile int*)&sm.abort) { ok = false; break; }
+          const int id = ids[e];
+          int k0, len;
+          if (id < 0) { k0 = 0; len = 1; }
+          else if (id == info.nvis) { k0 = (int)info.vstart; len = (int)(info.t - info.vstart + 1); }
+          else { k0 = id * kLeaf; len = kLeaf; }
+          sm.meta[s] = make_int2(len, (int)msk[e]);
+          mbar_arrive_tx(&sm.full[s], kTxBytes);
+          unsigned char* st = sm.stage[s];
+          const int z = (int)info.unit_kv;
+          tma_load_3d(st + 0 * kBoxBytes, &kmap, 0, k0, z, &sm.full[s]);
+          tma_load_3d(st + 1 * kBoxBytes, &kmap, 64, k0, z, &sm.full[s]);
+          tma_load_3d(st + 2 * kBoxBytes, &vmap, 0, k0, z, &sm.full[s]);
+          tma_load_3d(st + 3 * kBoxBytes, &vmap, 64, k0, z, &sm.full[s]);
+          ++issued[s];
+        }
+      }
+      // drain: no TMA write may land after the CTA exits (the copies complete on their
+      // own; this wait ignores `abort`)
+      for (int s = 0; s < kStages; ++s)
+        if (issued[s] > 0 && !mbar_wait(&sm.full[s], (uint32_t)((issued[s] - 1) & 1), &sm.zero))
+          set_status(a.dev_status, ZHA_ERR_DEVICE);
+    }
+    return;
+  }
+
+  // ---------------- consumers: 4 warps, warp w owns keys [16w, 16w + 16) ----------------
+  const int g = lane >> 2, t4 = lane & 3;
+  const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
+  long long it_count = 0;
+  for (int64_t item = blockIdx.x; item < total_items; item += gridDim.x) {
+    const ItemInfo info = item_info(a, item);
+    // B fragments of Q^T: head g, dims 16kk + 2t4 (+1) and + 8 (heads >= G are zero)
+    uint32_t qb[8][2];
+    {
+      const int h = g;
+      const __nv_bfloat16* qrow = a.Q + ((info.bq * a.Hq) + info.hk * a.G + (h < a.G ? h : 0)) * kD;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        uint32_t w0 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t4);
+        uint32_t w1 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t4 + 8);
+        qb[kk][0] = h < a.G ? w0 : 0u;
+        qb[kk][1] = h < a.G ? w1 : 0u;
+      }
+    }
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // heads 2t4, 2t4+1
+    float o[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    for (int e = info.e0; e < info.e1; ++e, ++it_count) {
+      const int s = (int)(it_count % kStages);
+      if (!mbar_wait(&sm.full[s], (uint32_t)((it_count / kStages) & 1), &sm.abort)) {
+        set_status(a.dev_status, ZHA_ERR_DEVICE);
+        atomicExch(&sm.abort, 1);
+        continue;      // every later wait of the CTA now fails at once; barriers stay aligned
+      }
+      const int2 meta = sm.meta[s];
+      const uint32_t base = smem_u32(sm.stage[s]);
+      // S^T = K . Q^T for keys 16w + [0, 16)
+      float sc[4] = {0.f, 0.f, 0.f, 0.f};
+      {
+        const int mi = lane >> 3, r8 = lane & 7;
+        const int row = warp * 16 + r8 + ((mi & 1) << 3);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int box = kk >> 2;                       // dims 0-63 | 64-127
+          const int chunk = ((kk & 3) << 1) + (mi >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(base + box * kBoxBytes + swz(row, chunk), a0, a1, a2, a3);
+          mma_bf16(sc, a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+        }
+      }
+      // mask: keys beyond the block's length, heads outside its mask
+      const int key0 = warp * 16 + g, key1 = key0 + 8;
+      const int hA = 2 * t4, hB = hA + 1;
+      const bool hAok = (meta.y >> hA) & 1, hBok = (meta.y >> hB) & 1;
+      float s00 = (key0 < meta.x && hAok) ? sc[0] * sl2 : -INFINITY;
+      float s01 = (key0 < meta.x && hBok) ? sc[1] * sl2 : -INFINITY;
+      float s10 = (key1 < meta.x && hAok) ? sc[2] * sl2 : -INFINITY;
+      float s11 = (key1 < meta.x && hBok) ? sc[3] * sl2 : -INFINITY;
+      float mxA = fmaxf(s00, s10), mxB = fmaxf(s01, s11);
+#pragma unroll
+      for (int x = 4; x < 32; x <<= 1) {
+        mxA = fmaxf(mxA, __shfl_xor_sync(0xffffffffu, mxA, x));
+        mxB = fmaxf(mxB, __shfl_xor_sync(0xffffffffu, mxB, x));
+      }
+      const float nA = fmaxf(m0, mxA), nB = fmaxf(m1, mxB);
+      const float uA = nA == -INFINITY ? 0.f : nA, uB = nB == -INFINITY ? 0.f : nB;
+      const float aA = exp2f(m0 - uA), aB = exp2f(m1 - uB);      // m = -inf -> 0
+      const float p00 = exp2f(s00 - uA), p10 = exp2f(s10 - uA);
+      const float p01 = exp2f(s01 - uB), p11 = exp2f(s11 - uB);
+      float sA = p00 + p10, sB = p01 + p11;
+#pragma unroll
+      for (int x = 4; x < 32; x <<= 1) {
+        sA += __shfl_xor_sync(0xffffffffu, sA, x);
+        sB += __shfl_xor_sync(0xffffffffu, sB, x);
+      }
+      l0 = l0 * aA + sA;
+      l1 = l1 * aB + sB;
+      m0 = nA;
+      m1 = nB;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { o[i][0] *= aA; o[i][1] *= aB; o[i][2] *= aA; o[i][3] *= aB; }
+      // P^T (keys x heads) as the B fragment: lane needs head g, keys 2t4, 2t4+1 (+8)
+      const uint32_t pk_lo = pack_bf16(p00, p01);      // key g,     heads 2t4, 2t4+1
+      const uint32_t pk_hi = pack_bf16(p10, p11);      // key g + 8, heads 2t4, 2t4+1
+      const int src0 = ((2 * t4) << 2) + (g >> 1), src1 = ((2 * t4 + 1) << 2) + (g >> 1);
+      const uint32_t v0 = __shfl_sync(0xffffffffu, pk_lo, src0);
+      const uint32_t v1 = __shfl_sync(0xffffffffu, pk_lo, src1);
+      const uint32_t v2 = __shfl_sync(0xffffffffu, pk_hi, src0);
+      const uint32_t v3 = __shfl_sync(0xffffffffu, pk_hi, src1);
+      const uint32_t sel = (g & 1) ? 0x7632u : 0x5410u;
+      const uint32_t pb0 = __byte_perm(v0, v1, sel);
+      const uint32_t pb1 = __byte_perm(v2, v3, sel);
+      // O^T += V^T . P^T for d = 16mt + [0, 16)
+      {
+        const int mi = lane >> 3, r8 = lane & 7;
+        const int key = warp * 16 + r8 + ((mi >> 1) << 3);
+#pragma unroll
+        for (int mt = 0; mt < 8; ++mt) {
+          const int box = mt >> 2;
+          const int chunk = ((mt & 3) << 1) + (mi & 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(base + 2 * kBoxBytes + box * kBoxBytes + swz(key, chunk), a0, a1, a2, a3);
+          mma_bf16(o[mt], a0, a1, a2, a3, pb0, pb1);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+    }
+    // merge the four warps' states into the item's partial; this lane holds O^T at
+    // d = 16mt + g (+8) for heads 2t4 and 2t4 + 1
+#pragma unroll
+    for (int mt = 0; mt < 8; ++mt) {
+      sm.o[warp][2 * t4][mt * 16 + g] = o[mt][0];
+      sm.o[warp][2 * t4 + 1][mt * 16 + g] = o[mt][1];
+      sm.o[warp][2 * t4][mt * 16 + g + 8] = o[mt][2];
+      sm.o[warp][2 * t4 + 1][mt * 16 + g + 8] = o[mt][3];
+    }
+    if (g == 0) {
+      sm.ml[warp][2 * t4][0] = m0; sm.ml[warp][2 * t4][1] = l0;
+      sm.ml[warp][2 * t4 + 1][0] = m1; sm.ml[warp][2 * t4 + 1][1] = l1;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+    {
+      const int d = threadIdx.x;                       // 0..127
+      for (int h = 0; h < a.G; ++h) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, sm.ml[w][h][0]);
+        float L = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float f = exp2f(sm.ml[w][h][0] - M);
+            L = fmaf(f, sm.ml[w][h][1], L);
+            acc = fmaf(f, sm.o[w][h][d], acc);
+          }
+        }
+        float* P = a.partials + ((int64_t)item * a.G + h) * kPartStride;
+        P[d] = acc;
+        if (d == 0) { P[kD] = M; P[kD + 1] = L; }
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerWarps * 32) : "memory");
+  }
+}
+
+}  // namespace tc
+
+// ---------------------------------------------------------------------------
+// host side: tensor maps and launch
+// ---------------------------------------------------------------------------
+
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// [units, t_cap, 128] bf16 cache as a 3-D tensor map with 64 x 64 boxes, 128B swizzle.
+static bool make_kv_map(CUtensorMap* map, const void* base, int64_t units, int64_t t_cap) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)t_cap, (cuuint64_t)units};
+  const cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)t_cap * kD * 2};
+  const cuuint32_t box[3] = {64, 64, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n;
+}
+
+cudaError_t attn_tc_launch(const AttnCall& c, const AttnWs& w, const int* stage_ids,
+                           const unsigned int* stage_mask, const int* stage_cnt, const int* pair_off,
+                           float* partials) {
+  const zha_geom& g = *c.g;
+  CUtensorMap km, vm;
+  const int64_t units_kv = (int64_t)g.B * g.Hkv;
+  if (!make_kv_map(&km, c.K, units_kv, g.t_cap) || !make_kv_map(&vm, c.V, units_kv, g.t_cap)) {
+    note_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+    return cudaErrorInvalidValue;
+  }
+  tc::Args a{};
+  a.B = g.B; a.nq = c.nq; a.Hq = g.Hq; a.Hkv = g.Hkv; a.G = g.Hq / g.Hkv; a.t_cap = g.t_cap;
+  a.q_pos = c.q_pos; a.pos_uniform = c.pos_uniform; a.nr = w.nr; a.cps = w.cps;
+  a.Q = (const __nv_bfloat16*)c.Q;
+  a.stage_ids = stage_ids; a.stage_mask = stage_mask; a.stage_cnt = stage_cnt; a.pair_off = pair_off;
+  a.pairs = w.pairs; a.partials = partials; a.dev_status = c.dev_status;
+  const size_t smem = sizeof(tc::Smem) + 1024;
+  cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int64_t grid = w.items_max < sm_count() ? w.items_max : sm_count();
+  tc::attn_tc_kernel<<<(unsigned)grid, tc::kThreads, smem, c.stream>>>(km, vm, a);
+  return cudaSuccess;
+}
+
+}  // namespace zha

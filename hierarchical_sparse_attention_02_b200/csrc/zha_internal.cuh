@@ -253,5 +253,9 @@ cudaError_t append_tokens(const zha_geom& g, void* K, void* V, const void* k_new
 cudaError_t route_all(const RouteCall& c);
 cudaError_t flat_select(const RouteCall& c);
 cudaError_t attention(const AttnCall& c);
+// bf16 split-KV gather on tensor cores (zha_attn_tc.cu)
+cudaError_t attn_tc_launch(const AttnCall& c, const AttnWs& w, const int* stage_ids,
+                           const unsigned int* stage_mask, const int* stage_cnt, const int* pair_off,
+                           float* partials);
 
 }  // namespace zha

@@ -34,7 +34,13 @@ __device__ __forceinline__ int top_level(const RouteGeom& g, int64_t t) {
 }
 
 // ---------------------------------------------------------------------------
-// score kernel: 128 threads, one candidate per thread; persistent over (qh, block)
+// score kernel: the G query heads of a (b, query, KV head) unit share every load.
+// A work item is 128 candidate slots of one unit: at the unit's top level 128
+// consecutive visible nodes; below it 128 / branch kept parents (their children) or the
+// unit's orphans.  Each thread converts one node's summaries once and scores them for
+// every head that has the node as a candidate; the score goes straight to that head's
+// compact candidate list (children of its i-th kept parent at i*branch + c, orphans
+// after all children), in ascending node order.
 // ---------------------------------------------------------------------------
 
 struct ScoreArgs {
@@ -49,73 +55,148 @@ struct ScoreArgs {
   int* cand_ids;                 // [nqh, C1]
   double* cand_score;            // [nqh, C1]
   int* cand_cnt;                 // [nqh]
-  int64_t nblk;                  // candidate blocks per query head
+  int64_t nblk;                  // work items per unit
   int32_t* dev_status;
 };
 
+constexpr int kScoreThreads = 128;
+
 template <typename KT>
-__global__ void __launch_bounds__(128) route_score_kernel(ScoreArgs a) {
-  __shared__ double qs[kD];
+__global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a) {
+  __shared__ __align__(16) double qs[kMaxG][kD];
+  __shared__ int rank[kScoreThreads][kMaxG];     // per parent slot: rank in each head's list
+  __shared__ int pcnt[kMaxG];
   const RouteGeom& g = a.g;
-  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
+  const int tid = threadIdx.x;
+  const int64_t units = (int64_t)g.B * g.nq * g.Hkv;
   const double scale = 1.0 / sqrt((double)kD);
-  for (int64_t w = blockIdx.x; w < nqh * a.nblk; w += gridDim.x) {
-    const int64_t qh = w / a.nblk;
+  const int per_blk = kScoreThreads / g.branch;          // parents per work item
+  for (int64_t w = blockIdx.x; w < units * a.nblk; w += gridDim.x) {
+    const int64_t u = w / a.nblk;
     const int64_t blk = w % a.nblk;
-    const int64_t bq = qh / g.Hq;
-    const int hq = (int)(qh % g.Hq);
+    const int64_t bq = u / g.Hkv;
+    const int hk = (int)(u % g.Hkv);
     const int64_t b = bq / g.nq;
-    const int hk = hq / g.G;
+    const int64_t qh0 = bq * g.Hq + (int64_t)hk * g.G;   // first head of the group
     const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
     if (!pos_ok(g, t)) {
-      if (blk == 0 && threadIdx.x == 0) set_status(a.dev_status, ZHA_ERR_INVALID_ARG);
+      if (blk == 0 && tid == 0) set_status(a.dev_status, ZHA_ERR_INVALID_ARG);
       continue;
     }
     const int top = top_level(g, t);
-    if (a.level > top) continue;                       // uniform over the CTA
+    if (a.level > top) continue;                         // uniform over the CTA
     const int64_t nvis = visible_nodes(t, g.span[a.level]);
-    int64_t n, nchild = 0, orph_lo = 0;
-    const int* par = a.parents + qh * a.C2;
-    if (a.level == top) {
-      n = nvis;
+    const bool at_top = a.level == top;
+    const int64_t npar = at_top ? 0 : visible_nodes(t, g.span[a.level + 1]);
+    const int64_t orph_lo = npar * g.branch;
+    const int64_t nb_par = (npar + per_blk - 1) / per_blk;
+    // which slots this item covers
+    int mode;                                            // 0 top nodes, 1 parents, 2 orphans
+    if (at_top) {
+      if (blk * kScoreThreads >= nvis) continue;
+      mode = 0;
+    } else if (blk < nb_par) {
+      mode = 1;
+    } else if (blk == nb_par && nvis > orph_lo) {
+      mode = 2;
+    } else if (blk == 0) {
+      mode = 3;                                          // nothing to score; counts only
     } else {
-      nchild = (int64_t)a.parents_cnt[qh] * g.branch;
-      orph_lo = visible_nodes(t, g.span[a.level + 1]) * g.branch;
-      n = nchild + (nvis - orph_lo);
+      continue;
     }
-    if (blk == 0 && threadIdx.x == 0) a.cand_cnt[qh] = (int)n;
-    const int64_t k = blk * 128 + threadIdx.x;
-    if (blk * 128 >= n) continue;                      // uniform over the CTA
+    __syncthreads();                                     // smem reuse across items
+    if (tid < g.G) pcnt[tid] = at_top ? 0 : a.parents_cnt[qh0 + tid];
+    for (int i = tid; i < g.G * kD; i += kScoreThreads) {
+      const KT* q = reinterpret_cast<const KT*>(a.Q) + qh0 * kD;
+      qs[i / kD][i % kD] = to_f64(q[i]);
+    }
     __syncthreads();
-    const KT* q = reinterpret_cast<const KT*>(a.Q) + qh * kD;
-    qs[threadIdx.x] = to_f64(q[threadIdx.x]);
-    __syncthreads();
-    if (k >= n) continue;
+    if (blk == 0 && tid < g.G)
+      a.cand_cnt[qh0 + tid] = (int)(at_top ? nvis : (int64_t)pcnt[tid] * g.branch + (nvis - orph_lo));
+    if (mode == 3) continue;
+    if (mode == 1) {
+      // rank of each parent of this item in each head's kept list (-1: not kept)
+      for (int i = tid; i < per_blk * g.G; i += kScoreThreads) {
+        const int j = i / g.G, h = i % g.G;
+        const int64_t p = blk * per_blk + j;
+        int r = -1;
+        if (p < npar) {
+          const int* lst = a.parents + (qh0 + h) * a.C2;
+          int lo = 0, hi = pcnt[h];
+          while (lo < hi) { const int m = (lo + hi) >> 1; if (lst[m] < p) lo = m + 1; else hi = m; }
+          if (lo < pcnt[h] && lst[lo] == p) r = lo;
+        }
+        rank[j][h] = r;
+      }
+      __syncthreads();
+    }
+    // this thread's node and the heads that have it as a candidate
     int64_t id;
-    if (a.level == top) id = k;
-    else if (k < nchild) id = (int64_t)par[k / g.branch] * g.branch + k % g.branch;
-    else id = orph_lo + (k - nchild);
-    const int64_t node = ((b * g.Hkv + hk) * g.ncap[a.level] + id);
+    unsigned int mask = 0;
+    int j = 0, c = 0;
+    if (mode == 0) {
+      id = blk * kScoreThreads + tid;
+      if (id < nvis) mask = (1u << g.G) - 1u;
+    } else if (mode == 1) {
+      j = tid / g.branch;
+      c = tid % g.branch;
+      id = (blk * per_blk + j) * g.branch + c;
+      if (j < per_blk)
+        for (int h = 0; h < g.G; ++h) mask |= (rank[j][h] >= 0 ? 1u : 0u) << h;
+    } else {
+      id = orph_lo + tid;
+      if (id < nvis) mask = (1u << g.G) - 1u;
+    }
+    if (!mask) continue;
+    const int64_t node = (b * g.Hkv + hk) * g.ncap[a.level] + id;
     const KT* kr = reinterpret_cast<const KT*>(a.k_route) + node * g.R * kD;
     const float* bh = a.b_hat + node * g.R;
-    double best = -INFINITY;
+    double best[kMaxG];
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) best[h] = -INFINITY;
     for (int r = 0; r < g.R; ++r) {
-      double acc = 0.0;
+      double acc[kMaxG];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.0;
       const KT* row = kr + r * kD;
       constexpr int kVec = 16 / sizeof(KT);
-#pragma unroll 4
-      for (int c = 0; c < kD; c += kVec) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + c);
+#pragma unroll 2
+      for (int cc = 0; cc < kD; cc += kVec) {
+        const uint4 v = *reinterpret_cast<const uint4*>(row + cc);
         const KT* e = reinterpret_cast<const KT*>(&v);
+        double x[kVec];
 #pragma unroll
-        for (int u = 0; u < kVec; ++u) acc = fma(qs[c + u], to_f64(e[u]), acc);
+        for (int uu = 0; uu < kVec; ++uu) x[uu] = to_f64(e[uu]);
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+          if (h < g.G && ((mask >> h) & 1u)) {
+            const double2* q2 = reinterpret_cast<const double2*>(&qs[h][cc]);
+#pragma unroll
+            for (int uu = 0; uu < kVec; uu += 2) {
+              const double2 qq = q2[uu / 2];
+              acc[h] = fma(qq.x, x[uu], acc[h]);
+              acc[h] = fma(qq.y, x[uu + 1], acc[h]);
+            }
+          }
+        }
       }
-      const double s = fma(acc, scale, (double)bh[r]);
-      best = fmax(best, s);
+      const double bb = (double)bh[r];
+#pragma unroll
+      for (int h = 0; h < kMaxG; ++h) best[h] = fmax(best[h], fma(acc[h], scale, bb));
     }
-    if (best == 0.0) best = 0.0;                       // one zero (no -0.0) for the key order
-    a.cand_ids[qh * a.C1 + k] = (int)id;
-    a.cand_score[qh * a.C1 + k] = best;
+#pragma unroll
+    for (int h = 0; h < kMaxG; ++h) {
+      if (h < g.G && ((mask >> h) & 1u)) {
+        int64_t pos;
+        if (mode == 0) pos = id;
+        else if (mode == 1) pos = (int64_t)rank[j][h] * g.branch + c;
+        else pos = (int64_t)pcnt[h] * g.branch + (id - orph_lo);
+        double s = best[h];
+        if (s == 0.0) s = 0.0;                           // one zero (no -0.0) for the key order
+        a.cand_ids[(qh0 + h) * a.C1 + pos] = (int)id;
+        a.cand_score[(qh0 + h) * a.C1 + pos] = s;
+      }
+    }
   }
 }
 
@@ -508,10 +589,18 @@ static cudaError_t route_levels(const RouteCall& c) {
     sa.cand_score = (double*)(c.ws + w.cand_score);
     sa.cand_cnt = (int*)(c.ws + w.cand_cnt);
     sa.dev_status = c.dev_status;
-    sa.nblk = (L.lv[l].n_cap + 127) / 128;
-    if (sa.nblk < 1) sa.nblk = 1;
+    {
+      const int64_t per_blk = kScoreThreads / g.branch;
+      int64_t nb = (L.lv[l].n_cap + kScoreThreads - 1) / kScoreThreads;
+      if (l < g.depth) {
+        const int64_t nbp = (L.lv[l + 1].n_cap + per_blk - 1) / per_blk + 1;
+        if (nbp > nb) nb = nbp;
+      }
+      sa.nblk = nb < 1 ? 1 : nb;
+    }
+    const int64_t units = (int64_t)g.B * c.nq * g.Hkv;
     trace_begin(ZHA_TRACE_ROUTE_SCORE, c.stream);
-    route_score_kernel<KT><<<grid_for(nqh * sa.nblk, 16), 128, 0, c.stream>>>(sa);
+    route_score_kernel<KT><<<grid_for(units * sa.nblk, 8), kScoreThreads, 0, c.stream>>>(sa);
     trace_end(ZHA_TRACE_ROUTE_SCORE, c.stream);
     count_launch();
     cudaError_t e = launch_status("route_score_kernel");

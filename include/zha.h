@@ -68,7 +68,7 @@ typedef enum zha_op {
 } zha_op;
 
 /* Geometry of one attention layer and its tree (host struct).
- * d must be 128; leaf must be 64; branch >= 2; 1 <= depth <= 8; 1 <= R <= 16;
+ * d must be 128; leaf must be 64; 2 <= branch <= 64; 1 <= depth <= 8; R in {1, 2, 4, 8, 16};
  * Hq % Hkv == 0 and Hq / Hkv <= 8; t_cap % leaf == 0; dtype a zha_dtype. */
 typedef struct zha_geom {
   int32_t B, Hq, Hkv, d;

@@ -46,7 +46,7 @@ def test_status_strings(lib):
 
 @pytest.mark.parametrize("kw,code", [
     ({}, 0), ({"d": 64}, 2), ({"leaf": 32}, 2), ({"Hq": 15}, 1), ({"Hq": 64, "Hkv": 2}, 2),
-    ({"R": 17}, 2), ({"R": 0}, 1), ({"depth": 9}, 2), ({"branch": 1}, 2), ({"t_cap": 1000}, 1),
+    ({"R": 17}, 2), ({"R": 0}, 1), ({"R": 3}, 2), ({"R": 16}, 0), ({"R": 1}, 0), ({"depth": 9}, 2), ({"branch": 1}, 2), ({"t_cap": 1000}, 1),
     ({"dtype": 7}, 2), ({"reserved": 1}, 1), ({"B": 0}, 1),
 ])
 def test_check_geom(lib, kw, code):

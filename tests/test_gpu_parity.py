@@ -161,10 +161,13 @@ def _check_tree(w, K, qref, tree, T, units):
             np.testing.assert_allclose(F[b, hk, :n].cpu().numpy(), L.F, rtol=1e-4, atol=0)
 
 
-@pytest.mark.parametrize("name,T,B", [("tiny-decode-f32", 8192, None), ("batched-decode-128k", 16384 + 64 * 5, 2),
-                                      ("deep-tree-16m", 70000, None)])
-def test_tree_build_parity(name, T, B):
+@pytest.mark.parametrize("name,T,B,R", [("tiny-decode-f32", 8192, None, 4), ("batched-decode-128k", 16384 + 64 * 5, 2, 4),
+                                        ("deep-tree-16m", 70000, None, 4), ("batched-decode-128k", 20000, 1, 1),
+                                        ("batched-decode-128k", 20000, 1, 16), ("tiny-decode-f32", 8192, None, 16)])
+def test_tree_build_parity(name, T, B, R):
+    import dataclasses
     w = S.scaled(S.workload(name), T=T, B=B, n_centres=min(S.workload(name).n_centres, 1024))
+    w = dataclasses.replace(w, R=R)
     g = geometry(w)
     C, K, V = S.clustered_kv(w, DEV)
     qref = S.reference_queries(w, DEV)
@@ -210,9 +213,15 @@ def test_append_equals_rebuild():
     ("long-decode-1m", 65536 + 64 * 7 + 63, 1, 0.99),    # the new token completes a leaf
     ("long-decode-1m", 65536 + 37, 1, 0.95),             # a partial chunk of 38 keys
     ("deep-tree-16m", 300000, None, 0.95),               # empty top levels
+    ("batched-decode-128k@R1", 32768, 1, 0.95),
+    ("batched-decode-128k@R16", 32768, 1, 0.9),
 ])
 def test_decode_parity(name, T, B, p):
-    w = S.scaled(S.workload(name), T=T, B=B, n_centres=min(S.workload(name).n_centres, 1024))
+    import dataclasses
+    base, _, rr = name.partition("@R")
+    w = S.scaled(S.workload(base), T=T, B=B, n_centres=min(S.workload(base).n_centres, 1024))
+    if rr:
+        w = dataclasses.replace(w, R=int(rr))
     run = DecodeRun(w, p)
     cmp = check_decode(run, [(b, h) for b in range(w.B) for h in range(w.Hkv)])
     print(f"{w.name} p={p}: {cmp.exact} exact, {cmp.near_cutoff} near-cutoff of {cmp.heads}")
