@@ -382,7 +382,7 @@ def main():
             entries += len(u) + (1 if sink else 0) + 1
     units = w.B * w.Hkv
     c1 = w.t_cap // 64
-    cps = max(16, -(-units * (c1 + 2) // 16384))
+    cps = max(16, -(-units * (c1 + 2) // 4096))                     # the library's split size
     items = -(-entries // cps)                                        # ranges: one per unit here
     gathered = union_rows * 2 * w.d * es
     partial_bytes = items * w.G * (w.d + 2) * 4          # o[d], m, l written per head and split

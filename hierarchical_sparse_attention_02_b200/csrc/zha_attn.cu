@@ -65,20 +65,37 @@ __global__ void __launch_bounds__(256) union_kernel(UnionArgs a) {
   if (a.dense) {
     for (int64_t i = lo + tid; i < hi && i < nvis; i += 256) mask[i - lo] = full;
   } else {
-    for (int h = 0; h < g.G; ++h) {
-      const int64_t qh = bq * g.Hq + hk * g.G + h;
+    // each head's slice [lower_bound(lo), lower_bound(hi)) of its ascending list, then
+    // one flat pass over all slices so that every thread's loads are independent
+    __shared__ int s_b0[kMaxG], s_off[kMaxG + 1];
+    if (tid < g.G) {
+      const int64_t qh = bq * g.Hq + hk * g.G + tid;
       const int* lst = a.leaf_ids + qh * a.leaf_cap;
       int cnt = a.leaf_cnt[qh];
       if (cnt > a.leaf_cap) cnt = a.leaf_cap;
-      // lower_bound(lo)
-      int b0 = 0, b1 = cnt;
-      while (b0 < b1) { const int m = (b0 + b1) >> 1; if (lst[m] < lo) b0 = m + 1; else b1 = m; }
-      for (int k = b0 + tid; k < cnt; k += 256) {
-        const int id = lst[k];
-        if (id >= hi) break;
-        if (id < 0 || id >= nvis) { set_status(a.dev_status, ZHA_ERR_INVALID_ARG); continue; }
-        atomicOr(&mask[id - lo], 1u << h);
-      }
+      if (cnt < 0) cnt = 0;
+      int x0 = 0, x1 = cnt;
+      while (x0 < x1) { const int m = (x0 + x1) >> 1; if (lst[m] < lo) x0 = m + 1; else x1 = m; }
+      int y0 = x0, y1 = cnt;
+      while (y0 < y1) { const int m = (y0 + y1) >> 1; if (lst[m] < hi) y0 = m + 1; else y1 = m; }
+      s_b0[tid] = x0;
+      s_off[tid + 1] = y0 - x0;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      s_off[0] = 0;
+      for (int h = 0; h < g.G; ++h) s_off[h + 1] += s_off[h];
+    }
+    __syncthreads();
+    const int total_ids = s_off[g.G];
+    for (int i = tid; i < total_ids; i += 256) {
+      int h = 0;
+      while (i >= s_off[h + 1]) ++h;
+      const int64_t qh = bq * g.Hq + hk * g.G + h;
+      const int id = a.leaf_ids[qh * a.leaf_cap + s_b0[h] + (i - s_off[h])];
+      // ids outside [lo, hi) mean an unsorted list; outside [0, nvis) an invisible chunk
+      if (id < lo || id >= hi || id >= nvis) { set_status(a.dev_status, ZHA_ERR_INVALID_ARG); continue; }
+      atomicOr(&mask[id - lo], 1u << h);
     }
   }
   __syncthreads();

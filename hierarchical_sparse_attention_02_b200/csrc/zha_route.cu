@@ -158,24 +158,32 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a)
       double acc[kMaxG];
 #pragma unroll
       for (int h = 0; h < kMaxG; ++h) acc[h] = 0.0;
-      const KT* row = kr + r * kD;
+      const uint4* row = reinterpret_cast<const uint4*>(kr + r * kD);
       constexpr int kVec = 16 / sizeof(KT);
-#pragma unroll 2
-      for (int cc = 0; cc < kD; cc += kVec) {
-        const uint4 v = *reinterpret_cast<const uint4*>(row + cc);
-        const KT* e = reinterpret_cast<const KT*>(&v);
-        double x[kVec];
+      constexpr int kRowVec = kD / kVec;                  // 16-byte vectors per row
+      constexpr int kPart = kRowVec < 16 ? kRowVec : 16;  // loaded together (in flight at once)
 #pragma unroll
-        for (int uu = 0; uu < kVec; ++uu) x[uu] = to_f64(e[uu]);
+      for (int part = 0; part < kRowVec; part += kPart) {
+        uint4 buf[kPart];
 #pragma unroll
-        for (int h = 0; h < kMaxG; ++h) {
-          if (h < g.G && ((mask >> h) & 1u)) {
-            const double2* q2 = reinterpret_cast<const double2*>(&qs[h][cc]);
+        for (int i = 0; i < kPart; ++i) buf[i] = __ldg(row + part + i);
 #pragma unroll
-            for (int uu = 0; uu < kVec; uu += 2) {
-              const double2 qq = q2[uu / 2];
-              acc[h] = fma(qq.x, x[uu], acc[h]);
-              acc[h] = fma(qq.y, x[uu + 1], acc[h]);
+        for (int i = 0; i < kPart; ++i) {
+          const int cc = (part + i) * kVec;
+          const KT* e = reinterpret_cast<const KT*>(&buf[i]);
+          double x[kVec];
+#pragma unroll
+          for (int uu = 0; uu < kVec; ++uu) x[uu] = to_f64(e[uu]);
+#pragma unroll
+          for (int h = 0; h < kMaxG; ++h) {
+            if (h < g.G && ((mask >> h) & 1u)) {
+              const double2* q2 = reinterpret_cast<const double2*>(&qs[h][cc]);
+#pragma unroll
+              for (int uu = 0; uu < kVec; uu += 2) {
+                const double2 qq = q2[uu / 2];
+                acc[h] = fma(qq.x, x[uu], acc[h]);
+                acc[h] = fma(qq.y, x[uu + 1], acc[h]);
+              }
             }
           }
         }
@@ -291,7 +299,7 @@ __global__ void __launch_bounds__(256) flat_score_kernel(FlatArgs a) {
 // select kernel: one CTA of 512 threads per query head (persistent)
 // ---------------------------------------------------------------------------
 
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = 256;
 constexpr int kDigit = 11;
 constexpr int kBuckets = 1 << kDigit;
 
@@ -377,6 +385,206 @@ __device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, SelSmem&
   return before + x - v;
 }
 
+// Candidates of one head: with kReg, thread tid holds the scores of the contiguous
+// candidates [tid * kSelPer, tid * kSelPer + kSelPer) in registers (n <= kSelThreads *
+// kSelPer) and compacts them in one ordered scan; otherwise every pass reads the
+// workspace and the compaction walks tiles of kSelThreads candidates.
+constexpr int kSelPer = 16;
+
+template <bool kReg>
+__device__ __forceinline__ void select_head(const SelectArgs& a, SelSmem& sm, int64_t qh, int n, int* lc) {
+  const int tid = threadIdx.x;
+  const double* s = a.cand_score + qh * a.C1;
+  const int* ids = a.cand_ids + qh * a.C1;
+  unsigned long long* E = a.cand_mass + qh * a.C1;
+  double rs[kReg ? kSelPer : 1];
+  const int i0 = tid * kSelPer;                      // first candidate of this thread (kReg)
+  if (kReg) {
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) rs[j] = (i0 + j < n) ? s[i0 + j] : 0.0;
+  }
+  // visit every candidate i of this thread with its score sv
+#define SEL_LOOP(BODY)                                                              \
+  if (kReg) {                                                                       \
+    _Pragma("unroll") for (int j = 0; j < kSelPer; ++j) {                           \
+      const int i = i0 + j;                                                         \
+      if (i < n) { const double sv = rs[j]; BODY }                                  \
+    }                                                                               \
+  } else {                                                                          \
+    for (int i = tid; i < n; i += kSelThreads) { const double sv = s[i]; BODY }     \
+  }
+  // 1. maximum and minimum score
+  double mx = -INFINITY, mn = INFINITY;
+  SEL_LOOP({ mx = fmax(mx, sv); mn = fmin(mn, sv); })
+  const double M = block_max_f64(mx, sm);
+  const double Mn = -block_max_f64(-mn, sm);
+  // 2. fixed-point masses and their exact total
+  unsigned long long z = 0;
+  SEL_LOOP({
+    const unsigned long long e = __double2ull_rn(ldexp(exp(sv - M), a.mass_shift));
+    E[i] = e;
+    z += e;
+  })
+  const unsigned long long Z = block_sum_u64(z, sm);
+  __syncthreads();   // E[] written by this block is visible to all its threads
+
+  // 3. cutoff: key threshold and the number of tied elements to keep
+  const bool keep_all = a.p >= 1.0 || n == 0;
+  unsigned long long pfx = 0, need = 0;
+  int shift = 0;
+  if (!keep_all) {
+    double tg = ceil(a.p * (double)Z);
+    unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
+    if (tgt > Z) tgt = Z;
+    const unsigned long long kmax = order_key(M), kmin = order_key(Mn);
+    unsigned long long above = 0;
+    unsigned int cnt_b = (unsigned int)n;
+    unsigned long long mass_b = Z;
+    if (kmax == kmin) {
+      shift = 0;
+      pfx = kmax;
+    } else {
+      // skip the leading bits every candidate shares, then 11-bit digits
+      int hi = 63 - __clzll((long long)(kmax ^ kmin));
+      pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
+      while (true) {
+        const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
+        const int lo = hi + 1 - width;
+        for (int i = tid; i < kBuckets; i += kSelThreads) { sm.cnt[i] = 0; sm.mass[i] = 0; }
+        if (tid == 0) { sm.bc_int[0] = 0; sm.bc_u64[0] = above; }
+        __syncthreads();
+        SEL_LOOP({
+          const unsigned long long key = order_key(sv);
+          if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+            const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+            atomicAdd(&sm.cnt[bkt], 1u);
+            atomicAdd(&sm.mass[bkt], E[i]);
+          }
+        })
+        __syncthreads();
+        // thread j owns kPer buckets, counted from the top (highest scores first)
+        constexpr int kPer = kBuckets / kSelThreads;
+        unsigned long long local = 0;
+        for (int q = 0; q < kPer; ++q) local += sm.mass[kBuckets - 1 - (tid * kPer + q)];
+        unsigned long long x = local;
+        const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (lane == 31) sm.wsum[warp] = x;
+        __syncthreads();
+        unsigned long long before = above;
+        for (int i = 0; i < warp; ++i) before += sm.wsum[i];
+        before += x - local;
+        if (before < tgt && before + local >= tgt) {
+          unsigned long long acc = before;
+          for (int q = 0; q < kPer; ++q) {
+            const int bkt = kBuckets - 1 - (tid * kPer + q);
+            if (acc + sm.mass[bkt] >= tgt) {
+              sm.bc_int[0] = bkt;
+              sm.bc_u64[0] = acc;       // mass strictly above the boundary bucket
+              break;
+            }
+            acc += sm.mass[bkt];
+          }
+        }
+        __syncthreads();
+        const int bstar = sm.bc_int[0];
+        above = sm.bc_u64[0];
+        cnt_b = sm.cnt[bstar];
+        mass_b = sm.mass[bstar];
+        pfx = (pfx << width) | (unsigned long long)bstar;
+        __syncthreads();
+        if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
+        hi = lo - 1;
+      }
+    }
+    // number of boundary-group elements to keep (exact ties share one mass value)
+    if (cnt_b <= 1) {
+      need = 1;
+    } else {
+      const unsigned long long e1 = mass_b / cnt_b;
+      need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
+      if (need < 1) need = 1;
+      if (need > cnt_b) need = cnt_b;
+    }
+  }
+
+  // 4. ordered compaction of the kept ids
+  int* outp = a.out_ids + qh * a.out_stride;
+  unsigned int written = 0;
+  bool overflow = false;
+  auto emit = [&](unsigned int pos, int id) {
+    if ((int64_t)pos < a.out_cap) outp[pos] = id;
+    else overflow = true;
+    if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
+      a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
+  };
+  if (kReg) {
+    // 0: drop, 1: keep, 2: tie (kept while its rank among ties is below `need`)
+    unsigned int cls = 0, ntie = 0;
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+      if (i0 + j < n) {
+        unsigned int c = 1;
+        if (!keep_all) {
+          const unsigned long long kk = order_key(rs[j]) >> shift;
+          c = kk > pfx ? 1u : (kk == pfx ? 2u : 0u);
+        }
+        cls |= c << (2 * j);
+        ntie += c == 2u;
+      }
+    }
+    unsigned int tie_total;
+    unsigned int tie_rank = block_excl_scan(ntie, sm, &tie_total);
+    unsigned int nkeep = 0;
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j) {
+      const unsigned int c = (cls >> (2 * j)) & 3u;
+      if (c == 2u) { if (tie_rank < need) { cls ^= 3u << (2 * j); /* -> 1 */ } else cls &= ~(3u << (2 * j)); ++tie_rank; }
+      nkeep += ((cls >> (2 * j)) & 3u) == 1u;
+    }
+    unsigned int keep_total;
+    unsigned int pos = block_excl_scan(nkeep, sm, &keep_total);
+#pragma unroll
+    for (int j = 0; j < kSelPer; ++j)
+      if (((cls >> (2 * j)) & 3u) == 1u) emit(pos++, ids[i0 + j]);
+    written = keep_total;
+  } else {
+    unsigned int ties_seen = 0;
+    const int ntiles = (n + kSelThreads - 1) / kSelThreads;
+    for (int tile = 0; tile < ntiles; ++tile) {
+      const int i = tile * kSelThreads + tid;
+      bool keep = false, tie = false;
+      if (i < n) {
+        if (keep_all) keep = true;
+        else {
+          const unsigned long long kk = order_key(s[i]) >> shift;
+          if (kk > pfx) keep = true;
+          else if (kk == pfx) tie = true;
+        }
+      }
+      unsigned int tie_total;
+      const unsigned int tie_rank = block_excl_scan(tie ? 1u : 0u, sm, &tie_total) + ties_seen;
+      if (tie && tie_rank < need) keep = true;
+      unsigned int keep_total;
+      const unsigned int pos = block_excl_scan(keep ? 1u : 0u, sm, &keep_total) + written;
+      if (keep) emit(pos, ids[i]);
+      written += keep_total;
+      ties_seen += tie_total;
+    }
+  }
+  if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
+  if (tid == 0) {
+    a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
+    if (lc) { lc[0] = n; lc[1] = (int)written; }
+  }
+  __syncthreads();
+#undef SEL_LOOP
+}
+
 __global__ void __launch_bounds__(kSelThreads) route_select_kernel(SelectArgs a) {
   __shared__ SelSmem sm;
   const RouteGeom& g = a.g;
@@ -395,146 +603,8 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(SelectArgs a)
       continue;
     }
     const int n = a.cand_cnt[qh];
-    const double* s = a.cand_score + qh * a.C1;
-    const int* ids = a.cand_ids + qh * a.C1;
-    unsigned long long* E = a.cand_mass + qh * a.C1;
-
-    // 1. maximum and minimum score
-    double mx = -INFINITY, mn = INFINITY;
-    for (int i = tid; i < n; i += kSelThreads) { mx = fmax(mx, s[i]); mn = fmin(mn, s[i]); }
-    const double M = block_max_f64(mx, sm);
-    const double Mn = -block_max_f64(-mn, sm);
-    // 2. fixed-point masses and their exact total
-    unsigned long long z = 0;
-    for (int i = tid; i < n; i += kSelThreads) {
-      const unsigned long long e = __double2ull_rn(ldexp(exp(s[i] - M), a.mass_shift));
-      E[i] = e;
-      z += e;
-    }
-    const unsigned long long Z = block_sum_u64(z, sm);
-    __syncthreads();   // E[] written by this block is visible to all its threads
-
-    // 3. cutoff: key threshold and the number of tied elements to keep
-    bool keep_all = a.p >= 1.0 || n == 0;
-    unsigned long long pfx = 0, need = 0;
-    int shift = 0;
-    if (!keep_all) {
-      double tg = ceil(a.p * (double)Z);
-      unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
-      if (tgt > Z) tgt = Z;
-      const unsigned long long kmax = order_key(M), kmin = order_key(Mn);
-      unsigned long long above = 0;
-      unsigned int cnt_b = (unsigned int)n;
-      unsigned long long mass_b = Z;
-      if (kmax == kmin) {
-        shift = 0;
-        pfx = kmax;
-      } else {
-        int hi = 63 - __clzll((long long)(kmax ^ kmin));
-        pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
-        while (true) {
-          const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
-          const int lo = hi + 1 - width;
-          for (int i = tid; i < kBuckets; i += kSelThreads) { sm.cnt[i] = 0; sm.mass[i] = 0; }
-          if (tid == 0) { sm.bc_int[0] = 0; sm.bc_u64[0] = above; }
-          __syncthreads();
-          for (int i = tid; i < n; i += kSelThreads) {
-            const unsigned long long key = order_key(s[i]);
-            if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
-              const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
-              atomicAdd(&sm.cnt[bkt], 1u);
-              atomicAdd(&sm.mass[bkt], E[i]);
-            }
-          }
-          __syncthreads();
-          // thread j owns the 4 buckets [kBuckets-4(j+1), kBuckets-4j), scanned from the top
-          constexpr int kPer = kBuckets / kSelThreads;
-          unsigned long long local = 0;
-          for (int q = 0; q < kPer; ++q) local += sm.mass[kBuckets - 1 - (tid * kPer + q)];
-          // exclusive scan of the u64 partials in thread order
-          unsigned long long x = local;
-          const int lane = tid & 31, warp = tid >> 5;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
-          }
-          if (lane == 31) sm.wsum[warp] = x;
-          __syncthreads();
-          unsigned long long before = above;
-          for (int i = 0; i < warp; ++i) before += sm.wsum[i];
-          before += x - local;
-          if (before < tgt && before + local >= tgt) {
-            unsigned long long acc = before;
-            unsigned int cacc = 0;
-            for (int q = 0; q < kPer; ++q) {
-              const int bkt = kBuckets - 1 - (tid * kPer + q);
-              if (acc + sm.mass[bkt] >= tgt) {
-                sm.bc_int[0] = bkt;
-                sm.bc_u64[0] = acc;       // mass strictly above the boundary bucket
-                break;
-              }
-              acc += sm.mass[bkt];
-              cacc += sm.cnt[bkt];
-            }
-          }
-          __syncthreads();
-          const int bstar = sm.bc_int[0];
-          above = sm.bc_u64[0];
-          cnt_b = sm.cnt[bstar];
-          mass_b = sm.mass[bstar];
-          pfx = (pfx << width) | (unsigned long long)bstar;
-          __syncthreads();
-          if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
-          hi = lo - 1;
-        }
-      }
-      // number of boundary-group elements to keep (exact ties share one mass value)
-      if (cnt_b <= 1) {
-        need = 1;
-      } else {
-        const unsigned long long e1 = mass_b / cnt_b;
-        need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
-        if (need < 1) need = 1;
-        if (need > cnt_b) need = cnt_b;
-      }
-    }
-
-    // 4. ordered compaction of the kept ids
-    int* outp = a.out_ids + qh * a.out_stride;
-    unsigned int written = 0, ties_seen = 0;
-    bool overflow = false;
-    for (int base = 0; base < n; base += kSelThreads) {
-      const int i = base + tid;
-      bool keep = false, tie = false;
-      if (i < n) {
-        if (keep_all) keep = true;
-        else {
-          const unsigned long long kk = order_key(s[i]) >> shift;
-          if (kk > pfx) keep = true;
-          else if (kk == pfx) tie = true;
-        }
-      }
-      unsigned int tie_total;
-      const unsigned int tie_rank = block_excl_scan(tie ? 1u : 0u, sm, &tie_total) + ties_seen;
-      if (tie && tie_rank < need) keep = true;
-      unsigned int keep_total;
-      const unsigned int pos = block_excl_scan(keep ? 1u : 0u, sm, &keep_total) + written;
-      if (keep) {
-        if ((int64_t)pos < a.out_cap) outp[pos] = ids[i];
-        else overflow = true;
-        if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
-          a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = ids[i];
-      }
-      written += keep_total;
-      ties_seen += tie_total;
-    }
-    if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
-    if (tid == 0) {
-      a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
-      if (lc) { lc[0] = n; lc[1] = (int)written; }
-    }
-    __syncthreads();
+    if (n <= kSelThreads * kSelPer) select_head<true>(a, sm, qh, n, lc);
+    else select_head<false>(a, sm, qh, n, lc);
   }
 }
 
