@@ -3,7 +3,7 @@
 //
 // The G query heads of one KV head share one gather: for each (b, query, KV head) unit
 // the heads' ascending leaf lists are merged into a union of chunk ids, each with a
-// bit mask of the heads that selected it.  The union is built per block of 4096 chunk
+// bit mask of the heads that selected it.  The union is built per block of kRange chunk
 // ids (no global zeroing, one pass), split into work items of `cps` entries, and a
 // persistent kernel walks the items: each item streams its K/V blocks once and keeps
 // an online softmax (m, l, o[d]) per head; a combine kernel merges the items' partials
@@ -88,8 +88,9 @@ __global__ void __launch_bounds__(256) union_kernel(UnionArgs a) {
     }
     __syncthreads();
     const int total_ids = s_off[g.G];
+    int h = 0;                                    // i only grows: the head index follows it
+#pragma unroll 4
     for (int i = tid; i < total_ids; i += 256) {
-      int h = 0;
       while (i >= s_off[h + 1]) ++h;
       const int64_t qh = bq * g.Hq + hk * g.G + h;
       const int id = a.leaf_ids[qh * a.leaf_cap + s_b0[h] + (i - s_off[h])];
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(256) union_kernel(UnionArgs a) {
     if (tid == 0) { out_ids[0] = -1; out_mask[0] = sink_mask; }
     base = 1;
   }
-  constexpr int kPer = kRange / 256;     // 16 consecutive ids per thread
+  constexpr int kPer = kRange / 256;     // consecutive ids per thread
   unsigned int cntl = 0;
   for (int q = 0; q < kPer; ++q) cntl += mask[tid * kPer + q] != 0;
   unsigned int x = cntl;

@@ -17,7 +17,7 @@ constexpr int kLeaf = 64;        // keys per leaf chunk
 constexpr int kMaxR = 16;        // reference queries per KV head
 constexpr int kMaxG = 8;         // query heads per KV head
 constexpr int kMaxDepth = 8;
-constexpr int kRange = 4096;     // chunk ids per union-building block
+constexpr int kRange = 1024;     // chunk ids per union-building block
 constexpr size_t kAlign = 256;
 // Floats per split-KV partial: o[d], the running max m and sum l, padded so that every
 // partial starts on a 16-byte boundary (vector stores).

@@ -59,6 +59,13 @@ struct ScoreArgs {
   int32_t* dev_status;
 };
 
+// D[8x8] += A[8x4] . B[4x8] in fp64 on the tensor cores (lane layout of mma.m8n8k4.f64:
+// a = A[lane/4][lane%4], b = B[lane%4][lane/4], (d0, d1) = D[lane/4][2*(lane%4) + {0,1}]).
+__device__ __forceinline__ void mma_f64(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
+}
+
 constexpr int kScoreThreads = 128;
 
 template <typename KT>
@@ -130,79 +137,71 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a)
       }
       __syncthreads();
     }
-    // this thread's node and the heads that have it as a candidate
-    int64_t id;
-    unsigned int mask = 0;
-    int j = 0, c = 0;
-    if (mode == 0) {
-      id = blk * kScoreThreads + tid;
-      if (id < nvis) mask = (1u << g.G) - 1u;
-    } else if (mode == 1) {
-      j = tid / g.branch;
-      c = tid % g.branch;
-      id = (blk * per_blk + j) * g.branch + c;
-      if (j < per_blk)
-        for (int h = 0; h < g.G; ++h) mask |= (rank[j][h] >= 0 ? 1u : 0u) << h;
-    } else {
-      id = orph_lo + tid;
-      if (id < nvis) mask = (1u << g.G) - 1u;
-    }
-    if (!mask) continue;
-    const int64_t node = (b * g.Hkv + hk) * g.ncap[a.level] + id;
-    const KT* kr = reinterpret_cast<const KT*>(a.k_route) + node * g.R * kD;
-    const float* bh = a.b_hat + node * g.R;
-    double best[kMaxG];
+    // Scores on the fp64 tensor cores: each warp takes its 32 slots as 4 groups of 8
+    // nodes; D[8 nodes x 8 heads] += A[8 nodes x 4 dims] . B[4 dims x 8 heads] per
+    // mma.m8n8k4.f64.  Lane L holds A[node L/4][dim 32*(L%4) + s] and B[dim][head L/4]
+    // at k-step s, so each lane reads 32 contiguous dims of its node's row.
+    const int lane = tid & 31, warp = tid >> 5;
+    const int hq_b = lane >> 2;                          // this lane's head in B
+    double qf[32];
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) best[h] = -INFINITY;
-    for (int r = 0; r < g.R; ++r) {
-      double acc[kMaxG];
-#pragma unroll
-      for (int h = 0; h < kMaxG; ++h) acc[h] = 0.0;
-      const uint4* row = reinterpret_cast<const uint4*>(kr + r * kD);
-      constexpr int kVec = 16 / sizeof(KT);
-      constexpr int kRowVec = kD / kVec;                  // 16-byte vectors per row
-      constexpr int kPart = kRowVec < 16 ? kRowVec : 16;  // loaded together (in flight at once)
-#pragma unroll
-      for (int part = 0; part < kRowVec; part += kPart) {
-        uint4 buf[kPart];
-#pragma unroll
-        for (int i = 0; i < kPart; ++i) buf[i] = __ldg(row + part + i);
-#pragma unroll
-        for (int i = 0; i < kPart; ++i) {
-          const int cc = (part + i) * kVec;
-          const KT* e = reinterpret_cast<const KT*>(&buf[i]);
-          double x[kVec];
-#pragma unroll
-          for (int uu = 0; uu < kVec; ++uu) x[uu] = to_f64(e[uu]);
-#pragma unroll
-          for (int h = 0; h < kMaxG; ++h) {
-            if (h < g.G && ((mask >> h) & 1u)) {
-              const double2* q2 = reinterpret_cast<const double2*>(&qs[h][cc]);
-#pragma unroll
-              for (int uu = 0; uu < kVec; uu += 2) {
-                const double2 qq = q2[uu / 2];
-                acc[h] = fma(qq.x, x[uu], acc[h]);
-                acc[h] = fma(qq.y, x[uu + 1], acc[h]);
-              }
-            }
-          }
-        }
+    for (int s2 = 0; s2 < 32; ++s2) qf[s2] = hq_b < g.G ? qs[hq_b][32 * (lane & 3) + s2] : 0.0;
+    const int h0 = 2 * (lane & 3), h1 = h0 + 1;         // this lane's heads in D
+    for (int grp = 0; grp < 4; ++grp) {
+      const int slot = warp * 32 + grp * 8 + (lane >> 2);
+      int64_t id = 0;
+      unsigned int mask = 0;
+      int j = 0, c = 0;
+      if (mode == 0) {
+        id = blk * kScoreThreads + slot;
+        if (id < nvis) mask = (1u << g.G) - 1u;
+      } else if (mode == 1) {
+        j = slot / g.branch;
+        c = slot % g.branch;
+        id = (blk * per_blk + j) * g.branch + c;
+        if (j < per_blk)
+          for (int h = 0; h < g.G; ++h) mask |= (rank[j][h] >= 0 ? 1u : 0u) << h;
+      } else {
+        id = orph_lo + slot;
+        if (id < nvis) mask = (1u << g.G) - 1u;
       }
-      const double bb = (double)bh[r];
+      if (!__any_sync(0xffffffffu, mask != 0)) continue; // warp-uniform
+      const int64_t node = (b * g.Hkv + hk) * g.ncap[a.level] + id;
+      const KT* kr = reinterpret_cast<const KT*>(a.k_route) + node * g.R * kD;
+      const float* bh = a.b_hat + node * g.R;
+      double best0 = -INFINITY, best1 = -INFINITY;
+      for (int r = 0; r < g.R; ++r) {
+        constexpr int kVec = 16 / sizeof(KT);
+        constexpr int kNv = 32 / kVec;                   // 16-byte vectors of 32 dims
+        uint4 v[kNv];
+        const uint4* src = reinterpret_cast<const uint4*>(kr + r * kD + 32 * (lane & 3));
 #pragma unroll
-      for (int h = 0; h < kMaxG; ++h) best[h] = fmax(best[h], fma(acc[h], scale, bb));
-    }
+        for (int i = 0; i < kNv; ++i) v[i] = mask ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+        double ca0 = 0.0, ca1 = 0.0, cb0 = 0.0, cb1 = 0.0;
 #pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-      if (h < g.G && ((mask >> h) & 1u)) {
-        int64_t pos;
-        if (mode == 0) pos = id;
-        else if (mode == 1) pos = (int64_t)rank[j][h] * g.branch + c;
-        else pos = (int64_t)pcnt[h] * g.branch + (id - orph_lo);
-        double s = best[h];
-        if (s == 0.0) s = 0.0;                           // one zero (no -0.0) for the key order
-        a.cand_ids[(qh0 + h) * a.C1 + pos] = (int)id;
-        a.cand_score[(qh0 + h) * a.C1 + pos] = s;
+        for (int s2 = 0; s2 < 32; ++s2) {
+          const KT* e = reinterpret_cast<const KT*>(&v[s2 / kVec]);
+          const double av = to_f64(e[s2 % kVec]);
+          if (s2 & 1) mma_f64(cb0, cb1, av, qf[s2]);
+          else mma_f64(ca0, ca1, av, qf[s2]);
+        }
+        const double bb = mask ? (double)bh[r] : 0.0;
+        best0 = fmax(best0, fma(ca0 + cb0, scale, bb));
+        best1 = fmax(best1, fma(ca1 + cb1, scale, bb));
+      }
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int h = q ? h1 : h0;
+        if (h < g.G && ((mask >> h) & 1u)) {
+          int64_t pos;
+          if (mode == 0) pos = id;
+          else if (mode == 1) pos = (int64_t)rank[j][h] * g.branch + c;
+          else pos = (int64_t)pcnt[h] * g.branch + (id - orph_lo);
+          double s = q ? best1 : best0;
+          if (s == 0.0) s = 0.0;                         // one zero (no -0.0) for the key order
+          a.cand_ids[(qh0 + h) * a.C1 + pos] = (int)id;
+          a.cand_score[(qh0 + h) * a.C1 + pos] = s;
+        }
       }
     }
   }
@@ -300,6 +299,7 @@ __global__ void __launch_bounds__(256) flat_score_kernel(FlatArgs a) {
 // ---------------------------------------------------------------------------
 
 constexpr int kSelThreads = 256;
+constexpr int kWarpSelMax = 16384;       // larger frontiers use the block-per-head kernel
 constexpr int kDigit = 11;
 constexpr int kBuckets = 1 << kDigit;
 
@@ -595,17 +595,229 @@ __global__ void __launch_bounds__(kSelThreads) route_select_kernel(SelectArgs a)
     const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
     const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
     int* lc = a.level_cnt ? a.level_cnt + (qh * g.depth + (a.level - 1)) * 2 : nullptr;
+    if (a.level > top) continue;                         // done by the warp kernel
+    const int n = a.cand_cnt[qh];
+    if (n <= kWarpSelMax) continue;                      // done by the warp kernel
+    select_head<false>(a, sm, qh, n, lc);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// warp select: one warp per query head for frontiers of up to kWarpSelMax candidates
+// (the common case).  Same algorithm as select_head with 8-bit digits, per-warp
+// histograms in shared memory and warp shuffles instead of block barriers.
+// ---------------------------------------------------------------------------
+
+constexpr int kWarpSelWarps = 8;
+constexpr int kWDigit = 8;
+constexpr int kWBuckets = 1 << kWDigit;
+
+struct WarpSelSmem {
+  unsigned int cnt[kWarpSelWarps][kWBuckets];
+  unsigned long long mass[kWarpSelWarps][kWBuckets];
+};
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ unsigned int warp_excl_scan(unsigned int v, unsigned int* total) {
+  const int lane = threadIdx.x & 31;
+  unsigned int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  *total = __shfl_sync(0xffffffffu, x, 31);
+  return x - v;
+}
+
+__global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(SelectArgs a) {
+  __shared__ WarpSelSmem sm;
+  const RouteGeom& g = a.g;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  unsigned int* hcnt = sm.cnt[wid];
+  unsigned long long* hmass = sm.mass[wid];
+  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
+  for (int64_t qh = (int64_t)blockIdx.x * kWarpSelWarps + wid; qh < nqh;
+       qh += (int64_t)gridDim.x * kWarpSelWarps) {
+    const int64_t bq = qh / g.Hq;
+    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
+    const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
+    int* lc = a.level_cnt ? a.level_cnt + (qh * g.depth + (a.level - 1)) * 2 : nullptr;
     if (a.level > top) {
-      if (tid == 0) {
+      if (lane == 0) {
         if (lc) { lc[0] = 0; lc[1] = 0; }
         if (a.level == 1) a.out_cnt[qh] = 0;
       }
       continue;
     }
     const int n = a.cand_cnt[qh];
-    if (n <= kSelThreads * kSelPer) select_head<true>(a, sm, qh, n, lc);
-    else select_head<false>(a, sm, qh, n, lc);
+    if (n > kWarpSelMax) continue;                      // the block kernel takes it
+    const double* s = a.cand_score + qh * a.C1;
+    const int* ids = a.cand_ids + qh * a.C1;
+    unsigned long long* E = a.cand_mass + qh * a.C1;
+    // 1. maximum and minimum
+    // every pass walks the candidates 8 per lane at a time, loads first (in flight together)
+#define WSEL_BATCH(LOADS, BODY)                                                     \
+    for (int base_ = 0; base_ < n; base_ += 32 * 8) {                               \
+      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
+        const int i = base_ + u_ * 32 + lane;                                       \
+        LOADS                                                                       \
+      }                                                                             \
+      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
+        const int i = base_ + u_ * 32 + lane;                                       \
+        if (i < n) { BODY }                                                         \
+      }                                                                             \
+    }
+    double sv[8];
+    unsigned long long ev[8];
+    double mx = -INFINITY, mn = INFINITY;
+    WSEL_BATCH({ sv[u_] = i < n ? s[i] : 0.0; }, { mx = fmax(mx, sv[u_]); mn = fmin(mn, sv[u_]); })
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mx = fmax(mx, shfl_xor_f64(mx, o));
+      mn = fmin(mn, shfl_xor_f64(mn, o));
+    }
+    // 2. fixed-point masses and their exact total
+    unsigned long long z = 0;
+    WSEL_BATCH({ sv[u_] = i < n ? s[i] : 0.0; }, {
+      const unsigned long long e = __double2ull_rn(ldexp(exp(sv[u_] - mx), a.mass_shift));
+      E[i] = e;
+      z += e;
+    })
+    const unsigned long long Z = warp_sum_u64(z);
+    __syncwarp();
+    // 3. cutoff
+    const bool keep_all = a.p >= 1.0 || n == 0;
+    unsigned long long pfx = 0, need = 0;
+    int shift = 0;
+    if (!keep_all) {
+      double tg = ceil(a.p * (double)Z);
+      unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
+      if (tgt > Z) tgt = Z;
+      const unsigned long long kmax = order_key(mx), kmin = order_key(mn);
+      unsigned long long above = 0;
+      unsigned int cnt_b = (unsigned int)n;
+      unsigned long long mass_b = Z;
+      if (kmax == kmin) {
+        pfx = kmax;
+      } else {
+        int hi = 63 - __clzll((long long)(kmax ^ kmin));
+        pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
+        while (true) {
+          const int width = (hi + 1) < kWDigit ? (hi + 1) : kWDigit;
+          const int lo = hi + 1 - width;
+#pragma unroll
+          for (int q = 0; q < kWBuckets / 32; ++q) { hcnt[lane + 32 * q] = 0; hmass[lane + 32 * q] = 0; }
+          __syncwarp();
+          WSEL_BATCH({ sv[u_] = i < n ? s[i] : 0.0; ev[u_] = i < n ? E[i] : 0ull; }, {
+            const unsigned long long key = order_key(sv[u_]);
+            if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+              const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+              atomicAdd(&hcnt[bkt], 1u);
+              atomicAdd(&hmass[bkt], ev[u_]);
+            }
+          })
+          __syncwarp();
+          // lane L owns the 8 buckets below kWBuckets - 8L (from the top: highest scores)
+          constexpr int kPer = kWBuckets / 32;
+          unsigned long long local = 0;
+#pragma unroll
+          for (int q = 0; q < kPer; ++q) local += hmass[kWBuckets - 1 - (lane * kPer + q)];
+          unsigned long long x = local;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+          }
+          const unsigned long long before = above + x - local;
+          const bool mine = before < tgt && before + local >= tgt;
+          int bstar = 0;
+          unsigned long long above_new = 0;
+          if (mine) {
+            unsigned long long acc = before;
+            for (int q = 0; q < kPer; ++q) {
+              const int bkt = kWBuckets - 1 - (lane * kPer + q);
+              if (acc + hmass[bkt] >= tgt) { bstar = bkt; above_new = acc; break; }
+              acc += hmass[bkt];
+            }
+          }
+          const unsigned int who = __ballot_sync(0xffffffffu, mine);
+          const int src = who ? __ffs(who) - 1 : 0;
+          bstar = __shfl_sync(0xffffffffu, bstar, src);
+          above = __shfl_sync(0xffffffffu, above_new, src);
+          cnt_b = hcnt[bstar];
+          mass_b = hmass[bstar];
+          pfx = (pfx << width) | (unsigned long long)bstar;
+          __syncwarp();
+          if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
+          hi = lo - 1;
+        }
+      }
+      if (cnt_b <= 1) {
+        need = 1;
+      } else {
+        const unsigned long long e1 = mass_b / cnt_b;
+        need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
+        if (need < 1) need = 1;
+        if (need > cnt_b) need = cnt_b;
+      }
+    }
+    // 4. ordered compaction: lane L owns the contiguous candidates [L*per, (L+1)*per)
+    const int per = (n + 31) / 32;
+    const int i0 = lane * per, i1 = (i0 + per < n) ? i0 + per : n;
+    unsigned int nt = 0;
+    if (!keep_all) {
+#pragma unroll 8
+      for (int i = i0; i < i1; ++i) nt += (order_key(s[i]) >> shift) == pfx;
+    }
+    unsigned int tie_total;
+    unsigned int tie_rank = warp_excl_scan(nt, &tie_total);
+    unsigned int nk = 0;
+    {
+      unsigned int tr = tie_rank;
+#pragma unroll 8
+      for (int i = i0; i < i1; ++i) {
+        bool keep = keep_all;
+        if (!keep_all) {
+          const unsigned long long kk = order_key(s[i]) >> shift;
+          keep = kk > pfx || (kk == pfx && tr++ < need);
+        }
+        nk += keep;
+      }
+    }
+    unsigned int written;
+    unsigned int pos = warp_excl_scan(nk, &written);
+    int* outp = a.out_ids + qh * a.out_stride;
+    bool overflow = false;
+#pragma unroll 4
+    for (int i = i0; i < i1; ++i) {
+      bool keep = keep_all;
+      if (!keep_all) {
+        const unsigned long long kk = order_key(s[i]) >> shift;
+        keep = kk > pfx || (kk == pfx && tie_rank++ < need);
+      }
+      if (keep) {
+        const int id = ids[i];
+        if ((int64_t)pos < a.out_cap) outp[pos] = id;
+        else overflow = true;
+        if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
+          a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
+        ++pos;
+      }
+    }
+    if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
+    if (lane == 0) {
+      a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
+      if (lc) { lc[0] = n; lc[1] = (int)written; }
+    }
+    __syncwarp();
   }
+#undef WSEL_BATCH
 }
 
 // ---------------------------------------------------------------------------
@@ -695,9 +907,16 @@ static cudaError_t route_levels(const RouteCall& c) {
     se.level_ids_cap = l >= 2 ? ncap_of(g, l) : 0;
     se.dev_status = c.dev_status;
     trace_begin(ZHA_TRACE_ROUTE_SELECT, c.stream);
-    route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+    route_select_warp_kernel<<<grid_for((nqh + kWarpSelWarps - 1) / kWarpSelWarps, 8), kWarpSelWarps * 32, 0,
+                               c.stream>>>(se);
     trace_end(ZHA_TRACE_ROUTE_SELECT, c.stream);
     count_launch();
+    e = launch_status("route_select_warp_kernel");
+    if (e != cudaSuccess) return e;
+    if (w.C1 > kWarpSelMax) {                            // frontiers too large for one warp
+      route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+      count_launch();
+    }
     e = launch_status("route_select_kernel");
     if (e != cudaSuccess) return e;
   }
@@ -734,8 +953,15 @@ static cudaError_t flat_select_t(const RouteCall& c) {
   se.cand_cnt = fa.cand_cnt; se.C1 = w.C1;
   se.out_ids = c.leaf_ids; se.out_cnt = c.leaf_cnt; se.out_stride = c.leaf_cap; se.out_cap = c.leaf_cap;
   se.dev_status = c.dev_status;
-  route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+  route_select_warp_kernel<<<grid_for((nqh + kWarpSelWarps - 1) / kWarpSelWarps, 8), kWarpSelWarps * 32, 0,
+                             c.stream>>>(se);
   count_launch();
+  e = launch_status("route_select_warp_kernel(flat)");
+  if (e != cudaSuccess) return e;
+  if (w.C1 > kWarpSelMax) {
+    route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+    count_launch();
+  }
   return launch_status("route_select_kernel(flat)");
 }
 

@@ -215,13 +215,18 @@ def test_append_equals_rebuild():
     ("deep-tree-16m", 300000, None, 0.95),               # empty top levels
     ("batched-decode-128k@R1", 32768, 1, 0.95),
     ("batched-decode-128k@R16", 32768, 1, 0.9),
+    ("deep-tree-16m@L1", 1200000 + 5, None, 0.95),       # one level: ~18.7K candidates per head
+    ("deep-tree-16m@L2", 1200000, None, 0.99),           # > 16K leaf candidates below the top
 ])
 def test_decode_parity(name, T, B, p):
     import dataclasses
     base, _, rr = name.partition("@R")
+    base, _, ll = base.partition("@L")
     w = S.scaled(S.workload(base), T=T, B=B, n_centres=min(S.workload(base).n_centres, 1024))
     if rr:
         w = dataclasses.replace(w, R=int(rr))
+    if ll:
+        w = dataclasses.replace(w, depth=int(ll))
     run = DecodeRun(w, p)
     cmp = check_decode(run, [(b, h) for b in range(w.B) for h in range(w.Hkv)])
     print(f"{w.name} p={p}: {cmp.exact} exact, {cmp.near_cutoff} near-cutoff of {cmp.heads}")
