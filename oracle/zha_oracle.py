@@ -195,10 +195,11 @@ def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
     for i0 in range(0, n1, block):
         i1 = min(n1, i0 + block)
         Kc = rows_f64(K, i0 * leaf, i1 * leaf).reshape(i1 - i0, leaf, d)
-        s = np.einsum("rd,ncd->nrc", qref, Kc) * scale
+        # s[n, r, c] = q_hat_r . k_{n,c} * scale  (a matrix product, then a reshape)
+        s = np.swapaxes((Kc.reshape(-1, d) @ qref.T).reshape(i1 - i0, leaf, -1), 1, 2) * scale
         F = lse(s, axis=-1)
         a = np.exp(s - F[..., None])
-        kh = np.einsum("nrc,ncd->nrd", a, Kc)
+        kh = np.matmul(a, Kc)                                   # [n, r, d] = a[n, r, c] . K[n, c, d]
         k1[i0:i1] = kh
         F1[i0:i1] = F
         b1[i0:i1] = F - np.einsum("rd,nrd->nr", qref, kh) * scale
