@@ -50,6 +50,8 @@ def parse():
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat"],
+                    help="zha: the hot path (default); dense / flat: the baselines on the same inputs")
     return ap.parse_args()
 
 
@@ -296,8 +298,21 @@ def main():
     build_ms = e0.elapsed_time(e1)
     k_bytes = w.B * w.Hkv * w.T * w.d * (2 if w.dtype == "bf16" else 4)
 
-    def step():
-        Z.zha_decode(g, q, k_new, v_new, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st)
+    if args.path == "zha":
+        def step():
+            Z.zha_decode(g, q, k_new, v_new, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st)
+    else:
+        # baselines attend from the same position over the same cache (new token appended once)
+        Z.zha_append(g, K, V, k_new, v_new, w.T, qref, tree, st)
+        qpos = torch.full((w.B, 1), w.T, dtype=torch.int64, device=dev)
+        op = Z.ZHA_OP_DENSE if args.path == "dense" else Z.ZHA_OP_FLAT
+        wsb = Z.empty_workspace(g, 1, op, dev)
+        if args.path == "dense":
+            def step():
+                Z.zha_dense_decode(g, q, K, V, qpos, O, wsb, st)
+        else:
+            def step():
+                Z.zha_flat_index(g, q, K, V, qpos, p, ids, cnt, O, wsb, st)
 
     for _ in range(args.warmup):
         step()
@@ -346,7 +361,12 @@ def main():
 
     def e2e_step():
         dq.copy_(hq, non_blocking=True); dk.copy_(hk, non_blocking=True); dv.copy_(hv, non_blocking=True)
-        Z.zha_decode(g, dq, dk, dv, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st)
+        if args.path == "zha":
+            Z.zha_decode(g, dq, dk, dv, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st)
+        elif args.path == "dense":
+            Z.zha_dense_decode(g, dq, K, V, qpos, O, wsb, st)
+        else:
+            Z.zha_flat_index(g, dq, K, V, qpos, p, ids, cnt, O, wsb, st)
         hO.copy_(O, non_blocking=True)
 
     for _ in range(2):
@@ -369,21 +389,31 @@ def main():
     vstart = (w.T // 64) * 64
     partial = w.T - vstart + 1
     ids_c, cnt_c = ids.cpu().numpy(), cnt.cpu().numpy()
-    per_head, union_rows, entries = [], 0, 0
-    for bb in range(w.B):
-        for hkv in range(w.Hkv):
-            lists = [ids_c[bb, 0, h, :cnt_c[bb, 0, h]] for h in range(hkv * w.G, (hkv + 1) * w.G)]
-            for lst in lists:
-                has0 = len(lst) and lst[0] == 0
-                per_head.append((len(lst) * 64 + (0 if has0 else 1) + partial) / T1)
-            u = np.unique(np.concatenate(lists)) if lists else np.zeros(0)
-            sink = any(not (len(l) and l[0] == 0) for l in lists) and vstart >= 64
-            union_rows += len(u) * 64 + (1 if sink else 0) + partial
-            entries += len(u) + (1 if sink else 0) + 1
+    nvis = vstart // 64
     units = w.B * w.Hkv
     c1 = w.t_cap // 64
     cps = max(16, -(-units * (c1 + 2) // 4096))                     # the library's split size
-    items = -(-entries // cps)                                        # ranges: one per unit here
+    krange = 1024                                                     # chunk ids per union block
+    per_head, union_rows, items = [], 0, 0
+    for bb in range(w.B):
+        for hkv in range(w.Hkv):
+            if args.path == "dense":
+                lists = [np.arange(nvis)] * w.G
+            else:
+                lists = [ids_c[bb, 0, h, :cnt_c[bb, 0, h]] for h in range(hkv * w.G, (hkv + 1) * w.G)]
+            for lst in lists:
+                has0 = len(lst) and lst[0] == 0
+                per_head.append((len(lst) * 64 + (0 if has0 or nvis == 0 else 1) + partial) / T1)
+            u = np.unique(np.concatenate(lists)) if lists else np.zeros(0, np.int64)
+            sink = any(not (len(l) and l[0] == 0) for l in lists) and nvis >= 1
+            union_rows += len(u) * 64 + (1 if sink else 0) + partial
+            # work items: per block of `krange` ids, ceil(entries / cps)
+            per_block = np.bincount(u // krange, minlength=nvis // krange + 1) if len(u) else np.zeros(1, np.int64)
+            per_block = per_block.astype(np.int64)
+            per_block[0] += 1 if sink else 0
+            per_block = np.concatenate([per_block, np.zeros(nvis // krange + 1, np.int64)])
+            per_block[nvis // krange] += 1                            # the query's own chunk
+            items += int(np.sum(-(-per_block // cps)))
     gathered = union_rows * 2 * w.d * es
     partial_bytes = items * w.G * (w.d + 2) * 4          # o[d], m, l written per head and split
     attn_bytes = gathered + partial_bytes
@@ -400,8 +430,9 @@ def main():
         "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": ws,
         "steps": Ksteps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": config_of(w, p),
-        "roofline": {"bound": "hbm", "kernel": "attn_split_kernel", "achieved": achieved, "peak": peak,
+        "config": {**config_of(w, p), "path": args.path},
+        "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel" if w.dtype == "bf16" else "attn_split_kernel",
+                     "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
                      "algorithmic_bytes_per_launch": attn_bytes, "kernel_ms": attn_ms},
         "step_hbm_gbs": attn_bytes / (ms * 1e-3) / 1e9,

@@ -290,29 +290,53 @@ __global__ void __launch_bounds__(256) attn_split_kernel(AttnArgs a) {
 // combine: one CTA of 128 threads per (unit, head); thread <-> dim
 // ---------------------------------------------------------------------------
 
+// 8 groups of 128 threads (thread <-> dim) each fold every 8th partial of the head with
+// a running maximum, then the groups are merged in a fixed order.
+constexpr int kCombGroups = 8;
+
 template <typename OT>
-__global__ void __launch_bounds__(128) combine_kernel(AttnGeom g, const int* pair_off, const float* partials,
-                                                      OT* O, float* lse) {
+__global__ void __launch_bounds__(kCombGroups * kD) combine_kernel(AttnGeom g, const int* pair_off,
+                                                                   const float* partials, OT* O, float* lse) {
+  __shared__ float gm[kCombGroups], gl[kCombGroups];
+  __shared__ float gacc[kCombGroups][kD];
   const int64_t uh = blockIdx.x;
   const int64_t u = uh / g.G;
   const int h = (int)(uh % g.G);
   const int64_t bq = u / g.Hkv;
   const int hk = (int)(u % g.Hkv);
+  const int d = threadIdx.x % kD, grp = threadIdx.x / kD;
   const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
-  float M = -INFINITY;
-  for (int64_t i = i0; i < i1; ++i) M = fmaxf(M, partials[(i * g.G + h) * kPartStride + kD]);
-  float L = 0.f, acc = 0.f;
-  if (M != -INFINITY) {
-    for (int64_t i = i0; i < i1; ++i) {
-      const float* P = partials + (i * g.G + h) * kPartStride;
-      const float w = exp2f(P[kD] - M);       // -inf partials weigh 0
-      L = fmaf(w, P[kD + 1], L);
-      acc = fmaf(w, P[threadIdx.x], acc);
-    }
+  float M = -INFINITY, L = 0.f, acc = 0.f;
+  for (int64_t i = i0 + grp; i < i1; i += kCombGroups) {
+    const float* P = partials + (i * g.G + h) * kPartStride;
+    const float m = P[kD];
+    const float Mn = fmaxf(M, m);
+    if (Mn == -INFINITY) continue;                 // nothing attended yet
+    const float a = exp2f(M - Mn), w = exp2f(m - Mn);
+    L = fmaf(L, a, w * P[kD + 1]);
+    acc = fmaf(acc, a, w * P[d]);
+    M = Mn;
   }
-  const int64_t qh = bq * g.Hq + hk * g.G + h;
-  O[qh * kD + threadIdx.x] = from_f32<OT>(L > 0.f ? acc / L : 0.f);
-  if (lse && threadIdx.x == 0) lse[qh] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+  gacc[grp][d] = acc;
+  if (d == 0) { gm[grp] = M; gl[grp] = L; }
+  __syncthreads();
+  if (grp == 0) {
+    float Mx = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kCombGroups; ++k) Mx = fmaxf(Mx, gm[k]);
+    float Lt = 0.f, At = 0.f;
+    if (Mx != -INFINITY) {
+#pragma unroll
+      for (int k = 0; k < kCombGroups; ++k) {
+        const float w = exp2f(gm[k] - Mx);        // -inf groups weigh 0
+        Lt = fmaf(w, gl[k], Lt);
+        At = fmaf(w, gacc[k][d], At);
+      }
+    }
+    const int64_t qh = bq * g.Hq + hk * g.G + h;
+    O[qh * kD + d] = from_f32<OT>(Lt > 0.f ? At / Lt : 0.f);
+    if (lse && d == 0) lse[qh] = Lt > 0.f ? (Mx + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -371,7 +395,7 @@ static cudaError_t attention_t(const AttnCall& c) {
     if ((e = launch_status("attn_split_kernel")) != cudaSuccess) return e;
   }
 
-  combine_kernel<KT><<<(unsigned)(w.units * ag.G), 128, 0, c.stream>>>(
+  combine_kernel<KT><<<(unsigned)(w.units * ag.G), kCombGroups * kD, 0, c.stream>>>(
       ag, pair_off, aa.partials, (KT*)c.O, c.lse);
   count_launch();
   return launch_status("combine_kernel");

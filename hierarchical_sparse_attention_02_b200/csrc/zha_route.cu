@@ -10,6 +10,8 @@
 //           integers 2^S * exp(s - max), so the sums are exact and order-free; the cutoff
 //           is found by a radix select over the order-preserving 64-bit key of s, and
 //           the kept ids are compacted in ascending order with a block scan.
+#include <cooperative_groups.h>
+
 #include "zha_internal.cuh"
 
 namespace zha {
@@ -299,7 +301,7 @@ __global__ void __launch_bounds__(256) flat_score_kernel(FlatArgs a) {
 // ---------------------------------------------------------------------------
 
 constexpr int kSelThreads = 256;
-constexpr int kWarpSelMax = 16384;       // larger frontiers use the block-per-head kernel
+constexpr int kWarpSelMax = 1024;        // larger frontiers use the cluster kernel
 constexpr int kDigit = 11;
 constexpr int kBuckets = 1 << kDigit;
 
@@ -821,6 +823,313 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
 }
 
 // ---------------------------------------------------------------------------
+// cluster select: one thread-block cluster (1..8 CTAs of kClThreads) per query head, for
+// frontiers above kWarpSelMax.  Each CTA takes a contiguous slice of the candidates; the
+// cluster's rank-0 CTA sums the per-CTA maxima, totals and digit histograms through
+// distributed shared memory and publishes every decision back into each CTA, so all CTAs
+// take identical decisions.  Cluster barriers are hardware barriers (no spin loops).
+// ---------------------------------------------------------------------------
+
+constexpr int kClThreads = 512;
+constexpr int kClMaxCta = 8;
+
+struct ClSmem {
+  unsigned int cnt[kBuckets];
+  unsigned long long mass[kBuckets];
+  unsigned long long wsum[kClThreads / 32];
+  double wd[kClThreads / 32];
+  unsigned int wcnt[kClThreads / 32];
+  // per-CTA contributions, written into the rank-0 CTA by every rank
+  unsigned long long slot_kmax[kClMaxCta], slot_kmin[kClMaxCta], slot_z[kClMaxCta];
+  unsigned int slot_tie[kClMaxCta], slot_keep[kClMaxCta];
+  // decisions published by rank 0
+  unsigned long long d_above, d_mass_b;
+  unsigned int d_cnt_b;
+  int d_bstar;
+};
+
+__device__ __forceinline__ double cl_block_max(double v, ClSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, shfl_xor_f64(v, o));
+  __syncthreads();
+  if (lane == 0) sm.wd[warp] = v;
+  __syncthreads();
+  double r = sm.wd[0];
+  for (int i = 1; i < kClThreads / 32; ++i) r = fmax(r, sm.wd[i]);
+  return r;
+}
+
+__device__ __forceinline__ unsigned long long cl_block_sum(unsigned long long v, ClSmem& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) sm.wsum[warp] = v;
+  __syncthreads();
+  unsigned long long r = 0;
+  for (int i = 0; i < kClThreads / 32; ++i) r += sm.wsum[i];
+  return r;
+}
+
+__device__ __forceinline__ unsigned int cl_excl_scan(unsigned int v, ClSmem& sm, unsigned int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  unsigned int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  __syncthreads();
+  if (lane == 31) sm.wcnt[warp] = x;
+  __syncthreads();
+  unsigned int before = 0, all = 0;
+  for (int i = 0; i < kClThreads / 32; ++i) {
+    if (i < warp) before += sm.wcnt[i];
+    all += sm.wcnt[i];
+  }
+  *total = all;
+  return before + x - v;
+}
+
+__global__ void __launch_bounds__(kClThreads) route_select_cluster_kernel(SelectArgs a) {
+  __shared__ ClSmem sm;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int CS = (int)cluster.num_blocks();
+  const int cr = (int)cluster.block_rank();
+  ClSmem* lead = cluster.map_shared_rank(&sm, 0);
+  const RouteGeom& g = a.g;
+  const int tid = threadIdx.x;
+  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
+  const int64_t nclusters = gridDim.x / CS;
+  for (int64_t qh = blockIdx.x / CS; qh < nqh; qh += nclusters) {
+    const int64_t bq = qh / g.Hq;
+    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
+    const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
+    if (a.level > top) continue;                         // the warp kernel writes the counts
+    const int n = a.cand_cnt[qh];
+    if (n <= kWarpSelMax) continue;                      // the warp kernel takes it
+    int* lc = a.level_cnt ? a.level_cnt + (qh * g.depth + (a.level - 1)) * 2 : nullptr;
+    const double* s = a.cand_score + qh * a.C1;
+    const int* ids = a.cand_ids + qh * a.C1;
+    unsigned long long* E = a.cand_mass + qh * a.C1;
+    const int chunk = (n + CS - 1) / CS;
+    const int r0 = cr * chunk < n ? cr * chunk : n;
+    const int r1 = r0 + chunk < n ? r0 + chunk : n;
+
+    // 1. maximum and minimum over the cluster
+    double mx = -INFINITY, mn = INFINITY;
+    for (int i = r0 + tid; i < r1; i += kClThreads) { const double v = s[i]; mx = fmax(mx, v); mn = fmin(mn, v); }
+    mx = cl_block_max(mx, sm);
+    mn = -cl_block_max(-mn, sm);
+    if (tid == 0) {
+      lead->slot_kmax[cr] = r1 > r0 ? order_key(mx) : 0ull;
+      lead->slot_kmin[cr] = r1 > r0 ? order_key(mn) : ~0ull;
+    }
+    cluster.sync();
+    unsigned long long kmax = 0, kmin = ~0ull;
+    for (int r = 0; r < CS; ++r) {
+      const unsigned long long x = lead->slot_kmax[r], y = lead->slot_kmin[r];
+      kmax = x > kmax ? x : kmax;
+      kmin = y < kmin ? y : kmin;
+    }
+    // back from the order key to the score
+    const unsigned long long mb = (kmax >> 63) ? (kmax & 0x7fffffffffffffffull) : ~kmax;
+    const double M = __longlong_as_double((long long)mb);
+    // 2. fixed-point masses and their exact total
+    unsigned long long z = 0;
+    for (int i = r0 + tid; i < r1; i += kClThreads) {
+      const unsigned long long e = __double2ull_rn(ldexp(exp(s[i] - M), a.mass_shift));
+      E[i] = e;
+      z += e;
+    }
+    z = cl_block_sum(z, sm);
+    if (tid == 0) lead->slot_z[cr] = z;
+    cluster.sync();
+    unsigned long long Z = 0;
+    for (int r = 0; r < CS; ++r) Z += lead->slot_z[r];
+
+    // 3. cutoff, with identical decisions in every CTA
+    const bool keep_all = a.p >= 1.0;
+    unsigned long long pfx = 0, need = 0;
+    int shift = 0;
+    if (!keep_all) {
+      double tg = ceil(a.p * (double)Z);
+      unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
+      if (tgt > Z) tgt = Z;
+      unsigned long long above = 0, mass_b = Z;
+      unsigned int cnt_b = (unsigned int)n;
+      if (kmax == kmin) {
+        pfx = kmax;
+      } else {
+        int hi = 63 - __clzll((long long)(kmax ^ kmin));
+        pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
+        while (true) {
+          const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
+          const int lo = hi + 1 - width;
+          for (int i = tid; i < kBuckets; i += kClThreads) { sm.cnt[i] = 0; sm.mass[i] = 0; }
+          __syncthreads();
+          for (int i = r0 + tid; i < r1; i += kClThreads) {
+            const unsigned long long key = order_key(s[i]);
+            if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+              const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+              atomicAdd(&sm.cnt[bkt], 1u);
+              atomicAdd(&sm.mass[bkt], E[i]);
+            }
+          }
+          cluster.sync();                                // every CTA's histogram is complete
+          if (cr == 0) {
+            // sum the CTAs' histograms (rank order) and find the boundary bucket
+            constexpr int kPer = kBuckets / kClThreads;
+            unsigned long long bm[kPer];
+            unsigned int bc[kPer];
+            unsigned long long local = 0;
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+              const int bkt = kBuckets - 1 - (tid * kPer + q);
+              unsigned long long m2 = 0;
+              unsigned int c2 = 0;
+              for (int r = 0; r < CS; ++r) {
+                ClSmem* o = cluster.map_shared_rank(&sm, r);
+                m2 += o->mass[bkt];
+                c2 += o->cnt[bkt];
+              }
+              bm[q] = m2;
+              bc[q] = c2;
+              local += m2;
+            }
+            unsigned long long x = local;
+            const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+              const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+              if (lane >= o) x += y;
+            }
+            if (lane == 31) sm.wsum[warp] = x;
+            __syncthreads();
+            unsigned long long before = above;
+            for (int i = 0; i < warp; ++i) before += sm.wsum[i];
+            before += x - local;
+            if (before < tgt && before + local >= tgt) {
+              unsigned long long acc = before;
+              for (int q = 0; q < kPer; ++q) {
+                if (acc + bm[q] >= tgt) {
+                  for (int r = 0; r < CS; ++r) {
+                    ClSmem* o = cluster.map_shared_rank(&sm, r);
+                    o->d_bstar = kBuckets - 1 - (tid * kPer + q);
+                    o->d_above = acc;
+                    o->d_cnt_b = bc[q];
+                    o->d_mass_b = bm[q];
+                  }
+                  break;
+                }
+                acc += bm[q];
+              }
+            }
+          }
+          cluster.sync();                                // decision published; histograms free
+          const int bstar = sm.d_bstar;
+          above = sm.d_above;
+          cnt_b = sm.d_cnt_b;
+          mass_b = sm.d_mass_b;
+          pfx = (pfx << width) | (unsigned long long)bstar;
+          if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
+          hi = lo - 1;
+        }
+      }
+      if (cnt_b <= 1) {
+        need = 1;
+      } else {
+        const unsigned long long e1 = mass_b / cnt_b;
+        need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
+        if (need < 1) need = 1;
+        if (need > cnt_b) need = cnt_b;
+      }
+    }
+
+    // 4. ordered compaction: thread t of CTA r owns a contiguous piece of the CTA's slice
+    const int len = r1 - r0;
+    const int per = (len + kClThreads - 1) / kClThreads;
+    const int i0 = r0 + tid * per < r1 ? r0 + tid * per : r1;
+    const int i1 = i0 + per < r1 ? i0 + per : r1;
+    unsigned int nt = 0;
+    if (!keep_all)
+      for (int i = i0; i < i1; ++i) nt += (order_key(s[i]) >> shift) == pfx;
+    unsigned int tie_cta;
+    unsigned int tie_rank = cl_excl_scan(nt, sm, &tie_cta);
+    if (tid == 0) lead->slot_tie[cr] = tie_cta;
+    cluster.sync();
+    for (int r = 0; r < cr; ++r) tie_rank += lead->slot_tie[r];
+    unsigned int nk = 0;
+    {
+      unsigned int tr = tie_rank;
+      for (int i = i0; i < i1; ++i) {
+        bool keep = keep_all;
+        if (!keep_all) {
+          const unsigned long long kk = order_key(s[i]) >> shift;
+          keep = kk > pfx || (kk == pfx && tr++ < need);
+        }
+        nk += keep;
+      }
+    }
+    unsigned int keep_cta;
+    unsigned int pos = cl_excl_scan(nk, sm, &keep_cta);
+    if (tid == 0) lead->slot_keep[cr] = keep_cta;
+    cluster.sync();
+    unsigned int written = 0;
+    for (int r = 0; r < CS; ++r) {
+      const unsigned int k = lead->slot_keep[r];
+      if (r < cr) pos += k;
+      written += k;
+    }
+    int* outp = a.out_ids + qh * a.out_stride;
+    bool overflow = false;
+    for (int i = i0; i < i1; ++i) {
+      bool keep = keep_all;
+      if (!keep_all) {
+        const unsigned long long kk = order_key(s[i]) >> shift;
+        keep = kk > pfx || (kk == pfx && tie_rank++ < need);
+      }
+      if (keep) {
+        const int id = ids[i];
+        if ((int64_t)pos < a.out_cap) outp[pos] = id;
+        else overflow = true;
+        if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
+          a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
+        ++pos;
+      }
+    }
+    if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
+    if (cr == 0 && tid == 0) {
+      a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
+      if (lc) { lc[0] = n; lc[1] = (int)written; }
+    }
+    cluster.sync();                                      // slots and smem reused by the next head
+  }
+}
+
+static cudaError_t launch_select_cluster(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
+  int cs = (int)((ncap + 8191) / 8192);
+  cs = cs < 1 ? 1 : (cs > kClMaxCta ? kClMaxCta : (cs > 4 ? 8 : (cs > 2 ? 4 : cs)));
+  int64_t clusters = nqh < (2 * 148) / cs ? nqh : (2 * 148) / cs;
+  if (clusters < 1) clusters = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(clusters * cs), 1, 1);
+  cfg.blockDim = dim3(kClThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, route_select_cluster_kernel, se);
+}
+
+// ---------------------------------------------------------------------------
 // host driver
 // ---------------------------------------------------------------------------
 
@@ -913,9 +1222,10 @@ static cudaError_t route_levels(const RouteCall& c) {
     count_launch();
     e = launch_status("route_select_warp_kernel");
     if (e != cudaSuccess) return e;
-    if (w.C1 > kWarpSelMax) {                            // frontiers too large for one warp
-      route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+    if (L.lv[l].n_cap > kWarpSelMax) {                   // frontiers too large for one warp
+      e = launch_select_cluster(se, nqh, L.lv[l].n_cap, c.stream);
       count_launch();
+      if (e != cudaSuccess) { note_cuda_error(e, "route_select_cluster_kernel"); return e; }
     }
     e = launch_status("route_select_kernel");
     if (e != cudaSuccess) return e;
@@ -959,10 +1269,11 @@ static cudaError_t flat_select_t(const RouteCall& c) {
   e = launch_status("route_select_warp_kernel(flat)");
   if (e != cudaSuccess) return e;
   if (w.C1 > kWarpSelMax) {
-    route_select_kernel<<<grid_for(nqh, 4), kSelThreads, 0, c.stream>>>(se);
+    e = launch_select_cluster(se, nqh, w.C1, c.stream);
     count_launch();
+    if (e != cudaSuccess) { note_cuda_error(e, "route_select_cluster_kernel(flat)"); return e; }
   }
-  return launch_status("route_select_kernel(flat)");
+  return launch_status("route_select_cluster_kernel(flat)");
 }
 
 // Flat indexer: `c.tree` carries the K cache pointer.
