@@ -290,53 +290,99 @@ __global__ void __launch_bounds__(256) attn_split_kernel(AttnArgs a) {
 // combine: one CTA of 128 threads per (unit, head); thread <-> dim
 // ---------------------------------------------------------------------------
 
-// 8 groups of 128 threads (thread <-> dim) each fold every 8th partial of the head with
-// a running maximum, then the groups are merged in a fixed order.
-constexpr int kCombGroups = 8;
+// Combine of the split partials, in up to two stages.  Stage 1: one CTA per (unit, head,
+// block of kCombBlock consecutive items); 4 groups of 128 threads (thread <-> dim) fold
+// every 4th partial of the block with a running maximum, then merge in a fixed order.  A
+// head with a single block writes O directly; otherwise the block's (o, m, l) replaces its
+// first partial and stage 2 merges the blocks.  Both stages use fixed orders (deterministic).
+constexpr int kCombGroups = 4;
+constexpr int kCombBlock = 128;
+
+struct Fold {
+  float M, L, acc;
+};
+
+__device__ __forceinline__ void fold_in(Fold& f, float m, float l, float o) {
+  const float Mn = fmaxf(f.M, m);
+  if (Mn == -INFINITY) return;                     // nothing attended yet
+  const float a = exp2f(f.M - Mn), w = exp2f(m - Mn);
+  f.L = fmaf(f.L, a, w * l);
+  f.acc = fmaf(f.acc, a, w * o);
+  f.M = Mn;
+}
+
+// Merges the groups' folds (in group order) into thread (group 0, dim d)'s result.
+__device__ __forceinline__ Fold merge_groups(const Fold& f, float (&gm)[kCombGroups], float (&gl)[kCombGroups],
+                                             float (&gacc)[kCombGroups][kD], int grp, int d) {
+  gacc[grp][d] = f.acc;
+  if (d == 0) { gm[grp] = f.M; gl[grp] = f.L; }
+  __syncthreads();
+  Fold r{-INFINITY, 0.f, 0.f};
+  if (grp == 0) {
+#pragma unroll
+    for (int k = 0; k < kCombGroups; ++k) fold_in(r, gm[k], gl[k], gacc[k][d]);
+  }
+  return r;
+}
 
 template <typename OT>
-__global__ void __launch_bounds__(kCombGroups * kD) combine_kernel(AttnGeom g, const int* pair_off,
-                                                                   const float* partials, OT* O, float* lse) {
+__device__ __forceinline__ void write_out(const AttnGeom& g, int64_t u, int h, int d, const Fold& r, OT* O,
+                                          float* lse) {
+  const int64_t bq = u / g.Hkv;
+  const int hk = (int)(u % g.Hkv);
+  const int64_t qh = bq * g.Hq + hk * g.G + h;
+  O[qh * kD + d] = from_f32<OT>(r.L > 0.f ? r.acc / r.L : 0.f);
+  if (lse && d == 0) lse[qh] = r.L > 0.f ? (r.M + log2f(r.L)) * 0.6931471805599453f : -INFINITY;
+}
+
+template <typename OT>
+__global__ void __launch_bounds__(kCombGroups * kD) combine_kernel(AttnGeom g, const int* pair_off, float* partials,
+                                                                   int64_t nb_max, OT* O, float* lse) {
+  __shared__ float gm[kCombGroups], gl[kCombGroups];
+  __shared__ float gacc[kCombGroups][kD];
+  const int64_t uh = blockIdx.x / nb_max;
+  const int64_t blk = blockIdx.x % nb_max;
+  const int64_t u = uh / g.G;
+  const int h = (int)(uh % g.G);
+  const int d = threadIdx.x % kD, grp = threadIdx.x / kD;
+  const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
+  const int64_t b0 = i0 + blk * kCombBlock;
+  if (b0 >= i1 && !(blk == 0)) return;             // uniform over the CTA
+  const int64_t b1 = b0 + kCombBlock < i1 ? b0 + kCombBlock : i1;
+  Fold f{-INFINITY, 0.f, 0.f};
+  for (int64_t i = b0 + grp; i < b1; i += kCombGroups) {
+    const float* P = partials + (i * g.G + h) * kPartStride;
+    fold_in(f, P[kD], P[kD + 1], P[d]);
+  }
+  const Fold r = merge_groups(f, gm, gl, gacc, grp, d);
+  if (grp != 0) return;
+  if (i1 - i0 <= kCombBlock) {
+    write_out(g, u, h, d, r, O, lse);
+  } else {
+    float* P = partials + (b0 * g.G + h) * kPartStride;
+    P[d] = r.acc;
+    if (d == 0) { P[kD] = r.M; P[kD + 1] = r.L; }
+  }
+}
+
+template <typename OT>
+__global__ void __launch_bounds__(kCombGroups * kD) combine_blocks_kernel(AttnGeom g, const int* pair_off,
+                                                                          const float* partials, OT* O, float* lse) {
   __shared__ float gm[kCombGroups], gl[kCombGroups];
   __shared__ float gacc[kCombGroups][kD];
   const int64_t uh = blockIdx.x;
   const int64_t u = uh / g.G;
   const int h = (int)(uh % g.G);
-  const int64_t bq = u / g.Hkv;
-  const int hk = (int)(u % g.Hkv);
   const int d = threadIdx.x % kD, grp = threadIdx.x / kD;
   const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
-  float M = -INFINITY, L = 0.f, acc = 0.f;
-  for (int64_t i = i0 + grp; i < i1; i += kCombGroups) {
-    const float* P = partials + (i * g.G + h) * kPartStride;
-    const float m = P[kD];
-    const float Mn = fmaxf(M, m);
-    if (Mn == -INFINITY) continue;                 // nothing attended yet
-    const float a = exp2f(M - Mn), w = exp2f(m - Mn);
-    L = fmaf(L, a, w * P[kD + 1]);
-    acc = fmaf(acc, a, w * P[d]);
-    M = Mn;
+  if (i1 - i0 <= kCombBlock) return;               // written by the first stage
+  Fold f{-INFINITY, 0.f, 0.f};
+  for (int64_t b0 = i0 + grp * kCombBlock; b0 < i1; b0 += kCombGroups * kCombBlock) {
+    const float* P = partials + (b0 * g.G + h) * kPartStride;
+    fold_in(f, P[kD], P[kD + 1], P[d]);
   }
-  gacc[grp][d] = acc;
-  if (d == 0) { gm[grp] = M; gl[grp] = L; }
-  __syncthreads();
-  if (grp == 0) {
-    float Mx = -INFINITY;
-#pragma unroll
-    for (int k = 0; k < kCombGroups; ++k) Mx = fmaxf(Mx, gm[k]);
-    float Lt = 0.f, At = 0.f;
-    if (Mx != -INFINITY) {
-#pragma unroll
-      for (int k = 0; k < kCombGroups; ++k) {
-        const float w = exp2f(gm[k] - Mx);        // -inf groups weigh 0
-        Lt = fmaf(w, gl[k], Lt);
-        At = fmaf(w, gacc[k][d], At);
-      }
-    }
-    const int64_t qh = bq * g.Hq + hk * g.G + h;
-    O[qh * kD + d] = from_f32<OT>(Lt > 0.f ? At / Lt : 0.f);
-    if (lse && d == 0) lse[qh] = Lt > 0.f ? (Mx + log2f(Lt)) * 0.6931471805599453f : -INFINITY;
-  }
+  const Fold r = merge_groups(f, gm, gl, gacc, grp, d);
+  if (grp == 0) write_out(g, u, h, d, r, O, lse);
 }
 
 // ---------------------------------------------------------------------------
@@ -395,10 +441,20 @@ static cudaError_t attention_t(const AttnCall& c) {
     if ((e = launch_status("attn_split_kernel")) != cudaSuccess) return e;
   }
 
-  combine_kernel<KT><<<(unsigned)(w.units * ag.G), kCombGroups * kD, 0, c.stream>>>(
-      ag, pair_off, aa.partials, (KT*)c.O, c.lse);
+  // items of one unit: at most ceil((C1 + 2) / cps) + nr
+  const int64_t items_unit = (w.C1 + 2 + w.cps - 1) / w.cps + w.nr;
+  const int64_t nb_max = (items_unit + kCombBlock - 1) / kCombBlock;
+  combine_kernel<KT><<<(unsigned)(w.units * ag.G * nb_max), kCombGroups * kD, 0, c.stream>>>(
+      ag, pair_off, aa.partials, nb_max, (KT*)c.O, c.lse);
   count_launch();
-  return launch_status("combine_kernel");
+  if ((e = launch_status("combine_kernel")) != cudaSuccess) return e;
+  if (nb_max > 1) {
+    combine_blocks_kernel<KT><<<(unsigned)(w.units * ag.G), kCombGroups * kD, 0, c.stream>>>(
+        ag, pair_off, aa.partials, (KT*)c.O, c.lse);
+    count_launch();
+    return launch_status("combine_blocks_kernel");
+  }
+  return cudaSuccess;
 }
 
 cudaError_t attention(const AttnCall& c) {

@@ -72,7 +72,7 @@ constexpr int kScoreThreads = 128;
 
 template <typename KT>
 __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a) {
-  __shared__ __align__(16) double qs[kMaxG][kD];
+  __shared__ __align__(16) double qfs[32][32];
   __shared__ int rank[kScoreThreads][kMaxG];     // per parent slot: rank in each head's list
   __shared__ int pcnt[kMaxG];
   const RouteGeom& g = a.g;
@@ -115,9 +115,11 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a)
     }
     __syncthreads();                                     // smem reuse across items
     if (tid < g.G) pcnt[tid] = at_top ? 0 : a.parents_cnt[qh0 + tid];
-    for (int i = tid; i < g.G * kD; i += kScoreThreads) {
+    // B fragments of the mma: qfs[s][L] = q[head L/4][32 * (L%4) + s] (0 for heads >= G)
+    for (int i = tid; i < 32 * 32; i += kScoreThreads) {
+      const int s2 = i / 32, L = i % 32, h = L >> 2;
       const KT* q = reinterpret_cast<const KT*>(a.Q) + qh0 * kD;
-      qs[i / kD][i % kD] = to_f64(q[i]);
+      qfs[s2][L] = h < g.G ? to_f64(q[h * kD + 32 * (L & 3) + s2]) : 0.0;
     }
     __syncthreads();
     if (blk == 0 && tid < g.G)
@@ -142,18 +144,17 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a)
     // Scores on the fp64 tensor cores: each warp takes its 32 slots as 4 groups of 8
     // nodes; D[8 nodes x 8 heads] += A[8 nodes x 4 dims] . B[4 dims x 8 heads] per
     // mma.m8n8k4.f64.  Lane L holds A[node L/4][dim 32*(L%4) + s] and B[dim][head L/4]
-    // at k-step s, so each lane reads 32 contiguous dims of its node's row.
+    // at k-step s (qf[s][L] in shared memory), so each lane reads 32 contiguous dims of
+    // its node's row.  The (group, reference) steps are software-pipelined: the next
+    // step's row is in flight while the current step's 32 mma run.
     const int lane = tid & 31, warp = tid >> 5;
-    const int hq_b = lane >> 2;                          // this lane's head in B
-    double qf[32];
-#pragma unroll
-    for (int s2 = 0; s2 < 32; ++s2) qf[s2] = hq_b < g.G ? qs[hq_b][32 * (lane & 3) + s2] : 0.0;
     const int h0 = 2 * (lane & 3), h1 = h0 + 1;         // this lane's heads in D
-    for (int grp = 0; grp < 4; ++grp) {
+    // node of this lane's row in group grp, and the heads that have it as a candidate
+    auto slot_of = [&](int grp, int64_t& id, unsigned int& mask, int& j, int& c) {
       const int slot = warp * 32 + grp * 8 + (lane >> 2);
-      int64_t id = 0;
-      unsigned int mask = 0;
-      int j = 0, c = 0;
+      mask = 0;
+      j = 0;
+      c = 0;
       if (mode == 0) {
         id = blk * kScoreThreads + slot;
         if (id < nvis) mask = (1u << g.G) - 1u;
@@ -167,44 +168,70 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a)
         id = orph_lo + slot;
         if (id < nvis) mask = (1u << g.G) - 1u;
       }
-      if (!__any_sync(0xffffffffu, mask != 0)) continue; // warp-uniform
-      const int64_t node = (b * g.Hkv + hk) * g.ncap[a.level] + id;
-      const KT* kr = reinterpret_cast<const KT*>(a.k_route) + node * g.R * kD;
-      const float* bh = a.b_hat + node * g.R;
-      double best0 = -INFINITY, best1 = -INFINITY;
-      for (int r = 0; r < g.R; ++r) {
-        constexpr int kVec = 16 / sizeof(KT);
-        constexpr int kNv = 32 / kVec;                   // 16-byte vectors of 32 dims
-        uint4 v[kNv];
-        const uint4* src = reinterpret_cast<const uint4*>(kr + r * kD + 32 * (lane & 3));
+    };
+    unsigned int any_mask = 0;
+    for (int grp = 0; grp < 4; ++grp) {
+      int64_t id; unsigned int m; int jj, cc;
+      slot_of(grp, id, m, jj, cc);
+      any_mask |= m;
+    }
+    if (!__any_sync(0xffffffffu, any_mask != 0)) continue;   // warp-uniform
+    constexpr int kVec = 16 / sizeof(KT);
+    constexpr int kNv = 32 / kVec;                       // 16-byte vectors of 32 dims
+    const int R = g.R;
+    const int nsteps = 4 * R;                            // even
+    const int64_t node0 = (b * g.Hkv + hk) * g.ncap[a.level];
+    auto load_step = [&](uint4 (&v)[kNv], int st) {
+      const int grp = st / R, r = st - grp * R;
+      int64_t id; unsigned int m; int jj, cc;
+      slot_of(grp, id, m, jj, cc);
+      const uint4* src = reinterpret_cast<const uint4*>(
+          reinterpret_cast<const KT*>(a.k_route) + ((node0 + id) * R + r) * kD + 32 * (lane & 3));
 #pragma unroll
-        for (int i = 0; i < kNv; ++i) v[i] = mask ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
-        double ca0 = 0.0, ca1 = 0.0, cb0 = 0.0, cb1 = 0.0;
+      for (int i = 0; i < kNv; ++i) v[i] = m ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+    };
+    double best0 = -INFINITY, best1 = -INFINITY;
+    auto compute_step = [&](const uint4 (&v)[kNv], int st) {
+      const int grp = st / R, r = st - grp * R;
+      double ca0 = 0.0, ca1 = 0.0, cb0 = 0.0, cb1 = 0.0;
 #pragma unroll
-        for (int s2 = 0; s2 < 32; ++s2) {
-          const KT* e = reinterpret_cast<const KT*>(&v[s2 / kVec]);
-          const double av = to_f64(e[s2 % kVec]);
-          if (s2 & 1) mma_f64(cb0, cb1, av, qf[s2]);
-          else mma_f64(ca0, ca1, av, qf[s2]);
-        }
-        const double bb = mask ? (double)bh[r] : 0.0;
-        best0 = fmax(best0, fma(ca0 + cb0, scale, bb));
-        best1 = fmax(best1, fma(ca1 + cb1, scale, bb));
+      for (int s2 = 0; s2 < 32; ++s2) {
+        const KT* e = reinterpret_cast<const KT*>(&v[s2 / kVec]);
+        const double av = (double)to_f32(e[s2 % kVec]);  // exact: bf16 / fp32 -> fp32 -> fp64
+        const double qv = qfs[s2][lane];
+        if (s2 & 1) mma_f64(cb0, cb1, av, qv);
+        else mma_f64(ca0, ca1, av, qv);
       }
+      int64_t id; unsigned int m; int jj, cc;
+      slot_of(grp, id, m, jj, cc);
+      const double bb = m ? (double)a.b_hat[(node0 + id) * R + r] : 0.0;
+      best0 = fmax(best0, fma(ca0 + cb0, scale, bb));
+      best1 = fmax(best1, fma(ca1 + cb1, scale, bb));
+      if (r == R - 1) {
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int h = q ? h1 : h0;
-        if (h < g.G && ((mask >> h) & 1u)) {
-          int64_t pos;
-          if (mode == 0) pos = id;
-          else if (mode == 1) pos = (int64_t)rank[j][h] * g.branch + c;
-          else pos = (int64_t)pcnt[h] * g.branch + (id - orph_lo);
-          double s = q ? best1 : best0;
-          if (s == 0.0) s = 0.0;                         // one zero (no -0.0) for the key order
-          a.cand_ids[(qh0 + h) * a.C1 + pos] = (int)id;
-          a.cand_score[(qh0 + h) * a.C1 + pos] = s;
+        for (int q = 0; q < 2; ++q) {
+          const int h = q ? h1 : h0;
+          if (h < g.G && ((m >> h) & 1u)) {
+            int64_t pos;
+            if (mode == 0) pos = id;
+            else if (mode == 1) pos = (int64_t)rank[jj][h] * g.branch + cc;
+            else pos = (int64_t)pcnt[h] * g.branch + (id - orph_lo);
+            double sc = q ? best1 : best0;
+            if (sc == 0.0) sc = 0.0;                     // one zero (no -0.0) for the key order
+            a.cand_ids[(qh0 + h) * a.C1 + pos] = (int)id;
+            a.cand_score[(qh0 + h) * a.C1 + pos] = sc;
+          }
         }
+        best0 = best1 = -INFINITY;
       }
+    };
+    uint4 vA[kNv], vB[kNv];
+    load_step(vA, 0);
+    for (int st = 0; st < nsteps; st += 2) {
+      load_step(vB, st + 1);
+      compute_step(vA, st);
+      if (st + 2 < nsteps) load_step(vA, st + 2);
+      compute_step(vB, st + 1);
     }
   }
 }
