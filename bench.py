@@ -165,6 +165,31 @@ class ClockSampler:
                 "samples": len(rows)}
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the attention
+# gather kernel, from the ncu capture summarised in
+# profiles/attn_tc_kernel.batched-decode-128k.md (batch 4, i.e. 16 of the 128 KV units),
+# valid while the kernel source is the one that was captured.
+PROFILED_TRAFFIC = {
+    "batched-decode-128k": {"bytes": 1.075265e9 + 11.197696e6, "units": 16,
+                            "source": "hierarchical_sparse_attention_02_b200/csrc/zha_attn_tc.cu",
+                            "sha1": "1a1445435c7ded07e36083d341e509ede65d6b56"},
+}
+
+
+def profiled_traffic(w, units: int):
+    import hashlib
+    rec = PROFILED_TRAFFIC.get(w.name)
+    if rec is None:
+        return None
+    try:
+        digest = hashlib.sha1(open(os.path.join(ROOT, rec["source"]), "rb").read()).hexdigest()
+    except OSError:
+        return None
+    if digest != rec["sha1"]:
+        return None                                      # the kernel changed since the capture
+    return rec["bytes"] * units / rec["units"]           # traffic grows with the units gathered
+
+
 def hbm_peak():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -433,7 +458,8 @@ def main():
         "config": {**config_of(w, p), "path": args.path},
         "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel" if w.dtype == "bf16" else "attn_split_kernel",
                      "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": profiled_traffic(w, units) if args.path == "zha" and w.dtype == "bf16" else None,
                      "algorithmic_bytes_per_launch": attn_bytes, "kernel_ms": attn_ms},
         "step_hbm_gbs": attn_bytes / (ms * 1e-3) / 1e9,
         "kv_touched": {"mean": float(np.mean(per_head)), "p50": float(np.median(per_head)),
