@@ -82,12 +82,21 @@ def barrier(ws):
 
 
 def max_over_ranks(x: float, ws: int) -> float:
+    """The maximum of x over the ranks (NCCL on the GPU, gloo on the host)."""
     if ws == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(units_per_rank: int, ms_local: float, ws: int) -> tuple:
+    """(slowest rank's ms per step, whole-job units per second): every rank processes
+    `units_per_rank` units per step (weak scaling), the job takes as long as its slowest rank."""
+    ms = max_over_ranks(ms_local, ws)
+    return ms, ws * units_per_rank / (ms * 1e-3)
 
 
 # ---------------------------------------------------------------------------
@@ -376,7 +385,7 @@ def main():
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(starts[:traced], stops[:traced])) / max(1, traced)
     if st.item() != 0:
         raise RuntimeError(f"device status {st.item()} in the timed region")
-    ms = max_over_ranks(ms_local, ws)
+    ms, value = whole_job_rate(w.B * w.Hq, ms_local, ws)
 
     # end to end through the public API with host buffers
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
@@ -444,7 +453,6 @@ def main():
     attn_bytes = gathered + partial_bytes
     peak, peak_kind = hbm_peak()
     achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
-    value = ws * w.B * w.Hq / (ms * 1e-3)
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda")

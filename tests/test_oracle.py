@@ -219,8 +219,9 @@ def test_stored_tree_rounds_where_stored():
 # ---------------------------------------------------------------------------
 
 
-def test_top_p_closed_form_with_ties(golden):
-    g = golden["top_p_ties"]
+@pytest.mark.parametrize("case", ["top_p_ties", "top_p_exact_boundary"])
+def test_top_p_closed_form_with_ties(golden, case):
+    g = golden[case]
     sel = zo.top_p(np.array([_ev(s) for s in g["scores"]]), np.array(g["ids"]), g["p"])
     assert sel.m == g["m"]
     assert sel.ids.tolist() == g["selected"]
