@@ -52,6 +52,8 @@ def parse():
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat"],
                     help="zha: the hot path (default); dense / flat: the baselines on the same inputs")
+    ap.add_argument("--sweep", action="store_true",
+                    help="crossover sweep over T and depth against the dense kernel (one JSON line each)")
     return ap.parse_args()
 
 
@@ -290,8 +292,73 @@ def config_of(w, p):
 # ---------------------------------------------------------------------------
 
 
+SWEEP_T = (16384, 32768, 65536, 131072, 262144, 524288, 1048576, 2097152)
+
+
+def run_sweep(args):
+    """Crossover sweep: ms per decode step of zha_decode at every depth L = 1..6 and of the
+    dense kernel, for T in SWEEP_T at the long-decode head geometry (B=4, Hq=32, Hkv=4),
+    on the same seeded inputs per T.  One JSON line per (T, path, depth)."""
+    import dataclasses
+    import hierarchical_sparse_attention_02_b200 as Z
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    base = S.workload("long-decode-1m")
+    p = args.p if args.p is not None else base.p[0]
+    for T in SWEEP_T:
+        w = S.scaled(base, T=T)
+        C, K, V = S.clustered_kv(w, dev)
+        qref = S.reference_queries(w, dev)
+        k_new, v_new = S.new_tokens(w, C, 1, dev)
+        q = S.queries(w, C, 1, dev)
+        del C
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        O = torch.empty(w.B, 1, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+
+        def timed(fn):
+            for _ in range(args.warmup):
+                fn()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            for _ in range(args.steps):
+                fn()
+            b.record()
+            torch.cuda.synchronize()
+            if st.item() != 0:
+                raise RuntimeError(f"device status {st.item()}")
+            return a.elapsed_time(b) / args.steps
+
+        best = None
+        for L in range(1, 7):
+            wl = dataclasses.replace(w, depth=L)
+            g = Z.Geometry(B=w.B, Hq=w.Hq, Hkv=w.Hkv, t_cap=w.t_cap, depth=L, R=w.R)
+            tree = Z.empty_tree(g, dev)
+            Z.zha_build_tree(g, K, w.T, qref, tree, st)
+            wsb = Z.empty_workspace(g, 1, Z.ZHA_OP_DECODE, dev)
+            ids = torch.empty(w.B, 1, w.Hq, Z.leaf_cap(g), dtype=torch.int32, device=dev)
+            cnt = torch.empty(w.B, 1, w.Hq, dtype=torch.int32, device=dev)
+            ms = timed(lambda: Z.zha_decode(g, q, k_new, v_new, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st))
+            touched = float((cnt.double() * 64 + 1).mean().item()) / (w.T + 1)
+            print(json.dumps({"sweep": "crossover", "T": T, "path": "zha", "depth": L, "p": p,
+                              "ms_per_step": ms, "kv_touched_approx": touched}), flush=True)
+            best = min(best, ms) if best is not None else ms
+            del tree, wsb, ids, cnt
+        g = Z.Geometry(B=w.B, Hq=w.Hq, Hkv=w.Hkv, t_cap=w.t_cap, depth=1, R=w.R)
+        wsd = Z.empty_workspace(g, 1, Z.ZHA_OP_DENSE, dev)
+        pos = torch.full((w.B, 1), w.T, dtype=torch.int64, device=dev)
+        ms_dense = timed(lambda: Z.zha_dense_decode(g, q, K, V, pos, O, wsd, st))
+        print(json.dumps({"sweep": "crossover", "T": T, "path": "dense", "ms_per_step": ms_dense,
+                          "zha_best_ms": best, "zha_faster": best < ms_dense}), flush=True)
+        del K, V, wsd
+        torch.cuda.empty_cache()
+
+
 def main():
     args = parse()
+    if args.sweep:
+        run_sweep(args)
+        return
     w = S.workload(args.workload)
     if args.batch is not None:
         w = S.scaled(w, T=w.T, B=args.batch)
