@@ -180,6 +180,20 @@ __device__ __forceinline__ double to_f64(__nv_bfloat16 x) {
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
+// Element i of a 16-byte vector of KT, without taking the vector's address (i is a
+// compile-time constant after unrolling, so this folds to a register move or shift).
+__device__ __forceinline__ uint32_t u4_word(const uint4& v, int w) {
+  return w == 0 ? v.x : w == 1 ? v.y : w == 2 ? v.z : v.w;
+}
+template <typename KT> __device__ __forceinline__ float u4_elem(const uint4& v, int i);
+template <> __device__ __forceinline__ float u4_elem<float>(const uint4& v, int i) {
+  return __uint_as_float(u4_word(v, i));
+}
+template <> __device__ __forceinline__ float u4_elem<__nv_bfloat16>(const uint4& v, int i) {
+  const uint32_t w = u4_word(v, i >> 1);
+  return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+}
+
 // fp64 -> storage type, a single round-to-nearest-even.
 __device__ __forceinline__ __nv_bfloat16 f64_to_bf16_rn(double x) {
   unsigned short r;
@@ -194,6 +208,13 @@ template <> __device__ __forceinline__ float from_f32<float>(float x) { return x
 template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) { return __float2bfloat16_rn(x); }
 
 __device__ __forceinline__ double shfl_xor_f64(double v, int m) { return __shfl_xor_sync(0xffffffffu, v, m); }
+
+// D[8x8] += A[8x4] . B[4x8] in fp64 on the tensor cores (lane layout of mma.m8n8k4.f64:
+// a = A[lane/4][lane%4], b = B[lane%4][lane/4], (d0, d1) = D[lane/4][2*(lane%4) + {0,1}]).
+__device__ __forceinline__ void mma_f64(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
+}
 
 // Position of the query of (b, qi): from q_pos, or the uniform position when q_pos is null.
 __device__ __forceinline__ int64_t query_pos(const int64_t* q_pos, int64_t uniform, int64_t bq) {

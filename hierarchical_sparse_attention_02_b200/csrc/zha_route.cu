@@ -61,13 +61,6 @@ struct ScoreArgs {
   int32_t* dev_status;
 };
 
-// D[8x8] += A[8x4] . B[4x8] in fp64 on the tensor cores (lane layout of mma.m8n8k4.f64:
-// a = A[lane/4][lane%4], b = B[lane%4][lane/4], (d0, d1) = D[lane/4][2*(lane%4) + {0,1}]).
-__device__ __forceinline__ void mma_f64(double& d0, double& d1, double a, double b) {
-  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
-               : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
-}
-
 constexpr int kScoreThreads = 128;
 
 template <typename KT>
@@ -196,8 +189,7 @@ __global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a)
       double ca0 = 0.0, ca1 = 0.0, cb0 = 0.0, cb1 = 0.0;
 #pragma unroll
       for (int s2 = 0; s2 < 32; ++s2) {
-        const KT* e = reinterpret_cast<const KT*>(&v[s2 / kVec]);
-        const double av = (double)to_f32(e[s2 % kVec]);  // exact: bf16 / fp32 -> fp32 -> fp64
+        const double av = (double)u4_elem<KT>(v[s2 / kVec], s2 % kVec);  // exact widening
         const double qv = qfs[s2][lane];
         if (s2 & 1) mma_f64(cb0, cb1, av, qv);
         else mma_f64(ca0, ca1, av, qv);
@@ -324,10 +316,11 @@ __global__ void __launch_bounds__(256) flat_score_kernel(FlatArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// select kernel: one CTA of 512 threads per query head (persistent)
+// top-p select over one level's candidates: exact radix select on the fp64 order key
+// with fixed-point masses (a warp per query head up to kWarpSelMax candidates, a
+// cluster of CTAs per query head above)
 // ---------------------------------------------------------------------------
 
-constexpr int kSelThreads = 256;
 constexpr int kWarpSelMax = 1024;        // larger frontiers use the cluster kernel
 constexpr int kDigit = 11;
 constexpr int kBuckets = 1 << kDigit;
@@ -358,283 +351,10 @@ __device__ __forceinline__ unsigned long long order_key(double s) {
   return (b >> 63) ? ~b : (b | 0x8000000000000000ull);
 }
 
-struct SelSmem {
-  unsigned int cnt[kBuckets];
-  unsigned long long mass[kBuckets];
-  unsigned long long wsum[kSelThreads / 32];
-  double wd[kSelThreads / 32];
-  unsigned int wcnt[kSelThreads / 32];
-  unsigned long long bc_u64[4];
-  double bc_f64[2];
-  int bc_int[4];
-};
-
-__device__ __forceinline__ double block_max_f64(double v, SelSmem& sm) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, shfl_xor_f64(v, o));
-  __syncthreads();
-  if (lane == 0) sm.wd[warp] = v;
-  __syncthreads();
-  double r = sm.wd[0];
-  for (int i = 1; i < kSelThreads / 32; ++i) r = fmax(r, sm.wd[i]);
-  return r;
-}
-
-__device__ __forceinline__ unsigned long long block_sum_u64(unsigned long long v, SelSmem& sm) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  __syncthreads();
-  if (lane == 0) sm.wsum[warp] = v;
-  __syncthreads();
-  unsigned long long r = 0;
-  for (int i = 0; i < kSelThreads / 32; ++i) r += sm.wsum[i];
-  return r;
-}
-
-// Exclusive block scan of small counts in thread order; returns the block total in *total.
-__device__ __forceinline__ unsigned int block_excl_scan(unsigned int v, SelSmem& sm, unsigned int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  __syncthreads();
-  if (lane == 31) sm.wcnt[warp] = x;
-  __syncthreads();
-  unsigned int before = 0, all = 0;
-  for (int i = 0; i < kSelThreads / 32; ++i) {
-    if (i < warp) before += sm.wcnt[i];
-    all += sm.wcnt[i];
-  }
-  *total = all;
-  return before + x - v;
-}
-
-// Candidates of one head: with kReg, thread tid holds the scores of the contiguous
-// candidates [tid * kSelPer, tid * kSelPer + kSelPer) in registers (n <= kSelThreads *
-// kSelPer) and compacts them in one ordered scan; otherwise every pass reads the
-// workspace and the compaction walks tiles of kSelThreads candidates.
-constexpr int kSelPer = 16;
-
-template <bool kReg>
-__device__ __forceinline__ void select_head(const SelectArgs& a, SelSmem& sm, int64_t qh, int n, int* lc) {
-  const int tid = threadIdx.x;
-  const double* s = a.cand_score + qh * a.C1;
-  const int* ids = a.cand_ids + qh * a.C1;
-  unsigned long long* E = a.cand_mass + qh * a.C1;
-  double rs[kReg ? kSelPer : 1];
-  const int i0 = tid * kSelPer;                      // first candidate of this thread (kReg)
-  if (kReg) {
-#pragma unroll
-    for (int j = 0; j < kSelPer; ++j) rs[j] = (i0 + j < n) ? s[i0 + j] : 0.0;
-  }
-  // visit every candidate i of this thread with its score sv
-#define SEL_LOOP(BODY)                                                              \
-  if (kReg) {                                                                       \
-    _Pragma("unroll") for (int j = 0; j < kSelPer; ++j) {                           \
-      const int i = i0 + j;                                                         \
-      if (i < n) { const double sv = rs[j]; BODY }                                  \
-    }                                                                               \
-  } else {                                                                          \
-    for (int i = tid; i < n; i += kSelThreads) { const double sv = s[i]; BODY }     \
-  }
-  // 1. maximum and minimum score
-  double mx = -INFINITY, mn = INFINITY;
-  SEL_LOOP({ mx = fmax(mx, sv); mn = fmin(mn, sv); })
-  const double M = block_max_f64(mx, sm);
-  const double Mn = -block_max_f64(-mn, sm);
-  // 2. fixed-point masses and their exact total
-  unsigned long long z = 0;
-  SEL_LOOP({
-    const unsigned long long e = __double2ull_rn(ldexp(exp(sv - M), a.mass_shift));
-    E[i] = e;
-    z += e;
-  })
-  const unsigned long long Z = block_sum_u64(z, sm);
-  __syncthreads();   // E[] written by this block is visible to all its threads
-
-  // 3. cutoff: key threshold and the number of tied elements to keep
-  const bool keep_all = a.p >= 1.0 || n == 0;
-  unsigned long long pfx = 0, need = 0;
-  int shift = 0;
-  if (!keep_all) {
-    double tg = ceil(a.p * (double)Z);
-    unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
-    if (tgt > Z) tgt = Z;
-    const unsigned long long kmax = order_key(M), kmin = order_key(Mn);
-    unsigned long long above = 0;
-    unsigned int cnt_b = (unsigned int)n;
-    unsigned long long mass_b = Z;
-    if (kmax == kmin) {
-      shift = 0;
-      pfx = kmax;
-    } else {
-      // skip the leading bits every candidate shares, then 11-bit digits
-      int hi = 63 - __clzll((long long)(kmax ^ kmin));
-      pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
-      while (true) {
-        const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
-        const int lo = hi + 1 - width;
-        for (int i = tid; i < kBuckets; i += kSelThreads) { sm.cnt[i] = 0; sm.mass[i] = 0; }
-        if (tid == 0) { sm.bc_int[0] = 0; sm.bc_u64[0] = above; }
-        __syncthreads();
-        SEL_LOOP({
-          const unsigned long long key = order_key(sv);
-          if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
-            const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
-            atomicAdd(&sm.cnt[bkt], 1u);
-            atomicAdd(&sm.mass[bkt], E[i]);
-          }
-        })
-        __syncthreads();
-        // thread j owns kPer buckets, counted from the top (highest scores first)
-        constexpr int kPer = kBuckets / kSelThreads;
-        unsigned long long local = 0;
-        for (int q = 0; q < kPer; ++q) local += sm.mass[kBuckets - 1 - (tid * kPer + q)];
-        unsigned long long x = local;
-        const int lane = tid & 31, warp = tid >> 5;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += y;
-        }
-        if (lane == 31) sm.wsum[warp] = x;
-        __syncthreads();
-        unsigned long long before = above;
-        for (int i = 0; i < warp; ++i) before += sm.wsum[i];
-        before += x - local;
-        if (before < tgt && before + local >= tgt) {
-          unsigned long long acc = before;
-          for (int q = 0; q < kPer; ++q) {
-            const int bkt = kBuckets - 1 - (tid * kPer + q);
-            if (acc + sm.mass[bkt] >= tgt) {
-              sm.bc_int[0] = bkt;
-              sm.bc_u64[0] = acc;       // mass strictly above the boundary bucket
-              break;
-            }
-            acc += sm.mass[bkt];
-          }
-        }
-        __syncthreads();
-        const int bstar = sm.bc_int[0];
-        above = sm.bc_u64[0];
-        cnt_b = sm.cnt[bstar];
-        mass_b = sm.mass[bstar];
-        pfx = (pfx << width) | (unsigned long long)bstar;
-        __syncthreads();
-        if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
-        hi = lo - 1;
-      }
-    }
-    // number of boundary-group elements to keep (exact ties share one mass value)
-    if (cnt_b <= 1) {
-      need = 1;
-    } else {
-      const unsigned long long e1 = mass_b / cnt_b;
-      need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
-      if (need < 1) need = 1;
-      if (need > cnt_b) need = cnt_b;
-    }
-  }
-
-  // 4. ordered compaction of the kept ids
-  int* outp = a.out_ids + qh * a.out_stride;
-  unsigned int written = 0;
-  bool overflow = false;
-  auto emit = [&](unsigned int pos, int id) {
-    if ((int64_t)pos < a.out_cap) outp[pos] = id;
-    else overflow = true;
-    if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
-      a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
-  };
-  if (kReg) {
-    // 0: drop, 1: keep, 2: tie (kept while its rank among ties is below `need`)
-    unsigned int cls = 0, ntie = 0;
-#pragma unroll
-    for (int j = 0; j < kSelPer; ++j) {
-      if (i0 + j < n) {
-        unsigned int c = 1;
-        if (!keep_all) {
-          const unsigned long long kk = order_key(rs[j]) >> shift;
-          c = kk > pfx ? 1u : (kk == pfx ? 2u : 0u);
-        }
-        cls |= c << (2 * j);
-        ntie += c == 2u;
-      }
-    }
-    unsigned int tie_total;
-    unsigned int tie_rank = block_excl_scan(ntie, sm, &tie_total);
-    unsigned int nkeep = 0;
-#pragma unroll
-    for (int j = 0; j < kSelPer; ++j) {
-      const unsigned int c = (cls >> (2 * j)) & 3u;
-      if (c == 2u) { if (tie_rank < need) { cls ^= 3u << (2 * j); /* -> 1 */ } else cls &= ~(3u << (2 * j)); ++tie_rank; }
-      nkeep += ((cls >> (2 * j)) & 3u) == 1u;
-    }
-    unsigned int keep_total;
-    unsigned int pos = block_excl_scan(nkeep, sm, &keep_total);
-#pragma unroll
-    for (int j = 0; j < kSelPer; ++j)
-      if (((cls >> (2 * j)) & 3u) == 1u) emit(pos++, ids[i0 + j]);
-    written = keep_total;
-  } else {
-    unsigned int ties_seen = 0;
-    const int ntiles = (n + kSelThreads - 1) / kSelThreads;
-    for (int tile = 0; tile < ntiles; ++tile) {
-      const int i = tile * kSelThreads + tid;
-      bool keep = false, tie = false;
-      if (i < n) {
-        if (keep_all) keep = true;
-        else {
-          const unsigned long long kk = order_key(s[i]) >> shift;
-          if (kk > pfx) keep = true;
-          else if (kk == pfx) tie = true;
-        }
-      }
-      unsigned int tie_total;
-      const unsigned int tie_rank = block_excl_scan(tie ? 1u : 0u, sm, &tie_total) + ties_seen;
-      if (tie && tie_rank < need) keep = true;
-      unsigned int keep_total;
-      const unsigned int pos = block_excl_scan(keep ? 1u : 0u, sm, &keep_total) + written;
-      if (keep) emit(pos, ids[i]);
-      written += keep_total;
-      ties_seen += tie_total;
-    }
-  }
-  if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
-  if (tid == 0) {
-    a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
-    if (lc) { lc[0] = n; lc[1] = (int)written; }
-  }
-  __syncthreads();
-#undef SEL_LOOP
-}
-
-__global__ void __launch_bounds__(kSelThreads) route_select_kernel(SelectArgs a) {
-  __shared__ SelSmem sm;
-  const RouteGeom& g = a.g;
-  const int tid = threadIdx.x;
-  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
-  for (int64_t qh = blockIdx.x; qh < nqh; qh += gridDim.x) {
-    const int64_t bq = qh / g.Hq;
-    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
-    const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
-    int* lc = a.level_cnt ? a.level_cnt + (qh * g.depth + (a.level - 1)) * 2 : nullptr;
-    if (a.level > top) continue;                         // done by the warp kernel
-    const int n = a.cand_cnt[qh];
-    if (n <= kWarpSelMax) continue;                      // done by the warp kernel
-    select_head<false>(a, sm, qh, n, lc);
-  }
-}
-
 // ---------------------------------------------------------------------------
 // warp select: one warp per query head for frontiers of up to kWarpSelMax candidates
-// (the common case).  Same algorithm as select_head with 8-bit digits, per-warp
-// histograms in shared memory and warp shuffles instead of block barriers.
+// (the common case): 8-bit digits, per-warp histograms in shared memory and warp
+// shuffles for every reduction and scan.
 // ---------------------------------------------------------------------------
 
 constexpr int kWarpSelWarps = 8;
@@ -685,7 +405,7 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
       continue;
     }
     const int n = a.cand_cnt[qh];
-    if (n > kWarpSelMax) continue;                      // the block kernel takes it
+    if (n > kWarpSelMax) continue;                      // the cluster kernel takes it
     const double* s = a.cand_score + qh * a.C1;
     const int* ids = a.cand_ids + qh * a.C1;
     unsigned long long* E = a.cand_mass + qh * a.C1;
@@ -1254,8 +974,6 @@ static cudaError_t route_levels(const RouteCall& c) {
       count_launch();
       if (e != cudaSuccess) { note_cuda_error(e, "route_select_cluster_kernel"); return e; }
     }
-    e = launch_status("route_select_kernel");
-    if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
 }

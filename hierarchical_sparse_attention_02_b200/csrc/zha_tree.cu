@@ -29,128 +29,168 @@ inline LevelPtrs level_ptrs(const zha_geom& g, const TreeLayout& L, void* base, 
 }
 
 // ---------------------------------------------------------------------------
-// leaf summaries: one CTA of 64 threads per leaf chunk (thread j <-> key j, then
-// thread i <-> dims 2i, 2i+1)
+// leaf summaries on the fp64 tensor cores: one CTA of 4 warps per leaf chunk.
+//   phase 1  S^T[64 keys x R] = K[64 x 128] . q_hat^T      (mma.m8n8k4.f64, 8 keys per tile)
+//   softmax  per reference over the 64 keys (fixed-order warp reductions)
+//   phase 2  k_hat^T[128 x R] = K^T[128 x 64] . a^T        (8 dims per tile, 4 keys per step)
+// References are padded to a multiple of 8 (the mma's N); the padding columns are zero.
+// In phase 1 lane L holds A[key L/4][dim 32*(L%4) + s] at k-step s: 32 contiguous dims of its
+// key; the B fragments (q_hat, then a) sit in shared memory as [step][lane].
 // ---------------------------------------------------------------------------
 
 template <typename KT, int R>
-struct alignas(16) LeafSmem {
-  KT keys[kLeaf][kD];           // the chunk, raw
-  double qref[R][kD];           // reference queries in fp64
-  double w[R][kLeaf];           // attention weights a_rj
-  double red[2][R];             // cross-warp partials
+struct alignas(16) LeafTcSmem {
+  static constexpr int NT = (R + 7) / 8;             // N-tiles of references
+  static constexpr int kRow = kD + 16 / sizeof(KT) * (sizeof(KT) == 2 ? 1 : 2);  // padded row
+  KT keys[kLeaf][kRow];                              // first: 16-byte aligned rows (272 / 544 B)
+  double qf[NT][32][32];                             // q_hat B fragments: [tile][step][lane]
+  double af[NT][16][32];                             // a B fragments:     [tile][step][lane]
+  double sS[R][kLeaf];                               // scaled scores
   double Fr[R];
+  double red[4][R];                                  // per-warp q_hat . k_hat partials
 };
 
 template <typename KT, int R>
-__global__ void __launch_bounds__(64) leaf_summarize_kernel(
+__global__ void __launch_bounds__(128) leaf_summarize_tc_kernel(
     const KT* __restrict__ K, const float* __restrict__ qref, int Hkv, int64_t t_cap,
     int64_t leaf_lo, int64_t nleaf, LevelPtrs out, double scale) {
+  using Sm = LeafTcSmem<KT, R>;
+  constexpr int NT = Sm::NT;
+  constexpr int kRow = Sm::kRow;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  LeafSmem<KT, R>& sm = *reinterpret_cast<LeafSmem<KT, R>*>(smem_raw);
+  Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t unit = blockIdx.x / nleaf;          // b * Hkv + h
+  const int64_t unit = blockIdx.x / nleaf;           // b * Hkv + h
   const int64_t leaf = leaf_lo + blockIdx.x % nleaf;
   const int h = (int)(unit % Hkv);
-
-  for (int i = tid; i < R * kD; i += 64) sm.qref[i / kD][i % kD] = (double)qref[(int64_t)h * R * kD + i];
+  const float* q = qref + (int64_t)h * R * kD;
+  for (int i = tid; i < NT * 32 * 32; i += 128) {
+    const int nt = i / 1024, s = (i / 32) % 32, L = i % 32;
+    const int r = nt * 8 + (L >> 2);
+    sm.qf[nt][s][L] = r < R ? (double)q[r * kD + 32 * (L & 3) + s] : 0.0;
+  }
   __syncthreads();
 
-  // phase 1: scores of key j against every reference, streaming the key row once
-  const KT* krow = K + (unit * t_cap + leaf * kLeaf + tid) * kD;
-  double acc[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) acc[r] = 0.0;
+  // phase 1: warp w takes keys [16w, 16w + 16) as two tiles of 8, interleaved (two
+  // independent accumulator chains per tile and reference tile)
   constexpr int kVec = 16 / sizeof(KT);
-#pragma unroll 2
-  for (int c = 0; c < kD; c += kVec) {
-    const uint4 v = *reinterpret_cast<const uint4*>(krow + c);
-    *reinterpret_cast<uint4*>(&sm.keys[tid][c]) = v;
-    const KT* e = reinterpret_cast<const KT*>(&v);
+  constexpr int kNv = 32 / kVec;
+  const KT* kbase = K + (unit * t_cap + leaf * kLeaf) * kD;
+  uint4 v[2][kNv];
 #pragma unroll
-    for (int u = 0; u < kVec; ++u) {
-      const double x = to_f64(e[u]);
+  for (int tile = 0; tile < 2; ++tile) {
+    const int key = warp * 16 + tile * 8 + (lane >> 2);
+    const uint4* src = reinterpret_cast<const uint4*>(kbase + key * kD + 32 * (lane & 3));
 #pragma unroll
-      for (int r = 0; r < R; ++r) acc[r] = fma(sm.qref[r][c + u], x, acc[r]);
+    for (int i = 0; i < kNv; ++i) v[tile][i] = __ldg(src + i);
+  }
+#pragma unroll
+  for (int tile = 0; tile < 2; ++tile) {
+    const int key = warp * 16 + tile * 8 + (lane >> 2);
+#pragma unroll
+    for (int i = 0; i < kNv; ++i)
+      *reinterpret_cast<uint4*>(&sm.keys[key][32 * (lane & 3) + i * kVec]) = v[tile][i];
+  }
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+    double c[2][2][2] = {};                          // [tile][chain][d0/d1]
+#pragma unroll
+    for (int s = 0; s < 32; ++s) {
+      const double b = sm.qf[nt][s][lane];
+#pragma unroll
+      for (int tile = 0; tile < 2; ++tile) {
+        mma_f64(c[tile][s & 1][0], c[tile][s & 1][1], (double)u4_elem<KT>(v[tile][s / kVec], s % kVec), b);
+      }
     }
-  }
-  // per-reference max over the 64 keys (fixed-order tree over lanes, then warps)
-  double m[R];
+    const int r0 = nt * 8 + 2 * (lane & 3);
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    acc[r] *= scale;
-    double v = acc[r];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v = fmax(v, shfl_xor_f64(v, o));
-    m[r] = v;
-  }
-  if (lane == 0) {
-#pragma unroll
-    for (int r = 0; r < R; ++r) sm.red[warp][r] = m[r];
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < R; ++r) m[r] = fmax(sm.red[0][r], sm.red[1][r]);
-  __syncthreads();
-  // exponentials and their sum
-  double e[R];
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    e[r] = exp(acc[r] - m[r]);
-    double v = e[r];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += shfl_xor_f64(v, o);
-    if (lane == 0) sm.red[warp][r] = v;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    const double Z = sm.red[0][r] + sm.red[1][r];
-    sm.w[r][tid] = e[r] / Z;
-    if (tid == 0) sm.Fr[r] = m[r] + log(Z);
+    for (int tile = 0; tile < 2; ++tile) {
+      const int krow = warp * 16 + tile * 8 + (lane >> 2);
+      if (r0 < R) sm.sS[r0][krow] = (c[tile][0][0] + c[tile][1][0]) * scale;
+      if (r0 + 1 < R) sm.sS[r0 + 1][krow] = (c[tile][0][1] + c[tile][1][1]) * scale;
+    }
   }
   __syncthreads();
 
-  // phase 2: k_hat_r[2i, 2i+1] = sum_j a_rj k_j
-  double k0[R], k1[R];
+  // softmax of each reference over the 64 keys: warp w takes references w, w + 4, ...
+  for (int r = warp; r < R; r += 4) {
+    const double v0 = sm.sS[r][lane], v1 = sm.sS[r][lane + 32];
+    double m = fmax(v0, v1);
 #pragma unroll
-  for (int r = 0; r < R; ++r) k0[r] = k1[r] = 0.0;
-#pragma unroll 4
-  for (int j = 0; j < kLeaf; ++j) {
-    const double x0 = to_f64(sm.keys[j][2 * tid]);
-    const double x1 = to_f64(sm.keys[j][2 * tid + 1]);
+    for (int o = 16; o > 0; o >>= 1) m = fmax(m, shfl_xor_f64(m, o));
+    const double e0 = exp(v0 - m), e1 = exp(v1 - m);
+    double z = e0 + e1;
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const double a = sm.w[r][j];
-      k0[r] = fma(a, x0, k0[r]);
-      k1[r] = fma(a, x1, k1[r]);
-    }
+    for (int o = 16; o > 0; o >>= 1) z += shfl_xor_f64(z, o);
+    if (lane == 0) sm.Fr[r] = m + log(z);
+    // a[r][key] -> B fragment of phase 2: step key / 4, lane (r % 8) * 4 + key % 4
+    sm.af[r / 8][lane >> 2][(r & 7) * 4 + (lane & 3)] = e0 / z;
+    sm.af[r / 8][(lane + 32) >> 2][(r & 7) * 4 + (lane & 3)] = e1 / z;
   }
-  // b_hat_r = F_r - scale * q_hat_r . k_hat_r
-  __syncthreads();
-#pragma unroll
-  for (int r = 0; r < R; ++r) {
-    double v = fma(sm.qref[r][2 * tid], k0[r], sm.qref[r][2 * tid + 1] * k1[r]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += shfl_xor_f64(v, o);
-    if (lane == 0) sm.red[warp][r] = v;
+  for (int i = tid; i < NT * 16 * 32; i += 128) {      // zero the padding references
+    const int nt = i / 512, s = (i / 32) % 16, L = i % 32;
+    if (nt * 8 + (L >> 2) >= R) sm.af[nt][s][L] = 0.0;
   }
   __syncthreads();
+
+  // phase 2: warp w takes the dim tiles w, w + 4, w + 8, w + 12
   const int64_t node = unit * out.n_cap + leaf;
   KT* kr = reinterpret_cast<KT*>(out.k_route) + node * R * kD;
   float* ks = out.k_state + node * R * kD;
+  double qk[NT][2];
 #pragma unroll
-  for (int r = 0; r < R; ++r) {
-    kr[r * kD + 2 * tid] = from_f64<KT>(k0[r]);
-    kr[r * kD + 2 * tid + 1] = from_f64<KT>(k1[r]);
-    *reinterpret_cast<float2*>(ks + r * kD + 2 * tid) =
-        make_float2(__double2float_rn(k0[r]), __double2float_rn(k1[r]));
+  for (int nt = 0; nt < NT; ++nt) qk[nt][0] = qk[nt][1] = 0.0;
+  double c4[4][NT][2] = {};                          // the warp's 4 dim tiles, interleaved
+#pragma unroll
+  for (int s = 0; s < 16; ++s) {
+    double b[NT];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) b[nt] = sm.af[nt][s][lane];
+#pragma unroll
+    for (int mi = 0; mi < 4; ++mi) {
+      const double av = (double)to_f32(sm.keys[4 * s + (lane & 3)][(warp + 4 * mi) * 8 + (lane >> 2)]);
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) mma_f64(c4[mi][nt][0], c4[mi][nt][1], av, b[nt]);
+    }
   }
+#pragma unroll
+  for (int mi = 0; mi < 4; ++mi) {
+    const int mt = warp + 4 * mi;
+    const int dim = mt * 8 + (lane >> 2);
+    double (&c)[NT][2] = c4[mi];
+    // lane holds k_hat[dim][refs nt*8 + 2*(lane%4) + {0, 1}]
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+      for (int x = 0; x < 2; ++x) {
+        const int r = nt * 8 + 2 * (lane & 3) + x;
+        if (r < R) {
+          kr[r * kD + dim] = from_f64<KT>(c[nt][x]);
+          ks[r * kD + dim] = __double2float_rn(c[nt][x]);
+          // q_hat[r][dim] from the phase-1 fragments: step dim % 32, lane (r % 8) * 4 + dim / 32
+          qk[nt][x] = fma(sm.qf[nt][dim & 31][(r & 7) * 4 + (dim >> 5)], c[nt][x], qk[nt][x]);
+        }
+      }
+    }
+  }
+  // b_hat_r = F_r - scale * q_hat_r . k_hat_r: lanes with the same lane % 4 hold one reference
+#pragma unroll
+  for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      double v = qk[nt][x];
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) v += shfl_xor_f64(v, o);
+      const int r = nt * 8 + 2 * (lane & 3) + x;
+      if (lane < 4 && r < R) sm.red[warp][r] = v;
+    }
+  }
+  __syncthreads();
   if (tid < R) {
     const double F = sm.Fr[tid];
-    const double qk = sm.red[0][tid] + sm.red[1][tid];
+    const double qkt = (sm.red[0][tid] + sm.red[1][tid]) + (sm.red[2][tid] + sm.red[3][tid]);
     out.F[node * R + tid] = __double2float_rn(F);
-    out.b_hat[node * R + tid] = __double2float_rn(F - scale * qk);
+    out.b_hat[node * R + tid] = __double2float_rn(F - scale * qkt);
   }
 }
 
@@ -255,13 +295,13 @@ static cudaError_t launch_leaves(const zha_geom& g, const TreeLayout& L, const v
                                  cudaStream_t s) {
   const int64_t n = hi - lo;
   const int64_t blocks = (int64_t)g.B * g.Hkv * n;
-  const size_t smem = sizeof(LeafSmem<KT, R>);
-  cudaFuncSetAttribute(leaf_summarize_kernel<KT, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  const size_t smem = sizeof(LeafTcSmem<KT, R>);
+  cudaFuncSetAttribute(leaf_summarize_tc_kernel<KT, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)smem);
-  leaf_summarize_kernel<KT, R><<<(unsigned)blocks, 64, smem, s>>>(
+  leaf_summarize_tc_kernel<KT, R><<<(unsigned)blocks, 128, smem, s>>>(
       (const KT*)K, qref, g.Hkv, g.t_cap, lo, n, level_ptrs(g, L, tree, 1), 1.0 / sqrt((double)g.d));
   count_launch();
-  return launch_status("leaf_summarize_kernel");
+  return launch_status("leaf_summarize_tc_kernel");
 }
 
 template <typename KT, int R>
