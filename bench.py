@@ -255,6 +255,45 @@ def oracle_rate(w: S.Workload, p: float, seconds: float, device: str):
     return heads / spent, heads, spent
 
 
+def stage_breakdown(lib, step, stream, nb, ms_step):
+    """Per-step GPU time of the traced kernels, from nb extra (untimed) steps whose
+    score, select and attention launches are bracketed by CUDA events on their stream.
+    With a chunked decode the routing of later chunks runs concurrently with attention,
+    so the stage sum exceeds the step time by the overlap."""
+    from hierarchical_sparse_attention_02_b200 import _lib
+    kinds = {"route_score": _lib.ZHA_TRACE_ROUTE_SCORE, "route_select": _lib.ZHA_TRACE_ROUTE_SELECT,
+             "attention": _lib.ZHA_TRACE_ATTN}
+    cap = nb * 64                     # <= 8 chunks x 8 levels per step
+    ev = {}
+    for name, kid in kinds.items():
+        a = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+        b = [torch.cuda.Event(enable_timing=True) for _ in range(cap)]
+        for e in a + b:
+            e.record(stream)
+        ev[name] = (a, b)
+    torch.cuda.synchronize()
+    keep = []
+    for name, kid in kinds.items():
+        a, b = ev[name]
+        arr_s = (ctypes.c_void_p * cap)(*[ctypes.c_void_p(e.cuda_event) for e in a])
+        arr_e = (ctypes.c_void_p * cap)(*[ctypes.c_void_p(e.cuda_event) for e in b])
+        keep.append((arr_s, arr_e))
+        lib.zha_trace(kid, arr_s, arr_e, cap)
+    for _ in range(nb):
+        step()
+    torch.cuda.synchronize()
+    out = {}
+    for name, kid in kinds.items():
+        n = lib.zha_trace_count(kid)
+        lib.zha_trace(kid, None, None, 0)
+        a, b = ev[name]
+        out[name] = sum(x.elapsed_time(y) for x, y in zip(a[:n], b[:n])) / nb
+    out["stage_sum"] = sum(out.values())
+    out["step"] = ms_step
+    out["steps"] = nb
+    return out
+
+
 def run_reference(args, w, p, ws, rank):
     if rank != 0:
         return
@@ -422,19 +461,20 @@ def main():
         raise RuntimeError(f"device status {st.item()} after warm-up")
 
     Ksteps = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(Ksteps)]
-    stops = [torch.cuda.Event(enable_timing=True) for _ in range(Ksteps)]
+    n_ev = Ksteps * 8                 # a decode step launches the attention once per chunk (<= 8)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+    stops = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
     for e in starts + stops:          # torch creates the CUDA event at its first record
         e.record(stream)
     torch.cuda.synchronize()
-    arr_s = (ctypes.c_void_p * Ksteps)(*[ctypes.c_void_p(e.cuda_event) for e in starts])
-    arr_e = (ctypes.c_void_p * Ksteps)(*[ctypes.c_void_p(e.cuda_event) for e in stops])
+    arr_s = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(e.cuda_event) for e in starts])
+    arr_e = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(e.cuda_event) for e in stops])
     lib = _lib.load()
     clocks = ClockSampler(torch.cuda.current_device())
     time.sleep(0.3)
     barrier(ws)
     torch.cuda.synchronize()
-    lib.zha_trace(_lib.ZHA_TRACE_ATTN, arr_s, arr_e, Ksteps)
+    lib.zha_trace(_lib.ZHA_TRACE_ATTN, arr_s, arr_e, n_ev)
     n_launch0 = Z.launch_count()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark_start()
@@ -449,10 +489,12 @@ def main():
     traced = lib.zha_trace_count(_lib.ZHA_TRACE_ATTN)
     lib.zha_trace(_lib.ZHA_TRACE_ATTN, None, None, 0)
     ms_local = t_start.elapsed_time(t_end) / Ksteps
+    attn_launches = traced / Ksteps                        # attention launches per step
     attn_ms = sum(a.elapsed_time(b) for a, b in zip(starts[:traced], stops[:traced])) / max(1, traced)
     if st.item() != 0:
         raise RuntimeError(f"device status {st.item()} in the timed region")
     ms, value = whole_job_rate(w.B * w.Hq, ms_local, ws)
+    stages = stage_breakdown(lib, step, stream, min(Ksteps, 20), ms_local)
 
     # end to end through the public API with host buffers
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
@@ -519,7 +561,10 @@ def main():
     partial_bytes = items * w.G * (w.d + 2) * 4          # o[d], m, l written per head and split
     attn_bytes = gathered + partial_bytes
     peak, peak_kind = hbm_peak()
-    achieved = attn_bytes / (attn_ms * 1e-3) / 1e9
+    # per launch: a decode step attends in `attn_launches` chunk launches (whole-step bytes
+    # split by chunk; the chunks are equal in size up to a ragged last one)
+    per_launch = attn_bytes / max(1.0, attn_launches)
+    achieved = per_launch / (attn_ms * 1e-3) / 1e9
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda")
@@ -534,12 +579,15 @@ def main():
         "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel" if w.dtype == "bf16" else "attn_split_kernel",
                      "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": profiled_traffic(w, units) if args.path == "zha" and w.dtype == "bf16" else None,
-                     "algorithmic_bytes_per_launch": attn_bytes, "kernel_ms": attn_ms},
+                     "traffic": (profiled_traffic(w, units / max(1.0, attn_launches))
+                                 if args.path == "zha" and w.dtype == "bf16" else None),
+                     "algorithmic_bytes_per_launch": per_launch, "kernel_ms": attn_ms,
+                     "launches_per_step": attn_launches},
         "step_hbm_gbs": attn_bytes / (ms * 1e-3) / 1e9,
         "kv_touched": {"mean": float(np.mean(per_head)), "p50": float(np.median(per_head)),
                        "p99": float(np.percentile(per_head, 99)),
                        "group_union": union_rows / (units * T1)},
+        "stages_ms": stages,
         "tree_build": {"ms": build_ms, "gbs": k_bytes / (build_ms * 1e-3) / 1e9},
         "e2e": {"value": ws * w.B * w.Hq / (e2e_ms * 1e-3), "unit": "query-heads/s",
                 "h2d_bytes_per_step": (q.numel() + k_new.numel() + v_new.numel()) * es,

@@ -23,7 +23,10 @@ namespace zha {
 
 namespace tc {
 
-constexpr int kStages = 6;
+#ifndef ZHA_ATTN_STAGES
+#define ZHA_ATTN_STAGES 4
+#endif
+constexpr int kStages = ZHA_ATTN_STAGES;         // 32 KiB each; 4..6 keep HBM saturated
 constexpr int kConsumerWarps = 4;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kBoxBytes = 64 * 128;              // 64 rows x 64 bf16, one swizzled box

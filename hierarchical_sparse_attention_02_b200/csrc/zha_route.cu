@@ -965,7 +965,6 @@ static cudaError_t route_levels(const RouteCall& c) {
     trace_begin(ZHA_TRACE_ROUTE_SELECT, c.stream);
     route_select_warp_kernel<<<grid_for((nqh + kWarpSelWarps - 1) / kWarpSelWarps, 8), kWarpSelWarps * 32, 0,
                                c.stream>>>(se);
-    trace_end(ZHA_TRACE_ROUTE_SELECT, c.stream);
     count_launch();
     e = launch_status("route_select_warp_kernel");
     if (e != cudaSuccess) return e;
@@ -974,6 +973,7 @@ static cudaError_t route_levels(const RouteCall& c) {
       count_launch();
       if (e != cudaSuccess) { note_cuda_error(e, "route_select_cluster_kernel"); return e; }
     }
+    trace_end(ZHA_TRACE_ROUTE_SELECT, c.stream);
   }
   return cudaSuccess;
 }

@@ -56,7 +56,6 @@ __global__ void __launch_bounds__(128) leaf_summarize_tc_kernel(
     int64_t leaf_lo, int64_t nleaf, LevelPtrs out, double scale) {
   using Sm = LeafTcSmem<KT, R>;
   constexpr int NT = Sm::NT;
-  constexpr int kRow = Sm::kRow;
   extern __shared__ __align__(16) unsigned char smem_raw[];
   Sm& sm = *reinterpret_cast<Sm*>(smem_raw);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

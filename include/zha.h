@@ -263,7 +263,7 @@ const char* zha_last_error(void);
 typedef enum zha_trace_kernel {
   ZHA_TRACE_ATTN = 1,        /* the split-KV gather kernel of the sparse / dense attention */
   ZHA_TRACE_ROUTE_SCORE = 2, /* the routing score kernel (every level)                      */
-  ZHA_TRACE_ROUTE_SELECT = 3 /* the routing top-p select kernel (every level)               */
+  ZHA_TRACE_ROUTE_SELECT = 3 /* the routing top-p select kernels (every level; both kinds)  */
 } zha_trace_kernel;
 
 /* Until n launches of kernel `which` have been traced, record start[i] just before and
