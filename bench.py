@@ -287,8 +287,12 @@ def stage_breakdown(lib, step, stream, nb, ms_step):
         n = lib.zha_trace_count(kid)
         lib.zha_trace(kid, None, None, 0)
         a, b = ev[name]
-        out[name] = sum(x.elapsed_time(y) for x, y in zip(a[:n], b[:n])) / nb
-    out["stage_sum"] = sum(out.values())
+        t = [x.elapsed_time(y) for x, y in zip(a[:n], b[:n])]
+        out[name] = sum(t) / nb
+        per = n // nb                 # launches per step, in launch order (top level first)
+        if per > 1:
+            out[name + "_per_launch"] = [round(sum(t[j::per]) / nb, 4) for j in range(per)]
+    out["stage_sum"] = sum(out[k] for k in kinds)
     out["step"] = ms_step
     out["steps"] = nb
     return out

@@ -62,9 +62,12 @@ struct ScoreArgs {
 };
 
 constexpr int kScoreThreads = 128;
+#ifndef ZHA_SCORE_MIN_BLOCKS
+#define ZHA_SCORE_MIN_BLOCKS 5                   // resident CTAs per SM the registers allow
+#endif
 
 template <typename KT>
-__global__ void __launch_bounds__(kScoreThreads) route_score_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads, ZHA_SCORE_MIN_BLOCKS) route_score_kernel(ScoreArgs a) {
   __shared__ __align__(16) double qfs[32][32];
   __shared__ int rank[kScoreThreads][kMaxG];     // per parent slot: rank in each head's list
   __shared__ int pcnt[kMaxG];
@@ -316,12 +319,10 @@ __global__ void __launch_bounds__(256) flat_score_kernel(FlatArgs a) {
 }
 
 // ---------------------------------------------------------------------------
-// top-p select over one level's candidates: exact radix select on the fp64 order key
-// with fixed-point masses (a warp per query head up to kWarpSelMax candidates, a
-// cluster of CTAs per query head above)
+// top-p select over one level's candidates with fixed-point masses; launch_select picks a
+// warp, a CTA or a cluster of CTAs per query head from the level's frontier capacity
 // ---------------------------------------------------------------------------
 
-constexpr int kWarpSelMax = 1024;        // larger frontiers use the cluster kernel
 constexpr int kDigit = 11;
 constexpr int kBuckets = 1 << kDigit;
 
@@ -352,18 +353,144 @@ __device__ __forceinline__ unsigned long long order_key(double s) {
 }
 
 // ---------------------------------------------------------------------------
-// warp select: one warp per query head for frontiers of up to kWarpSelMax candidates
-// (the common case): 8-bit digits, per-warp histograms in shared memory and warp
-// shuffles for every reduction and scan.
+// The select of every level, in four steps per query head:
+//   1. maximum M and minimum of the scores;
+//   2. fixed-point masses E_i = round(2^S exp(s_i - M)), their exact total Z, and a
+//      histogram of (count, mass) over linear buckets of [min, M] (the map from score to
+//      bucket is monotone, so each bucket is an interval of the descending order);
+//   3. the boundary bucket, where the cumulative mass from the top reaches ceil(p Z);
+//      when it holds more than one candidate, an exact radix select on the 64-bit order
+//      key of the score resolves it (digits below the common prefix of its keys);
+//   4. ordered compaction of the kept candidates (ascending position = ascending id).
+// The selected set is the one of the descending (score, then ascending id) order: the
+// linear buckets only replace the first radix passes.
 // ---------------------------------------------------------------------------
 
-constexpr int kWarpSelWarps = 8;
+struct LinBuckets {
+  double M, inv_w;
+  int nb;
+  __device__ __forceinline__ void init(double mx, double mn, int nbuckets) {
+    M = mx;
+    nb = nbuckets;
+    const double r = mx - mn;
+    const double iw = r > 0.0 ? (double)nbuckets / r : 0.0;
+    inv_w = isfinite(iw) ? iw : 0.0;                 // 0: one bucket (the radix resolves it)
+  }
+  // nb - 1 for the highest scores, 0 for the lowest
+  __device__ __forceinline__ int digit(double s) const {
+    if (inv_w == 0.0) return nb - 1;
+    const double x = (M - s) * inv_w;                // >= 0, monotone non-increasing in s
+    return x < (double)(nb - 1) ? nb - 1 - (int)x : 0;
+  }
+};
+
+// The cutoff, as every CTA / lane holds it after step 3.
+struct Cutoff {
+  bool keep_all;
+  int d1;                        // boundary linear bucket
+  int shift;                     // 64: every candidate of bucket d1 is kept
+  unsigned long long pfx;        // key prefix (order_key >> shift) of the tie group
+  unsigned long long need;       // candidates of the tie group kept, in position order
+  unsigned int cnt_t;            // candidates of the tie group
+};
+
+// 0: dropped, 1: kept, 2: in the tie group
+__device__ __forceinline__ int classify(const Cutoff& c, const LinBuckets& lb, double s) {
+  if (c.keep_all) return 1;
+  const int d = lb.digit(s);
+  if (d != c.d1) return d > c.d1 ? 1 : 0;
+  if (c.shift == 64) return 1;
+  const unsigned long long kk = order_key(s) >> c.shift;
+  return kk > c.pfx ? 1 : (kk == c.pfx ? 2 : 0);
+}
+
+__device__ __forceinline__ unsigned long long need_of(unsigned int cnt_b, unsigned long long mass_b,
+                                                      unsigned long long tgt, unsigned long long above) {
+  if (cnt_b <= 1) return 1;
+  const unsigned long long e1 = mass_b / cnt_b;          // equal keys: equal masses
+  unsigned long long need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
+  if (need < 1) need = 1;
+  if (need > cnt_b) need = cnt_b;
+  return need;
+}
+
+__device__ __forceinline__ unsigned long long target_of(double p, unsigned long long Z) {
+  const double tg = ceil(p * (double)Z);
+  unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
+  return tgt > Z ? Z : tgt;
+}
+
+template <typename M>
+__device__ __forceinline__ M lowest_bits(M m, long long r) {   // the r lowest set bits of m
+  M out = 0;
+  while (r > 0 && m) {
+    const M b = m & (~m + 1);
+    out |= b;
+    m ^= b;
+    --r;
+  }
+  return out;
+}
+
+// A boundary bucket of up to kMaxMembers candidates is resolved directly: its members
+// (position, order key, mass) are gathered into a list and one warp walks them in the
+// descending (key, then ascending position) order.  The member at which the cumulative
+// mass from `above` first reaches tgt is the last kept; the cutoff becomes its key (pfx,
+// shift 0), the members sharing that key (cnt_t) and how many of them, in position
+// order, are kept (need).  Larger boundary buckets take the radix refinement.
+constexpr int kMaxMembers = 32;
+
+__device__ __forceinline__ void resolve_members(int m, const int* mpos, const unsigned long long* mkey,
+                                                const unsigned long long* mmass, unsigned long long above,
+                                                unsigned long long tgt, unsigned long long& pfx,
+                                                unsigned long long& need, unsigned int& cnt_t) {
+  const int lane = threadIdx.x & 31;
+  const bool on = lane < m;
+  const int p = on ? mpos[lane] : 0x7fffffff;
+  const unsigned long long k = on ? mkey[lane] : 0ull;
+  const unsigned long long e = on ? mmass[lane] : 0ull;
+  unsigned long long cum = above;                      // mass up to and including this member
+  for (int j = 0; j < m; ++j) {
+    const unsigned long long kj = __shfl_sync(0xffffffffu, k, j);
+    const int pj = __shfl_sync(0xffffffffu, p, j);
+    const unsigned long long ej = __shfl_sync(0xffffffffu, e, j);
+    if (kj > k || (kj == k && pj <= p)) cum += ej;
+  }
+  // the earliest member (in the order) whose cumulative mass reaches tgt
+  const bool reach = on && cum >= tgt;
+  unsigned long long kb = reach ? k : 0ull;
+  bool any = reach;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long x = __shfl_xor_sync(0xffffffffu, kb, o);
+    const bool ax = __shfl_xor_sync(0xffffffffu, any, o);
+    if (ax && (!any || x > kb)) { kb = x; any = true; }
+  }
+  int pb = (reach && k == kb) ? p : 0x7fffffff;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) pb = min(pb, __shfl_xor_sync(0xffffffffu, pb, o));
+  pfx = kb;
+  cnt_t = __popc(__ballot_sync(0xffffffffu, on && k == kb));
+  need = __popc(__ballot_sync(0xffffffffu, on && k == kb && p <= pb));
+}
+
+// ---------------------------------------------------------------------------
+// warp select: one warp per query head: 256 linear buckets, 8-bit radix digits, per-warp
+// histograms in shared memory, warp shuffles for every reduction and scan.
+// ---------------------------------------------------------------------------
+
+constexpr int kWarpSelWarps = 4;
 constexpr int kWDigit = 8;
 constexpr int kWBuckets = 1 << kWDigit;
+constexpr int kWarpCap = 1024;           // candidates a warp holds in shared memory
 
-struct WarpSelSmem {
+struct WarpSelSmem {                     // 4 warps: 62 KiB (dynamic shared memory)
+  double sc[kWarpSelWarps][kWarpCap];
+  int sid[kWarpSelWarps][kWarpCap];
   unsigned int cnt[kWarpSelWarps][kWBuckets];
   unsigned long long mass[kWarpSelWarps][kWBuckets];
+  unsigned long long m_key[kWarpSelWarps][32], m_mass[kWarpSelWarps][32];
+  int m_pos[kWarpSelWarps][32];
 };
 
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
@@ -384,218 +511,287 @@ __device__ __forceinline__ unsigned int warp_excl_scan(unsigned int v, unsigned 
   return x - v;
 }
 
+// The bucket where the cumulative mass from the top bucket, starting at `above`, reaches
+// tgt.  Lane L owns the 8 buckets below kWBuckets - 8L.  Returns the bucket; `above`
+// becomes the mass of the buckets above it.
+__device__ __forceinline__ int warp_boundary(const unsigned long long* hmass, unsigned long long& above,
+                                             unsigned long long tgt) {
+  const int lane = threadIdx.x & 31;
+  constexpr int kPer = kWBuckets / 32;
+  unsigned long long local = 0;
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) local += hmass[kWBuckets - 1 - (lane * kPer + q)];
+  unsigned long long x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  const unsigned long long before = above + x - local;
+  const bool mine = before < tgt && before + local >= tgt;
+  int bstar = 0;
+  unsigned long long above_new = 0;
+  if (mine) {
+    unsigned long long acc = before;
+    for (int q = 0; q < kPer; ++q) {
+      const int bkt = kWBuckets - 1 - (lane * kPer + q);
+      if (acc + hmass[bkt] >= tgt) { bstar = bkt; above_new = acc; break; }
+      acc += hmass[bkt];
+    }
+  }
+  const unsigned int who = __ballot_sync(0xffffffffu, mine);
+  const int src = who ? __ffs(who) - 1 : 0;
+  above = __shfl_sync(0xffffffffu, above_new, src);
+  return __shfl_sync(0xffffffffu, bstar, src);
+}
+
+__device__ __forceinline__ int* level_counts(const SelectArgs& a, int64_t qh) {
+  return a.level_cnt ? a.level_cnt + (qh * a.g.depth + (a.level - 1)) * 2 : nullptr;
+}
+
+// Candidates of head qh at this level, or -1 when its query sees no node of the level
+// (then `writer` records the empty selection).
+__device__ __forceinline__ int head_candidates(const SelectArgs& a, int64_t qh, bool writer) {
+  const RouteGeom& g = a.g;
+  const int64_t t = query_pos(g.q_pos, g.pos_uniform, qh / g.Hq);
+  const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
+  if (a.level > top) {
+    if (writer) {
+      int* lc = level_counts(a, qh);
+      if (lc) { lc[0] = 0; lc[1] = 0; }
+      if (a.level == 1) a.out_cnt[qh] = 0;
+    }
+    return -1;
+  }
+  return a.cand_cnt[qh];
+}
+
+__device__ __forceinline__ unsigned long long mass_of(double s, double M, int shift) {
+  return __double2ull_rn(ldexp(exp(s - M), shift));
+}
+
+// Writes the kept candidate `i` (id ids[i]) at output position pos.
+__device__ __forceinline__ void emit_kept(const SelectArgs& a, int64_t qh, const int* ids, int i,
+                                          unsigned int pos, bool& overflow) {
+  const int id = ids[i];
+  if ((int64_t)pos < a.out_cap) a.out_ids[qh * a.out_stride + pos] = id;
+  else overflow = true;
+  if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
+    a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
+}
+
+// One warp per query head with its scores in shared memory (n <= kWarpCap): read once,
+// every later pass walks shared memory; the compaction goes in rounds of 32 positions.
 __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(SelectArgs a) {
-  __shared__ WarpSelSmem sm;
+  extern __shared__ __align__(16) unsigned char wsel_raw[];
+  WarpSelSmem& sm = *reinterpret_cast<WarpSelSmem*>(wsel_raw);
   const RouteGeom& g = a.g;
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const unsigned int lt = (1u << lane) - 1u;
+  double* sc = sm.sc[wid];
+  int* sid = sm.sid[wid];
   unsigned int* hcnt = sm.cnt[wid];
   unsigned long long* hmass = sm.mass[wid];
   const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
   for (int64_t qh = (int64_t)blockIdx.x * kWarpSelWarps + wid; qh < nqh;
        qh += (int64_t)gridDim.x * kWarpSelWarps) {
-    const int64_t bq = qh / g.Hq;
-    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
-    const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
-    int* lc = a.level_cnt ? a.level_cnt + (qh * g.depth + (a.level - 1)) * 2 : nullptr;
-    if (a.level > top) {
-      if (lane == 0) {
-        if (lc) { lc[0] = 0; lc[1] = 0; }
-        if (a.level == 1) a.out_cnt[qh] = 0;
-      }
+    const int n = head_candidates(a, qh, lane == 0);
+    if (n < 0) continue;
+    if (n > kWarpCap) {                                  // the host picks a larger kernel
+      if (lane == 0) set_status(a.dev_status, ZHA_ERR_CAPACITY);
       continue;
     }
-    const int n = a.cand_cnt[qh];
-    if (n > kWarpSelMax) continue;                      // the cluster kernel takes it
     const double* s = a.cand_score + qh * a.C1;
     const int* ids = a.cand_ids + qh * a.C1;
-    unsigned long long* E = a.cand_mass + qh * a.C1;
-    // 1. maximum and minimum
-    // every pass walks the candidates 8 per lane at a time, loads first (in flight together)
-#define WSEL_BATCH(LOADS, BODY)                                                     \
-    for (int base_ = 0; base_ < n; base_ += 32 * 8) {                               \
-      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
-        const int i = base_ + u_ * 32 + lane;                                       \
-        LOADS                                                                       \
-      }                                                                             \
-      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
-        const int i = base_ + u_ * 32 + lane;                                       \
-        if (i < n) { BODY }                                                         \
-      }                                                                             \
-    }
-    double sv[8];
-    unsigned long long ev[8];
+    // 1. scores and ids into shared memory; maximum and minimum
     double mx = -INFINITY, mn = INFINITY;
-    WSEL_BATCH({ sv[u_] = i < n ? s[i] : 0.0; }, { mx = fmax(mx, sv[u_]); mn = fmin(mn, sv[u_]); })
+#pragma unroll 4
+    for (int i = lane; i < n; i += 32) {
+      const double v = s[i];
+      sc[i] = v;
+      sid[i] = ids[i];
+      mx = fmax(mx, v);
+      mn = fmin(mn, v);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       mx = fmax(mx, shfl_xor_f64(mx, o));
       mn = fmin(mn, shfl_xor_f64(mn, o));
     }
-    // 2. fixed-point masses and their exact total
+    // 2. masses, their total and the linear histogram
+    LinBuckets lb;
+    lb.init(mx, mn, kWBuckets);
+#pragma unroll
+    for (int q = 0; q < kWBuckets / 32; ++q) { hcnt[lane + 32 * q] = 0; hmass[lane + 32 * q] = 0; }
+    __syncwarp();
     unsigned long long z = 0;
-    WSEL_BATCH({ sv[u_] = i < n ? s[i] : 0.0; }, {
-      const unsigned long long e = __double2ull_rn(ldexp(exp(sv[u_] - mx), a.mass_shift));
-      E[i] = e;
+    for (int i = lane; i < n; i += 32) {
+      const double v = sc[i];
+      const unsigned long long e = mass_of(v, mx, a.mass_shift);
       z += e;
-    })
+      const int d = lb.digit(v);
+      atomicAdd(&hcnt[d], 1u);
+      atomicAdd(&hmass[d], e);
+    }
     const unsigned long long Z = warp_sum_u64(z);
     __syncwarp();
-    // 3. cutoff
-    const bool keep_all = a.p >= 1.0 || n == 0;
-    unsigned long long pfx = 0, need = 0;
-    int shift = 0;
-    if (!keep_all) {
-      double tg = ceil(a.p * (double)Z);
-      unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
-      if (tgt > Z) tgt = Z;
-      const unsigned long long kmax = order_key(mx), kmin = order_key(mn);
+    // 3. the cutoff
+    Cutoff c{};
+    c.keep_all = a.p >= 1.0 || n == 0;
+    c.shift = 64;
+    if (!c.keep_all) {
+      const unsigned long long tgt = target_of(a.p, Z);
       unsigned long long above = 0;
-      unsigned int cnt_b = (unsigned int)n;
-      unsigned long long mass_b = Z;
-      if (kmax == kmin) {
-        pfx = kmax;
-      } else {
-        int hi = 63 - __clzll((long long)(kmax ^ kmin));
-        pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
-        while (true) {
-          const int width = (hi + 1) < kWDigit ? (hi + 1) : kWDigit;
-          const int lo = hi + 1 - width;
-#pragma unroll
-          for (int q = 0; q < kWBuckets / 32; ++q) { hcnt[lane + 32 * q] = 0; hmass[lane + 32 * q] = 0; }
-          __syncwarp();
-          WSEL_BATCH({ sv[u_] = i < n ? s[i] : 0.0; ev[u_] = i < n ? E[i] : 0ull; }, {
-            const unsigned long long key = order_key(sv[u_]);
-            if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
-              const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
-              atomicAdd(&hcnt[bkt], 1u);
-              atomicAdd(&hmass[bkt], ev[u_]);
-            }
-          })
-          __syncwarp();
-          // lane L owns the 8 buckets below kWBuckets - 8L (from the top: highest scores)
-          constexpr int kPer = kWBuckets / 32;
-          unsigned long long local = 0;
-#pragma unroll
-          for (int q = 0; q < kPer; ++q) local += hmass[kWBuckets - 1 - (lane * kPer + q)];
-          unsigned long long x = local;
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
-            if (lane >= o) x += y;
+      c.d1 = warp_boundary(hmass, above, tgt);
+      unsigned int cnt_b = hcnt[c.d1];
+      unsigned long long mass_b = hmass[c.d1];
+      __syncwarp();
+      if (cnt_b > 1 && cnt_b <= kMaxMembers) {
+        // gather the boundary bucket's members and walk them in order
+        unsigned int m = 0;
+        for (int b0 = 0; b0 < n; b0 += 32) {
+          const int i = b0 + lane;
+          const bool mem = i < n && lb.digit(sc[i]) == c.d1;
+          const unsigned int mb = __ballot_sync(0xffffffffu, mem);
+          if (mem) {
+            const unsigned int slot = m + __popc(mb & lt);
+            sm.m_pos[wid][slot] = i;
+            sm.m_key[wid][slot] = order_key(sc[i]);
+            sm.m_mass[wid][slot] = mass_of(sc[i], mx, a.mass_shift);
           }
-          const unsigned long long before = above + x - local;
-          const bool mine = before < tgt && before + local >= tgt;
-          int bstar = 0;
-          unsigned long long above_new = 0;
-          if (mine) {
-            unsigned long long acc = before;
-            for (int q = 0; q < kPer; ++q) {
-              const int bkt = kWBuckets - 1 - (lane * kPer + q);
-              if (acc + hmass[bkt] >= tgt) { bstar = bkt; above_new = acc; break; }
-              acc += hmass[bkt];
-            }
+          m += __popc(mb);
+        }
+        __syncwarp();
+        c.shift = 0;
+        resolve_members((int)m, sm.m_pos[wid], sm.m_key[wid], sm.m_mass[wid], above, tgt, c.pfx, c.need,
+                        c.cnt_t);
+        __syncwarp();
+      } else if (cnt_b > 1) {
+        // key range of the boundary bucket, then radix digits of the order key within it
+        unsigned long long kmx = 0, kmn = ~0ull;
+        for (int i = lane; i < n; i += 32) {
+          const double v = sc[i];
+          if (lb.digit(v) == c.d1) {
+            const unsigned long long k = order_key(v);
+            kmx = k > kmx ? k : kmx;
+            kmn = k < kmn ? k : kmn;
           }
-          const unsigned int who = __ballot_sync(0xffffffffu, mine);
-          const int src = who ? __ffs(who) - 1 : 0;
-          bstar = __shfl_sync(0xffffffffu, bstar, src);
-          above = __shfl_sync(0xffffffffu, above_new, src);
-          cnt_b = hcnt[bstar];
-          mass_b = hmass[bstar];
-          pfx = (pfx << width) | (unsigned long long)bstar;
-          __syncwarp();
-          if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
-          hi = lo - 1;
         }
-      }
-      if (cnt_b <= 1) {
-        need = 1;
-      } else {
-        const unsigned long long e1 = mass_b / cnt_b;
-        need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
-        if (need < 1) need = 1;
-        if (need > cnt_b) need = cnt_b;
-      }
-    }
-    // 4. ordered compaction: lane L owns the contiguous candidates [L*per, (L+1)*per)
-    const int per = (n + 31) / 32;
-    const int i0 = lane * per, i1 = (i0 + per < n) ? i0 + per : n;
-    unsigned int nt = 0;
-    if (!keep_all) {
-#pragma unroll 8
-      for (int i = i0; i < i1; ++i) nt += (order_key(s[i]) >> shift) == pfx;
-    }
-    unsigned int tie_total;
-    unsigned int tie_rank = warp_excl_scan(nt, &tie_total);
-    unsigned int nk = 0;
-    {
-      unsigned int tr = tie_rank;
-#pragma unroll 8
-      for (int i = i0; i < i1; ++i) {
-        bool keep = keep_all;
-        if (!keep_all) {
-          const unsigned long long kk = order_key(s[i]) >> shift;
-          keep = kk > pfx || (kk == pfx && tr++ < need);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long x = __shfl_xor_sync(0xffffffffu, kmx, o);
+          const unsigned long long y = __shfl_xor_sync(0xffffffffu, kmn, o);
+          kmx = x > kmx ? x : kmx;
+          kmn = y < kmn ? y : kmn;
         }
-        nk += keep;
+        if (kmx == kmn) {
+          c.pfx = kmx;
+          c.shift = 0;
+        } else {
+          int hi = 63 - __clzll((long long)(kmx ^ kmn));
+          unsigned long long pfx = (hi == 63) ? 0ull : (kmx >> (hi + 1));
+          while (true) {
+            const int width = (hi + 1) < kWDigit ? (hi + 1) : kWDigit;
+            const int lo = hi + 1 - width;
+#pragma unroll
+            for (int q = 0; q < kWBuckets / 32; ++q) { hcnt[lane + 32 * q] = 0; hmass[lane + 32 * q] = 0; }
+            __syncwarp();
+            for (int i = lane; i < n; i += 32) {
+              const double v = sc[i];
+              if (lb.digit(v) != c.d1) continue;
+              const unsigned long long key = order_key(v);
+              if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+                const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+                atomicAdd(&hcnt[bkt], 1u);
+                atomicAdd(&hmass[bkt], mass_of(v, mx, a.mass_shift));
+              }
+            }
+            __syncwarp();
+            const int bstar = warp_boundary(hmass, above, tgt);
+            cnt_b = hcnt[bstar];
+            mass_b = hmass[bstar];
+            pfx = (pfx << width) | (unsigned long long)bstar;
+            __syncwarp();
+            if (cnt_b <= 1 || lo == 0) { c.shift = lo; break; }
+            hi = lo - 1;
+          }
+          c.pfx = pfx;
+        }
+        c.cnt_t = cnt_b;
+        c.need = need_of(cnt_b, mass_b, tgt, above);
       }
     }
-    unsigned int written;
-    unsigned int pos = warp_excl_scan(nk, &written);
-    int* outp = a.out_ids + qh * a.out_stride;
+    // 4. ordered compaction, 32 positions per round
+    const bool partial = c.shift != 64 && c.cnt_t > 1 && c.need < c.cnt_t;
+    unsigned int written = 0, ties = 0;
     bool overflow = false;
-#pragma unroll 4
-    for (int i = i0; i < i1; ++i) {
-      bool keep = keep_all;
-      if (!keep_all) {
-        const unsigned long long kk = order_key(s[i]) >> shift;
-        keep = kk > pfx || (kk == pfx && tie_rank++ < need);
-      }
-      if (keep) {
-        const int id = ids[i];
-        if ((int64_t)pos < a.out_cap) outp[pos] = id;
-        else overflow = true;
-        if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
-          a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
-        ++pos;
-      }
+    for (int b0 = 0; b0 < n; b0 += 32) {
+      const int i = b0 + lane;
+      const int k = i < n ? classify(c, lb, sc[i]) : 0;
+      const unsigned int tb = __ballot_sync(0xffffffffu, k == 2);
+      const bool keep = k == 1 || (k == 2 && (!partial || ties + __popc(tb & lt) < c.need));
+      ties += __popc(tb);
+      const unsigned int kb = __ballot_sync(0xffffffffu, keep);
+      if (keep) emit_kept(a, qh, sid, i, written + __popc(kb & lt), overflow);
+      written += __popc(kb);
     }
     if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
     if (lane == 0) {
       a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
+      int* lc = level_counts(a, qh);
       if (lc) { lc[0] = n; lc[1] = (int)written; }
     }
     __syncwarp();
   }
-#undef WSEL_BATCH
 }
 
 // ---------------------------------------------------------------------------
-// cluster select: one thread-block cluster (1..8 CTAs of kClThreads) per query head, for
-// frontiers above kWarpSelMax.  Each CTA takes a contiguous slice of the candidates; the
-// cluster's rank-0 CTA sums the per-CTA maxima, totals and digit histograms through
-// distributed shared memory and publishes every decision back into each CTA, so all CTAs
-// take identical decisions.  Cluster barriers are hardware barriers (no spin loops).
+// cluster select: one thread-block cluster (1..8 CTAs of T threads) per query head.  The
+// cluster's rank-0 CTA sums the per-CTA maxima, totals and histograms through distributed
+// shared memory and publishes every decision back into each CTA, so all CTAs take
+// identical decisions.  Cluster barriers are hardware barriers (no spin loops).  The
+// streaming kernel re-reads the scores (and the masses it stored) in every pass, for
+// frontiers beyond what the register-resident kernel holds.
 // ---------------------------------------------------------------------------
 
-constexpr int kClThreads = 512;
 constexpr int kClMaxCta = 8;
 
+template <int T>
 struct ClSmem {
   unsigned int cnt[kBuckets];
   unsigned long long mass[kBuckets];
-  unsigned long long wsum[kClThreads / 32];
-  double wd[kClThreads / 32];
-  unsigned int wcnt[kClThreads / 32];
+  unsigned long long wsum[T / 32];
+  unsigned long long wu[T / 32];
+  double wd[T / 32];
+  unsigned int wcnt[T / 32];
+  unsigned int wdef[T / 32], wtie[T / 32], wkeep[T / 32];
   // per-CTA contributions, written into the rank-0 CTA by every rank
   unsigned long long slot_kmax[kClMaxCta], slot_kmin[kClMaxCta], slot_z[kClMaxCta];
   unsigned int slot_tie[kClMaxCta], slot_keep[kClMaxCta];
+  // boundary-bucket members, gathered into rank 0
+  unsigned int m_cnt;
+  int m_pos[kMaxMembers];
+  unsigned long long m_key[kMaxMembers], m_mass[kMaxMembers];
   // decisions published by rank 0
-  unsigned long long d_above, d_mass_b;
-  unsigned int d_cnt_b;
+  unsigned long long d_above, d_mass_b, d_pfx, d_need;
+  unsigned int d_cnt_b, d_cnt_t;
   int d_bstar;
 };
 
-__device__ __forceinline__ double cl_block_max(double v, ClSmem& sm) {
+// Barrier and shared-memory view of rank r: across the cluster (CL) or within the CTA.
+template <bool CL>
+__device__ __forceinline__ void csync() {
+  if constexpr (CL) cooperative_groups::this_cluster().sync();
+  else __syncthreads();
+}
+template <bool CL, typename S>
+__device__ __forceinline__ S* peer(S& sm, int r) {
+  if constexpr (CL) return cooperative_groups::this_cluster().map_shared_rank(&sm, r);
+  else return &sm;
+}
+
+template <int T>
+__device__ __forceinline__ double cl_block_max(double v, ClSmem<T>& sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmax(v, shfl_xor_f64(v, o));
@@ -603,11 +799,28 @@ __device__ __forceinline__ double cl_block_max(double v, ClSmem& sm) {
   if (lane == 0) sm.wd[warp] = v;
   __syncthreads();
   double r = sm.wd[0];
-  for (int i = 1; i < kClThreads / 32; ++i) r = fmax(r, sm.wd[i]);
+  for (int i = 1; i < T / 32; ++i) r = fmax(r, sm.wd[i]);
   return r;
 }
 
-__device__ __forceinline__ unsigned long long cl_block_sum(unsigned long long v, ClSmem& sm) {
+template <int T>
+__device__ __forceinline__ unsigned long long cl_block_max_u64(unsigned long long v, ClSmem<T>& sm) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long x = __shfl_xor_sync(0xffffffffu, v, o);
+    v = x > v ? x : v;
+  }
+  __syncthreads();
+  if (lane == 0) sm.wu[warp] = v;
+  __syncthreads();
+  unsigned long long r = sm.wu[0];
+  for (int i = 1; i < T / 32; ++i) r = sm.wu[i] > r ? sm.wu[i] : r;
+  return r;
+}
+
+template <int T>
+__device__ __forceinline__ unsigned long long cl_block_sum(unsigned long long v, ClSmem<T>& sm) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -615,11 +828,12 @@ __device__ __forceinline__ unsigned long long cl_block_sum(unsigned long long v,
   if (lane == 0) sm.wsum[warp] = v;
   __syncthreads();
   unsigned long long r = 0;
-  for (int i = 0; i < kClThreads / 32; ++i) r += sm.wsum[i];
+  for (int i = 0; i < T / 32; ++i) r += sm.wsum[i];
   return r;
 }
 
-__device__ __forceinline__ unsigned int cl_excl_scan(unsigned int v, ClSmem& sm, unsigned int* total) {
+template <int T>
+__device__ __forceinline__ unsigned int cl_excl_scan(unsigned int v, ClSmem<T>& sm, unsigned int* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   unsigned int x = v;
 #pragma unroll
@@ -631,7 +845,7 @@ __device__ __forceinline__ unsigned int cl_excl_scan(unsigned int v, ClSmem& sm,
   if (lane == 31) sm.wcnt[warp] = x;
   __syncthreads();
   unsigned int before = 0, all = 0;
-  for (int i = 0; i < kClThreads / 32; ++i) {
+  for (int i = 0; i < T / 32; ++i) {
     if (i < warp) before += sm.wcnt[i];
     all += sm.wcnt[i];
   }
@@ -639,41 +853,125 @@ __device__ __forceinline__ unsigned int cl_excl_scan(unsigned int v, ClSmem& sm,
   return before + x - v;
 }
 
-__global__ void __launch_bounds__(kClThreads) route_select_cluster_kernel(SelectArgs a) {
-  __shared__ ClSmem sm;
+// Cluster-wide boundary of the histograms every CTA has just filled: rank 0 sums them in
+// rank order, finds the bucket where the cumulative mass from the top (starting at
+// `above`) reaches tgt and publishes (bucket, mass above it, its count and mass) to every
+// CTA.  Contains the two cluster barriers around the decision.
+template <int T, bool CL>
+__device__ __forceinline__ int cl_boundary(ClSmem<T>& sm, int CS, int cr, unsigned long long& above,
+                                           unsigned long long tgt, unsigned int& cnt_b,
+                                           unsigned long long& mass_b) {
+  const int tid = threadIdx.x;
+  csync<CL>();                                        // every CTA's histogram is complete
+  if (cr == 0) {
+    constexpr int kPer = kBuckets / T;
+    unsigned long long bm[kPer];
+    unsigned int bc[kPer];
+    unsigned long long local = 0;
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const int bkt = kBuckets - 1 - (tid * kPer + q);
+      unsigned long long m2 = 0;
+      unsigned int c2 = 0;
+      for (int r = 0; r < CS; ++r) {
+        ClSmem<T>* o = peer<CL>(sm, r);
+        m2 += o->mass[bkt];
+        c2 += o->cnt[bkt];
+      }
+      bm[q] = m2;
+      bc[q] = c2;
+      local += m2;
+    }
+    unsigned long long x = local;
+    const int lane = tid & 31, warp = tid >> 5;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if (lane >= o) x += y;
+    }
+    if (lane == 31) sm.wsum[warp] = x;
+    __syncthreads();
+    unsigned long long before = above;
+    for (int i = 0; i < warp; ++i) before += sm.wsum[i];
+    before += x - local;
+    if (before < tgt && before + local >= tgt) {
+      unsigned long long acc = before;
+      for (int q = 0; q < kPer; ++q) {
+        if (acc + bm[q] >= tgt) {
+          for (int r = 0; r < CS; ++r) {
+            ClSmem<T>* o = peer<CL>(sm, r);
+            o->d_bstar = kBuckets - 1 - (tid * kPer + q);
+            o->d_above = acc;
+            o->d_cnt_b = bc[q];
+            o->d_mass_b = bm[q];
+          }
+          break;
+        }
+        acc += bm[q];
+      }
+    }
+  }
+  csync<CL>();                                           // decision published; histograms free
+  above = sm.d_above;
+  cnt_b = sm.d_cnt_b;
+  mass_b = sm.d_mass_b;
+  return sm.d_bstar;
+}
+
+template <int T>
+__device__ __forceinline__ void cl_clear(ClSmem<T>& sm) {
+  for (int i = threadIdx.x; i < kBuckets; i += T) { sm.cnt[i] = 0; sm.mass[i] = 0; }
+  __syncthreads();
+}
+
+template <int T>
+__global__ void __launch_bounds__(T, 1) route_select_stream_kernel(SelectArgs a) {
+  constexpr bool CLK = true;
+  __shared__ ClSmem<T> sm;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int CS = (int)cluster.num_blocks();
   const int cr = (int)cluster.block_rank();
-  ClSmem* lead = cluster.map_shared_rank(&sm, 0);
+  ClSmem<T>* lead = cluster.map_shared_rank(&sm, 0);
   const RouteGeom& g = a.g;
   const int tid = threadIdx.x;
   const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
   const int64_t nclusters = gridDim.x / CS;
   for (int64_t qh = blockIdx.x / CS; qh < nqh; qh += nclusters) {
-    const int64_t bq = qh / g.Hq;
-    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
-    const int top = !pos_ok(g, t) ? 0 : a.flat ? (visible_nodes(t, kLeaf) >= 1 ? 1 : 0) : top_level(g, t);
-    if (a.level > top) continue;                         // the warp kernel writes the counts
-    const int n = a.cand_cnt[qh];
-    if (n <= kWarpSelMax) continue;                      // the warp kernel takes it
-    int* lc = a.level_cnt ? a.level_cnt + (qh * g.depth + (a.level - 1)) * 2 : nullptr;
+    const int n = head_candidates(a, qh, cr == 0 && tid == 0);
+    if (n < 0) continue;                                 // uniform over the cluster
+    int* lc = level_counts(a, qh);
     const double* s = a.cand_score + qh * a.C1;
     const int* ids = a.cand_ids + qh * a.C1;
     unsigned long long* E = a.cand_mass + qh * a.C1;
     const int chunk = (n + CS - 1) / CS;
     const int r0 = cr * chunk < n ? cr * chunk : n;
     const int r1 = r0 + chunk < n ? r0 + chunk : n;
+    // every pass walks the CTA's slice 8 candidates per thread at a time, loads first
+#define CL_BATCH(LOADS, BODY)                                                       \
+    for (int base_ = r0; base_ < r1; base_ += T * 8) {                              \
+      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
+        const int i = base_ + u_ * T + tid;                                         \
+        LOADS                                                                       \
+      }                                                                             \
+      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
+        const int i = base_ + u_ * T + tid;                                         \
+        if (i < r1) { BODY }                                                        \
+      }                                                                             \
+    }
+    double sv[8];
+    unsigned long long ev[8];
 
     // 1. maximum and minimum over the cluster
     double mx = -INFINITY, mn = INFINITY;
-    for (int i = r0 + tid; i < r1; i += kClThreads) { const double v = s[i]; mx = fmax(mx, v); mn = fmin(mn, v); }
+    CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; }, { mx = fmax(mx, sv[u_]); mn = fmin(mn, sv[u_]); })
     mx = cl_block_max(mx, sm);
     mn = -cl_block_max(-mn, sm);
     if (tid == 0) {
       lead->slot_kmax[cr] = r1 > r0 ? order_key(mx) : 0ull;
       lead->slot_kmin[cr] = r1 > r0 ? order_key(mn) : ~0ull;
     }
+    cl_clear(sm);
     cluster.sync();
     unsigned long long kmax = 0, kmin = ~0ull;
     for (int r = 0; r < CS; ++r) {
@@ -682,146 +980,122 @@ __global__ void __launch_bounds__(kClThreads) route_select_cluster_kernel(Select
       kmin = y < kmin ? y : kmin;
     }
     // back from the order key to the score
-    const unsigned long long mb = (kmax >> 63) ? (kmax & 0x7fffffffffffffffull) : ~kmax;
-    const double M = __longlong_as_double((long long)mb);
-    // 2. fixed-point masses and their exact total
+    const double M = __longlong_as_double((long long)((kmax >> 63) ? (kmax & 0x7fffffffffffffffull) : ~kmax));
+    const double Mn = __longlong_as_double((long long)((kmin >> 63) ? (kmin & 0x7fffffffffffffffull) : ~kmin));
+    // 2. masses, their total and the linear histogram
+    LinBuckets lb;
+    lb.init(M, Mn, kBuckets);
     unsigned long long z = 0;
-    for (int i = r0 + tid; i < r1; i += kClThreads) {
-      const unsigned long long e = __double2ull_rn(ldexp(exp(s[i] - M), a.mass_shift));
+    CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; }, {
+      const unsigned long long e = __double2ull_rn(ldexp(exp(sv[u_] - M), a.mass_shift));
       E[i] = e;
       z += e;
-    }
+      const int d = lb.digit(sv[u_]);
+      atomicAdd(&sm.cnt[d], 1u);
+      atomicAdd(&sm.mass[d], e);
+    })
     z = cl_block_sum(z, sm);
     if (tid == 0) lead->slot_z[cr] = z;
     cluster.sync();
     unsigned long long Z = 0;
     for (int r = 0; r < CS; ++r) Z += lead->slot_z[r];
 
-    // 3. cutoff, with identical decisions in every CTA
-    const bool keep_all = a.p >= 1.0;
-    unsigned long long pfx = 0, need = 0;
-    int shift = 0;
-    if (!keep_all) {
-      double tg = ceil(a.p * (double)Z);
-      unsigned long long tgt = tg < 1.0 ? 1ull : (unsigned long long)tg;
-      if (tgt > Z) tgt = Z;
-      unsigned long long above = 0, mass_b = Z;
-      unsigned int cnt_b = (unsigned int)n;
-      if (kmax == kmin) {
-        pfx = kmax;
-      } else {
-        int hi = 63 - __clzll((long long)(kmax ^ kmin));
-        pfx = (hi == 63) ? 0ull : (kmax >> (hi + 1));
-        while (true) {
-          const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
-          const int lo = hi + 1 - width;
-          for (int i = tid; i < kBuckets; i += kClThreads) { sm.cnt[i] = 0; sm.mass[i] = 0; }
-          __syncthreads();
-          for (int i = r0 + tid; i < r1; i += kClThreads) {
-            const unsigned long long key = order_key(s[i]);
-            if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
-              const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
-              atomicAdd(&sm.cnt[bkt], 1u);
-              atomicAdd(&sm.mass[bkt], E[i]);
-            }
+    // 3. the cutoff, with identical decisions in every CTA
+    Cutoff c{};
+    c.keep_all = a.p >= 1.0 || n == 0;
+    c.shift = 64;
+    if (!c.keep_all) {
+      const unsigned long long tgt = target_of(a.p, Z);
+      unsigned long long above = 0, mass_b = 0;
+      unsigned int cnt_b = 0;
+      c.d1 = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
+      if (cnt_b > 1) {
+        // key range of the boundary bucket over the cluster
+        unsigned long long kmx = 0, kmn = ~0ull;
+        CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; }, {
+          if (lb.digit(sv[u_]) == c.d1) {
+            const unsigned long long k = order_key(sv[u_]);
+            kmx = k > kmx ? k : kmx;
+            kmn = k < kmn ? k : kmn;
           }
-          cluster.sync();                                // every CTA's histogram is complete
-          if (cr == 0) {
-            // sum the CTAs' histograms (rank order) and find the boundary bucket
-            constexpr int kPer = kBuckets / kClThreads;
-            unsigned long long bm[kPer];
-            unsigned int bc[kPer];
-            unsigned long long local = 0;
-#pragma unroll
-            for (int q = 0; q < kPer; ++q) {
-              const int bkt = kBuckets - 1 - (tid * kPer + q);
-              unsigned long long m2 = 0;
-              unsigned int c2 = 0;
-              for (int r = 0; r < CS; ++r) {
-                ClSmem* o = cluster.map_shared_rank(&sm, r);
-                m2 += o->mass[bkt];
-                c2 += o->cnt[bkt];
-              }
-              bm[q] = m2;
-              bc[q] = c2;
-              local += m2;
-            }
-            unsigned long long x = local;
-            const int lane = tid & 31, warp = tid >> 5;
-#pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-              const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
-              if (lane >= o) x += y;
-            }
-            if (lane == 31) sm.wsum[warp] = x;
-            __syncthreads();
-            unsigned long long before = above;
-            for (int i = 0; i < warp; ++i) before += sm.wsum[i];
-            before += x - local;
-            if (before < tgt && before + local >= tgt) {
-              unsigned long long acc = before;
-              for (int q = 0; q < kPer; ++q) {
-                if (acc + bm[q] >= tgt) {
-                  for (int r = 0; r < CS; ++r) {
-                    ClSmem* o = cluster.map_shared_rank(&sm, r);
-                    o->d_bstar = kBuckets - 1 - (tid * kPer + q);
-                    o->d_above = acc;
-                    o->d_cnt_b = bc[q];
-                    o->d_mass_b = bm[q];
-                  }
-                  break;
-                }
-                acc += bm[q];
-              }
-            }
-          }
-          cluster.sync();                                // decision published; histograms free
-          const int bstar = sm.d_bstar;
-          above = sm.d_above;
-          cnt_b = sm.d_cnt_b;
-          mass_b = sm.d_mass_b;
-          pfx = (pfx << width) | (unsigned long long)bstar;
-          if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
-          hi = lo - 1;
+        })
+        kmx = cl_block_max_u64(kmx, sm);
+        kmn = ~cl_block_max_u64(~kmn, sm);
+        if (tid == 0) { lead->slot_kmax[cr] = kmx; lead->slot_kmin[cr] = kmn; }
+        cl_clear(sm);
+        cluster.sync();
+        kmx = 0;
+        kmn = ~0ull;
+        for (int r = 0; r < CS; ++r) {
+          const unsigned long long x = lead->slot_kmax[r], y = lead->slot_kmin[r];
+          kmx = x > kmx ? x : kmx;
+          kmn = y < kmn ? y : kmn;
         }
-      }
-      if (cnt_b <= 1) {
-        need = 1;
-      } else {
-        const unsigned long long e1 = mass_b / cnt_b;
-        need = e1 == 0 ? cnt_b : (tgt - above + e1 - 1) / e1;
-        if (need < 1) need = 1;
-        if (need > cnt_b) need = cnt_b;
+        if (kmx == kmn) {
+          c.pfx = kmx;
+          c.shift = 0;
+        } else {
+          int hi = 63 - __clzll((long long)(kmx ^ kmn));
+          unsigned long long pfx = (hi == 63) ? 0ull : (kmx >> (hi + 1));
+          while (true) {
+            const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
+            const int lo = hi + 1 - width;
+            CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; ev[u_] = i < r1 ? E[i] : 0ull; }, {
+              if (lb.digit(sv[u_]) == c.d1) {
+                const unsigned long long key = order_key(sv[u_]);
+                if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+                  const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+                  atomicAdd(&sm.cnt[bkt], 1u);
+                  atomicAdd(&sm.mass[bkt], ev[u_]);
+                }
+              }
+            })
+            const int bstar = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
+            pfx = (pfx << width) | (unsigned long long)bstar;
+            if (cnt_b <= 1 || lo == 0) { c.shift = lo; break; }
+            cl_clear(sm);                                // rank 0 is done reading (cl_boundary)
+            hi = lo - 1;
+          }
+          c.pfx = pfx;
+        }
+        c.cnt_t = cnt_b;
+        c.need = need_of(cnt_b, mass_b, tgt, above);
       }
     }
 
     // 4. ordered compaction: thread t of CTA r owns a contiguous piece of the CTA's slice
+    //    (flags of its first 64 candidates kept as bit masks)
     const int len = r1 - r0;
-    const int per = (len + kClThreads - 1) / kClThreads;
+    const int per = (len + T - 1) / T;
     const int i0 = r0 + tid * per < r1 ? r0 + tid * per : r1;
     const int i1 = i0 + per < r1 ? i0 + per : r1;
-    unsigned int nt = 0;
-    if (!keep_all)
-      for (int i = i0; i < i1; ++i) nt += (order_key(s[i]) >> shift) == pfx;
-    unsigned int tie_cta;
-    unsigned int tie_rank = cl_excl_scan(nt, sm, &tie_cta);
-    if (tid == 0) lead->slot_tie[cr] = tie_cta;
-    cluster.sync();
-    for (int r = 0; r < cr; ++r) tie_rank += lead->slot_tie[r];
-    unsigned int nk = 0;
-    {
-      unsigned int tr = tie_rank;
-      for (int i = i0; i < i1; ++i) {
-        bool keep = keep_all;
-        if (!keep_all) {
-          const unsigned long long kk = order_key(s[i]) >> shift;
-          keep = kk > pfx || (kk == pfx && tr++ < need);
-        }
-        nk += keep;
+    unsigned long long defm = 0, tiem = 0;
+    unsigned int ndef = 0, ntie = 0;
+#pragma unroll 8
+    for (int i = i0; i < i1; ++i) {
+      const int k = classify(c, lb, s[i]);
+      const int j = i - i0;
+      ndef += k == 1;
+      ntie += k == 2;
+      if (j < 64) {
+        defm |= (unsigned long long)(k == 1) << j;
+        tiem |= (unsigned long long)(k == 2) << j;
       }
     }
+    const bool partial = c.shift != 64 && c.cnt_t > 1 && c.need < c.cnt_t;
+    long long take = ntie;                               // ties this thread keeps
+    unsigned int tie_before = 0;
+    if (partial) {
+      unsigned int tie_cta;
+      tie_before = cl_excl_scan(ntie, sm, &tie_cta);
+      if (tid == 0) lead->slot_tie[cr] = tie_cta;
+      cluster.sync();
+      for (int r = 0; r < cr; ++r) tie_before += lead->slot_tie[r];
+      take = (long long)c.need - (long long)tie_before;
+      take = take < 0 ? 0 : (take > (long long)ntie ? (long long)ntie : take);
+    }
     unsigned int keep_cta;
-    unsigned int pos = cl_excl_scan(nk, sm, &keep_cta);
+    unsigned int pos = cl_excl_scan(ndef + (unsigned int)take, sm, &keep_cta);
     if (tid == 0) lead->slot_keep[cr] = keep_cta;
     cluster.sync();
     unsigned int written = 0;
@@ -832,19 +1106,26 @@ __global__ void __launch_bounds__(kClThreads) route_select_cluster_kernel(Select
     }
     int* outp = a.out_ids + qh * a.out_stride;
     bool overflow = false;
-    for (int i = i0; i < i1; ++i) {
-      bool keep = keep_all;
-      if (!keep_all) {
-        const unsigned long long kk = order_key(s[i]) >> shift;
-        keep = kk > pfx || (kk == pfx && tie_rank++ < need);
+    auto emit = [&](int i) {
+      const int id = ids[i];
+      if ((int64_t)pos < a.out_cap) outp[pos] = id;
+      else overflow = true;
+      if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
+        a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
+      ++pos;
+    };
+    if (per <= 64) {
+      unsigned long long keepm = defm | lowest_bits(tiem, take);
+      while (keepm) {
+        const int j = __ffsll((long long)keepm) - 1;
+        keepm &= keepm - 1;
+        emit(i0 + j);
       }
-      if (keep) {
-        const int id = ids[i];
-        if ((int64_t)pos < a.out_cap) outp[pos] = id;
-        else overflow = true;
-        if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
-          a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
-        ++pos;
+    } else {
+      long long left = take;
+      for (int i = i0; i < i1; ++i) {
+        const int k = classify(c, lb, s[i]);
+        if (k == 1 || (k == 2 && left-- > 0)) emit(i);
       }
     }
     if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
@@ -854,26 +1135,298 @@ __global__ void __launch_bounds__(kClThreads) route_select_cluster_kernel(Select
     }
     cluster.sync();                                      // slots and smem reused by the next head
   }
+#undef CL_BATCH
 }
 
-static cudaError_t launch_select_cluster(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
-  int cs = (int)((ncap + 8191) / 8192);
-  cs = cs < 1 ? 1 : (cs > kClMaxCta ? kClMaxCta : (cs > 4 ? 8 : (cs > 2 ? 4 : cs)));
-  int64_t clusters = nqh < (2 * 148) / cs ? nqh : (2 * 148) / cs;
-  if (clusters < 1) clusters = 1;
+// Shared-memory-resident cluster select: CTA r of the cluster holds the contiguous slice
+// [r*CAP, r*CAP + CAP) of the candidates' scores in (dynamic) shared memory, read once;
+// every later pass walks shared memory.  The compaction gives warp w of each CTA a
+// contiguous chunk of the slice, counted first, then written in rounds of 32 positions.
+// n <= CS*CAP.
+template <int T, int CAP, bool CL>
+__global__ void __launch_bounds__(T) route_select_block_kernel(SelectArgs a) {
+  constexpr bool CLK = CL;
+  __shared__ ClSmem<T> sm;
+  extern __shared__ __align__(16) double sc[];           // [CAP] scores, then [CAP] ids
+  int CS = 1, cr = 0;
+  if constexpr (CL) {
+    CS = (int)cooperative_groups::this_cluster().num_blocks();
+    cr = (int)cooperative_groups::this_cluster().block_rank();
+  }
+  ClSmem<T>* lead = peer<CL>(sm, 0);
+  const RouteGeom& g = a.g;
+  const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+  constexpr int W = T / 32;
+  const unsigned int lt = (1u << lane) - 1u;
+  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
+  const int64_t nclusters = gridDim.x / CS;
+  int* sid = reinterpret_cast<int*>(sc + CAP);
+  for (int64_t qh = blockIdx.x / CS; qh < nqh; qh += nclusters) {
+    const int n = head_candidates(a, qh, cr == 0 && tid == 0);
+    if (n < 0) continue;                                 // uniform over the cluster
+    if (n > CS * CAP) {                                  // the host sizes the cluster from n_cap
+      if (cr == 0 && tid == 0) set_status(a.dev_status, ZHA_ERR_CAPACITY);
+      continue;
+    }
+    const int r0 = cr * CAP < n ? cr * CAP : n;
+    const int len = (r0 + CAP < n ? r0 + CAP : n) - r0;
+    const double* s = a.cand_score + qh * a.C1 + r0;
+    const int* ids = a.cand_ids + qh * a.C1 + r0;
+
+    // 1. scores into shared memory; maximum and minimum over the cluster
+    double mx = -INFINITY, mn = INFINITY;
+#pragma unroll 4
+    for (int i = tid; i < len; i += T) {
+      const double v = s[i];
+      sc[i] = v;
+      sid[i] = ids[i];
+      mx = fmax(mx, v);
+      mn = fmin(mn, v);
+    }
+    if (tid == 0) sm.m_cnt = 0;
+    mx = cl_block_max(mx, sm);                           // (its barriers also publish sc)
+    mn = -cl_block_max(-mn, sm);
+    if (tid == 0) {
+      lead->slot_kmax[cr] = order_key(mx);
+      lead->slot_kmin[cr] = order_key(mn);
+    }
+    cl_clear(sm);
+    csync<CL>();
+    unsigned long long kmax = 0, kmin = ~0ull;
+    for (int r = 0; r < CS; ++r) {
+      const unsigned long long x = lead->slot_kmax[r], y = lead->slot_kmin[r];
+      kmax = x > kmax ? x : kmax;
+      kmin = y < kmin ? y : kmin;
+    }
+    const double M = __longlong_as_double((long long)((kmax >> 63) ? (kmax & 0x7fffffffffffffffull) : ~kmax));
+    const double Mn = __longlong_as_double((long long)((kmin >> 63) ? (kmin & 0x7fffffffffffffffull) : ~kmin));
+
+    // 2. masses, their total and the linear histogram
+    LinBuckets lb;
+    lb.init(M, Mn, kBuckets);
+    unsigned long long z = 0;
+    for (int i = tid; i < len; i += T) {
+      const double v = sc[i];
+      const unsigned long long e = mass_of(v, M, a.mass_shift);
+      z += e;
+      const int d = lb.digit(v);
+      atomicAdd(&sm.cnt[d], 1u);
+      atomicAdd(&sm.mass[d], e);
+    }
+    z = cl_block_sum(z, sm);
+    if (tid == 0) lead->slot_z[cr] = z;
+    csync<CL>();
+    unsigned long long Z = 0;
+    for (int r = 0; r < CS; ++r) Z += lead->slot_z[r];
+
+    // 3. the cutoff, with identical decisions in every CTA
+    Cutoff c{};
+    c.keep_all = a.p >= 1.0 || n == 0;
+    c.shift = 64;
+    if (!c.keep_all) {
+      const unsigned long long tgt = target_of(a.p, Z);
+      unsigned long long above = 0, mass_b = 0;
+      unsigned int cnt_b = 0;
+      c.d1 = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
+      if (cnt_b > 1 && cnt_b <= kMaxMembers) {
+        // gather the boundary bucket's members into rank 0, which walks them in order
+        for (int i = tid; i < len; i += T) {
+          const double v = sc[i];
+          if (lb.digit(v) == c.d1) {
+            const unsigned int slot = atomicAdd(&lead->m_cnt, 1u);
+            lead->m_pos[slot] = r0 + i;
+            lead->m_key[slot] = order_key(v);
+            lead->m_mass[slot] = mass_of(v, M, a.mass_shift);
+          }
+        }
+        csync<CL>();                                     // every member is in rank 0's list
+        if (cr == 0 && wid == 0) {
+          unsigned long long pfx, need;
+          unsigned int cnt_t;
+          resolve_members((int)sm.m_cnt, sm.m_pos, sm.m_key, sm.m_mass, above, tgt, pfx, need, cnt_t);
+          if (lane < CS) {
+            ClSmem<T>* o = peer<CL>(sm, lane);
+            o->d_pfx = pfx;
+            o->d_need = need;
+            o->d_cnt_t = cnt_t;
+          }
+        }
+        csync<CL>();                                     // decision published
+        c.shift = 0;
+        c.pfx = sm.d_pfx;
+        c.need = sm.d_need;
+        c.cnt_t = sm.d_cnt_t;
+      } else if (cnt_b > 1) {
+        unsigned long long kmx = 0, kmn = ~0ull;
+        for (int i = tid; i < len; i += T) {
+          const double v = sc[i];
+          if (lb.digit(v) == c.d1) {
+            const unsigned long long k = order_key(v);
+            kmx = k > kmx ? k : kmx;
+            kmn = k < kmn ? k : kmn;
+          }
+        }
+        kmx = cl_block_max_u64(kmx, sm);
+        kmn = ~cl_block_max_u64(~kmn, sm);
+        if (tid == 0) { lead->slot_kmax[cr] = kmx; lead->slot_kmin[cr] = kmn; }
+        cl_clear(sm);
+        csync<CL>();
+        kmx = 0;
+        kmn = ~0ull;
+        for (int r = 0; r < CS; ++r) {
+          const unsigned long long x = lead->slot_kmax[r], y = lead->slot_kmin[r];
+          kmx = x > kmx ? x : kmx;
+          kmn = y < kmn ? y : kmn;
+        }
+        if (kmx == kmn) {
+          c.pfx = kmx;
+          c.shift = 0;
+        } else {
+          int hi = 63 - __clzll((long long)(kmx ^ kmn));
+          unsigned long long pfx = (hi == 63) ? 0ull : (kmx >> (hi + 1));
+          while (true) {
+            const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
+            const int lo = hi + 1 - width;
+            for (int i = tid; i < len; i += T) {
+              const double v = sc[i];
+              if (lb.digit(v) != c.d1) continue;
+              const unsigned long long key = order_key(v);
+              if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+                const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+                atomicAdd(&sm.cnt[bkt], 1u);
+                atomicAdd(&sm.mass[bkt], mass_of(v, M, a.mass_shift));
+              }
+            }
+            const int bstar = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
+            pfx = (pfx << width) | (unsigned long long)bstar;
+            if (cnt_b <= 1 || lo == 0) { c.shift = lo; break; }
+            cl_clear(sm);                                // rank 0 is done reading (cl_boundary)
+            hi = lo - 1;
+          }
+          c.pfx = pfx;
+        }
+        c.cnt_t = cnt_b;
+        c.need = need_of(cnt_b, mass_b, tgt, above);
+      }
+    }
+
+    // 4. ordered compaction: warp w owns [c0, c1) of the slice (a multiple of 32 wide)
+    const bool partial = c.shift != 64 && c.cnt_t > 1 && c.need < c.cnt_t;
+    const int C = ((len + W - 1) / W + 31) & ~31;
+    const int c0 = wid * C < len ? wid * C : len;
+    const int c1 = c0 + C < len ? c0 + C : len;
+    unsigned int ndef = 0, ntie = 0;
+    for (int b0 = c0; b0 < c1; b0 += 32) {
+      const int i = b0 + lane;
+      const int k = i < c1 ? classify(c, lb, sc[i]) : 0;
+      ndef += __popc(__ballot_sync(0xffffffffu, k == 1));
+      ntie += __popc(__ballot_sync(0xffffffffu, k == 2));
+    }
+    if (lane == 0) { sm.wdef[wid] = ndef; sm.wtie[wid] = ntie; }
+    __syncthreads();
+    long long take = ntie;                               // ties this warp keeps
+    if (partial) {
+      unsigned int tie_before = 0, tie_cta = 0;
+      for (int w2 = 0; w2 < W; ++w2) {
+        if (w2 < wid) tie_before += sm.wtie[w2];
+        tie_cta += sm.wtie[w2];
+      }
+      if (tid == 0) lead->slot_tie[cr] = tie_cta;
+      csync<CL>();
+      for (int r = 0; r < cr; ++r) tie_before += lead->slot_tie[r];
+      take = (long long)c.need - (long long)tie_before;
+      take = take < 0 ? 0 : (take > (long long)ntie ? (long long)ntie : take);
+    }
+    if (lane == 0) sm.wkeep[wid] = ndef + (unsigned int)take;
+    __syncthreads();
+    unsigned int pos = 0, keep_cta = 0;
+    for (int w2 = 0; w2 < W; ++w2) {
+      if (w2 < wid) pos += sm.wkeep[w2];
+      keep_cta += sm.wkeep[w2];
+    }
+    if (tid == 0) lead->slot_keep[cr] = keep_cta;
+    csync<CL>();
+    unsigned int written = 0;
+    for (int r = 0; r < CS; ++r) {
+      const unsigned int k = lead->slot_keep[r];
+      if (r < cr) pos += k;
+      written += k;
+    }
+    bool overflow = false;
+    unsigned int ties = 0;
+    for (int b0 = c0; b0 < c1; b0 += 32) {
+      const int i = b0 + lane;
+      const int k = i < c1 ? classify(c, lb, sc[i]) : 0;
+      const unsigned int tb = __ballot_sync(0xffffffffu, k == 2);
+      const bool keep = k == 1 || (k == 2 && (long long)(ties + __popc(tb & lt)) < take);
+      ties += __popc(tb);
+      const unsigned int kb = __ballot_sync(0xffffffffu, keep);
+      if (keep) emit_kept(a, qh, sid, i, pos + __popc(kb & lt), overflow);
+      pos += __popc(kb);
+    }
+    if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
+    if (cr == 0 && tid == 0) {
+      a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
+      int* lc = level_counts(a, qh);
+      if (lc) { lc[0] = n; lc[1] = (int)written; }
+    }
+    csync<CL>();                                      // slots, sc and smem reused by the next head
+  }
+}
+
+static int grid_for(int64_t work, int per_sm) {
+  int64_t cap = 148ll * per_sm;
+  return (int)(work < cap ? (work < 1 ? 1 : work) : cap);
+}
+
+template <typename K>
+static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t clusters, int cs, int threads,
+                                  size_t smem, cudaStream_t s) {
+  if (smem > 0) {
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)(clusters * cs), 1, 1);
-  cfg.blockDim = dim3(kClThreads, 1, 1);
-  cfg.dynamicSmemBytes = 0;
-  cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, route_select_cluster_kernel, se);
+  cfg.numAttrs = cs > 1 ? 1 : 0;                       // a CTA per head: no cluster
+  cfg.gridDim = dim3((unsigned)((clusters < 1 ? 1 : clusters) * cs), 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  return cudaLaunchKernelEx(&cfg, kernel, se);
+}
+
+// One select launch for a level whose frontier holds up to ncap candidates per head:
+//   ncap <= 1024    a warp per head (scores in shared memory)
+//   ncap <= 4096    a CTA of 256 threads per head (48 KiB of scores and ids)
+//   ncap <= 65536   a cluster of 2 / 4 / 8 CTAs of 512 threads per head (96 KiB of scores and ids each)
+//   above           a cluster of 8 CTAs of 512 threads streaming the scores from memory
+static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
+  if (ncap <= kWarpCap) {
+    const size_t smem = sizeof(WarpSelSmem);
+    cudaError_t e = cudaFuncSetAttribute(route_select_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    route_select_warp_kernel<<<grid_for((nqh + kWarpSelWarps - 1) / kWarpSelWarps, 3), kWarpSelWarps * 32, smem,
+                               s>>>(se);
+    return cudaGetLastError();
+  }
+  if (ncap <= 4096)
+    return launch_cluster(route_select_block_kernel<256, 4096, false>, se, nqh < 148 * 3 ? nqh : 148 * 3, 1, 256,
+                          4096 * (sizeof(double) + sizeof(int)), s);
+  if (ncap <= 8 * 8192) {
+    const int cs = ncap <= 2 * 8192 ? 2 : (ncap <= 4 * 8192 ? 4 : 8);
+    const int64_t per = 148 / cs;
+    return launch_cluster(route_select_block_kernel<512, 8192, true>, se, nqh < per ? nqh : per, cs, 512,
+                          8192 * (sizeof(double) + sizeof(int)), s);
+  }
+  const int64_t per = (2 * 148) / kClMaxCta;
+  return launch_cluster(route_select_stream_kernel<512>, se, nqh < per ? nqh : per, kClMaxCta, 512, 0, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -898,10 +1451,6 @@ static int mass_shift_for(int64_t n) {
   return 62 - bits;
 }
 
-static int grid_for(int64_t work, int per_sm) {
-  int64_t cap = 148ll * per_sm;
-  return (int)(work < cap ? (work < 1 ? 1 : work) : cap);
-}
 
 template <typename KT>
 static cudaError_t route_levels(const RouteCall& c) {
@@ -963,16 +1512,9 @@ static cudaError_t route_levels(const RouteCall& c) {
     se.level_ids_cap = l >= 2 ? ncap_of(g, l) : 0;
     se.dev_status = c.dev_status;
     trace_begin(ZHA_TRACE_ROUTE_SELECT, c.stream);
-    route_select_warp_kernel<<<grid_for((nqh + kWarpSelWarps - 1) / kWarpSelWarps, 8), kWarpSelWarps * 32, 0,
-                               c.stream>>>(se);
+    e = launch_select(se, nqh, L.lv[l].n_cap, c.stream);
     count_launch();
-    e = launch_status("route_select_warp_kernel");
-    if (e != cudaSuccess) return e;
-    if (L.lv[l].n_cap > kWarpSelMax) {                   // frontiers too large for one warp
-      e = launch_select_cluster(se, nqh, L.lv[l].n_cap, c.stream);
-      count_launch();
-      if (e != cudaSuccess) { note_cuda_error(e, "route_select_cluster_kernel"); return e; }
-    }
+    if (e != cudaSuccess) { note_cuda_error(e, "route select"); return e; }
     trace_end(ZHA_TRACE_ROUTE_SELECT, c.stream);
   }
   return cudaSuccess;
@@ -1008,17 +1550,10 @@ static cudaError_t flat_select_t(const RouteCall& c) {
   se.cand_cnt = fa.cand_cnt; se.C1 = w.C1;
   se.out_ids = c.leaf_ids; se.out_cnt = c.leaf_cnt; se.out_stride = c.leaf_cap; se.out_cap = c.leaf_cap;
   se.dev_status = c.dev_status;
-  route_select_warp_kernel<<<grid_for((nqh + kWarpSelWarps - 1) / kWarpSelWarps, 8), kWarpSelWarps * 32, 0,
-                             c.stream>>>(se);
+  e = launch_select(se, nqh, w.C1, c.stream);
   count_launch();
-  e = launch_status("route_select_warp_kernel(flat)");
-  if (e != cudaSuccess) return e;
-  if (w.C1 > kWarpSelMax) {
-    e = launch_select_cluster(se, nqh, w.C1, c.stream);
-    count_launch();
-    if (e != cudaSuccess) { note_cuda_error(e, "route_select_cluster_kernel(flat)"); return e; }
-  }
-  return launch_status("route_select_cluster_kernel(flat)");
+  if (e != cudaSuccess) note_cuda_error(e, "route select (flat)");
+  return e;
 }
 
 // Flat indexer: `c.tree` carries the K cache pointer.

@@ -48,10 +48,12 @@ def out_tol(w):
 class DecodeRun:
     """One decode step on the GPU plus everything the oracle needs."""
 
-    def __init__(self, w: S.Workload, p: float, with_levels=True):
+    def __init__(self, w: S.Workload, p: float, with_levels=True, k_transform=None):
         self.w, self.p = w, p
         self.g = g = geometry(w)
         self.C, self.K, self.V = S.clustered_kv(w, DEV)
+        if k_transform is not None:
+            k_transform(self.K)
         self.qref = S.reference_queries(w, DEV)
         self.k_new, self.v_new = S.new_tokens(w, self.C, 1, DEV)
         self.q = S.queries(w, self.C, 1, DEV)
@@ -245,6 +247,25 @@ def test_decode_p1_is_dense():
     torch.cuda.synchronize()
     assert (O2.float() - run.O.float()).abs().max().item() <= 2e-2
     check_decode(run, [(0, h) for h in range(w.Hkv)])
+
+
+@pytest.mark.parametrize("T,p", [(16384 + 64 * 3 + 17, 0.9), (70000 + 17, 0.95)])
+def test_decode_tied_chunks(T, p):
+    """Leaf chunks repeated with period 5: exact score ties at level 1 (and, with period 5
+    over the parents, at level 2), boundaries inside tie groups; the select must keep the
+    lowest ids of a tie group like the oracle.  T = 70017 puts level 1 (1094 candidates)
+    on the cluster select, the other case on the warp select."""
+    w = S.scaled(S.workload("batched-decode-128k"), T=T, B=1, n_centres=256)
+
+    def tie(K):
+        n = w.T // 64
+        src = torch.arange(n, device=K.device) % 5
+        Kv = K[:, :, :n * 64].view(K.shape[0], K.shape[1], n, 64, K.shape[-1])
+        Kv.copy_(Kv[:, :, src].clone())
+
+    run = DecodeRun(w, p, k_transform=tie)
+    cmp = check_decode(run, [(0, h) for h in range(w.Hkv)])
+    print(f"tied chunks T={T} p={p}: {cmp.exact} exact, {cmp.near_cutoff} near-cutoff of {cmp.heads}")
 
 
 def test_decode_is_deterministic():
