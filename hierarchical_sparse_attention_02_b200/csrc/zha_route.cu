@@ -63,11 +63,11 @@ struct ScoreArgs {
 
 constexpr int kScoreThreads = 128;
 #ifndef ZHA_SCORE_MIN_BLOCKS
-#define ZHA_SCORE_MIN_BLOCKS 5                   // resident CTAs per SM the registers allow
+#define ZHA_SCORE_MIN_BLOCKS 4                   // resident CTAs per SM the registers allow
 #endif
 
 template <typename KT>
-__global__ void __launch_bounds__(kScoreThreads, ZHA_SCORE_MIN_BLOCKS) route_score_kernel(ScoreArgs a) {
+__global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN_BLOCKS : 3) route_score_kernel(ScoreArgs a) {
   __shared__ __align__(16) double qfs[32][32];
   __shared__ int rank[kScoreThreads][kMaxG];     // per parent slot: rank in each head's list
   __shared__ int pcnt[kMaxG];
@@ -175,9 +175,10 @@ __global__ void __launch_bounds__(kScoreThreads, ZHA_SCORE_MIN_BLOCKS) route_sco
     constexpr int kVec = 16 / sizeof(KT);
     constexpr int kNv = 32 / kVec;                       // 16-byte vectors of 32 dims
     const int R = g.R;
-    const int nsteps = 4 * R;                            // even
+    const int nsteps = 4 * R;
     const int64_t node0 = (b * g.Hkv + hk) * g.ncap[a.level];
-    auto load_step = [&](uint4 (&v)[kNv], int st) {
+    // a step's row and its b_hat are loaded together, one step ahead of their use
+    auto load_step = [&](uint4 (&v)[kNv], float& bh, int st) {
       const int grp = st / R, r = st - grp * R;
       int64_t id; unsigned int m; int jj, cc;
       slot_of(grp, id, m, jj, cc);
@@ -185,23 +186,22 @@ __global__ void __launch_bounds__(kScoreThreads, ZHA_SCORE_MIN_BLOCKS) route_sco
           reinterpret_cast<const KT*>(a.k_route) + ((node0 + id) * R + r) * kD + 32 * (lane & 3));
 #pragma unroll
       for (int i = 0; i < kNv; ++i) v[i] = m ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+      bh = m ? __ldg(a.b_hat + (node0 + id) * R + r) : 0.f;
     };
     double best0 = -INFINITY, best1 = -INFINITY;
-    auto compute_step = [&](const uint4 (&v)[kNv], int st) {
+    auto compute_step = [&](const uint4 (&v)[kNv], float bh, int st) {
       const int grp = st / R, r = st - grp * R;
-      double ca0 = 0.0, ca1 = 0.0, cb0 = 0.0, cb1 = 0.0;
+      double c0[4] = {0.0, 0.0, 0.0, 0.0}, c1[4] = {0.0, 0.0, 0.0, 0.0};   // 4 independent chains
 #pragma unroll
       for (int s2 = 0; s2 < 32; ++s2) {
         const double av = (double)u4_elem<KT>(v[s2 / kVec], s2 % kVec);  // exact widening
-        const double qv = qfs[s2][lane];
-        if (s2 & 1) mma_f64(cb0, cb1, av, qv);
-        else mma_f64(ca0, ca1, av, qv);
+        mma_f64(c0[s2 & 3], c1[s2 & 3], av, qfs[s2][lane]);
       }
       int64_t id; unsigned int m; int jj, cc;
       slot_of(grp, id, m, jj, cc);
-      const double bb = m ? (double)a.b_hat[(node0 + id) * R + r] : 0.0;
-      best0 = fmax(best0, fma(ca0 + cb0, scale, bb));
-      best1 = fmax(best1, fma(ca1 + cb1, scale, bb));
+      const double bb = (double)bh;
+      best0 = fmax(best0, fma((c0[0] + c0[1]) + (c0[2] + c0[3]), scale, bb));
+      best1 = fmax(best1, fma((c1[0] + c1[1]) + (c1[2] + c1[3]), scale, bb));
       if (r == R - 1) {
 #pragma unroll
         for (int q = 0; q < 2; ++q) {
@@ -220,13 +220,18 @@ __global__ void __launch_bounds__(kScoreThreads, ZHA_SCORE_MIN_BLOCKS) route_sco
         best0 = best1 = -INFINITY;
       }
     };
-    uint4 vA[kNv], vB[kNv];
-    load_step(vA, 0);
-    for (int st = 0; st < nsteps; st += 2) {
-      load_step(vB, st + 1);
-      compute_step(vA, st);
-      if (st + 2 < nsteps) load_step(vA, st + 2);
-      compute_step(vB, st + 1);
+    // three row buffers: the rows of the next two steps are in flight during each step
+    uint4 vA[kNv], vB[kNv], vC[kNv];
+    float bA, bB, bC;
+    load_step(vA, bA, 0);
+    load_step(vB, bB, 1);                                // nsteps = 4R >= 4
+    for (int st = 0; st < nsteps; st += 3) {
+      if (st + 2 < nsteps) load_step(vC, bC, st + 2);
+      compute_step(vA, bA, st);
+      if (st + 3 < nsteps) load_step(vA, bA, st + 3);
+      if (st + 1 < nsteps) compute_step(vB, bB, st + 1);
+      if (st + 4 < nsteps) load_step(vB, bB, st + 4);
+      if (st + 2 < nsteps) compute_step(vC, bC, st + 2);
     }
   }
 }
@@ -755,6 +760,7 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
 // ---------------------------------------------------------------------------
 
 constexpr int kClMaxCta = 8;
+constexpr int kStreamCta = 8;
 
 template <int T>
 struct ClSmem {
@@ -1379,15 +1385,12 @@ static int grid_for(int64_t work, int per_sm) {
   return (int)(work < cap ? (work < 1 ? 1 : work) : cap);
 }
 
+constexpr int kCta1024Cap = 16896;       // candidates a 1024-thread select CTA holds
+
 template <typename K>
-static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t clusters, int cs, int threads,
-                                  size_t smem, cudaStream_t s) {
-  if (smem > 0) {
-    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-  }
+static cudaLaunchConfig_t cluster_config(K kernel, cudaLaunchAttribute* attr, int64_t clusters, int cs,
+                                         int threads, size_t smem, cudaStream_t s) {
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = cs;
   attr[0].val.clusterDim.y = 1;
@@ -1398,16 +1401,41 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
   cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
+  return cfg;
+}
+
+template <typename K>
+static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t clusters, int cs, int threads,
+                                  size_t smem, cudaStream_t s) {
+  if (smem > 0) {
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchAttribute attr[1];
+  const cudaLaunchConfig_t cfg = cluster_config(kernel, attr, clusters, cs, threads, smem, s);
   return cudaLaunchKernelEx(&cfg, kernel, se);
 }
 
-// One select launch for a level whose frontier holds up to ncap candidates per head:
-//   ncap <= 1024    a warp per head (scores in shared memory)
-//   ncap <= 4096    a CTA of 256 threads per head (48 KiB of scores and ids)
-//   ncap <= 65536   a cluster of 2 / 4 / 8 CTAs of 512 threads per head (96 KiB of scores and ids each)
-//   above           a cluster of 8 CTAs of 512 threads streaming the scores from memory
+// One select launch per level.  Kernels, by the frontier capacity ncap they hold:
+//   warp     a warp per head (scores in shared memory)            ncap <= 1024
+//   cta256   a CTA of 256 threads per head (48 KiB)               ncap <= 4096
+//   cta1024  a CTA of 1024 threads per head (198 KiB)             ncap <= 16896
+//   cluster  2 / 4 / 8 CTAs of 1024 threads per head              ncap <= 8 * 16896
+//   stream   8 CTAs of 512 threads re-reading the scores          above
+// The widest kernel whose resident heads (148 SMs x CTAs per SM) cover every head of the
+// level runs them in one wave at the lowest latency per head; when none does, the
+// narrowest one that holds ncap takes the most heads at once.
 static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
-  if (ncap <= kWarpCap) {
+  const int64_t res_warp = 148ll * 3 * kWarpSelWarps, res256 = 148ll * 3, res1024 = 148;
+  int kind;                                            // 0 warp, 1 cta256, 2 cta1024, 3 cluster, 4 stream
+  if (ncap <= kCta1024Cap && nqh <= res1024) kind = 2;
+  else if (ncap <= 4096 && nqh <= res256) kind = 1;
+  else if (ncap <= kWarpCap) kind = 0;
+  else if (ncap <= 4096) kind = 1;
+  else if (ncap <= kCta1024Cap) kind = 2;
+  else if (ncap <= 8ll * kCta1024Cap) kind = 3;
+  else kind = 4;
+  if (kind == 0) {
     const size_t smem = sizeof(WarpSelSmem);
     cudaError_t e = cudaFuncSetAttribute(route_select_warp_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
@@ -1416,17 +1444,20 @@ static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap
                                s>>>(se);
     return cudaGetLastError();
   }
-  if (ncap <= 4096)
-    return launch_cluster(route_select_block_kernel<256, 4096, false>, se, nqh < 148 * 3 ? nqh : 148 * 3, 1, 256,
+  if (kind == 1)
+    return launch_cluster(route_select_block_kernel<256, 4096, false>, se, nqh < res256 ? nqh : res256, 1, 256,
                           4096 * (sizeof(double) + sizeof(int)), s);
-  if (ncap <= 8 * 8192) {
-    const int cs = ncap <= 2 * 8192 ? 2 : (ncap <= 4 * 8192 ? 4 : 8);
+  if (kind == 2)
+    return launch_cluster(route_select_block_kernel<1024, kCta1024Cap, false>, se, nqh < res1024 ? nqh : res1024,
+                          1, 1024, kCta1024Cap * (sizeof(double) + sizeof(int)), s);
+  if (kind == 3) {
+    const int cs = ncap <= 2 * kCta1024Cap ? 2 : ncap <= 4 * kCta1024Cap ? 4 : 8;
     const int64_t per = 148 / cs;
-    return launch_cluster(route_select_block_kernel<512, 8192, true>, se, nqh < per ? nqh : per, cs, 512,
-                          8192 * (sizeof(double) + sizeof(int)), s);
+    return launch_cluster(route_select_block_kernel<1024, kCta1024Cap, true>, se, nqh < per ? nqh : per, cs,
+                          1024, kCta1024Cap * (sizeof(double) + sizeof(int)), s);
   }
-  const int64_t per = (2 * 148) / kClMaxCta;
-  return launch_cluster(route_select_stream_kernel<512>, se, nqh < per ? nqh : per, kClMaxCta, 512, 0, s);
+  const int64_t per = (2 * 148) / kStreamCta;
+  return launch_cluster(route_select_stream_kernel<512>, se, nqh < per ? nqh : per, kStreamCta, 512, 0, s);
 }
 
 // ---------------------------------------------------------------------------
