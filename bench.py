@@ -181,9 +181,9 @@ class ClockSampler:
 # profiles/attn_tc_kernel.batched-decode-128k.md (batch 4, i.e. 16 of the 128 KV units),
 # valid while the kernel source is the one that was captured.
 PROFILED_TRAFFIC = {
-    "batched-decode-128k": {"bytes": 1.075265e9 + 11.197696e6, "units": 16,
+    "batched-decode-128k": {"bytes": 1.075072e9 + 11.166976e6, "units": 16,
                             "source": "hierarchical_sparse_attention_02_b200/csrc/zha_attn_tc.cu",
-                            "sha1": "1a1445435c7ded07e36083d341e509ede65d6b56"},
+                            "sha1": "cff5ce98064c40fbb38bc64c4047b9cf46b050f3"},
 }
 
 

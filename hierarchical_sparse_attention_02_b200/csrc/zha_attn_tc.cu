@@ -368,6 +368,194 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__
   }
 }
 
+// ---------------------------------------------------------------------------
+// Flat indexer scores (the exact-chunk-score baseline) on the same TMA ring: every
+// visible 64-key chunk of a KV group streams through shared memory once; consumer warp w
+// takes the chunks w, w + 4, ... of the CTA's sequence (ring stage s always belongs to warp
+// s % 4), computes S^T[64 keys x 8 heads] = K_chunk . Q^T with mma.sync bf16 (fp32
+// accumulate) and reduces it to F_C(q) = max + log(sum exp(s - max)) per head.
+// ---------------------------------------------------------------------------
+
+constexpr int kFlatStages = 8;                   // a multiple of the consumer warps
+constexpr int kFlatChunksPerItem = 64;
+constexpr uint32_t kFlatTxBytes = 2 * kBoxBytes;
+
+struct FlatSmem {
+  unsigned char stage[kFlatStages][2 * kBoxBytes];   // K dims 0-63 | 64-127 of one chunk
+  unsigned long long full[kFlatStages];
+  unsigned long long empty[kFlatStages];
+  int abort;
+  int zero;
+};
+
+struct FlatTcArgs {
+  int B, nq, Hq, Hkv, G;
+  int64_t t_cap;
+  const int64_t* q_pos;
+  int64_t pos_uniform;
+  const __nv_bfloat16* Q;
+  int64_t C1, nblk;                              // chunk blocks (of kFlatChunksPerItem) per unit
+  int* cand_ids;
+  double* cand_score;
+  int* cand_cnt;
+  int32_t* dev_status;
+};
+
+struct FlatItem {
+  int64_t bq, unit_kv, blk, nvis;
+  int hk, c0, c1;
+};
+
+__device__ __forceinline__ FlatItem flat_item(const FlatTcArgs& a, int64_t item) {
+  FlatItem f;
+  const int64_t u = item / a.nblk;
+  f.blk = item % a.nblk;
+  f.bq = u / a.Hkv;
+  f.hk = (int)(u % a.Hkv);
+  f.unit_kv = (f.bq / a.nq) * a.Hkv + f.hk;
+  const int64_t t = query_pos(a.q_pos, a.pos_uniform, f.bq);
+  f.nvis = (t >= 0 && t < a.t_cap) ? visible_nodes(t, kLeaf) : 0;
+  const int64_t lo = f.blk * kFlatChunksPerItem;
+  f.c0 = (int)(lo < f.nvis ? lo : f.nvis);
+  f.c1 = (int)(lo + kFlatChunksPerItem < f.nvis ? lo + kFlatChunksPerItem : f.nvis);
+  return f;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+flat_tc_kernel(const __grid_constant__ CUtensorMap kmap, FlatTcArgs a) {
+  extern __shared__ unsigned char smem_raw[];
+  FlatSmem& sm = *reinterpret_cast<FlatSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t total_items = (int64_t)a.B * a.nq * a.Hkv * a.nblk;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kFlatStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
+    sm.abort = 0;
+    sm.zero = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ---------------- producer: one lane issues the TMA loads ----------------
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"((unsigned long long)&kmap) : "memory");
+      long long it_count = 0;
+      long long issued[kFlatStages];
+      for (int s = 0; s < kFlatStages; ++s) issued[s] = 0;
+      bool ok = true;
+      for (int64_t item = blockIdx.x; item < total_items && ok; item += gridDim.x) {
+        const FlatItem f = flat_item(a, item);
+        for (int c = f.c0; c < f.c1; ++c, ++it_count) {
+          const int s = (int)(it_count % kFlatStages);
+          if (it_count >= kFlatStages) {
+            if (!mbar_wait(&sm.empty[s], (uint32_t)(((it_count / kFlatStages) - 1) & 1), &sm.abort)) {
+              set_status(a.dev_status, ZHA_ERR_DEVICE);
+              atomicExch(&sm.abort, 1);
+              ok = false;
+              break;
+            }
+          }
+          if (*(volatile int*)&sm.abort) { ok = false; break; }
+          mbar_arrive_tx(&sm.full[s], kFlatTxBytes);
+          tma_load_3d(sm.stage[s], &kmap, 0, c * kLeaf, (int)f.unit_kv, &sm.full[s]);
+          tma_load_3d(sm.stage[s] + kBoxBytes, &kmap, 64, c * kLeaf, (int)f.unit_kv, &sm.full[s]);
+          ++issued[s];
+        }
+      }
+      // drain: no TMA write may land after the CTA exits
+      for (int s = 0; s < kFlatStages; ++s)
+        if (issued[s] > 0 && !mbar_wait(&sm.full[s], (uint32_t)((issued[s] - 1) & 1), &sm.zero))
+          set_status(a.dev_status, ZHA_ERR_DEVICE);
+    }
+    return;
+  }
+
+  // ---------------- consumers ----------------
+  const int g = lane >> 2, t4 = lane & 3;
+  const float scale = 1.0f / sqrtf((float)kD);
+  long long it_count = 0;
+  for (int64_t item = blockIdx.x; item < total_items; item += gridDim.x) {
+    const FlatItem f = flat_item(a, item);
+    const int64_t qh0 = f.bq * a.Hq + (int64_t)f.hk * a.G;
+    if (f.blk == 0 && warp == 0 && lane < a.G) a.cand_cnt[qh0 + lane] = (int)f.nvis;
+    if (f.c0 >= f.c1) continue;
+    uint32_t qb[8][2];
+    {
+      const __nv_bfloat16* qrow = a.Q + (qh0 + (g < a.G ? g : 0)) * kD;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t w0 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t4);
+        const uint32_t w1 = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * t4 + 8);
+        qb[kk][0] = g < a.G ? w0 : 0u;
+        qb[kk][1] = g < a.G ? w1 : 0u;
+      }
+    }
+    for (int c = f.c0; c < f.c1; ++c, ++it_count) {
+      if ((int)(it_count % kConsumerWarps) != warp) continue;
+      const int s = (int)(it_count % kFlatStages);
+      if (!mbar_wait(&sm.full[s], (uint32_t)((it_count / kFlatStages) & 1), &sm.abort)) {
+        set_status(a.dev_status, ZHA_ERR_DEVICE);
+        atomicExch(&sm.abort, 1);
+        continue;
+      }
+      const uint32_t base = smem_u32(sm.stage[s]);
+      float sc[4][4];
+      const int mi = lane >> 3, r8 = lane & 7;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
+        const int row = 16 * j + r8 + ((mi & 1) << 3);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const int box = kk >> 2;
+          const int chunk = ((kk & 3) << 1) + (mi >> 1);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(base + box * kBoxBytes + swz(row, chunk), a0, a1, a2, a3);
+          mma_bf16(sc[j], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[s]);
+      // lane holds keys 16j + g (+8) for heads 2t4 (values 0, 2) and 2t4 + 1 (values 1, 3)
+      float mA = -INFINITY, mB = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        mA = fmaxf(mA, fmaxf(sc[j][0] * scale, sc[j][2] * scale));
+        mB = fmaxf(mB, fmaxf(sc[j][1] * scale, sc[j][3] * scale));
+      }
+#pragma unroll
+      for (int x = 4; x < 32; x <<= 1) {
+        mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, x));
+        mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, x));
+      }
+      float zA = 0.f, zB = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        zA += expf(sc[j][0] * scale - mA) + expf(sc[j][2] * scale - mA);
+        zB += expf(sc[j][1] * scale - mB) + expf(sc[j][3] * scale - mB);
+      }
+#pragma unroll
+      for (int x = 4; x < 32; x <<= 1) {
+        zA += __shfl_xor_sync(0xffffffffu, zA, x);
+        zB += __shfl_xor_sync(0xffffffffu, zB, x);
+      }
+      if (g == 0) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int h = 2 * t4 + q;
+          if (h < a.G) {
+            double F = (double)(q ? mB : mA) + log((double)(q ? zB : zA));
+            if (F == 0.0) F = 0.0;
+            a.cand_ids[(qh0 + h) * a.C1 + c] = c;
+            a.cand_score[(qh0 + h) * a.C1 + c] = F;
+          }
+        }
+      }
+    }
+  }
+}
+
 }  // namespace tc
 
 // ---------------------------------------------------------------------------
@@ -426,6 +614,30 @@ cudaError_t attn_tc_launch(const AttnCall& c, const AttnWs& w, const int* stage_
   cudaFuncSetAttribute(tc::attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   const int64_t grid = w.items_max < sm_count() ? w.items_max : sm_count();
   tc::attn_tc_kernel<<<(unsigned)grid, tc::kThreads, smem, c.stream>>>(km, vm, a);
+  return cudaSuccess;
+}
+
+cudaError_t flat_tc_launch(const zha_geom& g, int nq, const void* Q, const void* K, const int64_t* q_pos,
+                          int64_t pos_uniform, int64_t C1, int* cand_ids, double* cand_score, int* cand_cnt,
+                          int32_t* dev_status, cudaStream_t stream) {
+  CUtensorMap km;
+  if (!make_kv_map(&km, K, (int64_t)g.B * g.Hkv, g.t_cap)) {
+    note_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+    return cudaErrorInvalidValue;
+  }
+  tc::FlatTcArgs a{};
+  a.B = g.B; a.nq = nq; a.Hq = g.Hq; a.Hkv = g.Hkv; a.G = g.Hq / g.Hkv; a.t_cap = g.t_cap;
+  a.q_pos = q_pos; a.pos_uniform = pos_uniform;
+  a.Q = (const __nv_bfloat16*)Q;
+  a.C1 = C1;
+  a.nblk = (C1 + tc::kFlatChunksPerItem - 1) / tc::kFlatChunksPerItem;
+  if (a.nblk < 1) a.nblk = 1;
+  a.cand_ids = cand_ids; a.cand_score = cand_score; a.cand_cnt = cand_cnt; a.dev_status = dev_status;
+  const size_t smem = sizeof(tc::FlatSmem) + 1024;
+  cudaFuncSetAttribute(tc::flat_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int64_t items = (int64_t)g.B * nq * g.Hkv * a.nblk;
+  const int64_t grid = items < sm_count() ? items : sm_count();
+  tc::flat_tc_kernel<<<(unsigned)(grid < 1 ? 1 : grid), tc::kThreads, smem, stream>>>(km, a);
   return cudaSuccess;
 }
 

@@ -276,6 +276,11 @@ cudaError_t route_all(const RouteCall& c);
 cudaError_t flat_select(const RouteCall& c);
 cudaError_t attention(const AttnCall& c);
 // bf16 split-KV gather on tensor cores (zha_attn_tc.cu)
+// Flat indexer scores of bf16 caches on the tensor cores: F_C(q) of every visible chunk of
+// every query head, into the routing workspace's candidate arrays (ids, scores, counts).
+cudaError_t flat_tc_launch(const zha_geom& g, int nq, const void* Q, const void* K, const int64_t* q_pos,
+                          int64_t pos_uniform, int64_t C1, int* cand_ids, double* cand_score, int* cand_cnt,
+                          int32_t* dev_status, cudaStream_t stream);
 cudaError_t attn_tc_launch(const AttnCall& c, const AttnWs& w, const int* stage_ids,
                            const unsigned int* stage_mask, const int* stage_cnt, const int* pair_off,
                            float* partials);

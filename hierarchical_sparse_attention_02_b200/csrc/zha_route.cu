@@ -1569,9 +1569,20 @@ static cudaError_t flat_select_t(const RouteCall& c) {
   fa.cand_cnt = (int*)(c.ws + w.cand_cnt);
   fa.nblk = (w.C1 + 7) / 8;
   if (fa.nblk < 1) fa.nblk = 1;
-  flat_score_kernel<KT><<<grid_for(units * fa.nblk, 8), 256, 0, c.stream>>>(fa);
-  count_launch();
-  cudaError_t e = launch_status("flat_score_kernel");
+  cudaError_t e;
+  if (g.dtype == ZHA_BF16) {                           // tensor cores, K streamed by TMA
+    trace_begin(ZHA_TRACE_ROUTE_SCORE, c.stream);
+    e = flat_tc_launch(g, c.nq, c.Q, c.tree, c.q_pos, c.pos_uniform, w.C1, fa.cand_ids, fa.cand_score,
+                       fa.cand_cnt, c.dev_status, c.stream);
+    trace_end(ZHA_TRACE_ROUTE_SCORE, c.stream);
+    count_launch();
+    if (e != cudaSuccess) return e;
+    e = launch_status("flat_tc_kernel");
+  } else {
+    flat_score_kernel<KT><<<grid_for(units * fa.nblk, 8), 256, 0, c.stream>>>(fa);
+    count_launch();
+    e = launch_status("flat_score_kernel");
+  }
   if (e != cudaSuccess) return e;
   SelectArgs se{};
   se.g = rg; se.level = 1; se.flat = 1; se.p = c.p;
