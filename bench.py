@@ -478,7 +478,9 @@ def main():
     time.sleep(0.3)
     barrier(ws)
     torch.cuda.synchronize()
-    lib.zha_trace(_lib.ZHA_TRACE_ATTN, arr_s, arr_e, n_ev)
+    # the dominant kernel is traced live: the attention, or the chunk scores of the flat path
+    dom = _lib.ZHA_TRACE_ROUTE_SCORE if args.path == "flat" and w.dtype == "bf16" else _lib.ZHA_TRACE_ATTN
+    lib.zha_trace(dom, arr_s, arr_e, n_ev)
     n_launch0 = Z.launch_count()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark_start()
@@ -490,11 +492,11 @@ def main():
     clocks.mark_end()
     barrier(ws)
     launches = Z.launch_count() - n_launch0
-    traced = lib.zha_trace_count(_lib.ZHA_TRACE_ATTN)
-    lib.zha_trace(_lib.ZHA_TRACE_ATTN, None, None, 0)
+    traced = lib.zha_trace_count(dom)
+    lib.zha_trace(dom, None, None, 0)
     ms_local = t_start.elapsed_time(t_end) / Ksteps
-    attn_launches = traced / Ksteps                        # attention launches per step
-    attn_ms = sum(a.elapsed_time(b) for a, b in zip(starts[:traced], stops[:traced])) / max(1, traced)
+    dom_launches = traced / Ksteps                         # launches of the traced kernel per step
+    dom_ms = sum(a.elapsed_time(b) for a, b in zip(starts[:traced], stops[:traced])) / max(1, traced)
     if st.item() != 0:
         raise RuntimeError(f"device status {st.item()} in the timed region")
     ms, value = whole_job_rate(w.B * w.Hq, ms_local, ws)
@@ -564,11 +566,16 @@ def main():
     gathered = union_rows * 2 * w.d * es
     partial_bytes = items * w.G * (w.d + 2) * 4          # o[d], m, l written per head and split
     attn_bytes = gathered + partial_bytes
+    # flat path: every visible chunk's keys read once, a score and an id written per head
+    flat_bytes = units * nvis * 64 * w.d * es + w.B * w.Hq * nvis * 12 if args.path == "flat" else 0
     peak, peak_kind = hbm_peak()
-    # per launch: a decode step attends in `attn_launches` chunk launches (whole-step bytes
-    # split by chunk; the chunks are equal in size up to a ragged last one)
-    per_launch = attn_bytes / max(1.0, attn_launches)
-    achieved = per_launch / (attn_ms * 1e-3) / 1e9
+    if dom == _lib.ZHA_TRACE_ATTN:
+        dom_name = "attn_tc_kernel" if w.dtype == "bf16" else "attn_split_kernel"
+        per_launch = attn_bytes / max(1.0, dom_launches)
+    else:
+        dom_name = "flat_tc_kernel"
+        per_launch = flat_bytes / max(1.0, dom_launches)
+    achieved = per_launch / (dom_ms * 1e-3) / 1e9
     cpu = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda")
@@ -580,14 +587,14 @@ def main():
         "steps": Ksteps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {**config_of(w, p), "path": args.path},
-        "roofline": {"bound": "hbm", "kernel": "attn_tc_kernel" if w.dtype == "bf16" else "attn_split_kernel",
+        "roofline": {"bound": "hbm", "kernel": dom_name,
                      "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": (profiled_traffic(w, units / max(1.0, attn_launches))
+                     "traffic": (profiled_traffic(w, units / max(1.0, dom_launches))
                                  if args.path == "zha" and w.dtype == "bf16" else None),
-                     "algorithmic_bytes_per_launch": per_launch, "kernel_ms": attn_ms,
-                     "launches_per_step": attn_launches},
-        "step_hbm_gbs": attn_bytes / (ms * 1e-3) / 1e9,
+                     "algorithmic_bytes_per_launch": per_launch, "kernel_ms": dom_ms,
+                     "launches_per_step": dom_launches},
+        "step_hbm_gbs": (attn_bytes + flat_bytes) / (ms * 1e-3) / 1e9,
         "kv_touched": {"mean": float(np.mean(per_head)), "p50": float(np.median(per_head)),
                        "p99": float(np.percentile(per_head, 99)),
                        "group_union": union_rows / (units * T1)},
