@@ -61,21 +61,26 @@ struct ScoreArgs {
   int32_t* dev_status;
 };
 
-constexpr int kScoreThreads = 128;
+constexpr int kScoreSlots = 128;                 // candidate slots per work item
 #ifndef ZHA_SCORE_MIN_BLOCKS
 #define ZHA_SCORE_MIN_BLOCKS 4                   // resident CTAs per SM the registers allow
 #endif
 
-template <typename KT>
-__global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN_BLOCKS : 3) route_score_kernel(ScoreArgs a) {
+// GPW = groups of 8 slots per warp: 4 (4 warps per item, for levels with many items) or 1
+// (16 warps per item: a quarter of the dependent steps per warp, for the few items of the
+// upper levels).
+template <typename KT, int GPW>
+__global__ void __launch_bounds__(kScoreSlots * 4 / GPW, GPW == 4 ? (sizeof(KT) == 2 ? ZHA_SCORE_MIN_BLOCKS : 3) : 1)
+route_score_kernel(ScoreArgs a) {
+  constexpr int kThreads = kScoreSlots * 4 / GPW;
   __shared__ __align__(16) double qfs[32][32];
-  __shared__ int rank[kScoreThreads][kMaxG];     // per parent slot: rank in each head's list
+  __shared__ int rank[kScoreSlots][kMaxG];       // per parent slot: rank in each head's list
   __shared__ int pcnt[kMaxG];
   const RouteGeom& g = a.g;
   const int tid = threadIdx.x;
   const int64_t units = (int64_t)g.B * g.nq * g.Hkv;
   const double scale = 1.0 / sqrt((double)kD);
-  const int per_blk = kScoreThreads / g.branch;          // parents per work item
+  const int per_blk = kScoreSlots / g.branch;            // parents per work item
   for (int64_t w = blockIdx.x; w < units * a.nblk; w += gridDim.x) {
     const int64_t u = w / a.nblk;
     const int64_t blk = w % a.nblk;
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
     // which slots this item covers
     int mode;                                            // 0 top nodes, 1 parents, 2 orphans
     if (at_top) {
-      if (blk * kScoreThreads >= nvis) continue;
+      if (blk * kScoreSlots >= nvis) continue;
       mode = 0;
     } else if (blk < nb_par) {
       mode = 1;
@@ -112,7 +117,7 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
     __syncthreads();                                     // smem reuse across items
     if (tid < g.G) pcnt[tid] = at_top ? 0 : a.parents_cnt[qh0 + tid];
     // B fragments of the mma: qfs[s][L] = q[head L/4][32 * (L%4) + s] (0 for heads >= G)
-    for (int i = tid; i < 32 * 32; i += kScoreThreads) {
+    for (int i = tid; i < 32 * 32; i += kThreads) {
       const int s2 = i / 32, L = i % 32, h = L >> 2;
       const KT* q = reinterpret_cast<const KT*>(a.Q) + qh0 * kD;
       qfs[s2][L] = h < g.G ? to_f64(q[h * kD + 32 * (L & 3) + s2]) : 0.0;
@@ -123,7 +128,7 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
     if (mode == 3) continue;
     if (mode == 1) {
       // rank of each parent of this item in each head's kept list (-1: not kept)
-      for (int i = tid; i < per_blk * g.G; i += kScoreThreads) {
+      for (int i = tid; i < per_blk * g.G; i += kThreads) {
         const int j = i / g.G, h = i % g.G;
         const int64_t p = blk * per_blk + j;
         int r = -1;
@@ -137,7 +142,7 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
       }
       __syncthreads();
     }
-    // Scores on the fp64 tensor cores: each warp takes its 32 slots as 4 groups of 8
+    // Scores on the fp64 tensor cores: each warp takes its 8*GPW slots as GPW groups of 8
     // nodes; D[8 nodes x 8 heads] += A[8 nodes x 4 dims] . B[4 dims x 8 heads] per
     // mma.m8n8k4.f64.  Lane L holds A[node L/4][dim 32*(L%4) + s] and B[dim][head L/4]
     // at k-step s (qf[s][L] in shared memory), so each lane reads 32 contiguous dims of
@@ -147,12 +152,12 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
     const int h0 = 2 * (lane & 3), h1 = h0 + 1;         // this lane's heads in D
     // node of this lane's row in group grp, and the heads that have it as a candidate
     auto slot_of = [&](int grp, int64_t& id, unsigned int& mask, int& j, int& c) {
-      const int slot = warp * 32 + grp * 8 + (lane >> 2);
+      const int slot = (warp * GPW + grp) * 8 + (lane >> 2);
       mask = 0;
       j = 0;
       c = 0;
       if (mode == 0) {
-        id = blk * kScoreThreads + slot;
+        id = blk * kScoreSlots + slot;
         if (id < nvis) mask = (1u << g.G) - 1u;
       } else if (mode == 1) {
         j = slot / g.branch;
@@ -166,7 +171,7 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
       }
     };
     unsigned int any_mask = 0;
-    for (int grp = 0; grp < 4; ++grp) {
+    for (int grp = 0; grp < GPW; ++grp) {
       int64_t id; unsigned int m; int jj, cc;
       slot_of(grp, id, m, jj, cc);
       any_mask |= m;
@@ -175,7 +180,7 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
     constexpr int kVec = 16 / sizeof(KT);
     constexpr int kNv = 32 / kVec;                       // 16-byte vectors of 32 dims
     const int R = g.R;
-    const int nsteps = 4 * R;
+    const int nsteps = GPW * R;
     const int64_t node0 = (b * g.Hkv + hk) * g.ncap[a.level];
     // a step's row and its b_hat are loaded together, one step ahead of their use
     auto load_step = [&](uint4 (&v)[kNv], float& bh, int st) {
@@ -224,7 +229,7 @@ __global__ void __launch_bounds__(kScoreThreads, sizeof(KT) == 2 ? ZHA_SCORE_MIN
     uint4 vA[kNv], vB[kNv], vC[kNv];
     float bA, bB, bC;
     load_step(vA, bA, 0);
-    load_step(vB, bB, 1);                                // nsteps = 4R >= 4
+    if (nsteps > 1) load_step(vB, bB, 1);
     for (int st = 0; st < nsteps; st += 3) {
       if (st + 2 < nsteps) load_step(vC, bC, st + 2);
       compute_step(vA, bA, st);
@@ -1508,8 +1513,8 @@ static cudaError_t route_levels(const RouteCall& c) {
     sa.cand_cnt = (int*)(c.ws + w.cand_cnt);
     sa.dev_status = c.dev_status;
     {
-      const int64_t per_blk = kScoreThreads / g.branch;
-      int64_t nb = (L.lv[l].n_cap + kScoreThreads - 1) / kScoreThreads;
+      const int64_t per_blk = kScoreSlots / g.branch;
+      int64_t nb = (L.lv[l].n_cap + kScoreSlots - 1) / kScoreSlots;
       if (l < g.depth) {
         const int64_t nbp = (L.lv[l + 1].n_cap + per_blk - 1) / per_blk + 1;
         if (nbp > nb) nb = nbp;
@@ -1518,7 +1523,10 @@ static cudaError_t route_levels(const RouteCall& c) {
     }
     const int64_t units = (int64_t)g.B * c.nq * g.Hkv;
     trace_begin(ZHA_TRACE_ROUTE_SCORE, c.stream);
-    route_score_kernel<KT><<<grid_for(units * sa.nblk, 8), kScoreThreads, 0, c.stream>>>(sa);
+    if (units * sa.nblk <= 2 * 148)                      // few items: shortest chains
+      route_score_kernel<KT, 1><<<grid_for(units * sa.nblk, 1), kScoreSlots * 4, 0, c.stream>>>(sa);
+    else
+      route_score_kernel<KT, 4><<<grid_for(units * sa.nblk, 8), kScoreSlots, 0, c.stream>>>(sa);
     trace_end(ZHA_TRACE_ROUTE_SCORE, c.stream);
     count_launch();
     cudaError_t e = launch_status("route_score_kernel");
