@@ -339,8 +339,8 @@ SWEEP_T = (16384, 32768, 65536, 131072, 262144, 524288, 1048576, 2097152)
 
 
 def run_sweep(args):
-    """Crossover sweep: ms per decode step of zha_decode at every depth L = 1..6 and of the
-    dense kernel, for T in SWEEP_T at the long-decode head geometry (B=4, Hq=32, Hkv=4),
+    """Crossover sweep: ms per decode step of zha_decode at every depth L = 1..6, of the
+    dense kernel and of the flat indexer, for T in SWEEP_T at the long-decode head geometry (B=4, Hq=32, Hkv=4),
     on the same seeded inputs per T.  One JSON line per (T, path, depth)."""
     import dataclasses
     import hierarchical_sparse_attention_02_b200 as Z
@@ -393,7 +393,14 @@ def run_sweep(args):
         ms_dense = timed(lambda: Z.zha_dense_decode(g, q, K, V, pos, O, wsd, st))
         print(json.dumps({"sweep": "crossover", "T": T, "path": "dense", "ms_per_step": ms_dense,
                           "zha_best_ms": best, "zha_faster": best < ms_dense}), flush=True)
-        del K, V, wsd
+        wsf = Z.empty_workspace(g, 1, Z.ZHA_OP_FLAT, dev)
+        ids = torch.empty(w.B, 1, w.Hq, Z.leaf_cap(g), dtype=torch.int32, device=dev)
+        cnt = torch.empty(w.B, 1, w.Hq, dtype=torch.int32, device=dev)
+        ms_flat = timed(lambda: Z.zha_flat_index(g, q, K, V, pos, p, ids, cnt, O, wsf, st))
+        touched = float((cnt.double() * 64 + 1).mean().item()) / (w.T + 1)
+        print(json.dumps({"sweep": "crossover", "T": T, "path": "flat", "ms_per_step": ms_flat,
+                          "kv_touched_approx": touched}), flush=True)
+        del K, V, wsd, wsf, ids, cnt
         torch.cuda.empty_cache()
 
 
