@@ -162,3 +162,49 @@ def test_prefill_append_256k_full(Z):
     e = np.stack(errs)
     assert e.max() <= 2e-2 and e.mean() <= 2e-3, (e.max(), e.mean())
     print(f"prefill-append-256k: {cmp.exact} exact, {cmp.near_cutoff} near-cutoff of {cmp.heads}")
+
+
+@pytest.mark.parametrize("name,units,heads", [("batched-decode-128k", [(0, 0), (31, 3)], None),
+                                              ("long-decode-1m", [(2, 1)], [0, 5])])
+def test_flat_index_full(Z, name, units, heads):
+    """The flat exact-LSE indexer at full size: tensor-core chunk scores over every visible
+    chunk, top-p select, sparse attention; sampled heads against the oracle's exact chunk
+    scores (fp32 chunk log-masses: sets may differ only among near-equal scores at the
+    boundary)."""
+    w = S.workload(name)
+    g = geometry(w)
+    p = w.p[0]
+    C, K, V = S.clustered_kv(w, DEV)
+    q = S.queries(w, C, 1, DEV)
+    del C
+    t = w.T - 1
+    pos = torch.full((w.B, 1), t, dtype=torch.int64, device=DEV)
+    cap = Z.leaf_cap(g)
+    ids = torch.full((w.B, 1, w.Hq, cap), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros(w.B, 1, w.Hq, dtype=torch.int32, device=DEV)
+    O = torch.empty(w.B, 1, w.Hq, w.d, dtype=g.dtype, device=DEV)
+    ws = Z.empty_workspace(g, 1, Z.ZHA_OP_FLAT, DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    Z.zha_flat_index(g, q, K, V, pos, p, ids, cnt, O, ws, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    qc = q.double().cpu().numpy()
+    exact = total = 0
+    for (b, hk) in units:
+        Kc, Vc = K[b, hk].cpu(), V[b, hk].cpu()
+        hs = range(hk * w.G, (hk + 1) * w.G) if heads is None else [hk * w.G + i for i in heads]
+        for h in hs:
+            total += 1
+            sel = zo.flat_select(qc[b, 0, h], Kc, t, p)
+            got = ids[b, 0, h, :int(cnt[b, 0, h])].cpu().numpy()
+            diff = np.setxor1d(sel.ids, got)
+            if len(diff) == 0:
+                exact += 1
+                o, _ = zo.attention(qc[b, 0, h], Kc, Vc, zo.index_set(sel.ids, t))
+                assert np.abs(O[b, 0, h].float().cpu().numpy() - o).max() <= 2e-2
+            else:
+                s = zo.flat_scores(qc[b, 0, h], Kc, t)
+                boundary = np.sort(s)[::-1][sel.m - 1]
+                assert np.abs(s[diff] - boundary).max() <= 1e-4 or sel.margin < 1e-4, (b, h, len(diff))
+    assert exact >= total // 2
+    print(f"{name} flat: {exact} exact of {total} heads")

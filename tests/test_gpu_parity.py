@@ -249,13 +249,20 @@ def test_decode_p1_is_dense():
     check_decode(run, [(0, h) for h in range(w.Hkv)])
 
 
-@pytest.mark.parametrize("T,p", [(16384 + 64 * 3 + 17, 0.9), (70000 + 17, 0.95)])
-def test_decode_tied_chunks(T, p):
+@pytest.mark.parametrize("name,T,p", [("batched-decode-128k", 16384 + 64 * 3 + 17, 0.9),
+                                      ("batched-decode-128k", 70000 + 17, 0.95),
+                                      ("deep-tree-16m@L1", 1200000 + 5, 0.9)])
+def test_decode_tied_chunks(name, T, p):
     """Leaf chunks repeated with period 5: exact score ties at level 1 (and, with period 5
     over the parents, at level 2), boundaries inside tie groups; the select must keep the
-    lowest ids of a tie group like the oracle.  T = 70017 puts level 1 (1094 candidates)
-    on the cluster select, the other case on the warp select."""
-    w = S.scaled(S.workload("batched-decode-128k"), T=T, B=1, n_centres=256)
+    lowest ids of a tie group like the oracle.  The three cases put level 1 on the warp
+    select (259 candidates), a 1024-thread CTA (1094) and a 2-CTA cluster (18750
+    candidates in 5 tie groups of 3750: the tie ranks run across the cluster)."""
+    import dataclasses
+    base, _, ll = name.partition("@L")
+    w = S.scaled(S.workload(base), T=T, B=1, n_centres=256)
+    if ll:
+        w = dataclasses.replace(w, depth=int(ll))
 
     def tie(K):
         n = w.T // 64
