@@ -385,6 +385,108 @@ __global__ void __launch_bounds__(kCombGroups * kD) combine_blocks_kernel(AttnGe
   if (grp == 0) write_out(g, u, h, d, r, O, lse);
 }
 
+// Combine for units of at most kCombBlock items (the common case): one CTA per unit, warp
+// h <-> head h, lane <-> 4 dims.  Two passes in item order: the maximum M of the partials'
+// m, then L = sum 2^(m_i - M) l_i and o = sum 2^(m_i - M) o_i with every load independent
+// of the running state (deterministic, fixed order).
+template <typename OT>
+__global__ void __launch_bounds__(kMaxG * 32) combine_warp_kernel(AttnGeom g, const int* pair_off,
+                                                                const float* partials, OT* O, float* lse) {
+  const int64_t u = blockIdx.x;
+  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (h >= g.G) return;
+  const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
+  float M = -INFINITY;
+  for (int64_t i = i0 + lane; i < i1; i += 32) M = fmaxf(M, partials[(i * g.G + h) * kPartStride + kD]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (M != -INFINITY) {
+#pragma unroll 4
+    for (int64_t i = i0; i < i1; ++i) {
+      const float* P = partials + (i * g.G + h) * kPartStride;
+      const float4 o4 = *reinterpret_cast<const float4*>(P + 4 * lane);
+      const float w = exp2f(P[kD] - M);                  // 0 for an empty partial (m = -inf)
+      L = fmaf(w, P[kD + 1], L);
+      acc.x = fmaf(w, o4.x, acc.x);
+      acc.y = fmaf(w, o4.y, acc.y);
+      acc.z = fmaf(w, o4.z, acc.z);
+      acc.w = fmaf(w, o4.w, acc.w);
+    }
+  }
+  const int64_t bq = u / g.Hkv;
+  const int hk = (int)(u % g.Hkv);
+  const int64_t qh = bq * g.Hq + hk * g.G + h;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  OT* out = O + qh * kD + 4 * lane;
+  out[0] = from_f32<OT>(acc.x * inv);
+  out[1] = from_f32<OT>(acc.y * inv);
+  out[2] = from_f32<OT>(acc.z * inv);
+  out[3] = from_f32<OT>(acc.w * inv);
+  if (lse && lane == 0) lse[qh] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+}
+
+// Combine for units of up to 4 * kCombBlock items: one CTA of 8 warps per (unit, head);
+// the CTA's maximum M first, then warp w sums the items w, w + 8, ... (lane <-> 4 dims)
+// and the eight warp sums are added in warp order (deterministic, fixed order).
+template <typename OT>
+__global__ void __launch_bounds__(256) combine_cta_kernel(AttnGeom g, const int* pair_off, const float* partials,
+                                                        OT* O, float* lse) {
+  __shared__ float wm[8], wl[8];
+  __shared__ float4 wacc[8][32];
+  const int64_t u = blockIdx.x / g.G;
+  const int h = (int)(blockIdx.x % g.G);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
+  float M = -INFINITY;
+  for (int64_t i = i0 + tid; i < i1; i += 256) M = fmaxf(M, partials[(i * g.G + h) * kPartStride + kD]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  if (lane == 0) wm[warp] = M;
+  __syncthreads();
+  M = wm[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) M = fmaxf(M, wm[w]);
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (M != -INFINITY) {
+#pragma unroll 4
+    for (int64_t i = i0 + warp; i < i1; i += 8) {
+      const float* P = partials + (i * g.G + h) * kPartStride;
+      const float4 o4 = *reinterpret_cast<const float4*>(P + 4 * lane);
+      const float w = exp2f(P[kD] - M);
+      L = fmaf(w, P[kD + 1], L);
+      acc.x = fmaf(w, o4.x, acc.x);
+      acc.y = fmaf(w, o4.y, acc.y);
+      acc.z = fmaf(w, o4.z, acc.z);
+      acc.w = fmaf(w, o4.w, acc.w);
+    }
+  }
+  wacc[warp][lane] = acc;
+  if (lane == 0) wl[warp] = L;
+  __syncthreads();
+  if (warp != 0) return;
+  L = 0.f;
+  acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+  for (int w = 0; w < 8; ++w) {
+    L += wl[w];
+    const float4 a4 = wacc[w][lane];
+    acc.x += a4.x; acc.y += a4.y; acc.z += a4.z; acc.w += a4.w;
+  }
+  const int64_t bq = u / g.Hkv;
+  const int hk = (int)(u % g.Hkv);
+  const int64_t qh = bq * g.Hq + hk * g.G + h;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  OT* out = O + qh * kD + 4 * lane;
+  out[0] = from_f32<OT>(acc.x * inv);
+  out[1] = from_f32<OT>(acc.y * inv);
+  out[2] = from_f32<OT>(acc.z * inv);
+  out[3] = from_f32<OT>(acc.w * inv);
+  if (lse && lane == 0) lse[qh] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+}
+
 // ---------------------------------------------------------------------------
 // host driver
 // ---------------------------------------------------------------------------
@@ -444,6 +546,18 @@ static cudaError_t attention_t(const AttnCall& c) {
   // items of one unit: at most ceil((C1 + 2) / cps) + nr
   const int64_t items_unit = (w.C1 + 2 + w.cps - 1) / w.cps + w.nr;
   const int64_t nb_max = (items_unit + kCombBlock - 1) / kCombBlock;
+  if (nb_max == 1) {
+    combine_warp_kernel<KT><<<(unsigned)w.units, kMaxG * 32, 0, c.stream>>>(ag, pair_off, aa.partials,
+                                                                            (KT*)c.O, c.lse);
+    count_launch();
+    return launch_status("combine_warp_kernel");
+  }
+  if (nb_max <= 4) {
+    combine_cta_kernel<KT><<<(unsigned)(w.units * ag.G), 256, 0, c.stream>>>(ag, pair_off, aa.partials,
+                                                                             (KT*)c.O, c.lse);
+    count_launch();
+    return launch_status("combine_cta_kernel");
+  }
   combine_kernel<KT><<<(unsigned)(w.units * ag.G * nb_max), kCombGroups * kD, 0, c.stream>>>(
       ag, pair_off, aa.partials, nb_max, (KT*)c.O, c.lse);
   count_launch();
