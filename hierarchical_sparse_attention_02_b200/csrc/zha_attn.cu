@@ -68,18 +68,35 @@ __global__ void __launch_bounds__(256) union_kernel(UnionArgs a) {
     // each head's slice [lower_bound(lo), lower_bound(hi)) of its ascending list, then
     // one flat pass over all slices so that every thread's loads are independent
     __shared__ int s_b0[kMaxG], s_off[kMaxG + 1];
-    if (tid < g.G) {
-      const int64_t qh = bq * g.Hq + hk * g.G + tid;
+    if (warp < g.G) {
+      // warp h finds its head's slice with a 32-way search (each round probes 32 positions
+      // and keeps the segment where the list crosses the bound: ~log32 dependent loads)
+      const int64_t qh = bq * g.Hq + hk * g.G + warp;
       const int* lst = a.leaf_ids + qh * a.leaf_cap;
       int cnt = a.leaf_cnt[qh];
       if (cnt > a.leaf_cap) cnt = a.leaf_cap;
       if (cnt < 0) cnt = 0;
-      int x0 = 0, x1 = cnt;
-      while (x0 < x1) { const int m = (x0 + x1) >> 1; if (lst[m] < lo) x0 = m + 1; else x1 = m; }
-      int y0 = x0, y1 = cnt;
-      while (y0 < y1) { const int m = (y0 + y1) >> 1; if (lst[m] < hi) y0 = m + 1; else y1 = m; }
-      s_b0[tid] = x0;
-      s_off[tid + 1] = y0 - x0;
+      int xb[2];
+      const int64_t bound[2] = {lo, hi};
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        int x0 = 0, x1 = cnt;                        // lower_bound(bound[k]) lies in [x0, x1]
+        while (x1 - x0 > 32) {
+          const int step = (x1 - x0 + 31) / 32;
+          const int idx = x0 + (lane + 1) * step - 1;
+          const bool below = idx < x1 && lst[idx] < bound[k];
+          const int c = __popc(__ballot_sync(0xffffffffu, below));
+          const int nx0 = x0 + c * step;
+          x1 = nx0 + step < x1 ? nx0 + step : x1;
+          x0 = nx0;
+        }
+        const bool below = x0 + lane < x1 && lst[x0 + lane] < bound[k];
+        xb[k] = x0 + __popc(__ballot_sync(0xffffffffu, below));
+      }
+      if (lane == 0) {
+        s_b0[warp] = xb[0];
+        s_off[warp + 1] = xb[1] - xb[0];
+      }
     }
     __syncthreads();
     if (tid == 0) {
@@ -89,7 +106,7 @@ __global__ void __launch_bounds__(256) union_kernel(UnionArgs a) {
     __syncthreads();
     const int total_ids = s_off[g.G];
     int h = 0;                                    // i only grows: the head index follows it
-#pragma unroll 4
+#pragma unroll 8
     for (int i = tid; i < total_ids; i += 256) {
       while (i >= s_off[h + 1]) ++h;
       const int64_t qh = bq * g.Hq + hk * g.G + h;
