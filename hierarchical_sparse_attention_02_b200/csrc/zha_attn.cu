@@ -69,33 +69,17 @@ __global__ void __launch_bounds__(256) union_kernel(UnionArgs a) {
     // one flat pass over all slices so that every thread's loads are independent
     __shared__ int s_b0[kMaxG], s_off[kMaxG + 1];
     if (warp < g.G) {
-      // warp h finds its head's slice with a 32-way search (each round probes 32 positions
-      // and keeps the segment where the list crosses the bound: ~log32 dependent loads)
+      // warp h finds its head's slice of its ascending list
       const int64_t qh = bq * g.Hq + hk * g.G + warp;
       const int* lst = a.leaf_ids + qh * a.leaf_cap;
       int cnt = a.leaf_cnt[qh];
       if (cnt > a.leaf_cap) cnt = a.leaf_cap;
       if (cnt < 0) cnt = 0;
-      int xb[2];
-      const int64_t bound[2] = {lo, hi};
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        int x0 = 0, x1 = cnt;                        // lower_bound(bound[k]) lies in [x0, x1]
-        while (x1 - x0 > 32) {
-          const int step = (x1 - x0 + 31) / 32;
-          const int idx = x0 + (lane + 1) * step - 1;
-          const bool below = idx < x1 && lst[idx] < bound[k];
-          const int c = __popc(__ballot_sync(0xffffffffu, below));
-          const int nx0 = x0 + c * step;
-          x1 = nx0 + step < x1 ? nx0 + step : x1;
-          x0 = nx0;
-        }
-        const bool below = x0 + lane < x1 && lst[x0 + lane] < bound[k];
-        xb[k] = x0 + __popc(__ballot_sync(0xffffffffu, below));
-      }
+      const int x0 = warp_lower_bound(lst, cnt, lo);
+      const int x1 = warp_lower_bound(lst, cnt, hi);
       if (lane == 0) {
-        s_b0[warp] = xb[0];
-        s_off[warp + 1] = xb[1] - xb[0];
+        s_b0[warp] = x0;
+        s_off[warp + 1] = x1 - x0;
       }
     }
     __syncthreads();

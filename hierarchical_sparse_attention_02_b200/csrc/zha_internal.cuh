@@ -216,6 +216,25 @@ __device__ __forceinline__ void mma_f64(double& d0, double& d1, double a, double
                : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
 }
 
+// First index i in [0, cnt) of an ascending list with lst[i] >= key (cnt if none), found by
+// the whole warp with a 32-way search: every round probes 32 positions and keeps the
+// segment where the list crosses key (about log32(cnt) dependent loads).  All lanes return
+// the same index.
+__device__ __forceinline__ int warp_lower_bound(const int* lst, int cnt, int64_t key) {
+  const int lane = threadIdx.x & 31;
+  int x0 = 0, x1 = cnt;                              // the answer lies in [x0, x1]
+  while (x1 - x0 > 32) {
+    const int step = (x1 - x0 + 31) / 32;
+    const int idx = x0 + (lane + 1) * step - 1;
+    const bool below = idx < x1 && lst[idx] < key;
+    const int nx0 = x0 + __popc(__ballot_sync(0xffffffffu, below)) * step;
+    x1 = nx0 + step < x1 ? nx0 + step : x1;
+    x0 = nx0;
+  }
+  const bool below = x0 + lane < x1 && lst[x0 + lane] < key;
+  return x0 + __popc(__ballot_sync(0xffffffffu, below));
+}
+
 // Position of the query of (b, qi): from q_pos, or the uniform position when q_pos is null.
 __device__ __forceinline__ int64_t query_pos(const int64_t* q_pos, int64_t uniform, int64_t bq) {
   return q_pos ? q_pos[bq] : uniform;

@@ -127,18 +127,23 @@ route_score_kernel(ScoreArgs a) {
       a.cand_cnt[qh0 + tid] = (int)(at_top ? nvis : (int64_t)pcnt[tid] * g.branch + (nvis - orph_lo));
     if (mode == 3) continue;
     if (mode == 1) {
-      // rank of each parent of this item in each head's kept list (-1: not kept)
-      for (int i = tid; i < per_blk * g.G; i += kThreads) {
-        const int j = i / g.G, h = i % g.G;
-        const int64_t p = blk * per_blk + j;
-        int r = -1;
-        if (p < npar) {
-          const int* lst = a.parents + (qh0 + h) * a.C2;
-          int lo = 0, hi = pcnt[h];
-          while (lo < hi) { const int m = (lo + hi) >> 1; if (lst[m] < p) lo = m + 1; else hi = m; }
-          if (lo < pcnt[h] && lst[lo] == p) r = lo;
+      // rank of each parent of this item in each head's kept list (-1: not kept): the kept
+      // parents in [p0, p0 + per_blk) are consecutive entries of the head's ascending list,
+      // from its lower bound of p0 on (one warp per head)
+      const int64_t p0 = blk * per_blk;
+      for (int i = tid; i < per_blk * g.G; i += kThreads) rank[i / g.G][i % g.G] = -1;
+      __syncthreads();
+      const int lane_ = tid & 31;
+      for (int h = tid >> 5; h < g.G; h += kThreads / 32) {
+        const int* lst = a.parents + (qh0 + h) * a.C2;
+        const int cnt = pcnt[h];
+        const int x = warp_lower_bound(lst, cnt, p0);
+        for (int j = lane_; j < per_blk; j += 32) {
+          if (x + j < cnt) {
+            const int v = lst[x + j];
+            if (v < p0 + per_blk && v < npar) rank[v - p0][h] = x + j;
+          }
         }
-        rank[j][h] = r;
       }
       __syncthreads();
     }
