@@ -82,8 +82,8 @@ route_score_kernel(ScoreArgs a) {
   const double scale = 1.0 / sqrt((double)kD);
   const int per_blk = kScoreSlots / g.branch;            // parents per work item
   for (int64_t w = blockIdx.x; w < units * a.nblk; w += gridDim.x) {
-    const int64_t u = w / a.nblk;
-    const int64_t blk = w % a.nblk;
+    const int64_t u = w % units;                         // block-major: the items of block 0
+    const int64_t blk = w / units;                       // of every unit come first
     const int64_t bq = u / g.Hkv;
     const int hk = (int)(u % g.Hkv);
     const int64_t b = bq / g.nq;
@@ -1428,7 +1428,7 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
 
 // One select launch per level.  Kernels, by the frontier capacity ncap they hold:
 //   warp     a warp per head (scores in shared memory)            ncap <= 1024
-//   cta256   a CTA of 256 threads per head (48 KiB)               ncap <= 4096
+//   cta256   a CTA of 256 threads per head (30 or 48 KiB)         ncap <= 2560 or 4096
 //   cta1024  a CTA of 1024 threads per head (198 KiB)             ncap <= 16896
 //   cluster  2 / 4 / 8 CTAs of 1024 threads per head              ncap <= 8 * 16896
 //   stream   8 CTAs of 512 threads re-reading the scores          above
@@ -1454,6 +1454,9 @@ static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap
                                s>>>(se);
     return cudaGetLastError();
   }
+  if (kind == 1 && ncap <= 2560)                       // 56 KiB per CTA: 4 resident per SM
+    return launch_cluster(route_select_block_kernel<256, 2560, false>, se, nqh < 4 * 148 ? nqh : 4 * 148, 1,
+                          256, 2560 * (sizeof(double) + sizeof(int)), s);
   if (kind == 1)
     return launch_cluster(route_select_block_kernel<256, 4096, false>, se, nqh < res256 ? nqh : res256, 1, 256,
                           4096 * (sizeof(double) + sizeof(int)), s);
