@@ -183,7 +183,7 @@ class ClockSampler:
 PROFILED_TRAFFIC = {
     "batched-decode-128k": {"bytes": 1.075072e9 + 11.166976e6, "units": 16,
                             "source": "hierarchical_sparse_attention_02_b200/csrc/zha_attn_tc.cu",
-                            "sha1": "cff5ce98064c40fbb38bc64c4047b9cf46b050f3"},
+                            "sha1": "7cd49e01f798c1e4020732017f021f6d675035d1"},
 }
 
 

@@ -2,7 +2,7 @@
 //
 // One persistent CTA per SM walks the work items (splits of the union-of-heads chunk
 // lists built by union_kernel / plan_kernel).  A producer warp streams every selected
-// 64-key block of K and V into a 6-stage shared-memory ring with 3-D TMA loads
+// 64-key block of K and V into a 4-stage shared-memory ring with 3-D TMA loads
 // (cp.async.bulk.tensor, 128-byte swizzle, completion on mbarriers; no multicast).  Four
 // consumer warps each own 16 keys of every block and run, for the G <= 8 query heads that
 // share the block (GQA),
