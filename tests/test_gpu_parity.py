@@ -333,7 +333,8 @@ def test_sparse_attn_on_oracle_lists(name, T):
 # ---------------------------------------------------------------------------
 
 
-@pytest.mark.parametrize("name,T", [("tiny-decode-f32", 8192), ("batched-decode-128k", 20000 + 17)])
+@pytest.mark.parametrize("name,T", [("tiny-decode-f32", 8192), ("batched-decode-128k", 20000 + 17),
+                                    ("batched-decode-128k", 140000 + 3)])   # > 128 splits: CTA combine
 def test_dense_decode_parity(name, T):
     w = S.scaled(S.workload(name), T=T, B=2, n_centres=256)
     g = geometry(w)
