@@ -1390,6 +1390,469 @@ __global__ void __launch_bounds__(T) route_select_block_kernel(SelectArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// wide select: frontiers beyond the clusters' shared memory (more than 8 x 16896 candidates
+// per head) as a chain of grid-wide kernels over (head, chunk of kWideChunk candidates), so
+// that every SM works on a few heads' candidates; the heads' running state lives at the
+// start of the head's row of the mass workspace (C1 x 8 bytes, C1 > 135168):
+//   init -> maxima -> masses + linear histogram (per-CTA histograms added with global
+//   atomics, integer sums: order-free) -> boundary bucket (a CTA per head) -> its members
+//   gathered -> resolved (a CTA per head: the members sorted in shared memory, or, for a
+//   boundary bucket of more than kWideMembers candidates, radix digits of the order key over
+//   a stream of the head's candidates) -> keeps counted per chunk -> written in order.
+// ---------------------------------------------------------------------------
+
+constexpr int kWideChunk = 4096;
+constexpr int kWideThreads = 256;                 // 16 candidates per thread
+constexpr int kWideMembers = 4096;
+constexpr int kWideMaxChunks = 1024;
+
+enum : int { kWideSkip = -1, kWideDone = 0, kWideAll = 1, kWideGather = 2, kWideRadix = 3 };
+
+struct WideHead {
+  unsigned long long kmax, kmin, Z, tgt, above, mass_b, pfx, need;
+  unsigned int mcount, cnt_b, cnt_t;
+  int mode, d1, shift, n, pad;
+  unsigned int cnt[kBuckets];
+  unsigned long long mass[kBuckets];
+  unsigned int chunk_def[kWideMaxChunks], chunk_tie[kWideMaxChunks];
+  int m_pos[kWideMembers];
+  unsigned long long m_key[kWideMembers], m_mass[kWideMembers];
+};
+
+__device__ __forceinline__ WideHead* wide_head(const SelectArgs& a, int64_t qh) {
+  return reinterpret_cast<WideHead*>(a.cand_mass + qh * a.C1);
+}
+
+__device__ __forceinline__ double key_to_score(unsigned long long k) {
+  return __longlong_as_double((long long)((k >> 63) ? (k & 0x7fffffffffffffffull) : ~k));
+}
+
+__device__ __forceinline__ LinBuckets wide_buckets(const WideHead* h) {
+  LinBuckets lb;
+  lb.init(key_to_score(h->kmax), key_to_score(h->kmin), kBuckets);
+  return lb;
+}
+
+__device__ __forceinline__ Cutoff wide_cutoff(const WideHead* h) {
+  Cutoff c{};
+  c.keep_all = h->mode == kWideAll;
+  c.d1 = h->d1;
+  c.shift = h->shift;
+  c.pfx = h->pfx;
+  c.need = h->need;
+  c.cnt_t = h->cnt_t;
+  return c;
+}
+
+// sum over the CTA (any T multiple of 32); the result is valid in every thread
+template <typename V, int T>
+__device__ __forceinline__ V wide_sum(V v, V* scratch) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  __syncthreads();
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  V r = 0;
+  for (int w = 0; w < T / 32; ++w) r += scratch[w];
+  return r;
+}
+
+__global__ void __launch_bounds__(kWideThreads) wide_init_kernel(SelectArgs a) {
+  const int64_t qh = blockIdx.x;
+  WideHead* h = wide_head(a, qh);
+  const int n = head_candidates(a, qh, threadIdx.x == 0);
+  if (threadIdx.x == 0) {
+    h->n = n;
+    h->mode = n < 0 ? kWideSkip : kWideDone;
+    h->kmax = 0ull;
+    h->kmin = ~0ull;
+    h->Z = 0ull;
+    h->mcount = 0u;
+    h->shift = 64;
+  }
+  if (n < 0) return;
+  for (int i = threadIdx.x; i < kBuckets; i += kWideThreads) { h->cnt[i] = 0u; h->mass[i] = 0ull; }
+  for (int i = threadIdx.x; i < kWideMaxChunks; i += kWideThreads) { h->chunk_def[i] = 0u; h->chunk_tie[i] = 0u; }
+}
+
+__global__ void __launch_bounds__(kWideThreads) wide_minmax_kernel(SelectArgs a, int nch) {
+  __shared__ unsigned long long red[kWideThreads / 32];
+  const int64_t qh = blockIdx.x / nch;
+  const int c = (int)(blockIdx.x % nch);
+  const WideHead* h = wide_head(a, qh);
+  if (h->mode == kWideSkip) return;
+  const int i0 = c * kWideChunk;
+  const int i1 = min(h->n, i0 + kWideChunk);
+  if (i0 >= i1) return;
+  const double* s = a.cand_score + qh * a.C1;
+  unsigned long long kx = 0ull, kn = ~0ull;
+#pragma unroll 8
+  for (int i = i0 + threadIdx.x; i < i1; i += kWideThreads) {
+    const unsigned long long k = order_key(s[i]);
+    kx = k > kx ? k : kx;
+    kn = k < kn ? k : kn;
+  }
+  // maxima of the keys (the minimum as the complement's maximum)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const unsigned long long x = __shfl_xor_sync(0xffffffffu, kx, o), y = __shfl_xor_sync(0xffffffffu, kn, o);
+    kx = x > kx ? x : kx;
+    kn = y < kn ? y : kn;
+  }
+  if (lane == 0) red[warp] = kx;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kWideThreads / 32; ++w) kx = red[w] > kx ? red[w] : kx;
+    atomicMax(&wide_head(a, qh)->kmax, kx);
+  }
+  __syncthreads();
+  if (lane == 0) red[warp] = kn;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kWideThreads / 32; ++w) kn = red[w] < kn ? red[w] : kn;
+    atomicMin(&wide_head(a, qh)->kmin, kn);
+  }
+}
+
+__global__ void __launch_bounds__(kWideThreads) wide_hist_kernel(SelectArgs a, int nch) {
+  __shared__ unsigned int cnt[kBuckets];
+  __shared__ unsigned long long mass[kBuckets];
+  __shared__ unsigned long long red[kWideThreads / 32];
+  const int64_t qh = blockIdx.x / nch;
+  const int c = (int)(blockIdx.x % nch);
+  WideHead* h = wide_head(a, qh);
+  if (h->mode == kWideSkip) return;
+  const int i0 = c * kWideChunk;
+  const int i1 = min(h->n, i0 + kWideChunk);
+  if (i0 >= i1) return;
+  const LinBuckets lb = wide_buckets(h);
+  const double M = lb.M;
+  for (int i = threadIdx.x; i < kBuckets; i += kWideThreads) { cnt[i] = 0u; mass[i] = 0ull; }
+  __syncthreads();
+  const double* s = a.cand_score + qh * a.C1;
+  unsigned long long z = 0ull;
+#pragma unroll 4
+  for (int i = i0 + threadIdx.x; i < i1; i += kWideThreads) {
+    const double v = s[i];
+    const unsigned long long e = mass_of(v, M, a.mass_shift);
+    z += e;
+    const int d = lb.digit(v);
+    atomicAdd(&cnt[d], 1u);
+    atomicAdd(&mass[d], e);
+  }
+  z = wide_sum<unsigned long long, kWideThreads>(z, red);    // contains the barriers
+  if (threadIdx.x == 0) atomicAdd(&h->Z, z);
+  for (int i = threadIdx.x; i < kBuckets; i += kWideThreads) {
+    if (cnt[i]) {
+      atomicAdd(&h->cnt[i], cnt[i]);
+      atomicAdd(&h->mass[i], mass[i]);
+    }
+  }
+}
+
+// One CTA of 1024 threads per head: the boundary bucket of the global histogram.
+__global__ void __launch_bounds__(1024) wide_boundary_kernel(SelectArgs a) {
+  __shared__ ClSmem<1024> sm;
+  const int64_t qh = blockIdx.x;
+  WideHead* h = wide_head(a, qh);
+  if (h->mode == kWideSkip) return;
+  if (a.p >= 1.0 || h->n == 0) {
+    if (threadIdx.x == 0) h->mode = kWideAll;
+    return;
+  }
+  for (int i = threadIdx.x; i < kBuckets; i += 1024) { sm.cnt[i] = h->cnt[i]; sm.mass[i] = h->mass[i]; }
+  const unsigned long long tgt = target_of(a.p, h->Z);
+  unsigned long long above = 0ull, mass_b = 0ull;
+  unsigned int cnt_b = 0u;
+  const int d1 = cl_boundary<1024, false>(sm, 1, 0, above, tgt, cnt_b, mass_b);   // syncs first
+  if (threadIdx.x == 0) {
+    h->tgt = tgt;
+    h->d1 = d1;
+    h->above = above;
+    h->cnt_b = cnt_b;
+    h->mass_b = mass_b;
+    h->shift = 64;                               // a single candidate: the whole bucket is kept
+    h->mode = cnt_b <= 1 ? kWideDone : (cnt_b <= (unsigned)kWideMembers ? kWideGather : kWideRadix);
+  }
+}
+
+__global__ void __launch_bounds__(kWideThreads) wide_gather_kernel(SelectArgs a, int nch) {
+  const int64_t qh = blockIdx.x / nch;
+  const int c = (int)(blockIdx.x % nch);
+  WideHead* h = wide_head(a, qh);
+  if (h->mode != kWideGather) return;
+  const int i0 = c * kWideChunk;
+  const int i1 = min(h->n, i0 + kWideChunk);
+  const LinBuckets lb = wide_buckets(h);
+  const int d1 = h->d1;
+  const double* s = a.cand_score + qh * a.C1;
+  for (int i = i0 + threadIdx.x; i < i1; i += kWideThreads) {
+    const double v = s[i];
+    if (lb.digit(v) != d1) continue;
+    const unsigned int slot = atomicAdd(&h->mcount, 1u);   // < cnt_b <= kWideMembers
+    if (slot >= (unsigned)kWideMembers) continue;          // (the histogram counted them all)
+    h->m_pos[slot] = i;
+    h->m_key[slot] = order_key(v);
+    h->m_mass[slot] = mass_of(v, lb.M, a.mass_shift);
+  }
+}
+
+// One CTA of 1024 threads per head: the boundary bucket resolved.
+__global__ void __launch_bounds__(1024) wide_resolve_kernel(SelectArgs a) {
+  extern __shared__ __align__(16) unsigned char wide_raw[];
+  __shared__ ClSmem<1024> sm;
+  const int64_t qh = blockIdx.x;
+  WideHead* h = wide_head(a, qh);
+  const int tid = threadIdx.x;
+  const int mode = h->mode;
+  if (mode != kWideGather && mode != kWideRadix) return;
+  const unsigned long long tgt = h->tgt;
+  unsigned long long above = h->above;
+  if (mode == kWideGather) {
+    // sort the members by (key descending, position ascending), then walk their masses
+    unsigned long long* key = reinterpret_cast<unsigned long long*>(wide_raw);
+    unsigned long long* ms = key + kWideMembers;
+    int* pos = reinterpret_cast<int*>(ms + kWideMembers);
+    const int m = (int)(h->mcount < (unsigned)kWideMembers ? h->mcount : (unsigned)kWideMembers);
+    int P = 1;
+    while (P < m) P <<= 1;
+    for (int i = tid; i < P; i += 1024) {
+      const bool on = i < m;
+      key[i] = on ? h->m_key[i] : 0ull;            // 0 is below every order key of a score
+      pos[i] = on ? h->m_pos[i] : 0x7fffffff;
+      ms[i] = on ? h->m_mass[i] : 0ull;
+    }
+    __syncthreads();
+    for (int k = 2; k <= P; k <<= 1) {
+      for (int j = k >> 1; j > 0; j >>= 1) {
+        for (int i = tid; i < P; i += 1024) {
+          const int l = i ^ j;
+          if (l > i) {
+            const bool first_before = key[i] > key[l] || (key[i] == key[l] && pos[i] < pos[l]);
+            const bool up = (i & k) == 0;          // this pair's run is in (descending) order
+            if (first_before != up) {
+              const unsigned long long tk = key[i]; key[i] = key[l]; key[l] = tk;
+              const int tp = pos[i]; pos[i] = pos[l]; pos[l] = tp;
+              const unsigned long long tm = ms[i]; ms[i] = ms[l]; ms[l] = tm;
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+    // the first member (in order) whose cumulative mass from `above` reaches tgt
+    if (tid == 0) {
+      unsigned long long acc = above;
+      int cidx = m - 1;
+      for (int i = 0; i < m; ++i) {
+        acc += ms[i];
+        if (acc >= tgt) { cidx = i; break; }
+      }
+      const unsigned long long kc = key[cidx];
+      const int pc = pos[cidx];
+      unsigned int cnt_t = 0;
+      unsigned long long need = 0;
+      for (int i = 0; i < m; ++i) {
+        if (key[i] == kc) {
+          ++cnt_t;
+          need += pos[i] <= pc;
+        }
+      }
+      h->pfx = kc;
+      h->shift = 0;
+      h->cnt_t = cnt_t;
+      h->need = need;
+      h->mode = kWideDone;
+    }
+    return;
+  }
+  // large boundary bucket: key range of its members, then radix digits of the order key
+  const LinBuckets lb = wide_buckets(h);
+  const int d1 = h->d1;
+  const int n = h->n;
+  const double* s = a.cand_score + qh * a.C1;
+  unsigned long long kmx = 0ull, kmn = ~0ull;
+  for (int i = tid; i < n; i += 1024) {
+    const double v = s[i];
+    if (lb.digit(v) == d1) {
+      const unsigned long long k = order_key(v);
+      kmx = k > kmx ? k : kmx;
+      kmn = k < kmn ? k : kmn;
+    }
+  }
+  kmx = cl_block_max_u64(kmx, sm);
+  kmn = ~cl_block_max_u64(~kmn, sm);
+  unsigned int cnt_b = h->cnt_b;
+  unsigned long long mass_b = h->mass_b;
+  unsigned long long pfx;
+  int shift;
+  if (kmx == kmn) {
+    pfx = kmx;
+    shift = 0;
+  } else {
+    int hi = 63 - __clzll((long long)(kmx ^ kmn));
+    pfx = (hi == 63) ? 0ull : (kmx >> (hi + 1));
+    while (true) {
+      const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
+      const int lo = hi + 1 - width;
+      cl_clear(sm);
+      for (int i = tid; i < n; i += 1024) {
+        const double v = s[i];
+        if (lb.digit(v) != d1) continue;
+        const unsigned long long key = order_key(v);
+        if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
+          const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
+          atomicAdd(&sm.cnt[bkt], 1u);
+          atomicAdd(&sm.mass[bkt], mass_of(v, lb.M, a.mass_shift));
+        }
+      }
+      const int bstar = cl_boundary<1024, false>(sm, 1, 0, above, tgt, cnt_b, mass_b);
+      pfx = (pfx << width) | (unsigned long long)bstar;
+      if (cnt_b <= 1 || lo == 0) { shift = lo; break; }
+      hi = lo - 1;
+    }
+  }
+  if (tid == 0) {
+    h->pfx = pfx;
+    h->shift = shift;
+    h->cnt_t = cnt_b;
+    h->need = need_of(cnt_b, mass_b, tgt, above);
+    h->mode = kWideDone;
+  }
+}
+
+// Keeps (definite and tie) of each chunk.
+__global__ void __launch_bounds__(kWideThreads) wide_count_kernel(SelectArgs a, int nch) {
+  __shared__ unsigned int red[kWideThreads / 32];
+  const int64_t qh = blockIdx.x / nch;
+  const int c = (int)(blockIdx.x % nch);
+  WideHead* h = wide_head(a, qh);
+  if (h->mode == kWideSkip) return;
+  const int i0 = c * kWideChunk;
+  const int i1 = min(h->n, i0 + kWideChunk);
+  const LinBuckets lb = wide_buckets(h);
+  const Cutoff cut = wide_cutoff(h);
+  const double* s = a.cand_score + qh * a.C1;
+  unsigned int nd = 0u, nt = 0u;
+#pragma unroll 4
+  for (int i = i0 + threadIdx.x; i < i1; i += kWideThreads) {
+    const int k = classify(cut, lb, s[i]);
+    nd += k == 1;
+    nt += k == 2;
+  }
+  nd = wide_sum<unsigned int, kWideThreads>(nd, red);
+  nt = wide_sum<unsigned int, kWideThreads>(nt, red);
+  if (threadIdx.x == 0) { h->chunk_def[c] = nd; h->chunk_tie[c] = nt; }
+}
+
+// Ordered write: warp w of chunk c's CTA owns a contiguous slice of the chunk.
+__global__ void __launch_bounds__(kWideThreads) wide_write_kernel(SelectArgs a, int nch) {
+  __shared__ unsigned int wdef[kWideThreads / 32], wtie[kWideThreads / 32];
+  __shared__ unsigned long long s_keep_before, s_tie_before, s_total;
+  const int64_t qh = blockIdx.x / nch;
+  const int c = (int)(blockIdx.x % nch);
+  const WideHead* h = wide_head(a, qh);
+  if (h->mode == kWideSkip) return;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int W = kWideThreads / 32;
+  const unsigned int lt = (1u << lane) - 1u;
+  const Cutoff cut = wide_cutoff(h);
+  const bool partial = cut.shift != 64 && cut.cnt_t > 1 && cut.need < cut.cnt_t;
+  // keeps and ties of the chunks before this one (and, in chunk 0, of all of them)
+  if (tid == 0) {
+    unsigned long long keep = 0, ties = 0, keep_c = 0, ties_c = 0;
+    for (int x = 0; x < nch; ++x) {
+      if (x == c) { keep_c = keep; ties_c = ties; }
+      const unsigned long long t = h->chunk_tie[x];
+      unsigned long long take = t;
+      if (partial) {
+        const long long r = (long long)cut.need - (long long)ties;
+        take = r <= 0 ? 0ull : ((unsigned long long)r < t ? (unsigned long long)r : t);
+      }
+      keep += h->chunk_def[x] + take;
+      ties += t;
+    }
+    s_keep_before = keep_c;
+    s_tie_before = ties_c;
+    s_total = keep;
+  }
+  const int i0 = c * kWideChunk;
+  const int i1 = min(h->n, i0 + kWideChunk);
+  const int len = i1 > i0 ? i1 - i0 : 0;
+  const LinBuckets lb = wide_buckets(h);
+  const double* s = a.cand_score + qh * a.C1;
+  const int* ids = a.cand_ids + qh * a.C1;
+  const int C = ((len + W - 1) / W + 31) & ~31;
+  const int c0 = i0 + (warp * C < len ? warp * C : len);
+  const int c1 = i0 + (warp * C + C < len ? warp * C + C : len);
+  unsigned int nd = 0, nt = 0;
+  for (int b0 = c0; b0 < c1; b0 += 32) {
+    const int i = b0 + lane;
+    const int k = i < c1 ? classify(cut, lb, s[i]) : 0;
+    nd += __popc(__ballot_sync(0xffffffffu, k == 1));
+    nt += __popc(__ballot_sync(0xffffffffu, k == 2));
+  }
+  if (lane == 0) { wdef[warp] = nd; wtie[warp] = nt; }
+  __syncthreads();
+  unsigned long long tie_before = s_tie_before, keep_before = s_keep_before;
+  for (int w = 0; w < warp; ++w) {
+    const unsigned long long t = wtie[w];
+    unsigned long long take = t;
+    if (partial) {
+      const long long r = (long long)cut.need - (long long)tie_before;
+      take = r <= 0 ? 0ull : ((unsigned long long)r < t ? (unsigned long long)r : t);
+    }
+    keep_before += wdef[w] + take;
+    tie_before += t;
+  }
+  long long take = nt;                                   // ties this warp keeps
+  if (partial) {
+    const long long r = (long long)cut.need - (long long)tie_before;
+    take = r <= 0 ? 0 : (r < (long long)nt ? r : (long long)nt);
+  }
+  unsigned int pos = (unsigned int)keep_before, ties = 0;
+  bool overflow = false;
+  for (int b0 = c0; b0 < c1; b0 += 32) {
+    const int i = b0 + lane;
+    const int k = i < c1 ? classify(cut, lb, s[i]) : 0;
+    const unsigned int tb = __ballot_sync(0xffffffffu, k == 2);
+    const bool keep = k == 1 || (k == 2 && (long long)(ties + __popc(tb & lt)) < take);
+    ties += __popc(tb);
+    const unsigned int kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) emit_kept(a, qh, ids, i, pos + __popc(kb & lt), overflow);
+    pos += __popc(kb);
+  }
+  if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
+  if (c == 0 && tid == 0) {
+    const unsigned long long written = s_total;
+    a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
+    int* lc = level_counts(a, qh);
+    if (lc) { lc[0] = h->n; lc[1] = (int)written; }
+  }
+}
+
+static cudaError_t launch_select_wide(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
+  const int nch = (int)((ncap + kWideChunk - 1) / kWideChunk);
+  const unsigned g1 = (unsigned)nqh, gc = (unsigned)(nqh * nch);
+  const size_t sort_smem = (size_t)kWideMembers * (2 * sizeof(unsigned long long) + sizeof(int));
+  cudaError_t e = cudaFuncSetAttribute(wide_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)sort_smem);
+  if (e != cudaSuccess) return e;
+  wide_init_kernel<<<g1, kWideThreads, 0, s>>>(se);
+  wide_minmax_kernel<<<gc, kWideThreads, 0, s>>>(se, nch);
+  wide_hist_kernel<<<gc, kWideThreads, 0, s>>>(se, nch);
+  wide_boundary_kernel<<<g1, 1024, 0, s>>>(se);
+  wide_gather_kernel<<<gc, kWideThreads, 0, s>>>(se, nch);
+  wide_resolve_kernel<<<g1, 1024, sort_smem, s>>>(se);
+  wide_count_kernel<<<gc, kWideThreads, 0, s>>>(se, nch);
+  wide_write_kernel<<<gc, kWideThreads, 0, s>>>(se, nch);
+  count_launch(7);                                       // with the caller's count: 8
+  return cudaGetLastError();
+}
+
 static int grid_for(int64_t work, int per_sm) {
   int64_t cap = 148ll * per_sm;
   return (int)(work < cap ? (work < 1 ? 1 : work) : cap);
@@ -1431,7 +1894,8 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
 //   cta256   a CTA of 256 threads per head (30 or 48 KiB)         ncap <= 2560 or 4096
 //   cta1024  a CTA of 1024 threads per head (198 KiB)             ncap <= 16896
 //   cluster  2 / 4 / 8 CTAs of 1024 threads per head              ncap <= 8 * 16896
-//   stream   8 CTAs of 512 threads re-reading the scores          above
+//   wide     a chain of grid-wide kernels over (head, chunk)      above
+//   stream   8 CTAs of 512 threads re-reading the scores          (beyond the wide chain's limits)
 // The widest kernel whose resident heads (148 SMs x CTAs per SM) cover every head of the
 // level runs them in one wave at the lowest latency per head; when none does, the
 // narrowest one that holds ncap takes the most heads at once.
@@ -1469,6 +1933,8 @@ static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap
     return launch_cluster(route_select_block_kernel<1024, kCta1024Cap, true>, se, nqh < per ? nqh : per, cs,
                           1024, kCta1024Cap * (sizeof(double) + sizeof(int)), s);
   }
+  if ((ncap + kWideChunk - 1) / kWideChunk <= kWideMaxChunks && se.C1 * 8 >= (int64_t)sizeof(WideHead))
+    return launch_select_wide(se, nqh, ncap, s);
   const int64_t per = (2 * 148) / kStreamCta;
   return launch_cluster(route_select_stream_kernel<512>, se, nqh < per ? nqh : per, kStreamCta, 512, 0, s);
 }

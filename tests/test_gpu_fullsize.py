@@ -208,3 +208,51 @@ def test_flat_index_full(Z, name, units, heads):
                 assert np.abs(s[diff] - boundary).max() <= 1e-4 or sel.margin < 1e-4, (b, h, len(diff))
     assert exact >= total // 2
     print(f"{name} flat: {exact} exact of {total} heads")
+
+
+@pytest.mark.parametrize("tie", [False, True])
+def test_flat_index_wide(Z, tie):
+    """The flat indexer over 8.7 M keys of one KV head: ~136 K candidate chunks per query
+    head, beyond what the clusters hold in shared memory, so the select runs as the chain
+    of grid-wide kernels over (head, chunk).  With tied chunks (period 5) every score comes
+    in groups of ~27 K equal values spread over all chunks and the boundary falls inside a
+    group: the lowest ids of the group must be kept, exactly as the oracle keeps them."""
+    w = S.scaled(S.workload("deep-tree-16m"), T=8_700_000 + 37, B=1)
+    g = geometry(w)
+    p = w.p[0]
+    C, K, V = S.clustered_kv(w, DEV)
+    q = S.queries(w, C, 1, DEV)
+    del C
+    if tie:
+        n = w.T // 64
+        src = torch.arange(n, device=DEV) % 5
+        Kv = K[:, :, :n * 64].view(K.shape[0], K.shape[1], n, 64, K.shape[-1])
+        Kv.copy_(Kv[:, :, src].clone())
+    t = w.T - 1
+    pos = torch.full((w.B, 1), t, dtype=torch.int64, device=DEV)
+    cap = Z.leaf_cap(g)
+    assert cap > 8 * 16896                             # beyond the cluster selects
+    ids = torch.full((w.B, 1, w.Hq, cap), -1, dtype=torch.int32, device=DEV)
+    cnt = torch.zeros(w.B, 1, w.Hq, dtype=torch.int32, device=DEV)
+    O = torch.empty(w.B, 1, w.Hq, w.d, dtype=g.dtype, device=DEV)
+    ws = Z.empty_workspace(g, 1, Z.ZHA_OP_FLAT, DEV)
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    Z.zha_flat_index(g, q, K, V, pos, p, ids, cnt, O, ws, st)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    qc = q.double().cpu().numpy()
+    Kc = K[0, 0].cpu()
+    del V, ws
+    exact = 0
+    for h in (0, 5):
+        sel = zo.flat_select(qc[0, 0, h], Kc, t, p)
+        got = ids[0, 0, h, :int(cnt[0, 0, h])].cpu().numpy()
+        diff = np.setxor1d(sel.ids, got)
+        if tie:
+            assert len(diff) == 0, (h, len(diff), len(sel.ids), len(got))
+        elif len(diff):
+            s = zo.flat_scores(qc[0, 0, h], Kc, t)
+            boundary = np.sort(s)[::-1][sel.m - 1]
+            assert np.abs(s[diff] - boundary).max() <= 1e-4 or sel.margin < 1e-4, (h, len(diff))
+        exact += len(diff) == 0
+    print(f"flat wide (tie={tie}): {exact} exact of 2 heads, {int(cnt[0, 0, 0])} chunks kept of {t // 64}")
