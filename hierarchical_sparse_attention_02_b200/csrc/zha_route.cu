@@ -1643,28 +1643,51 @@ __global__ void __launch_bounds__(1024) wide_resolve_kernel(SelectArgs a) {
         __syncthreads();
       }
     }
-    // the first member (in order) whose cumulative mass from `above` reaches tgt
+    // the first member (in order) whose cumulative mass from `above` reaches tgt: a block
+    // scan of the sorted masses, thread t owning the consecutive members [4t, 4t + 4)
+    __shared__ int s_cidx;
+    __shared__ unsigned int s_cnt, s_need;
+    constexpr int kPerT = kWideMembers / 1024;
+    unsigned long long loc[kPerT], lsum = 0;
+#pragma unroll
+    for (int q = 0; q < kPerT; ++q) {
+      const int i = tid * kPerT + q;
+      loc[q] = i < m ? ms[i] : 0ull;
+      lsum += loc[q];
+    }
+    if (tid == 0) { s_cidx = m - 1; s_cnt = 0u; s_need = 0u; }
+    unsigned long long x = lsum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const unsigned long long y = __shfl_up_sync(0xffffffffu, x, o);
+      if ((tid & 31) >= o) x += y;
+    }
+    if ((tid & 31) == 31) sm.wsum[tid >> 5] = x;
+    __syncthreads();
+    unsigned long long acc = above + x - lsum;
+    for (int w = 0; w < (tid >> 5); ++w) acc += sm.wsum[w];
+#pragma unroll
+    for (int q = 0; q < kPerT; ++q) {
+      const int i = tid * kPerT + q;
+      acc += loc[q];
+      if (i < m && acc >= tgt) { atomicMin(&s_cidx, i); break; }
+    }
+    __syncthreads();
+    const unsigned long long kc = key[s_cidx];
+    const int pc = pos[s_cidx];
+    unsigned int ct = 0, nd = 0;
+#pragma unroll
+    for (int q = 0; q < kPerT; ++q) {
+      const int i = tid * kPerT + q;
+      if (i < m && key[i] == kc) { ++ct; nd += pos[i] <= pc; }
+    }
+    if (ct) { atomicAdd(&s_cnt, ct); atomicAdd(&s_need, nd); }
+    __syncthreads();
     if (tid == 0) {
-      unsigned long long acc = above;
-      int cidx = m - 1;
-      for (int i = 0; i < m; ++i) {
-        acc += ms[i];
-        if (acc >= tgt) { cidx = i; break; }
-      }
-      const unsigned long long kc = key[cidx];
-      const int pc = pos[cidx];
-      unsigned int cnt_t = 0;
-      unsigned long long need = 0;
-      for (int i = 0; i < m; ++i) {
-        if (key[i] == kc) {
-          ++cnt_t;
-          need += pos[i] <= pc;
-        }
-      }
       h->pfx = kc;
       h->shift = 0;
-      h->cnt_t = cnt_t;
-      h->need = need;
+      h->cnt_t = s_cnt;
+      h->need = s_need;
       h->mode = kWideDone;
     }
     return;
@@ -1761,23 +1784,38 @@ __global__ void __launch_bounds__(kWideThreads) wide_write_kernel(SelectArgs a, 
   const unsigned int lt = (1u << lane) - 1u;
   const Cutoff cut = wide_cutoff(h);
   const bool partial = cut.shift != 64 && cut.cnt_t > 1 && cut.need < cut.cnt_t;
-  // keeps and ties of the chunks before this one (and, in chunk 0, of all of them)
-  if (tid == 0) {
-    unsigned long long keep = 0, ties = 0, keep_c = 0, ties_c = 0;
-    for (int x = 0; x < nch; ++x) {
-      if (x == c) { keep_c = keep; ties_c = ties; }
-      const unsigned long long t = h->chunk_tie[x];
+  // keeps and ties of the chunks before this one, and of all of them: warp 0 scans the
+  // chunks' counts 32 at a time
+  if (warp == 0) {
+    unsigned long long keep_run = 0, tie_run = 0;
+    for (int base = 0; base < nch; base += 32) {
+      const int x = base + lane;
+      const unsigned long long t = x < nch ? h->chunk_tie[x] : 0ull;
+      const unsigned long long dd = x < nch ? h->chunk_def[x] : 0ull;
+      unsigned long long tin = t;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, tin, o);
+        if (lane >= o) tin += y;
+      }
+      const unsigned long long tie_before_x = tie_run + tin - t;
       unsigned long long take = t;
       if (partial) {
-        const long long r = (long long)cut.need - (long long)ties;
+        const long long r = (long long)cut.need - (long long)tie_before_x;
         take = r <= 0 ? 0ull : ((unsigned long long)r < t ? (unsigned long long)r : t);
       }
-      keep += h->chunk_def[x] + take;
-      ties += t;
+      const unsigned long long k = dd + take;
+      unsigned long long kin = k;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const unsigned long long y = __shfl_up_sync(0xffffffffu, kin, o);
+        if (lane >= o) kin += y;
+      }
+      if (x == c) { s_keep_before = keep_run + kin - k; s_tie_before = tie_before_x; }
+      keep_run += __shfl_sync(0xffffffffu, kin, 31);
+      tie_run += __shfl_sync(0xffffffffu, tin, 31);
     }
-    s_keep_before = keep_c;
-    s_tie_before = ties_c;
-    s_total = keep;
+    if (lane == 0) s_total = keep_run;
   }
   const int i0 = c * kWideChunk;
   const int i1 = min(h->n, i0 + kWideChunk);
