@@ -764,13 +764,10 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
 // cluster select: one thread-block cluster (1..8 CTAs of T threads) per query head.  The
 // cluster's rank-0 CTA sums the per-CTA maxima, totals and histograms through distributed
 // shared memory and publishes every decision back into each CTA, so all CTAs take
-// identical decisions.  Cluster barriers are hardware barriers (no spin loops).  The
-// streaming kernel re-reads the scores (and the masses it stored) in every pass, for
-// frontiers beyond what the register-resident kernel holds.
+// identical decisions.  Cluster barriers are hardware barriers (no spin loops).
 // ---------------------------------------------------------------------------
 
 constexpr int kClMaxCta = 8;
-constexpr int kStreamCta = 8;
 
 template <int T>
 struct ClSmem {
@@ -848,27 +845,6 @@ __device__ __forceinline__ unsigned long long cl_block_sum(unsigned long long v,
   return r;
 }
 
-template <int T>
-__device__ __forceinline__ unsigned int cl_excl_scan(unsigned int v, ClSmem<T>& sm, unsigned int* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  unsigned int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  __syncthreads();
-  if (lane == 31) sm.wcnt[warp] = x;
-  __syncthreads();
-  unsigned int before = 0, all = 0;
-  for (int i = 0; i < T / 32; ++i) {
-    if (i < warp) before += sm.wcnt[i];
-    all += sm.wcnt[i];
-  }
-  *total = all;
-  return before + x - v;
-}
-
 // Cluster-wide boundary of the histograms every CTA has just filled: rank 0 sums them in
 // rank order, finds the bucket where the cumulative mass from the top (starting at
 // `above`) reaches tgt and publishes (bucket, mass above it, its count and mass) to every
@@ -938,220 +914,6 @@ template <int T>
 __device__ __forceinline__ void cl_clear(ClSmem<T>& sm) {
   for (int i = threadIdx.x; i < kBuckets; i += T) { sm.cnt[i] = 0; sm.mass[i] = 0; }
   __syncthreads();
-}
-
-template <int T>
-__global__ void __launch_bounds__(T, 1) route_select_stream_kernel(SelectArgs a) {
-  constexpr bool CLK = true;
-  __shared__ ClSmem<T> sm;
-  namespace cg = cooperative_groups;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int CS = (int)cluster.num_blocks();
-  const int cr = (int)cluster.block_rank();
-  ClSmem<T>* lead = cluster.map_shared_rank(&sm, 0);
-  const RouteGeom& g = a.g;
-  const int tid = threadIdx.x;
-  const int64_t nqh = (int64_t)g.B * g.nq * g.Hq;
-  const int64_t nclusters = gridDim.x / CS;
-  for (int64_t qh = blockIdx.x / CS; qh < nqh; qh += nclusters) {
-    const int n = head_candidates(a, qh, cr == 0 && tid == 0);
-    if (n < 0) continue;                                 // uniform over the cluster
-    int* lc = level_counts(a, qh);
-    const double* s = a.cand_score + qh * a.C1;
-    const int* ids = a.cand_ids + qh * a.C1;
-    unsigned long long* E = a.cand_mass + qh * a.C1;
-    const int chunk = (n + CS - 1) / CS;
-    const int r0 = cr * chunk < n ? cr * chunk : n;
-    const int r1 = r0 + chunk < n ? r0 + chunk : n;
-    // every pass walks the CTA's slice 8 candidates per thread at a time, loads first
-#define CL_BATCH(LOADS, BODY)                                                       \
-    for (int base_ = r0; base_ < r1; base_ += T * 8) {                              \
-      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
-        const int i = base_ + u_ * T + tid;                                         \
-        LOADS                                                                       \
-      }                                                                             \
-      _Pragma("unroll") for (int u_ = 0; u_ < 8; ++u_) {                            \
-        const int i = base_ + u_ * T + tid;                                         \
-        if (i < r1) { BODY }                                                        \
-      }                                                                             \
-    }
-    double sv[8];
-    unsigned long long ev[8];
-
-    // 1. maximum and minimum over the cluster
-    double mx = -INFINITY, mn = INFINITY;
-    CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; }, { mx = fmax(mx, sv[u_]); mn = fmin(mn, sv[u_]); })
-    mx = cl_block_max(mx, sm);
-    mn = -cl_block_max(-mn, sm);
-    if (tid == 0) {
-      lead->slot_kmax[cr] = r1 > r0 ? order_key(mx) : 0ull;
-      lead->slot_kmin[cr] = r1 > r0 ? order_key(mn) : ~0ull;
-    }
-    cl_clear(sm);
-    cluster.sync();
-    unsigned long long kmax = 0, kmin = ~0ull;
-    for (int r = 0; r < CS; ++r) {
-      const unsigned long long x = lead->slot_kmax[r], y = lead->slot_kmin[r];
-      kmax = x > kmax ? x : kmax;
-      kmin = y < kmin ? y : kmin;
-    }
-    // back from the order key to the score
-    const double M = __longlong_as_double((long long)((kmax >> 63) ? (kmax & 0x7fffffffffffffffull) : ~kmax));
-    const double Mn = __longlong_as_double((long long)((kmin >> 63) ? (kmin & 0x7fffffffffffffffull) : ~kmin));
-    // 2. masses, their total and the linear histogram
-    LinBuckets lb;
-    lb.init(M, Mn, kBuckets);
-    unsigned long long z = 0;
-    CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; }, {
-      const unsigned long long e = __double2ull_rn(ldexp(exp(sv[u_] - M), a.mass_shift));
-      E[i] = e;
-      z += e;
-      const int d = lb.digit(sv[u_]);
-      atomicAdd(&sm.cnt[d], 1u);
-      atomicAdd(&sm.mass[d], e);
-    })
-    z = cl_block_sum(z, sm);
-    if (tid == 0) lead->slot_z[cr] = z;
-    cluster.sync();
-    unsigned long long Z = 0;
-    for (int r = 0; r < CS; ++r) Z += lead->slot_z[r];
-
-    // 3. the cutoff, with identical decisions in every CTA
-    Cutoff c{};
-    c.keep_all = a.p >= 1.0 || n == 0;
-    c.shift = 64;
-    if (!c.keep_all) {
-      const unsigned long long tgt = target_of(a.p, Z);
-      unsigned long long above = 0, mass_b = 0;
-      unsigned int cnt_b = 0;
-      c.d1 = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
-      if (cnt_b > 1) {
-        // key range of the boundary bucket over the cluster
-        unsigned long long kmx = 0, kmn = ~0ull;
-        CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; }, {
-          if (lb.digit(sv[u_]) == c.d1) {
-            const unsigned long long k = order_key(sv[u_]);
-            kmx = k > kmx ? k : kmx;
-            kmn = k < kmn ? k : kmn;
-          }
-        })
-        kmx = cl_block_max_u64(kmx, sm);
-        kmn = ~cl_block_max_u64(~kmn, sm);
-        if (tid == 0) { lead->slot_kmax[cr] = kmx; lead->slot_kmin[cr] = kmn; }
-        cl_clear(sm);
-        cluster.sync();
-        kmx = 0;
-        kmn = ~0ull;
-        for (int r = 0; r < CS; ++r) {
-          const unsigned long long x = lead->slot_kmax[r], y = lead->slot_kmin[r];
-          kmx = x > kmx ? x : kmx;
-          kmn = y < kmn ? y : kmn;
-        }
-        if (kmx == kmn) {
-          c.pfx = kmx;
-          c.shift = 0;
-        } else {
-          int hi = 63 - __clzll((long long)(kmx ^ kmn));
-          unsigned long long pfx = (hi == 63) ? 0ull : (kmx >> (hi + 1));
-          while (true) {
-            const int width = (hi + 1) < kDigit ? (hi + 1) : kDigit;
-            const int lo = hi + 1 - width;
-            CL_BATCH({ sv[u_] = i < r1 ? s[i] : 0.0; ev[u_] = i < r1 ? E[i] : 0ull; }, {
-              if (lb.digit(sv[u_]) == c.d1) {
-                const unsigned long long key = order_key(sv[u_]);
-                if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
-                  const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
-                  atomicAdd(&sm.cnt[bkt], 1u);
-                  atomicAdd(&sm.mass[bkt], ev[u_]);
-                }
-              }
-            })
-            const int bstar = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
-            pfx = (pfx << width) | (unsigned long long)bstar;
-            if (cnt_b <= 1 || lo == 0) { c.shift = lo; break; }
-            cl_clear(sm);                                // rank 0 is done reading (cl_boundary)
-            hi = lo - 1;
-          }
-          c.pfx = pfx;
-        }
-        c.cnt_t = cnt_b;
-        c.need = need_of(cnt_b, mass_b, tgt, above);
-      }
-    }
-
-    // 4. ordered compaction: thread t of CTA r owns a contiguous piece of the CTA's slice
-    //    (flags of its first 64 candidates kept as bit masks)
-    const int len = r1 - r0;
-    const int per = (len + T - 1) / T;
-    const int i0 = r0 + tid * per < r1 ? r0 + tid * per : r1;
-    const int i1 = i0 + per < r1 ? i0 + per : r1;
-    unsigned long long defm = 0, tiem = 0;
-    unsigned int ndef = 0, ntie = 0;
-#pragma unroll 8
-    for (int i = i0; i < i1; ++i) {
-      const int k = classify(c, lb, s[i]);
-      const int j = i - i0;
-      ndef += k == 1;
-      ntie += k == 2;
-      if (j < 64) {
-        defm |= (unsigned long long)(k == 1) << j;
-        tiem |= (unsigned long long)(k == 2) << j;
-      }
-    }
-    const bool partial = c.shift != 64 && c.cnt_t > 1 && c.need < c.cnt_t;
-    long long take = ntie;                               // ties this thread keeps
-    unsigned int tie_before = 0;
-    if (partial) {
-      unsigned int tie_cta;
-      tie_before = cl_excl_scan(ntie, sm, &tie_cta);
-      if (tid == 0) lead->slot_tie[cr] = tie_cta;
-      cluster.sync();
-      for (int r = 0; r < cr; ++r) tie_before += lead->slot_tie[r];
-      take = (long long)c.need - (long long)tie_before;
-      take = take < 0 ? 0 : (take > (long long)ntie ? (long long)ntie : take);
-    }
-    unsigned int keep_cta;
-    unsigned int pos = cl_excl_scan(ndef + (unsigned int)take, sm, &keep_cta);
-    if (tid == 0) lead->slot_keep[cr] = keep_cta;
-    cluster.sync();
-    unsigned int written = 0;
-    for (int r = 0; r < CS; ++r) {
-      const unsigned int k = lead->slot_keep[r];
-      if (r < cr) pos += k;
-      written += k;
-    }
-    int* outp = a.out_ids + qh * a.out_stride;
-    bool overflow = false;
-    auto emit = [&](int i) {
-      const int id = ids[i];
-      if ((int64_t)pos < a.out_cap) outp[pos] = id;
-      else overflow = true;
-      if (a.level_ids && a.level >= 2 && (int64_t)pos < a.level_ids_cap)
-        a.level_ids[qh * a.level_ids_stride + a.level_ids_off + pos] = id;
-      ++pos;
-    };
-    if (per <= 64) {
-      unsigned long long keepm = defm | lowest_bits(tiem, take);
-      while (keepm) {
-        const int j = __ffsll((long long)keepm) - 1;
-        keepm &= keepm - 1;
-        emit(i0 + j);
-      }
-    } else {
-      long long left = take;
-      for (int i = i0; i < i1; ++i) {
-        const int k = classify(c, lb, s[i]);
-        if (k == 1 || (k == 2 && left-- > 0)) emit(i);
-      }
-    }
-    if (overflow) set_status(a.dev_status, ZHA_ERR_CAPACITY);
-    if (cr == 0 && tid == 0) {
-      a.out_cnt[qh] = (int64_t)written < a.out_cap ? (int)written : a.out_cap;
-      if (lc) { lc[0] = n; lc[1] = (int)written; }
-    }
-    cluster.sync();                                      // slots and smem reused by the next head
-  }
-#undef CL_BATCH
 }
 
 // Shared-memory-resident cluster select: CTA r of the cluster holds the contiguous slice
@@ -1405,7 +1167,6 @@ __global__ void __launch_bounds__(T) route_select_block_kernel(SelectArgs a) {
 constexpr int kWideChunk = 4096;
 constexpr int kWideThreads = 256;                 // 16 candidates per thread
 constexpr int kWideMembers = 4096;
-constexpr int kWideMaxChunks = 1024;
 
 enum : int { kWideSkip = -1, kWideDone = 0, kWideAll = 1, kWideGather = 2, kWideRadix = 3 };
 
@@ -1415,10 +1176,14 @@ struct WideHead {
   int mode, d1, shift, n, pad;
   unsigned int cnt[kBuckets];
   unsigned long long mass[kBuckets];
-  unsigned int chunk_def[kWideMaxChunks], chunk_tie[kWideMaxChunks];
   int m_pos[kWideMembers];
   unsigned long long m_key[kWideMembers], m_mass[kWideMembers];
+  // followed by the chunks' keep counts: [nch] definite, then [nch] ties
 };
+
+__device__ __forceinline__ unsigned int* wide_chunks(const WideHead* h) {
+  return reinterpret_cast<unsigned int*>(const_cast<WideHead*>(h) + 1);
+}
 
 __device__ __forceinline__ WideHead* wide_head(const SelectArgs& a, int64_t qh) {
   return reinterpret_cast<WideHead*>(a.cand_mass + qh * a.C1);
@@ -1459,7 +1224,7 @@ __device__ __forceinline__ V wide_sum(V v, V* scratch) {
   return r;
 }
 
-__global__ void __launch_bounds__(kWideThreads) wide_init_kernel(SelectArgs a) {
+__global__ void __launch_bounds__(kWideThreads) wide_init_kernel(SelectArgs a, int nch) {
   const int64_t qh = blockIdx.x;
   WideHead* h = wide_head(a, qh);
   const int n = head_candidates(a, qh, threadIdx.x == 0);
@@ -1474,7 +1239,7 @@ __global__ void __launch_bounds__(kWideThreads) wide_init_kernel(SelectArgs a) {
   }
   if (n < 0) return;
   for (int i = threadIdx.x; i < kBuckets; i += kWideThreads) { h->cnt[i] = 0u; h->mass[i] = 0ull; }
-  for (int i = threadIdx.x; i < kWideMaxChunks; i += kWideThreads) { h->chunk_def[i] = 0u; h->chunk_tie[i] = 0u; }
+  for (int i = threadIdx.x; i < 2 * nch; i += kWideThreads) wide_chunks(h)[i] = 0u;
 }
 
 __global__ void __launch_bounds__(kWideThreads) wide_minmax_kernel(SelectArgs a, int nch) {
@@ -1768,7 +1533,7 @@ __global__ void __launch_bounds__(kWideThreads) wide_count_kernel(SelectArgs a, 
   }
   nd = wide_sum<unsigned int, kWideThreads>(nd, red);
   nt = wide_sum<unsigned int, kWideThreads>(nt, red);
-  if (threadIdx.x == 0) { h->chunk_def[c] = nd; h->chunk_tie[c] = nt; }
+  if (threadIdx.x == 0) { wide_chunks(h)[c] = nd; wide_chunks(h)[nch + c] = nt; }
 }
 
 // Ordered write: warp w of chunk c's CTA owns a contiguous slice of the chunk.
@@ -1790,8 +1555,8 @@ __global__ void __launch_bounds__(kWideThreads) wide_write_kernel(SelectArgs a, 
     unsigned long long keep_run = 0, tie_run = 0;
     for (int base = 0; base < nch; base += 32) {
       const int x = base + lane;
-      const unsigned long long t = x < nch ? h->chunk_tie[x] : 0ull;
-      const unsigned long long dd = x < nch ? h->chunk_def[x] : 0ull;
+      const unsigned long long t = x < nch ? wide_chunks(h)[nch + x] : 0ull;
+      const unsigned long long dd = x < nch ? wide_chunks(h)[x] : 0ull;
       unsigned long long tin = t;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -1879,7 +1644,8 @@ static cudaError_t launch_select_wide(const SelectArgs& se, int64_t nqh, int64_t
   cudaError_t e = cudaFuncSetAttribute(wide_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)sort_smem);
   if (e != cudaSuccess) return e;
-  wide_init_kernel<<<g1, kWideThreads, 0, s>>>(se);
+  if (se.C1 * 8 < (int64_t)(sizeof(WideHead) + 8 * (size_t)nch)) return cudaErrorInvalidValue;   // C1 > 135168
+  wide_init_kernel<<<g1, kWideThreads, 0, s>>>(se, nch);
   wide_minmax_kernel<<<gc, kWideThreads, 0, s>>>(se, nch);
   wide_hist_kernel<<<gc, kWideThreads, 0, s>>>(se, nch);
   wide_boundary_kernel<<<g1, 1024, 0, s>>>(se);
@@ -1933,13 +1699,12 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
 //   cta1024  a CTA of 1024 threads per head (198 KiB)             ncap <= 16896
 //   cluster  2 / 4 / 8 CTAs of 1024 threads per head              ncap <= 8 * 16896
 //   wide     a chain of grid-wide kernels over (head, chunk)      above
-//   stream   8 CTAs of 512 threads re-reading the scores          (beyond the wide chain's limits)
 // The widest kernel whose resident heads (148 SMs x CTAs per SM) cover every head of the
 // level runs them in one wave at the lowest latency per head; when none does, the
 // narrowest one that holds ncap takes the most heads at once.
 static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
   const int64_t res_warp = 148ll * 3 * kWarpSelWarps, res256 = 148ll * 3, res1024 = 148;
-  int kind;                                            // 0 warp, 1 cta256, 2 cta1024, 3 cluster, 4 stream
+  int kind;                                            // 0 warp, 1 cta256, 2 cta1024, 3 cluster, 4 wide
   if (ncap <= kCta1024Cap && nqh <= res1024) kind = 2;
   else if (ncap <= 4096 && nqh <= res256) kind = 1;
   else if (ncap <= kWarpCap) kind = 0;
@@ -1971,10 +1736,7 @@ static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap
     return launch_cluster(route_select_block_kernel<1024, kCta1024Cap, true>, se, nqh < per ? nqh : per, cs,
                           1024, kCta1024Cap * (sizeof(double) + sizeof(int)), s);
   }
-  if ((ncap + kWideChunk - 1) / kWideChunk <= kWideMaxChunks && se.C1 * 8 >= (int64_t)sizeof(WideHead))
-    return launch_select_wide(se, nqh, ncap, s);
-  const int64_t per = (2 * 148) / kStreamCta;
-  return launch_cluster(route_select_stream_kernel<512>, se, nqh < per ? nqh : per, kStreamCta, 512, 0, s);
+  return launch_select_wide(se, nqh, ncap, s);
 }
 
 // ---------------------------------------------------------------------------
