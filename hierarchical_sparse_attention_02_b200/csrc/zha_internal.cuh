@@ -68,9 +68,12 @@ inline TreeLayout tree_layout(const zha_geom& g) {
 // Split size (chunks per attention work item) chosen from the geometry only, so that
 // the workspace bound is known on the host: about 4K items per call (a few dozen per
 // SM), >= 16 chunks each.
+#ifndef ZHA_SPLIT_ITEMS
+#define ZHA_SPLIT_ITEMS 4096                     // target number of attention work items
+#endif
 inline int64_t chunks_per_split(int64_t units, int64_t c1) {
   const int64_t total = units * (c1 + 2);
-  int64_t cps = (total + 4095) / 4096;
+  int64_t cps = (total + ZHA_SPLIT_ITEMS - 1) / ZHA_SPLIT_ITEMS;
   return cps < 16 ? 16 : cps;
 }
 

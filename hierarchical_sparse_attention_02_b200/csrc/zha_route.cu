@@ -1703,7 +1703,7 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
 // level runs them in one wave at the lowest latency per head; when none does, the
 // narrowest one that holds ncap takes the most heads at once.
 static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
-  const int64_t res_warp = 148ll * 3 * kWarpSelWarps, res256 = 148ll * 3, res1024 = 148;
+  const int64_t res256 = 148ll * 3, res1024 = 148;
   int kind;                                            // 0 warp, 1 cta256, 2 cta1024, 3 cluster, 4 wide
   if (ncap <= kCta1024Cap && nqh <= res1024) kind = 2;
   else if (ncap <= 4096 && nqh <= res256) kind = 1;
