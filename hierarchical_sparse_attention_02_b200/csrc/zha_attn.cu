@@ -291,100 +291,12 @@ __global__ void __launch_bounds__(256) attn_split_kernel(AttnArgs a) {
 // combine: one CTA of 128 threads per (unit, head); thread <-> dim
 // ---------------------------------------------------------------------------
 
-// Combine of the split partials, in up to two stages.  Stage 1: one CTA per (unit, head,
-// block of kCombBlock consecutive items); 4 groups of 128 threads (thread <-> dim) fold
-// every 4th partial of the block with a running maximum, then merge in a fixed order.  A
-// head with a single block writes O directly; otherwise the block's (o, m, l) replaces its
-// first partial and stage 2 merges the blocks.  Both stages use fixed orders (deterministic).
-constexpr int kCombGroups = 4;
+// Combine of the split partials (log-sum-exp of (o, m, l) per head, fixed orders, so the
+// result is deterministic).  Units of at most kCombBlock items: combine_warp_kernel; larger
+// ones: combine_cta_kernel over blocks of kCtaItems items (one block: the output directly;
+// several: block partials, then combine_cta_blocks_kernel over the blocks).
 constexpr int kCombBlock = 128;
-
-struct Fold {
-  float M, L, acc;
-};
-
-__device__ __forceinline__ void fold_in(Fold& f, float m, float l, float o) {
-  const float Mn = fmaxf(f.M, m);
-  if (Mn == -INFINITY) return;                     // nothing attended yet
-  const float a = exp2f(f.M - Mn), w = exp2f(m - Mn);
-  f.L = fmaf(f.L, a, w * l);
-  f.acc = fmaf(f.acc, a, w * o);
-  f.M = Mn;
-}
-
-// Merges the groups' folds (in group order) into thread (group 0, dim d)'s result.
-__device__ __forceinline__ Fold merge_groups(const Fold& f, float (&gm)[kCombGroups], float (&gl)[kCombGroups],
-                                             float (&gacc)[kCombGroups][kD], int grp, int d) {
-  gacc[grp][d] = f.acc;
-  if (d == 0) { gm[grp] = f.M; gl[grp] = f.L; }
-  __syncthreads();
-  Fold r{-INFINITY, 0.f, 0.f};
-  if (grp == 0) {
-#pragma unroll
-    for (int k = 0; k < kCombGroups; ++k) fold_in(r, gm[k], gl[k], gacc[k][d]);
-  }
-  return r;
-}
-
-template <typename OT>
-__device__ __forceinline__ void write_out(const AttnGeom& g, int64_t u, int h, int d, const Fold& r, OT* O,
-                                          float* lse) {
-  const int64_t bq = u / g.Hkv;
-  const int hk = (int)(u % g.Hkv);
-  const int64_t qh = bq * g.Hq + hk * g.G + h;
-  O[qh * kD + d] = from_f32<OT>(r.L > 0.f ? r.acc / r.L : 0.f);
-  if (lse && d == 0) lse[qh] = r.L > 0.f ? (r.M + log2f(r.L)) * 0.6931471805599453f : -INFINITY;
-}
-
-template <typename OT>
-__global__ void __launch_bounds__(kCombGroups * kD) combine_kernel(AttnGeom g, const int* pair_off, float* partials,
-                                                                   int64_t nb_max, OT* O, float* lse) {
-  __shared__ float gm[kCombGroups], gl[kCombGroups];
-  __shared__ float gacc[kCombGroups][kD];
-  const int64_t uh = blockIdx.x / nb_max;
-  const int64_t blk = blockIdx.x % nb_max;
-  const int64_t u = uh / g.G;
-  const int h = (int)(uh % g.G);
-  const int d = threadIdx.x % kD, grp = threadIdx.x / kD;
-  const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
-  const int64_t b0 = i0 + blk * kCombBlock;
-  if (b0 >= i1 && !(blk == 0)) return;             // uniform over the CTA
-  const int64_t b1 = b0 + kCombBlock < i1 ? b0 + kCombBlock : i1;
-  Fold f{-INFINITY, 0.f, 0.f};
-  for (int64_t i = b0 + grp; i < b1; i += kCombGroups) {
-    const float* P = partials + (i * g.G + h) * kPartStride;
-    fold_in(f, P[kD], P[kD + 1], P[d]);
-  }
-  const Fold r = merge_groups(f, gm, gl, gacc, grp, d);
-  if (grp != 0) return;
-  if (i1 - i0 <= kCombBlock) {
-    write_out(g, u, h, d, r, O, lse);
-  } else {
-    float* P = partials + (b0 * g.G + h) * kPartStride;
-    P[d] = r.acc;
-    if (d == 0) { P[kD] = r.M; P[kD + 1] = r.L; }
-  }
-}
-
-template <typename OT>
-__global__ void __launch_bounds__(kCombGroups * kD) combine_blocks_kernel(AttnGeom g, const int* pair_off,
-                                                                          const float* partials, OT* O, float* lse) {
-  __shared__ float gm[kCombGroups], gl[kCombGroups];
-  __shared__ float gacc[kCombGroups][kD];
-  const int64_t uh = blockIdx.x;
-  const int64_t u = uh / g.G;
-  const int h = (int)(uh % g.G);
-  const int d = threadIdx.x % kD, grp = threadIdx.x / kD;
-  const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
-  if (i1 - i0 <= kCombBlock) return;               // written by the first stage
-  Fold f{-INFINITY, 0.f, 0.f};
-  for (int64_t b0 = i0 + grp * kCombBlock; b0 < i1; b0 += kCombGroups * kCombBlock) {
-    const float* P = partials + (b0 * g.G + h) * kPartStride;
-    fold_in(f, P[kD], P[kD + 1], P[d]);
-  }
-  const Fold r = merge_groups(f, gm, gl, gacc, grp, d);
-  if (grp == 0) write_out(g, u, h, d, r, O, lse);
-}
+constexpr int kCtaItems = 512;
 
 // Combine for units of at most kCombBlock items (the common case): one CTA per unit, warp
 // h <-> head h, lane <-> 4 dims.  Two passes in item order: the maximum M of the partials'
@@ -428,20 +340,24 @@ __global__ void __launch_bounds__(kMaxG * 32) combine_warp_kernel(AttnGeom g, co
   if (lse && lane == 0) lse[qh] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
 }
 
-// Combine for units of up to 4 * kCombBlock items: one CTA of 8 warps per (unit, head);
-// the CTA's maximum M first, then warp w sums the items w, w + 8, ... (lane <-> 4 dims)
-// and the eight warp sums are added in warp order (deterministic, fixed order).
+// One CTA of 8 warps per (unit, head, block of kCtaItems items): the block's maximum M first,
+// then warp w sums the items w, w + 8, ... (lane <-> 4 dims) and the eight warp sums are
+// added in warp order.
 template <typename OT>
-__global__ void __launch_bounds__(256) combine_cta_kernel(AttnGeom g, const int* pair_off, const float* partials,
-                                                        OT* O, float* lse) {
+__global__ void __launch_bounds__(256) combine_cta_kernel(AttnGeom g, const int* pair_off, float* partials,
+                                                        int64_t nbl, OT* O, float* lse) {
   __shared__ float wm[8], wl[8];
   __shared__ float4 wacc[8][32];
-  const int64_t u = blockIdx.x / g.G;
-  const int h = (int)(blockIdx.x % g.G);
+  const int64_t uh = blockIdx.x / nbl, blk = blockIdx.x % nbl;
+  const int64_t u = uh / g.G;
+  const int h = (int)(uh % g.G);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
+  const int64_t b0 = i0 + blk * kCtaItems;
+  if (b0 >= i1 && blk > 0) return;                   // uniform over the CTA
+  const int64_t b1 = b0 + kCtaItems < i1 ? b0 + kCtaItems : i1;
   float M = -INFINITY;
-  for (int64_t i = i0 + tid; i < i1; i += 256) M = fmaxf(M, partials[(i * g.G + h) * kPartStride + kD]);
+  for (int64_t i = b0 + tid; i < b1; i += 256) M = fmaxf(M, partials[(i * g.G + h) * kPartStride + kD]);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   if (lane == 0) wm[warp] = M;
@@ -453,7 +369,7 @@ __global__ void __launch_bounds__(256) combine_cta_kernel(AttnGeom g, const int*
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
   if (M != -INFINITY) {
 #pragma unroll 4
-    for (int64_t i = i0 + warp; i < i1; i += 8) {
+    for (int64_t i = b0 + warp; i < b1; i += 8) {
       const float* P = partials + (i * g.G + h) * kPartStride;
       const float4 o4 = *reinterpret_cast<const float4*>(P + 4 * lane);
       const float w = exp2f(P[kD] - M);
@@ -475,6 +391,54 @@ __global__ void __launch_bounds__(256) combine_cta_kernel(AttnGeom g, const int*
     L += wl[w];
     const float4 a4 = wacc[w][lane];
     acc.x += a4.x; acc.y += a4.y; acc.z += a4.z; acc.w += a4.w;
+  }
+  if (i1 - i0 > kCtaItems) {
+    // the block's (o, m, l) replaces its first partial (every read of the block is done)
+    float* P = partials + (b0 * g.G + h) * kPartStride;
+    *reinterpret_cast<float4*>(P + 4 * lane) = acc;
+    if (lane == 0) { P[kD] = M; P[kD + 1] = L; }
+    return;
+  }
+  const int64_t bq = u / g.Hkv;
+  const int hk = (int)(u % g.Hkv);
+  const int64_t qh = bq * g.Hq + hk * g.G + h;
+  const float inv = L > 0.f ? 1.f / L : 0.f;
+  OT* out = O + qh * kD + 4 * lane;
+  out[0] = from_f32<OT>(acc.x * inv);
+  out[1] = from_f32<OT>(acc.y * inv);
+  out[2] = from_f32<OT>(acc.z * inv);
+  out[3] = from_f32<OT>(acc.w * inv);
+  if (lse && lane == 0) lse[qh] = L > 0.f ? (M + log2f(L)) * 0.6931471805599453f : -INFINITY;
+}
+
+// Second stage for units of more than kCtaItems items: one warp per (unit, head) merges the
+// block partials (at items i0, i0 + kCtaItems, ...) in block order, two passes as above.
+template <typename OT>
+__global__ void __launch_bounds__(kMaxG * 32) combine_cta_blocks_kernel(AttnGeom g, const int* pair_off,
+                                                                      const float* partials, OT* O, float* lse) {
+  const int64_t u = blockIdx.x;
+  const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (h >= g.G) return;
+  const int64_t i0 = pair_off[u * g.nr], i1 = pair_off[(u + 1) * g.nr];
+  if (i1 - i0 <= kCtaItems) return;                  // written by the first stage
+  float M = -INFINITY;
+  for (int64_t b = i0 + (int64_t)lane * kCtaItems; b < i1; b += 32ll * kCtaItems)
+    M = fmaxf(M, partials[(b * g.G + h) * kPartStride + kD]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  float L = 0.f;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (M != -INFINITY) {
+    for (int64_t b = i0; b < i1; b += kCtaItems) {
+      const float* P = partials + (b * g.G + h) * kPartStride;
+      const float4 o4 = *reinterpret_cast<const float4*>(P + 4 * lane);
+      const float w = exp2f(P[kD] - M);
+      L = fmaf(w, P[kD + 1], L);
+      acc.x = fmaf(w, o4.x, acc.x);
+      acc.y = fmaf(w, o4.y, acc.y);
+      acc.z = fmaf(w, o4.z, acc.z);
+      acc.w = fmaf(w, o4.w, acc.w);
+    }
   }
   const int64_t bq = u / g.Hkv;
   const int hk = (int)(u % g.Hkv);
@@ -546,28 +510,22 @@ static cudaError_t attention_t(const AttnCall& c) {
 
   // items of one unit: at most ceil((C1 + 2) / cps) + nr
   const int64_t items_unit = (w.C1 + 2 + w.cps - 1) / w.cps + w.nr;
-  const int64_t nb_max = (items_unit + kCombBlock - 1) / kCombBlock;
-  if (nb_max == 1) {
+  if (items_unit <= kCombBlock) {
     combine_warp_kernel<KT><<<(unsigned)w.units, kMaxG * 32, 0, c.stream>>>(ag, pair_off, aa.partials,
                                                                             (KT*)c.O, c.lse);
     count_launch();
     return launch_status("combine_warp_kernel");
   }
-  if (nb_max <= 4) {
-    combine_cta_kernel<KT><<<(unsigned)(w.units * ag.G), 256, 0, c.stream>>>(ag, pair_off, aa.partials,
-                                                                             (KT*)c.O, c.lse);
-    count_launch();
-    return launch_status("combine_cta_kernel");
-  }
-  combine_kernel<KT><<<(unsigned)(w.units * ag.G * nb_max), kCombGroups * kD, 0, c.stream>>>(
-      ag, pair_off, aa.partials, nb_max, (KT*)c.O, c.lse);
+  const int64_t nbl = (items_unit + kCtaItems - 1) / kCtaItems;
+  combine_cta_kernel<KT><<<(unsigned)(w.units * ag.G * nbl), 256, 0, c.stream>>>(ag, pair_off, aa.partials, nbl,
+                                                                                 (KT*)c.O, c.lse);
   count_launch();
-  if ((e = launch_status("combine_kernel")) != cudaSuccess) return e;
-  if (nb_max > 1) {
-    combine_blocks_kernel<KT><<<(unsigned)(w.units * ag.G), kCombGroups * kD, 0, c.stream>>>(
-        ag, pair_off, aa.partials, (KT*)c.O, c.lse);
+  if ((e = launch_status("combine_cta_kernel")) != cudaSuccess) return e;
+  if (nbl > 1) {
+    combine_cta_blocks_kernel<KT><<<(unsigned)w.units, kMaxG * 32, 0, c.stream>>>(ag, pair_off, aa.partials,
+                                                                                  (KT*)c.O, c.lse);
     count_launch();
-    return launch_status("combine_blocks_kernel");
+    return launch_status("combine_cta_blocks_kernel");
   }
   return cudaSuccess;
 }
