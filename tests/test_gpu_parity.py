@@ -219,6 +219,9 @@ def test_append_equals_rebuild():
     ("batched-decode-128k@R16", 32768, 1, 0.9),
     ("deep-tree-16m@L1", 1200000 + 5, None, 0.95),       # one level: ~18.7K candidates per head
     ("deep-tree-16m@L2", 1200000, None, 0.99),           # > 16K leaf candidates below the top
+    ("deep-tree-16m@L1", 2300000 + 5, None, 0.95),       # ~36K candidates: a 4-CTA cluster select
+    ("deep-tree-16m@L1", 4500000 + 5, None, 0.95),       # ~70K candidates: an 8-CTA cluster select
+    ("batched-decode-128k", 180000 + 9, 8, 0.95),        # 2813 candidates x 256 heads: 256-thread CTAs
 ])
 def test_decode_parity(name, T, B, p):
     import dataclasses
@@ -230,7 +233,8 @@ def test_decode_parity(name, T, B, p):
     if ll:
         w = dataclasses.replace(w, depth=int(ll))
     run = DecodeRun(w, p)
-    cmp = check_decode(run, [(b, h) for b in range(w.B) for h in range(w.Hkv)])
+    units = [(b, h) for b in range(w.B) for h in range(w.Hkv)]
+    cmp = check_decode(run, units if len(units) <= 8 else [units[0], units[len(units) // 2], units[-1]])
     print(f"{w.name} p={p}: {cmp.exact} exact, {cmp.near_cutoff} near-cutoff of {cmp.heads}")
 
 
