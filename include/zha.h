@@ -216,7 +216,8 @@ zha_status zha_dense_decode(const zha_geom* g, const void* Q, const void* K, con
  * every query head by its exact log mass F_C(q) = log sum_{j in C} exp(q . k_j / sqrt(d))
  * ("ZHA summary" page, Tree Construction; reading every key, as the flat sparse-attention
  * indexers of arXiv 2610.42112 §I do), keeps the top-p chunks as zha_route does for one
- * level, and attends as zha_sparse_attn.  Scores are computed in fp32.
+ * level, and attends as zha_sparse_attn.  Scores are computed in fp32 (bf16 caches: on the
+ * tensor cores, products of bf16 values accumulated in fp32), the log mass in fp64.
  *   ws >= zha_workspace_bytes(g, nq, ZHA_OP_FLAT).
  */
 zha_status zha_flat_index(const zha_geom* g, const void* Q, const void* K, const void* V,
@@ -262,7 +263,8 @@ const char* zha_last_error(void);
 /* Measurement hook.  Kernel ids for zha_trace. */
 typedef enum zha_trace_kernel {
   ZHA_TRACE_ATTN = 1,        /* the split-KV gather kernel of the sparse / dense attention */
-  ZHA_TRACE_ROUTE_SCORE = 2, /* the routing score kernel (every level)                      */
+  ZHA_TRACE_ROUTE_SCORE = 2, /* the routing score kernel (every level); the flat indexer's
+                                chunk scores                                                */
   ZHA_TRACE_ROUTE_SELECT = 3 /* the routing top-p select kernels (every level; both kinds)  */
 } zha_trace_kernel;
 
