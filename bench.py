@@ -48,6 +48,9 @@ def parse():
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--segment", type=int, default=0,
+                    help="structured keys: runs of this many positions share a cluster centre "
+                         "(a variant of the generator, not one of the five workloads)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat"],
@@ -327,7 +330,9 @@ def config_of(w, p):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "T": w.T, "depth": w.depth,
             "leaf": w.leaf, "branch": w.branch, "R": w.R, "p": p, "n_centres": w.n_centres,
             "kv_bytes": 2 * w.B * w.Hkv * w.T * w.d * (2 if w.dtype == "bf16" else 4),
-            "l2": "no flush: the KV cache read per step is larger than the 126 MB L2"}
+            "l2": "no flush: the KV cache read per step is larger than the 126 MB L2",
+            **({"segment": w.segment, "generator": "structured variant: keys share a centre over runs "
+                "of `segment` positions; queries take a segment's centre"} if w.segment else {})}
 
 
 # ---------------------------------------------------------------------------
@@ -412,6 +417,9 @@ def main():
     w = S.workload(args.workload)
     if args.batch is not None:
         w = S.scaled(w, T=w.T, B=args.batch)
+    if args.segment > 0:
+        import dataclasses
+        w = dataclasses.replace(w, segment=args.segment, name=f"{w.name}+seg{args.segment}")
     p = args.p if args.p is not None else w.p[0]
     ws, rank, local = dist_setup(args.gpus)
     if args.impl == "reference":

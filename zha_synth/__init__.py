@@ -13,6 +13,10 @@ Recipe (one independent draw per (batch, KV head) unit):
   * queries   q   = 2 * c_{z'} + 0.3 * N(0, I_d)      z' ~ U over the query's KV group
               (a fraction ``random_frac`` of queries instead use q = 2 * N(0, I_d))
   * reference queries  q_hat_r ~ N(0, I_d / d)        (randomly initialised, never trained)
+With ``segment`` > 0 (a structured variant, not one of the five workloads) the cluster of a
+key is drawn once per run of ``segment`` consecutive positions instead of per key, and a
+query takes the centre of a uniformly chosen segment of its cache: the keys that matter to a
+query then sit in a few contiguous chunks, as in text where a topic spans a passage.
 Keys, values and queries are drawn in fp32 and then stored in the workload's
 dtype (bf16 rounding is round-to-nearest-even, torch's ``.to(torch.bfloat16)``).
 
@@ -29,7 +33,7 @@ import torch
 
 __all__ = [
     "Workload", "WORKLOADS", "workload", "scaled",
-    "clustered_kv", "queries", "reference_queries", "new_tokens",
+    "clustered_kv", "queries", "reference_queries", "new_tokens", "segment_centres",
 ]
 
 _TAGS = {"centres": 11, "assign": 12, "knoise": 13, "values": 14, "qpick": 21,
@@ -57,6 +61,7 @@ class Workload:
     mode: str = "decode"   # "decode": one new token per sequence; "prefill": n_new causal tokens
     n_new: int = 1
     random_frac: float = 0.0
+    segment: int = 0       # > 0: keys share a centre over runs of this many positions
 
     @property
     def G(self) -> int:
@@ -120,6 +125,13 @@ def centres_of(w: Workload, device="cpu") -> torch.Tensor:
     return torch.randn(w.B, w.Hkv, w.n_centres, w.d, generator=g, device=device)
 
 
+def segment_centres(w: Workload, b: int, h: int, device="cpu") -> torch.Tensor:
+    """Centre index of every run of ``w.segment`` positions of unit (b, h), over t_cap."""
+    ga = _gen(device, w.seed, "assign", b * w.Hkv + h)
+    nseg = (w.t_cap + w.segment - 1) // w.segment
+    return torch.randint(0, w.n_centres, (nseg,), generator=ga, device=device)
+
+
 def clustered_kv(w: Workload, device="cpu", block: int = 1 << 20):
     """Keys/values for the existing cache, laid out [B, Hkv, t_cap, d].
 
@@ -137,9 +149,13 @@ def clustered_kv(w: Workload, device="cpu", block: int = 1 << 20):
             ga = _gen(device, w.seed, "assign", unit)
             gk = _gen(device, w.seed, "knoise", unit)
             gv = _gen(device, w.seed, "values", unit)
+            zs = segment_centres(w, b, h, device) if w.segment > 0 else None
             for t0 in range(0, w.T, block):
                 n = min(block, w.T - t0)
-                z = torch.randint(0, w.n_centres, (n,), generator=ga, device=device)
+                if zs is not None:
+                    z = zs[(t0 + torch.arange(n, device=device)) // w.segment]
+                else:
+                    z = torch.randint(0, w.n_centres, (n,), generator=ga, device=device)
                 k = C[b, h][z] + 0.3 * torch.randn(n, w.d, generator=gk, device=device)
                 K[b, h, t0:t0 + n] = k.to(dt)
                 V[b, h, t0:t0 + n] = torch.randn(n, w.d, generator=gv, device=device).to(dt)
@@ -153,6 +169,12 @@ def new_tokens(w: Workload, C: torch.Tensor, n_new: int, device="cpu", step: int
     gk = _gen(device, w.seed, "new_knoise", step)
     gv = _gen(device, w.seed, "new_values", step)
     z = torch.randint(0, w.n_centres, (w.B, n_new, w.Hkv), generator=ga, device=device)
+    if w.segment > 0:                                # the runs continue past T
+        pos = (w.T + step * n_new + torch.arange(n_new, device=device)) // w.segment
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                zs = segment_centres(w, b, h, device)
+                z[b, :, h] = zs[pos.clamp(max=len(zs) - 1)]
     bi = torch.arange(w.B, device=device).view(-1, 1, 1)
     hi = torch.arange(w.Hkv, device=device).view(1, 1, -1)
     k = C[bi, hi, z] + 0.3 * torch.randn(w.B, n_new, w.Hkv, w.d, generator=gk, device=device)
@@ -170,6 +192,13 @@ def queries(w: Workload, C: torch.Tensor, nq: int, device="cpu", step: int = 0):
     gp = _gen(device, w.seed, "qpick", step)
     gn = _gen(device, w.seed, "qnoise", step)
     z = torch.randint(0, w.n_centres, (w.B, nq, w.Hq), generator=gp, device=device)
+    if w.segment > 0:                                # the centre of a random full segment
+        nfull = max(1, w.T // w.segment)
+        pick = torch.randint(0, nfull, (w.B, nq, w.Hq), generator=gp, device=device)
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                zs = segment_centres(w, b, h, device)
+                z[b, :, h * w.G:(h + 1) * w.G] = zs[pick[b, :, h * w.G:(h + 1) * w.G]]
     bi = torch.arange(w.B, device=device).view(-1, 1, 1)
     gi = (torch.arange(w.Hq, device=device) // w.G).view(1, 1, -1)
     q = 2.0 * C[bi, gi, z] + 0.3 * torch.randn(w.B, nq, w.Hq, w.d, generator=gn, device=device)
