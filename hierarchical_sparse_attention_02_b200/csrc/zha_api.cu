@@ -16,14 +16,17 @@ void note_cuda_error(cudaError_t e, const char* where) {
   snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%s)", where, cudaGetErrorName(e), cudaGetErrorString(e));
 }
 
-
-
-
-
-
 static zha_status from_cuda(cudaError_t e) { return e == cudaSuccess ? ZHA_OK : ZHA_ERR_CUDA; }
 
 static bool valid_p(double p) { return p > 0.0 && p <= 1.0 && !isnan(p); }
+
+// The workspace check of every entry point: sizes whose arrays would not fit 64-bit byte
+// counts are unsupported (zha_workspace_bytes returns 0 for them), smaller buffers too small.
+static zha_status check_ws(const zha_geom* g, int32_t nq, int32_t op, const zha_buf& ws) {
+  const size_t need = zha_workspace_bytes(g, nq, op);
+  if (need == 0) return ZHA_ERR_UNSUPPORTED;
+  return ws.bytes < need ? ZHA_ERR_CAPACITY : ZHA_OK;
+}
 
 }  // namespace zha
 
@@ -56,6 +59,7 @@ zha_status zha_check_geom(const zha_geom* g) {
   if (g->dtype != ZHA_F32 && g->dtype != ZHA_BF16) return ZHA_ERR_UNSUPPORTED;
   if (g->t_cap % kLeaf != 0) return ZHA_ERR_INVALID_ARG;
   if (g->t_cap / kLeaf + 2 > (int64_t)INT32_MAX / 2) return ZHA_ERR_UNSUPPORTED;
+  if (!cache_fits(*g)) return ZHA_ERR_UNSUPPORTED;
   return ZHA_OK;
 }
 
@@ -78,7 +82,7 @@ int64_t zha_leaf_cap(const zha_geom* g) {
 }
 
 size_t zha_workspace_bytes(const zha_geom* g, int32_t nq, int32_t op) {
-  if (zha_check_geom(g) != ZHA_OK || nq < 1) return 0;
+  if (zha_check_geom(g) != ZHA_OK || nq < 1 || !call_fits(*g, nq)) return 0;
   switch (op) {
     case ZHA_OP_ROUTE: return route_ws(*g, nq).bytes;
     case ZHA_OP_ATTN:
@@ -141,8 +145,8 @@ zha_status zha_route(const zha_geom* g, const void* Q, const int64_t* q_pos, int
   if (!Q || !q_pos || nq < 1 || !valid_p(p) || !tree.base || !leaf_ids || !leaf_cnt || leaf_cap < 1 ||
       !ws.base || !dev_status)
     return ZHA_ERR_INVALID_ARG;
-  if (tree.bytes < zha_tree_bytes(g) || ws.bytes < zha_workspace_bytes(g, nq, ZHA_OP_ROUTE))
-    return ZHA_ERR_CAPACITY;
+  if (tree.bytes < zha_tree_bytes(g)) return ZHA_ERR_CAPACITY;
+  if ((s = check_ws(g, nq, ZHA_OP_ROUTE, ws)) != ZHA_OK) return s;
   RouteCall c{g, nq, Q, q_pos, 0, p, tree.base, leaf_ids, leaf_cnt, leaf_cap, level_cnt, level_ids,
               (char*)ws.base, dev_status, (cudaStream_t)stream};
   return from_cuda(route_all(c));
@@ -157,7 +161,7 @@ zha_status zha_sparse_attn(const zha_geom* g, const void* Q, const void* K, cons
   if (!Q || !K || !V || !q_pos || nq < 1 || !leaf_ids || !leaf_cnt || leaf_cap < 1 || !O ||
       !ws.base || !dev_status)
     return ZHA_ERR_INVALID_ARG;
-  if (ws.bytes < zha_workspace_bytes(g, nq, ZHA_OP_ATTN)) return ZHA_ERR_CAPACITY;
+  if ((s = check_ws(g, nq, ZHA_OP_ATTN, ws)) != ZHA_OK) return s;
   AttnCall c{g, nq, Q, K, V, q_pos, 0, 0, leaf_ids, leaf_cnt, leaf_cap, O, lse, (char*)ws.base,
              dev_status, (cudaStream_t)stream};
   return from_cuda(attention(c));
@@ -173,8 +177,8 @@ zha_status zha_decode(const zha_geom* g, const void* q, const void* k_new, const
       !leaf_cnt || leaf_cap < 1 || !O || !ws.base || !dev_status)
     return ZHA_ERR_INVALID_ARG;
   if (T < 0 || T + 1 > g->t_cap) return ZHA_ERR_INVALID_ARG;
-  if (tree.bytes < zha_tree_bytes(g) || ws.bytes < zha_workspace_bytes(g, 1, ZHA_OP_DECODE))
-    return ZHA_ERR_CAPACITY;
+  if (tree.bytes < zha_tree_bytes(g)) return ZHA_ERR_CAPACITY;
+  if ((s = check_ws(g, 1, ZHA_OP_DECODE, ws)) != ZHA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   cudaError_t e = append_tokens(*g, K, V, k_new, v_new, T, 1, st);
   if (e == cudaSuccess) e = tree_extend(*g, K, qref, tree.base, T, T + 1, st);
@@ -193,7 +197,7 @@ zha_status zha_dense_decode(const zha_geom* g, const void* Q, const void* K, con
   zha_status s = zha_check_geom(g);
   if (s != ZHA_OK) return s;
   if (!Q || !K || !V || !q_pos || nq < 1 || !O || !ws.base || !dev_status) return ZHA_ERR_INVALID_ARG;
-  if (ws.bytes < zha_workspace_bytes(g, nq, ZHA_OP_DENSE)) return ZHA_ERR_CAPACITY;
+  if ((s = check_ws(g, nq, ZHA_OP_DENSE, ws)) != ZHA_OK) return s;
   AttnCall c{g, nq, Q, K, V, q_pos, 0, 1, nullptr, nullptr, 1, O, lse, (char*)ws.base, dev_status,
              (cudaStream_t)stream};
   return from_cuda(attention(c));
@@ -208,7 +212,7 @@ zha_status zha_flat_index(const zha_geom* g, const void* Q, const void* K, const
   if (!Q || !K || !V || !q_pos || nq < 1 || !valid_p(p) || !leaf_ids || !leaf_cnt || leaf_cap < 1 ||
       !O || !ws.base || !dev_status)
     return ZHA_ERR_INVALID_ARG;
-  if (ws.bytes < zha_workspace_bytes(g, nq, ZHA_OP_FLAT)) return ZHA_ERR_CAPACITY;
+  if ((s = check_ws(g, nq, ZHA_OP_FLAT, ws)) != ZHA_OK) return s;
   cudaStream_t st = (cudaStream_t)stream;
   RouteCall rc{g, nq, Q, q_pos, 0, p, const_cast<void*>(K), leaf_ids, leaf_cnt, leaf_cap, nullptr,
                nullptr, (char*)ws.base, dev_status, st};

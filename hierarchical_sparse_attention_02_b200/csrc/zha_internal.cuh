@@ -12,7 +12,7 @@
 
 namespace zha {
 
-constexpr int kD = 128;          // head dimension supported by this build
+constexpr int kD = 128;          // head dimension the kernels support
 constexpr int kLeaf = 64;        // keys per leaf chunk
 constexpr int kMaxR = 16;        // reference queries per KV head
 constexpr int kMaxG = 8;         // query heads per KV head
@@ -38,6 +38,19 @@ inline int64_t span_of(const zha_geom& g, int level) {
 inline int64_t ncap_of(const zha_geom& g, int level) { return g.t_cap / span_of(g, level); }
 
 inline int elem_bytes(const zha_geom& g) { return g.dtype == ZHA_BF16 ? 2 : 4; }
+
+// Bounds that keep every byte count and offset the library forms far inside 64-bit
+// arithmetic (checked in double, which is exact at these magnitudes up to rounding that
+// cannot cross the bound by more than one part in 2^52): one layer's cache, counted at
+// 4 bytes per element, and the largest per-call array (8 bytes per query head per leaf
+// chunk) each at most 2^48 bytes.
+constexpr double kMaxBytes = 281474976710656.0;  // 2^48
+inline bool cache_fits(const zha_geom& g) {
+  return (double)g.B * g.Hkv * (double)g.t_cap * kD * 4.0 <= kMaxBytes;
+}
+inline bool call_fits(const zha_geom& g, int64_t nq) {
+  return (double)g.B * (double)nq * g.Hq * (double)(g.t_cap / kLeaf + 2) * 8.0 <= kMaxBytes;
+}
 
 struct TreeLayout {
   zha_level_layout lv[kMaxDepth + 1];  // index = level (1..depth)

@@ -71,6 +71,7 @@ extern "C" zha_status zha_sparse_attn_noalloc(const zha_geom* g, const void* Q, 
   if (!Q || !K || !V || !q_pos || nq < 1 || !leaf_ids || !leaf_cnt || leaf_cap < 1 || !O ||
       !dev_status)
     return ZHA_ERR_INVALID_ARG;
+  if (!call_fits(*g, nq)) return ZHA_ERR_UNSUPPORTED;
   const int64_t cps = fitting_cps(*g, nq);
   if (cps == 0) return ZHA_ERR_CAPACITY;
   void* scratch = nullptr;

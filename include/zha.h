@@ -69,7 +69,9 @@ typedef enum zha_op {
 
 /* Geometry of one attention layer and its tree (host struct).
  * d must be 128; leaf must be 64; 2 <= branch <= 64; 1 <= depth <= 8; R in {1, 2, 4, 8, 16};
- * Hq % Hkv == 0 and Hq / Hkv <= 8; t_cap % leaf == 0; dtype a zha_dtype. */
+ * Hq % Hkv == 0 and Hq / Hkv <= 8; t_cap % leaf == 0; dtype a zha_dtype;
+ * B * Hkv * t_cap * d * 4 <= 2^48 (bytes of the cache counted at 4 bytes per element),
+ * else ZHA_ERR_UNSUPPORTED, so that no byte count the library forms can overflow. */
 typedef struct zha_geom {
   int32_t B, Hq, Hkv, d;
   int32_t leaf;     /* keys per leaf chunk (level 1)                       */
@@ -110,7 +112,10 @@ size_t zha_tree_bytes(const zha_geom* g);
 /* Layout of level `level` (1..depth) inside the tree buffer. */
 zha_status zha_tree_level(const zha_geom* g, int32_t level, zha_level_layout* out);
 
-/* Bytes of the workspace `op` needs for `nq` queries per sequence (0 if invalid). */
+/* Bytes of the workspace `op` needs for `nq` queries per sequence.  0 for an invalid
+ * geometry, nq < 1, an unknown op, or B * nq * Hq * (t_cap / leaf + 2) * 8 > 2^48 (the
+ * per-call arrays would not fit 64-bit byte counts); the entry points then return
+ * ZHA_ERR_UNSUPPORTED (ZHA_ERR_INVALID_ARG for nq < 1) before anything is enqueued. */
 size_t zha_workspace_bytes(const zha_geom* g, int32_t nq, int32_t op);
 
 /* Leaf chunks a query can select at most (t_cap / leaf): a leaf_cap that never overflows. */

@@ -48,6 +48,10 @@ def test_status_strings(lib):
     ({}, 0), ({"d": 64}, 2), ({"leaf": 32}, 2), ({"Hq": 15}, 1), ({"Hq": 64, "Hkv": 2}, 2),
     ({"R": 17}, 2), ({"R": 0}, 1), ({"R": 3}, 2), ({"R": 16}, 0), ({"R": 1}, 0), ({"depth": 9}, 2), ({"branch": 1}, 2), ({"t_cap": 1000}, 1),
     ({"dtype": 7}, 2), ({"reserved": 1}, 1), ({"B": 0}, 1),
+    # a cache whose byte count (at 4 bytes per element) passes 2^48: 2^20 * 2 * 2^28 * 512 = 2^58
+    ({"B": 1 << 20, "t_cap": 1 << 28}, 2),
+    # the largest cache of the decode workloads (16M keys) is well inside the bound
+    ({"B": 1, "Hq": 8, "Hkv": 1, "depth": 6, "t_cap": 1 << 24}, 0),
 ])
 def test_check_geom(lib, kw, code):
     assert lib.zha_check_geom(ctypes.byref(geom(**kw))) == code
@@ -101,4 +105,27 @@ def test_host_side_rejections_enqueue_nothing(lib):
     bad = geom(d=256)
     assert lib.zha_decode(ctypes.byref(bad), fake, fake, fake, fake, fake, 5, fake, 0.9, buf, fake, fake, 8,
                           fake, buf, fake, None) == 2
+    assert lib.zha_launch_count() == n0
+
+
+def test_sizes_that_would_overflow_are_rejected(lib):
+    """Per-call arrays past 2^48 bytes: the workspace size is 0 and every entry point that
+    takes nq returns ZHA_ERR_UNSUPPORTED before it enqueues anything."""
+    g = geom()
+    fake = ctypes.c_void_p(0x1000)
+    buf = _lib.Buf(0x1000, (1 << 64) - 1)
+    huge = (1 << 31) - 1          # 2 * huge * 16 heads * 1026 chunks * 8 bytes > 2^48
+    for op in (1, 2, 3, 4, 5):
+        assert lib.zha_workspace_bytes(ctypes.byref(g), huge, op) == 0
+    assert lib.zha_workspace_bytes(ctypes.byref(g), 1 << 20, 1) > 0
+    n0 = lib.zha_launch_count()
+    assert lib.zha_route(ctypes.byref(g), fake, fake, huge, 0.9, buf, fake, fake, 8, None, None, buf, fake,
+                         None) == 2
+    assert lib.zha_sparse_attn(ctypes.byref(g), fake, fake, fake, fake, huge, fake, fake, 8, fake, None, buf,
+                               fake, None) == 2
+    assert lib.zha_dense_decode(ctypes.byref(g), fake, fake, fake, fake, huge, fake, None, buf, fake, None) == 2
+    assert lib.zha_flat_index(ctypes.byref(g), fake, fake, fake, fake, huge, 0.9, fake, fake, 8, fake, buf,
+                              fake, None) == 2
+    assert lib.zha_sparse_attn_noalloc(ctypes.byref(g), fake, fake, fake, fake, huge, fake, fake, 8, fake,
+                                       None, fake, None) == 2
     assert lib.zha_launch_count() == n0
