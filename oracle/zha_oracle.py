@@ -37,6 +37,11 @@ Readings where the pages are silent (each is listed in the design doc):
     rounded cumulative mass never does; p >= 1 keeps every candidate.
   * Scores, softmax and cumulative sums are float64 (the routing decision is
     made in float64 on both sides).
+  * Selector variants (``route(..., p=schedule)`` and ``route(..., k=...)``):
+    a per-level threshold p_l replaces the constant p level by level; the
+    "p**(1/L)" schedule takes L = the configured depth; the fixed-count
+    selector keeps the first min(K, n) candidates in the same (score desc,
+    id asc) order.
 """
 from __future__ import annotations
 
@@ -259,6 +264,43 @@ def top_p(scores: np.ndarray, ids: np.ndarray, p: float) -> Selection:
     return Selection(np.sort(ids[order[:m]]), m, n, float(margin), float(gap))
 
 
+def top_k(scores: np.ndarray, ids: np.ndarray, k: int) -> Selection:
+    """The fixed-count selector: the first min(k, n) candidates in (score desc,
+    id asc) order.
+
+    The roofline-model variables of arXiv 2610.42112 (App. D, Table VI) name a
+    fixed-count budget K beside the threshold p "when used by the chosen
+    selector"; §III-C contrasts it with top-p.  ``margin`` is inf (no mass
+    threshold); ``gap`` is pi_(m) - pi_(m+1) of the candidates' softmax, as for
+    top-p, so that near-ties at the boundary are counted the same way.
+    """
+    n = len(ids)
+    if n == 0 or k <= 0:
+        return Selection(np.zeros(0, np.int64), 0, n, math.inf, math.inf)
+    order = np.lexsort((ids, -scores))
+    m = min(int(k), n)
+    s = scores[order]
+    e = np.exp(s - s[0])
+    pi = e / np.sum(e)
+    gap = pi[m - 1] - pi[m] if m < n else math.inf
+    return Selection(np.sort(ids[order[:m]]), m, n, math.inf, float(gap))
+
+
+def p_root_schedule(p: float, depth: int) -> List[float]:
+    """Per-level thresholds p_l = p**(1/L), L = the configured depth, so that the
+    product of the per-level thresholds over all L levels is p (arXiv
+    2610.42112 §VII, "Asymptotic length scaling": a constant p gives a
+    cumulative p**L; rescaling each level to p**(1/L) undoes it).  Index l-1
+    holds level l."""
+    return [float(p) ** (1.0 / depth)] * depth
+
+
+def _at_level(x, level: int):
+    """A per-level parameter: a scalar applies to every level; a sequence holds
+    level l at index l-1."""
+    return x if np.ndim(x) == 0 else x[level - 1]
+
+
 def visible_count(t: int, span: int, leaf: int) -> int:
     """Full nodes of size ``span`` that end at or before the query's own chunk."""
     return (leaf * (t // leaf)) // span
@@ -272,12 +314,17 @@ class Route:
     leaves: np.ndarray                        # S_1(q), ascending chunk ids
 
 
-def route(q: np.ndarray, t: int, tree: Tree, p: float) -> Route:
+def route(q: np.ndarray, t: int, tree: Tree, p, k=None) -> Route:
     """Top-down top-p routing of one query head at position ``t``.
 
     The top level is the highest level with a visible node; all its visible
     nodes are candidates.  Below it, the candidates are the children of the
     selected nodes plus the visible nodes whose parent is not visible.
+
+    ``p`` is one threshold for every level (the pages' setting, §IV-A) or a
+    per-level schedule (index l-1 = level l, e.g. ``p_root_schedule``).  With
+    ``k`` (a count, or a per-level sequence of counts) each level keeps the
+    k best candidates instead (``top_k``) and ``p`` is ignored.
     """
     d = q.shape[0]
     scale = 1.0 / math.sqrt(d)
@@ -293,7 +340,7 @@ def route(q: np.ndarray, t: int, tree: Tree, p: float) -> Route:
     cand = np.arange(nvis[top], dtype=np.int64)
     for l in range(top, 0, -1):
         s = node_scores(q, tree.levels[l - 1], cand, scale)
-        sel = top_p(s, cand, p)
+        sel = top_p(s, cand, _at_level(p, l)) if k is None else top_k(s, cand, _at_level(k, l))
         out.cand[l] = cand
         out.sel[l] = sel
         if l > 1:

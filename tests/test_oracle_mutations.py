@@ -2,7 +2,7 @@
 
 Each case replaces one oracle function by a copy with one plausible slip (a dropped term, a
 wrong sign, an index off by one, a transposed operand, an unnormalised weight, a wrong tie
-order) and runs the pins of tests/test_oracle.py that cover it: at least one must fail.
+order) and runs the pins of tests/test_oracle.py or tests/test_oracle_selectors.py that cover it: at least one must fail.
 The mistakes are planted in the oracle only, on the CPU.
 """
 import numpy as np
@@ -10,6 +10,7 @@ import pytest
 
 from oracle import zha_oracle as zo
 from tests import test_oracle as pins
+from tests import test_oracle_selectors as sel_pins
 
 
 def _golden():
@@ -121,7 +122,29 @@ def round_bf16_via_f32(x):
     return torch.from_numpy(np.asarray(x, np.float64).astype(np.float32)).to(torch.bfloat16).double().numpy()
 
 
-_orig = {"leaf_summary": zo.leaf_summary, "top_p": zo.top_p}
+def top_k_ties_descending(scores, ids, k):
+    order = np.lexsort((-ids, -scores))                # wrong tie order
+    m = min(int(k), len(ids))
+    return zo.Selection(np.sort(ids[order[:m]]), m, len(ids), 0.0, 0.0)
+
+
+def top_k_one_too_few(scores, ids, k):
+    sel = _orig["top_k"](scores, ids, k)
+    if sel.m > 1:
+        order = np.lexsort((ids, -scores))
+        return zo.Selection(np.sort(ids[order[:sel.m - 1]]), sel.m - 1, sel.n, sel.margin, sel.gap)
+    return sel
+
+
+def at_level_reversed(x, level):
+    return x if np.ndim(x) == 0 else x[-level]         # level l read from the wrong end
+
+
+def p_root_power_not_root(p, depth):
+    return [float(p) ** depth] * depth
+
+
+_orig = {"leaf_summary": zo.leaf_summary, "top_p": zo.top_p, "top_k": zo.top_k}
 
 
 def _route_pins():
@@ -150,6 +173,11 @@ CASES = [
     ("visible_count", visible_count_off_by_one, _route_pins),
     ("attention", attention_no_scale, lambda: pins.test_p_one_routing_reproduces_dense_attention(8, 4096, 4095)),
     ("round_bf16", round_bf16_via_f32, pins.test_round_bf16_ties_to_even_and_no_double_rounding),
+    ("top_k", top_k_ties_descending, lambda: [sel_pins.test_top_k_by_brute_force(s) for s in range(30)]),
+    ("top_k", top_k_one_too_few, lambda: [sel_pins.test_top_k_by_brute_force(s) for s in range(30)]),
+    ("_at_level", at_level_reversed,
+     lambda: sel_pins.test_whole_route_with_per_level_parameters_by_brute_force("schedule")),
+    ("p_root_schedule", p_root_power_not_root, sel_pins.test_p_root_schedule),
 ]
 
 
