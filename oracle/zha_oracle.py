@@ -16,6 +16,9 @@ Plain numpy in float64, written step by step from the method's definitions:
   (stable-state merge of the children's per-reference state, without
   Taylor/RoPE re-anchoring), App. E-E (nodes without complete parents join the
   frontier; the first key and the partial chunk are always read).
+* Paper §III-B, models with RoPE: reference queries rotated to each node's
+  last position; children re-anchored to the parent's rotated reference
+  along their tangent planes before the merge (``rope``, ``reanchor``).
 * "ZHA summary" page, Methodology -> Routing: m_l(q), the final index set
   I(q) = {0} u (union of selected leaf chunks) u C_cur(q), o(q) = Attn(q, K_I, V_I).
 
@@ -42,6 +45,12 @@ Readings where the pages are silent (each is listed in the design doc):
     "p**(1/L)" schedule takes L = the configured depth; the fixed-count
     selector keeps the first min(K, n) candidates in the same (score desc,
     id asc) order.
+  * Rotary variant (``build_tree(..., inv_freq=...)``): the pages name RoPE
+    and partial RoPE but not the convention.  Dims (i, i + h), h =
+    len(inv_freq), rotate by pos * inv_freq[i] and the remaining dims pass
+    through (the "rotate half" pairing); the frequency table is an input (the
+    model's), not computed here.  Keys arrive rotated; queries at their own
+    position are rotated by the caller.
 """
 from __future__ import annotations
 
@@ -116,7 +125,47 @@ def leaf_summary(Kc: np.ndarray, qref: np.ndarray, scale: float):
     return k_hat, F, b_hat
 
 
-def merge_summaries(F_c: np.ndarray, k_hat_c: np.ndarray, qref: np.ndarray, scale: float):
+def rope(x: np.ndarray, pos, inv_freq) -> np.ndarray:
+    """Rotary position embedding of ``x`` [..., d] at position(s) ``pos``.
+
+    With h = len(inv_freq), dims i and i + h (i < h) are rotated together by the
+    angle pos * inv_freq[i]:
+      x'_i     = x_i cos - x_{i+h} sin,      x'_{i+h} = x_{i+h} cos + x_i sin;
+    dims >= 2h pass through unchanged (partial rotary).  ``pos`` broadcasts
+    against x.shape[:-1].  An empty ``inv_freq`` is the identity.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    f = np.asarray(inv_freq, dtype=np.float64)
+    h = len(f)
+    if h == 0:
+        return x.copy()
+    ang = np.asarray(pos, dtype=np.float64)[..., None] * f
+    c, sn = np.cos(ang), np.sin(ang)
+    out = np.array(np.broadcast_to(x, np.broadcast_shapes(x.shape, ang.shape[:-1] + x.shape[-1:])))
+    x1, x2 = out[..., :h].copy(), out[..., h:2 * h].copy()
+    out[..., :h] = x1 * c - x2 * sn
+    out[..., h:2 * h] = x2 * c + x1 * sn
+    return out
+
+
+def node_anchor(i, span: int):
+    """Position a node's reference queries are rotated to: the last key of its
+    span [i * span, (i + 1) * span) (paper §III-B)."""
+    return (np.asarray(i, dtype=np.int64) + 1) * span - 1
+
+
+def reanchor(F_c: np.ndarray, k_hat_c: np.ndarray, q_parent: np.ndarray, q_child: np.ndarray,
+             scale: float) -> np.ndarray:
+    """A child's log mass F_c, estimated at its own reference query q_child, moved
+    along its tangent plane to the parent's q_parent (paper §III-B): the
+    compressed key's score at the parent's reference minus its score at the
+    child's, F_c + <k_hat_c, q_parent - q_child> * scale.  Arrays broadcast;
+    the last axis is d."""
+    return F_c + np.sum(k_hat_c * (q_parent - q_child), axis=-1) * scale
+
+
+def merge_summaries(F_c: np.ndarray, k_hat_c: np.ndarray, qref: np.ndarray, scale: float,
+                    q_child: Optional[np.ndarray] = None):
     """Parent summary from its children's per-reference state.
 
     For each reference r independently (stable-state merge):
@@ -125,7 +174,15 @@ def merge_summaries(F_c: np.ndarray, k_hat_c: np.ndarray, qref: np.ndarray, scal
       k_hat = sum_c w_c k_hat_c
       b_hat = F_P - q_hat_r . k_hat * scale
     F_c: [C, R], k_hat_c: [C, R, d].  Returns (k_hat [R, d], F [R], b_hat [R]).
+
+    With rotary positions (paper §III-B) ``qref`` is the parent's rotated
+    reference query q_hat_{r,P} and ``q_child`` [C, R, d] the children's
+    q_hat_{r,c}: before the merge each child's log mass is moved to the parent's
+    reference query along its tangent plane,
+      F_c <- F_c + <k_hat_c, q_hat_{r,P} - q_hat_{r,c}> * scale.
     """
+    if q_child is not None:
+        F_c = reanchor(F_c, k_hat_c, qref[None, :, :], q_child, scale)
     F = lse(F_c, axis=0)                         # [R]
     w = np.exp(F_c - F[None, :])                 # [C, R]
     k_hat = np.einsum("cr,crd->rd", w, k_hat_c)
@@ -180,7 +237,7 @@ def rows_f64(K, a: int, b: int) -> np.ndarray:
 
 def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
                branch: int = 16, route_storage: str = "bf16", state_storage: str = "f32",
-               block: int = 4096) -> Tree:
+               block: int = 4096, inv_freq=None) -> Tree:
     """All full nodes over keys [0, T) of one unit.
 
     K: [>=T, d] keys (float64 values of the stored keys, or a CPU torch tensor
@@ -188,7 +245,23 @@ def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
     Level 1 summarises raw keys (``leaf_summary``); level l >= 2 merges the
     stored state of ``branch`` consecutive level-(l-1) nodes (``merge_summaries``).
     ``block`` only bounds the temporary memory of the vectorised leaf pass.
+
+    ``inv_freq`` (rotary frequencies, see ``rope``; None or empty: no rotation)
+    gives the RoPE variant of paper §III-B: node i of level l summarises at the
+    reference queries rotated to its last position, q_hat_{r,i} =
+    rope(q_hat_r, (i + 1) * span_l - 1), and a parent moves each child's log
+    mass to its own rotated reference before the merge (``merge_summaries``).
+    The keys are the cache's keys as stored (already rotated by the model).
     """
+    rot = inv_freq is not None and len(inv_freq) > 0
+
+    def rotated(level: int, n0: int, n1: int) -> np.ndarray:
+        """q_hat of nodes [n0, n1) of ``level``: [n, R, d] (rotated) or [1, R, d]."""
+        if not rot:
+            return qref[None, :, :]
+        last = node_anchor(np.arange(n0, n1, dtype=np.int64), tree.span(level))
+        return rope(qref[None, :, :], last[:, None], inv_freq)
+
     d = K.shape[1]
     scale = 1.0 / math.sqrt(d)
     R = qref.shape[0]
@@ -200,24 +273,31 @@ def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
     for i0 in range(0, n1, block):
         i1 = min(n1, i0 + block)
         Kc = rows_f64(K, i0 * leaf, i1 * leaf).reshape(i1 - i0, leaf, d)
-        # s[n, r, c] = q_hat_r . k_{n,c} * scale  (a matrix product, then a reshape)
-        s = np.swapaxes((Kc.reshape(-1, d) @ qref.T).reshape(i1 - i0, leaf, -1), 1, 2) * scale
+        qn = rotated(1, i0, i1)                                 # [n or 1, R, d]
+        if rot:   # s[n, r, c] = q_hat_{r,n} . k_{n,c} * scale
+            s = np.matmul(qn, np.swapaxes(Kc, 1, 2)) * scale
+        else:     # the same with one q_hat for every node: a matrix product, then a reshape
+            s = np.swapaxes((Kc.reshape(-1, d) @ qref.T).reshape(i1 - i0, leaf, -1), 1, 2) * scale
         F = lse(s, axis=-1)
         a = np.exp(s - F[..., None])
         kh = np.matmul(a, Kc)                                   # [n, r, d] = a[n, r, c] . K[n, c, d]
         k1[i0:i1] = kh
         F1[i0:i1] = F
-        b1[i0:i1] = F - np.einsum("rd,nrd->nr", qref, kh) * scale
+        b1[i0:i1] = F - (np.sum(qn * kh, axis=-1) if rot else np.einsum("rd,nrd->nr", qref, kh)) * scale
     tree.levels.append(_store_level(leaf, k1, F1, b1, route_storage, state_storage))
     for lvl in range(2, depth + 1):
         child = tree.levels[-1]
         n = child.n // branch
         Fc = child.F[:n * branch].reshape(n, branch, R)
         kc = child.k_state[:n * branch].reshape(n, branch, R, d)
+        qP = rotated(lvl, 0, n)                                 # [n or 1, R, d]
+        if rot:                                                 # each child's log mass at the parent's q_hat
+            qc = rotated(lvl - 1, 0, n * branch).reshape(n, branch, R, d)
+            Fc = reanchor(Fc, kc, qP[:, None], qc, scale)
         F = lse(Fc, axis=1)                                     # [n, R]
         w = np.exp(Fc - F[:, None, :])                          # [n, C, R]
         kh = np.einsum("ncr,ncrd->nrd", w, kc)
-        bh = F - np.einsum("rd,nrd->nr", qref, kh) * scale
+        bh = F - (np.sum(qP * kh, axis=-1) if rot else np.einsum("rd,nrd->nr", qref, kh)) * scale
         tree.levels.append(_store_level(tree.span(lvl), kh, F, bh, route_storage, state_storage))
     return tree
 

@@ -2,7 +2,8 @@
 
 Each case replaces one oracle function by a copy with one plausible slip (a dropped term, a
 wrong sign, an index off by one, a transposed operand, an unnormalised weight, a wrong tie
-order) and runs the pins of tests/test_oracle.py or tests/test_oracle_selectors.py that cover it: at least one must fail.
+order) and runs the pins of tests/test_oracle.py, tests/test_oracle_selectors.py or
+tests/test_oracle_rope.py that cover it: at least one must fail.
 The mistakes are planted in the oracle only, on the CPU.
 """
 import numpy as np
@@ -10,6 +11,7 @@ import pytest
 
 from oracle import zha_oracle as zo
 from tests import test_oracle as pins
+from tests import test_oracle_rope as rope_pins
 from tests import test_oracle_selectors as sel_pins
 
 
@@ -144,7 +146,29 @@ def p_root_power_not_root(p, depth):
     return [float(p) ** depth] * depth
 
 
-_orig = {"leaf_summary": zo.leaf_summary, "top_p": zo.top_p, "top_k": zo.top_k}
+def reanchor_missing(F_c, k_hat_c, q_parent, q_child, scale):
+    return F_c + 0.0 * np.sum(k_hat_c, axis=-1)        # the child's mass left at its own reference
+
+
+def reanchor_sign(F_c, k_hat_c, q_parent, q_child, scale):
+    return F_c + np.sum(k_hat_c * (q_child - q_parent), axis=-1) * scale
+
+
+def node_anchor_first_key(i, span):
+    return np.asarray(i, dtype=np.int64) * span         # rotated to the first key of the span
+
+
+def rope_clockwise(x, pos, inv_freq):
+    return _orig["rope"](x, -np.asarray(pos), inv_freq)  # the opposite sense of rotation
+
+
+_orig = {"leaf_summary": zo.leaf_summary, "top_p": zo.top_p, "top_k": zo.top_k, "rope": zo.rope}
+
+
+def _rope_tree_pins():
+    rope_pins.test_leaf_tangent_exact_at_its_rotated_reference()
+    for level in (2, 3):
+        rope_pins.test_parent_of_affine_children_equals_leaf_formula_over_span(level)
 
 
 def _route_pins():
@@ -178,6 +202,10 @@ CASES = [
     ("_at_level", at_level_reversed,
      lambda: sel_pins.test_whole_route_with_per_level_parameters_by_brute_force("schedule")),
     ("p_root_schedule", p_root_power_not_root, sel_pins.test_p_root_schedule),
+    ("reanchor", reanchor_missing, _rope_tree_pins),
+    ("reanchor", reanchor_sign, _rope_tree_pins),
+    ("node_anchor", node_anchor_first_key, _rope_tree_pins),
+    ("rope", rope_clockwise, rope_pins.test_rope_is_complex_multiplication),
 ]
 
 
