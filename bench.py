@@ -218,13 +218,48 @@ def hbm_peak():
 # ---------------------------------------------------------------------------
 
 
-def oracle_rate(w: S.Workload, p: float, seconds: float, device: str):
+NEAR_CUTOFF = 1e-4      # a level whose cutoff margin or boundary gap is below this is "near-cutoff"
+
+
+def near_cutoff_count(routes) -> dict:
+    """Near-cutoff levels among oracle routes: (query head, level) pairs whose cumulative
+    mass at the cutoff lies within NEAR_CUTOFF of p, or whose two candidates at the
+    boundary differ by less than NEAR_CUTOFF in softmax mass.  There a one-ulp difference
+    in a score may legitimately change the kept set."""
+    levels = near = 0
+    for r in routes:
+        for sel in r.sel.values():
+            levels += 1
+            near += int(min(sel.margin, sel.gap) < NEAR_CUTOFF)
+    return {"heads": len(routes), "levels": levels, "near_cutoff": near, "threshold": NEAR_CUTOFF}
+
+
+def frontier_stats(level_cnt: np.ndarray) -> list:
+    """Per-level frontier sizes from zha_route's level counts [..., depth, 2] (candidates,
+    kept) of every query head: mean / p50 / max over the heads that route that level."""
+    lc = np.asarray(level_cnt).reshape(-1, level_cnt.shape[-2], 2)
+    out = []
+    for l in range(lc.shape[1], 0, -1):
+        c, k = lc[:, l - 1, 0], lc[:, l - 1, 1]
+        on = c > 0
+        if not on.any():
+            continue
+        out.append({"level": l, "heads": int(on.sum()),
+                    "candidates_mean": float(c[on].mean()), "candidates_p50": float(np.median(c[on])),
+                    "candidates_max": int(c[on].max()),
+                    "kept_mean": float(k[on].mean()), "kept_p50": float(np.median(k[on])),
+                    "kept_max": int(k[on].max())})
+    return out
+
+
+def oracle_rate(w: S.Workload, p: float, seconds: float, device: str, routes: list = None):
     """Query-heads/s of the CPU oracle on a bounded sample of the decode step.
 
     The sample: whole KV groups (G query heads of one (sequence, KV head) unit) of the
     same seeded workload, routed and attended by the oracle one head at a time until
     ``seconds`` of CPU time have been spent (at least one group).  The oracle's tree of
     each sampled unit is built first, untimed (it is the decode step's prior state).
+    With ``routes`` (a list) the oracle's route of every sampled head is appended to it.
     """
     from oracle import zha_oracle as zo
     try:
@@ -248,8 +283,10 @@ def oracle_rate(w: S.Workload, p: float, seconds: float, device: str):
                              route_storage="bf16" if w.dtype == "bf16" else "f32")
         t0 = time.process_time()
         for h in range(hk * w.G, (hk + 1) * w.G):
-            zo.decode_head(qc[0, 0, h], Kc[0, hk], Vc[0, hk], w.T, tree, p)
+            r, _, _ = zo.decode_head(qc[0, 0, h], Kc[0, hk], Vc[0, hk], w.T, tree, p)
             heads += 1
+            if routes is not None:
+                routes.append(r)
         spent += time.process_time() - t0
         if spent >= seconds:
             break
@@ -591,12 +628,34 @@ def main():
         dom_name = "flat_tc_kernel"
         per_launch = flat_bytes / max(1.0, dom_launches)
     achieved = per_launch / (dom_ms * 1e-3) / 1e9
+    # per-level frontier sizes: one more (untimed) routing of the step's queries with the
+    # level counts switched on; its leaf lists must equal the decode step's
+    frontier = None
+    if args.path == "zha":
+        try:
+            lcnt = torch.zeros(w.B, 1, w.Hq, w.depth, 2, dtype=torch.int32, device=dev)
+            ids2, cnt2 = torch.empty_like(ids), torch.empty_like(cnt)
+            qpos = torch.full((w.B, 1), w.T, dtype=torch.int64, device=dev)
+            Z.zha_route(g, q, qpos, p, tree, ids2, cnt2, wsb, st, lcnt)
+            torch.cuda.synchronize()
+            ids2_c, cnt2_c = ids2.cpu().numpy(), cnt2.cpu().numpy()
+            same = bool(np.array_equal(cnt2_c, cnt_c)) and all(
+                np.array_equal(ids2_c[bb, 0, h, :cnt_c[bb, 0, h]], ids_c[bb, 0, h, :cnt_c[bb, 0, h]])
+                for bb in range(w.B) for h in range(w.Hq))
+            frontier = {"levels": frontier_stats(lcnt.cpu().numpy()), "route_matches_decode": same}
+            del lcnt, ids2, cnt2
+        except Exception as e:   # statistics outside the timed region: report, do not hide
+            frontier = {"error": repr(e)}
     cpu = None
+    near = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda")
+        routes = []
+        r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda", routes)
         cpu = {"value": r, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
                "sample": f"{heads} query heads (whole KV groups of sequence 0) of {w.name}, "
                          f"route + attention, fp64 numpy, 1 thread, {spent:.1f} s CPU"}
+        if args.path == "zha":
+            near = {**near_cutoff_count(routes), "sample": "the oracle's routes of the cpu_baseline sample"}
     line = {
         "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": ws,
         "steps": Ksteps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -614,6 +673,8 @@ def main():
                        "p99": float(np.percentile(per_head, 99)),
                        "group_union": union_rows / (units * T1)},
         "stages_ms": stages,
+        "frontier": frontier,
+        "near_cutoff": near,
         "tree_build": {"ms": build_ms, "gbs": k_bytes / (build_ms * 1e-3) / 1e9},
         "e2e": {"value": ws * w.B * w.Hq / (e2e_ms * 1e-3), "unit": "query-heads/s",
                 "h2d_bytes_per_step": (q.numel() + k_new.numel() + v_new.numel()) * es,
