@@ -125,6 +125,18 @@ def zha_route(g, Q, q_pos, p, tree, leaf_ids, leaf_cnt, ws, dev_status, level_cn
         _stream(stream)))
 
 
+def zha_route_schedule(g, Q, q_pos, p_levels, tree, leaf_ids, leaf_cnt, ws, dev_status, level_cnt=None,
+                       level_ids=None, stream=None):
+    """zha_route with one threshold per level: p_levels[l-1] for level l (len == depth)."""
+    if len(p_levels) != g.depth:
+        raise ValueError(f"p_levels holds {len(p_levels)} thresholds for {g.depth} levels")
+    arr = (ctypes.c_double * g.depth)(*[float(x) for x in p_levels])
+    _check("zha_route_schedule", _lib.load().zha_route_schedule(
+        ctypes.byref(g.c()), _ptr(Q), _ptr(q_pos), Q.shape[1], arr, _buf(tree), _ptr(leaf_ids),
+        _ptr(leaf_cnt), leaf_ids.shape[-1], _ptr(level_cnt), _ptr(level_ids), _buf(ws), _ptr(dev_status),
+        _stream(stream)))
+
+
 def zha_sparse_attn(g, Q, K, V, q_pos, leaf_ids, leaf_cnt, O, ws, dev_status, lse=None, stream=None):
     _check("zha_sparse_attn", _lib.load().zha_sparse_attn(
         ctypes.byref(g.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_pos), Q.shape[1], _ptr(leaf_ids),

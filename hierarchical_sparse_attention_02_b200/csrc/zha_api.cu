@@ -152,6 +152,25 @@ zha_status zha_route(const zha_geom* g, const void* Q, const int64_t* q_pos, int
   return from_cuda(route_all(c));
 }
 
+zha_status zha_route_schedule(const zha_geom* g, const void* Q, const int64_t* q_pos, int32_t nq,
+                              const double* p_levels, zha_buf tree, int32_t* leaf_ids,
+                              int32_t* leaf_cnt, int32_t leaf_cap, int32_t* level_cnt,
+                              int32_t* level_ids, zha_buf ws, int32_t* dev_status, void* stream) {
+  zha_status s = zha_check_geom(g);
+  if (s != ZHA_OK) return s;
+  if (!p_levels) return ZHA_ERR_INVALID_ARG;
+  for (int l = 0; l < g->depth; ++l)
+    if (!valid_p(p_levels[l])) return ZHA_ERR_INVALID_ARG;
+  if (!Q || !q_pos || nq < 1 || !tree.base || !leaf_ids || !leaf_cnt || leaf_cap < 1 || !ws.base ||
+      !dev_status)
+    return ZHA_ERR_INVALID_ARG;
+  if (tree.bytes < zha_tree_bytes(g)) return ZHA_ERR_CAPACITY;
+  if ((s = check_ws(g, nq, ZHA_OP_ROUTE, ws)) != ZHA_OK) return s;
+  RouteCall c{g, nq, Q, q_pos, 0, p_levels[0], tree.base, leaf_ids, leaf_cnt, leaf_cap, level_cnt,
+              level_ids, (char*)ws.base, dev_status, (cudaStream_t)stream, p_levels};
+  return from_cuda(route_all(c));
+}
+
 zha_status zha_sparse_attn(const zha_geom* g, const void* Q, const void* K, const void* V,
                            const int64_t* q_pos, int32_t nq, const int32_t* leaf_ids,
                            const int32_t* leaf_cnt, int32_t leaf_cap, void* O, float* lse,

@@ -281,6 +281,7 @@ struct RouteCall {
   char* ws;                      // workspace base, layout route_ws(g, nq, 0)
   int32_t* dev_status;
   cudaStream_t stream;
+  const double* p_levels = nullptr;  // host [depth]: level l selects with p_levels[l-1]; null: p
 };
 
 struct AttnCall {

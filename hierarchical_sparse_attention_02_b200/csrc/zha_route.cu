@@ -1807,7 +1807,7 @@ static cudaError_t route_levels(const RouteCall& c) {
     if (e != cudaSuccess) return e;
 
     SelectArgs se{};
-    se.g = rg; se.level = l; se.flat = 0; se.p = c.p;
+    se.g = rg; se.level = l; se.flat = 0; se.p = c.p_levels ? c.p_levels[l - 1] : c.p;
     se.mass_shift = mass_shift_for(w.C1);
     se.cand_ids = sa.cand_ids; se.cand_score = sa.cand_score;
     se.cand_mass = (unsigned long long*)(c.ws + w.cand_mass);

@@ -179,6 +179,20 @@ zha_status zha_route(const zha_geom* g, const void* Q, const int64_t* q_pos, int
                      int32_t* dev_status, void* stream);
 
 /*
+ * zha_route_schedule - zha_route with one threshold per level.
+ * Level l keeps the smallest prefix whose softmax mass reaches p_levels[l-1] instead of
+ * a single p (arXiv 2610.42112 §VII, "Asymptotic length scaling": a constant p compounds
+ * to p^L over L levels; a schedule such as p_l = p^(1/L) undoes that).  Candidates,
+ * order, expansion and outputs are those of zha_route.
+ *   p_levels  HOST array of g->depth doubles, each in (0, 1]; read before the call returns.
+ *   Other arguments as zha_route.
+ */
+zha_status zha_route_schedule(const zha_geom* g, const void* Q, const int64_t* q_pos, int32_t nq,
+                              const double* p_levels, zha_buf tree, int32_t* leaf_ids,
+                              int32_t* leaf_cnt, int32_t leaf_cap, int32_t* level_cnt,
+                              int32_t* level_ids, zha_buf ws, int32_t* dev_status, void* stream);
+
+/*
  * zha_sparse_attn - exact softmax attention over the index set
  * ("ZHA summary" page, Routing):  I(q) = {0} u (keys of the chunks in S_1(q)) u C_cur(q),
  * C_cur(q) = [V(t), t],   o(q) = sum_{j in I} softmax_j(q . k_j / sqrt(d)) v_j.

@@ -26,7 +26,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(lib):
     decl = declared_symbols()
-    assert len(decl) == 18
+    assert len(decl) == 19
     assert sorted(decl) == sorted(_lib.EXPORTS)
     for name in decl:
         assert hasattr(lib, name), name
@@ -128,4 +128,23 @@ def test_sizes_that_would_overflow_are_rejected(lib):
                               fake, None) == 2
     assert lib.zha_sparse_attn_noalloc(ctypes.byref(g), fake, fake, fake, fake, huge, fake, fake, 8, fake,
                                        None, fake, None) == 2
+    assert lib.zha_launch_count() == n0
+
+
+def test_route_schedule_rejections(lib):
+    """Per-level thresholds: a null array or any level outside (0, 1] is rejected before any
+    launch; only the first `depth` entries are read."""
+    g = geom()                                  # depth 3
+    fake = ctypes.c_void_p(0x1000)
+    buf = _lib.Buf(0x1000, 1 << 40)
+    n0 = lib.zha_launch_count()
+    arr = lambda *v: (ctypes.c_double * len(v))(*v)  # noqa: E731
+    for bad in (arr(0.9, 0.0, 0.9), arr(0.9, 0.9, 1.5), arr(float("nan"), 0.9, 0.9), arr(-1.0, 1.0, 1.0)):
+        assert lib.zha_route_schedule(ctypes.byref(g), fake, fake, 1, bad, buf, fake, fake, 8, None, None, buf,
+                                      fake, None) == 1
+    assert lib.zha_route_schedule(ctypes.byref(g), fake, fake, 1, None, buf, fake, fake, 8, None, None, buf,
+                                  fake, None) == 1
+    good = arr(0.9, 1.0, 0.5, 7.0)             # the fourth entry is past the depth: never read
+    assert lib.zha_route_schedule(ctypes.byref(g), fake, fake, 1, good, buf, fake, fake, 8, None, None,
+                                  _lib.Buf(0x1000, 16), fake, None) == 3
     assert lib.zha_launch_count() == n0
