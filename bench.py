@@ -57,6 +57,9 @@ def parse():
                     help="zha: the hot path (default); dense / flat: the baselines on the same inputs")
     ap.add_argument("--sweep", action="store_true",
                     help="crossover sweep over T and depth against the dense kernel (one JSON line each)")
+    ap.add_argument("--model", metavar="FILE", default=None,
+                    help="no GPU work: read bench JSON lines of the zha path from FILE and print the "
+                         "pages' roofline model of each beside its measured stage times")
     return ap.parse_args()
 
 
@@ -249,6 +252,127 @@ def frontier_stats(level_cnt: np.ndarray) -> list:
                     "candidates_max": int(c[on].max()),
                     "kept_mean": float(k[on].mean()), "kept_p50": float(np.median(k[on])),
                     "kept_max": int(k[on].max())})
+    return out
+
+
+FP64_TENSOR_TFLOPS = 40.0      # nominal dense fp64 tensor-core rate of a B200 (no measured figure here)
+
+
+def paper_model(line: dict, peaks: dict) -> dict:
+    """The pages' decode roofline model (arXiv 2610.42112 §V-A, App. D-B) with this GPU's
+    constants, set against the measured stage times of one bench line of the zha path.
+
+    Per stage x, Phi_x = max(FLOPs_x / P_x, bytes_x / BW, t_waves).  The worker-wave term
+    needs a per-block latency tau_x; it is calibrated here as the measured time of the same
+    kernel's launch at the top level, whose few candidates fit in one wave (so tau is the
+    kernel's fixed latency and the wave count is taken as 1).  Counts follow App. D-B1
+    with this implementation's element sizes:
+      routing, level l:  FLOPs = 2 B Hq R d K_l (every head scores its own candidates, on the
+                         fp64 tensor cores here); bytes = R (s d + 4) B Hkv K_l^grp + s d B Hq
+                         (each node of a KV group's candidate union K_l^grp is read once;
+                         without the union in the line, the largest per-head frontier, a
+                         lower bound, stands in for it);
+      scan, level l:     bytes = 12 B Hq K_l (an fp64 score and an int32 id per candidate,
+                         one pass: the select keeps the scores in shared memory);
+      attention:         FLOPs = 2 B Hq (d_k + d_v) K_0; bytes = the bench's gathered bytes
+                         (K_0 union rows of K and V per KV group) + split partials (d_v + 2
+                         fp32 values per head and split), i.e. bytes_attn,split;
+      tree (decode):     amortised: one leaf summary per `leaf` appended tokens per unit,
+                         64 d s read + R (d s + 4 d + 8) written (parents add 1/branch of it);
+      launches:          lambda = step time minus the traced kernels' time, plus the
+                         launches of levels above the top one (no visible node there).
+    """
+    cfg = line["config"]
+    B, Hq, Hkv, d, R = cfg["B"], cfg["Hq"], cfg["Hkv"], cfg["d"], cfg["R"]
+    leaf = cfg.get("leaf", 64)
+    s = 2 if line["dtype"] == "bf16" else 4
+    bw = peaks["hbm_gbs"] * 1e9
+    p16 = peaks["bf16_tflops"] * 1e12
+    p64 = FP64_TENSOR_TFLOPS * 1e12
+    st = line["stages_ms"]
+    levels = line["frontier"]["levels"]               # top level first
+    depth = cfg["depth"]
+    # one score and one select launch per level, from level `depth` down (empty levels too)
+    score_ms = lambda l: st["route_score_per_launch"][depth - l]     # noqa: E731
+    select_ms = lambda l: st["route_select_per_launch"][depth - l]   # noqa: E731
+    top = levels[0]["level"]
+    tau = {"score": score_ms(top), "select": select_ms(top)}
+
+    def row(stage, kind, flops, byts, peak, unit, measured):
+        t_f, t_b = 1e3 * flops / peak, 1e3 * byts / bw
+        t_w = tau.get(kind, 0.0)
+        model = max(t_f, t_b, t_w)
+        bound = "latency (one wave)" if model == t_w and t_w > 0 else (unit if t_f > t_b else "hbm")
+        return {"stage": stage, "flops": flops, "bytes": byts, "flops_ms": t_f, "bytes_ms": t_b,
+                "waves_ms": t_w, "model_ms": model, "bound": bound, "measured_ms": measured}
+
+    rows = []
+    for f in levels:
+        l = f["level"]
+        k_head = f["candidates_mean"]
+        k_grp = f.get("candidates_group_union", f["candidates_max"])
+        rows.append(row(f"route score L{l}", "score", 2.0 * B * Hq * R * d * k_head,
+                        R * (s * d + 4) * B * Hkv * k_grp + s * d * B * Hq, p64, "fp64 tensor", score_ms(l)))
+        rows.append(row(f"route select L{l}", "select", 0.0, 12.0 * B * Hq * k_head, p64, "alu",
+                        select_ms(l)))
+    T1 = cfg["T"] + 1
+    k0 = line["kv_touched"]["mean"] * T1
+    byts = line["roofline"]["algorithmic_bytes_per_launch"] * line["roofline"]["launches_per_step"]
+    rows.append(row("attention", "attention", 2.0 * B * Hq * 2 * d * k0, byts, p16, "bf16 tensor",
+                    st["attention"]))
+    leaf_bytes = leaf * d * s + R * (d * s + 4 * d + 8)
+    byts = B * Hkv * leaf_bytes / leaf * (1 + 1 / max(1, cfg.get("branch", 16) - 1))
+    rows.append(row("tree (amortised per step)", "tree", 4.0 * R * d * B * Hkv, byts, p64, "fp64 tensor",
+                    line["tree_build"]["ms"] / cfg["T"]))
+    # levels above the top one have no visible node: their score and select launches are
+    # launch overhead only (the lambda_l of the model), with the gaps between kernels
+    empty = 0.0
+    for l in range(depth, top, -1):
+        t = score_ms(l) + select_ms(l)
+        empty += t
+        rows.append({"stage": f"route L{l} (empty)", "flops": 0.0, "bytes": 0.0, "flops_ms": 0.0,
+                     "bytes_ms": 0.0, "waves_ms": 0.0, "model_ms": 0.0, "bound": "launch only",
+                     "measured_ms": t})
+    kernels = sum(r["model_ms"] for r in rows)
+    lam = max(0.0, st["step"] - st["stage_sum"]) + empty
+    for r in rows:
+        r["measured_over_model"] = r["measured_ms"] / r["model_ms"] if r["model_ms"] > 0 else None
+    return {"workload": cfg["workload"], "rows": rows, "model_kernels_ms": kernels,
+            "measured_step_ms": st["step"], "launch_gaps_ms": lam,
+            "launches_per_step": line["gpu_launches"] / line["steps"],
+            "model_step_ms": kernels + lam,
+            "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                      "fp64_tensor_tflops": FP64_TENSOR_TFLOPS}}
+
+
+def candidate_unions(level_cnt: np.ndarray, level_ids: np.ndarray, n_cap: dict, nvis: dict, G: int,
+                     branch: int) -> dict:
+    """Per level, the mean over KV groups of the size of the group's candidate union (the
+    nodes the score kernel reads once per group), from zha_route's level counts
+    [B, nq, Hq, depth, 2] and kept ids [B, nq, Hq, sum_{l>=2} n_cap(l)] (one query per
+    sequence).  At the top level every head's candidates are the visible nodes; below it,
+    the children of the union of the heads' kept parents plus the orphans (visible nodes
+    whose parent is not visible)."""
+    B, _, Hq, depth, _ = level_cnt.shape
+    offs, off = {}, 0
+    for l in range(2, depth + 1):
+        offs[l] = off
+        off += n_cap[l]
+    top = max((l for l in range(1, depth + 1) if nvis.get(l, 0) >= 1), default=0)
+    out = {}
+    for l in range(top, 0, -1):
+        sizes = []
+        for b in range(B):
+            for g0 in range(0, Hq, G):
+                if l == top:
+                    sizes.append(nvis[top])
+                    continue
+                kept = set()
+                for h in range(g0, g0 + G):
+                    n = int(level_cnt[b, 0, h, l, 1])            # kept at level l + 1
+                    kept.update(level_ids[b, 0, h, offs[l + 1]:offs[l + 1] + n].tolist())
+                sizes.append(branch * len(kept) + nvis[l] - branch * nvis[l + 1])
+        out[l] = float(np.mean(sizes))
     return out
 
 
@@ -448,6 +572,17 @@ def run_sweep(args):
 
 def main():
     args = parse()
+    if args.model:
+        peaks = {"hbm_gbs": hbm_peak()[0], "bf16_tflops": 1590.0}
+        try:
+            peaks["bf16_tflops"] = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["bf16_tflops"]
+        except (OSError, ValueError, KeyError):
+            pass
+        for raw in open(args.model):
+            raw = raw.strip()
+            if raw.startswith("{") and '"frontier"' in raw and '"path": "zha"' in raw:
+                print(json.dumps(paper_model(json.loads(raw), peaks)), flush=True)
+        return
     if args.sweep:
         run_sweep(args)
         return
@@ -634,16 +769,24 @@ def main():
     if args.path == "zha":
         try:
             lcnt = torch.zeros(w.B, 1, w.Hq, w.depth, 2, dtype=torch.int32, device=dev)
+            n_cap = {l: Z.tree_level(g, l).n_cap for l in range(2, w.depth + 1)}
+            lids = torch.zeros(w.B, 1, w.Hq, max(1, sum(n_cap.values())), dtype=torch.int32, device=dev)
             ids2, cnt2 = torch.empty_like(ids), torch.empty_like(cnt)
             qpos = torch.full((w.B, 1), w.T, dtype=torch.int64, device=dev)
-            Z.zha_route(g, q, qpos, p, tree, ids2, cnt2, wsb, st, lcnt)
+            Z.zha_route(g, q, qpos, p, tree, ids2, cnt2, wsb, st, lcnt, lids)
             torch.cuda.synchronize()
+            lc_np = lcnt.cpu().numpy()
+            nvis = {l: (64 * (w.T // 64)) // (64 * w.branch ** (l - 1)) for l in range(1, w.depth + 1)}
+            unions = candidate_unions(lc_np, lids.cpu().numpy(), n_cap, nvis, w.G, w.branch)
             ids2_c, cnt2_c = ids2.cpu().numpy(), cnt2.cpu().numpy()
             same = bool(np.array_equal(cnt2_c, cnt_c)) and all(
                 np.array_equal(ids2_c[bb, 0, h, :cnt_c[bb, 0, h]], ids_c[bb, 0, h, :cnt_c[bb, 0, h]])
                 for bb in range(w.B) for h in range(w.Hq))
-            frontier = {"levels": frontier_stats(lcnt.cpu().numpy()), "route_matches_decode": same}
-            del lcnt, ids2, cnt2
+            levels = frontier_stats(lc_np)
+            for f in levels:
+                f["candidates_group_union"] = unions.get(f["level"])
+            frontier = {"levels": levels, "route_matches_decode": same}
+            del lcnt, lids, ids2, cnt2
         except Exception as e:   # statistics outside the timed region: report, do not hide
             frontier = {"error": repr(e)}
     cpu = None

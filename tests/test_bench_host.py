@@ -7,6 +7,7 @@ import subprocess
 import sys
 
 import numpy as np
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 sys.path.insert(0, ROOT)
@@ -57,3 +58,74 @@ def test_reference_arm_line_on_cpu():
     for key in ("metric", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
                 "scaling", "dtype", "data", "config", "e2e"):
         assert key in line
+
+
+def _gpu_layout(routes_by_head, depth, n_cap):
+    """Oracle routes of one sequence's heads in zha_route's level_cnt / level_ids layout."""
+    Hq = len(routes_by_head)
+    lc = np.zeros((1, 1, Hq, depth, 2), np.int32)
+    lids = np.full((1, 1, Hq, sum(n_cap.values())), -1, np.int32)
+    for h, r in enumerate(routes_by_head):
+        off = 0
+        for l in range(2, depth + 1):
+            if l in r.sel:
+                lc[0, 0, h, l - 1] = (len(r.cand[l]), r.sel[l].m)
+                lids[0, 0, h, off:off + r.sel[l].m] = r.sel[l].ids
+            off += n_cap[l]
+        lc[0, 0, h, 0] = (len(r.cand[1]), r.sel[1].m)
+    return lc, lids
+
+
+def test_candidate_unions_match_the_oracle_candidate_sets():
+    d, leaf, branch, depth = 8, 4, 4, 3
+    T = 4 * 4 * 4 * 3 + 4 * 4 + 3 * 4 + 2          # orphans at levels 1 and 2
+    rng = np.random.default_rng(8)
+    C = rng.standard_normal((4, d))
+    K = C[rng.integers(0, 4, T + 1)] + 0.3 * rng.standard_normal((T + 1, d))
+    qref = rng.standard_normal((2, d)) / math.sqrt(d)
+    tree = zo.build_tree(K, T + 1, qref, depth=depth, leaf=leaf, branch=branch, route_storage="f64")
+    G = 4
+    routes = [zo.route(2 * C[h % 4] + 0.3 * rng.standard_normal(d), T, tree, 0.6) for h in range(2 * G)]
+    n_cap = {l: (T + 1) // (leaf * branch ** (l - 1)) for l in range(2, depth + 1)}
+    lc, lids = _gpu_layout(routes, depth, n_cap)
+    v = leaf * (T // leaf)
+    nvis = {l: v // (leaf * branch ** (l - 1)) for l in range(1, depth + 1)}
+    got = bench.candidate_unions(lc, lids, n_cap, nvis, G, branch)
+    assert sorted(got) == [1, 2, 3]
+    for l in (1, 2, 3):
+        want = np.mean([len(np.unique(np.concatenate([r.cand[l] for r in routes[g:g + G]])))
+                        for g in (0, G)])
+        assert got[l] == want
+
+
+def test_paper_model_terms():
+    line = {"dtype": "bf16", "steps": 10, "gpu_launches": 80,
+            "config": {"workload": "w", "B": 2, "Hq": 16, "Hkv": 2, "d": 128, "R": 4, "T": 65536,
+                       "leaf": 64, "branch": 16, "depth": 3},
+            "frontier": {"levels": [
+                {"level": 2, "candidates_mean": 64.0, "candidates_max": 64, "candidates_group_union": 64.0},
+                {"level": 1, "candidates_mean": 900.0, "candidates_max": 950, "candidates_group_union": 1000.0}]},
+            # depth 3 with an empty top level: three launches per kind, level 3 first
+            "stages_ms": {"route_score_per_launch": [0.004, 0.01, 0.02],
+                          "route_select_per_launch": [0.003, 0.005, 0.01],
+                          "attention": 0.05, "step": 0.1, "stage_sum": 0.095},
+            "kv_touched": {"mean": 0.5}, "tree_build": {"ms": 0.4},
+            "roofline": {"algorithmic_bytes_per_launch": 1e8, "launches_per_step": 1.0}}
+    peaks = {"hbm_gbs": 5000.0, "bf16_tflops": 1000.0}
+    m = bench.paper_model(line, peaks)
+    rows = {r["stage"]: r for r in m["rows"]}
+    r1 = rows["route score L1"]
+    # 2 B Hq R d K flops; R (s d + 4) B Hkv K_grp + s d B Hq bytes
+    assert r1["flops"] == 2 * 2 * 16 * 4 * 128 * 900.0
+    assert r1["bytes"] == 4 * (2 * 128 + 4) * 2 * 2 * 1000.0 + 2 * 128 * 2 * 16
+    assert r1["model_ms"] == pytest.approx(max(1e3 * r1["flops"] / 40e12, 1e3 * r1["bytes"] / 5e12, 0.01))
+    assert r1["measured_ms"] == 0.02 and rows["route score L2"]["measured_ms"] == 0.01
+    # the wave term: the top level's launch (level 2 here) calibrates tau
+    assert rows["route score L2"]["waves_ms"] == 0.01 and rows["route select L1"]["waves_ms"] == 0.005
+    assert rows["route select L2"]["bytes"] == 12 * 2 * 16 * 64.0
+    att = rows["attention"]
+    assert att["bytes"] == 1e8 and att["model_ms"] == pytest.approx(1e3 * 1e8 / 5e12)
+    assert att["measured_over_model"] == pytest.approx(0.05 / att["model_ms"])
+    # launch overhead: the gaps between kernels plus the launches of the empty level 3
+    assert m["launch_gaps_ms"] == pytest.approx(0.005 + 0.004 + 0.003) and m["launches_per_step"] == 8
+    assert rows["route L3 (empty)"]["measured_ms"] == pytest.approx(0.007)
