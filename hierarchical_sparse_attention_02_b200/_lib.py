@@ -30,7 +30,7 @@ class Geom(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32), ("d", ctypes.c_int32),
                 ("leaf", ctypes.c_int32), ("branch", ctypes.c_int32), ("depth", ctypes.c_int32),
                 ("R", ctypes.c_int32), ("t_cap", ctypes.c_int64), ("dtype", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("rope_pairs", ctypes.c_int32)]
 
 
 class Buf(ctypes.Structure):

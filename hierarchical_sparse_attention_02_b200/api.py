@@ -38,6 +38,7 @@ class Geometry:
     leaf: int = 64
     branch: int = 16
     dtype: torch.dtype = torch.bfloat16
+    rope_pairs: int = 0          # > 0: qref carries that many rotary frequencies after the references
 
     @property
     def G(self) -> int:
@@ -45,7 +46,18 @@ class Geometry:
 
     def c(self) -> _lib.Geom:
         return _lib.Geom(self.B, self.Hq, self.Hkv, self.d, self.leaf, self.branch, self.depth, self.R,
-                         self.t_cap, _lib.ZHA_BF16 if self.dtype == torch.bfloat16 else _lib.ZHA_F32, 0)
+                         self.t_cap, _lib.ZHA_BF16 if self.dtype == torch.bfloat16 else _lib.ZHA_F32,
+                         self.rope_pairs)
+
+
+def reference_block(qref: torch.Tensor, inv_freq: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The reference-query argument of the tree calls: q_hat [Hkv, R, d] fp32, followed by the
+    rotary frequencies (fp32) of a RoPE model when there are any (geometry rope_pairs =
+    len(inv_freq))."""
+    q = qref.float().contiguous().reshape(-1)
+    if inv_freq is None or inv_freq.numel() == 0:
+        return q
+    return torch.cat([q, inv_freq.to(device=q.device, dtype=torch.float32).reshape(-1)])
 
 
 def _ptr(t: Optional[torch.Tensor]):
@@ -106,15 +118,25 @@ def empty_workspace(g: Geometry, nq: int, op: int, device="cuda") -> torch.Tenso
     return torch.empty(workspace_bytes(g, nq, op), dtype=torch.uint8, device=device)
 
 
+def _qref(g, qref: torch.Tensor):
+    """The reference block the library reads: Hkv*R*d fp32 values, plus g.rope_pairs
+    frequencies (reference_block); a shorter tensor would be read past its end."""
+    need = g.Hkv * g.R * g.d + g.rope_pairs
+    if qref.dtype != torch.float32 or qref.numel() != need:
+        raise ValueError(f"qref: expected {need} fp32 values (Hkv*R*d references + {g.rope_pairs} "
+                         f"rotary frequencies), got {qref.numel()} {qref.dtype}")
+    return _ptr(qref)
+
+
 def zha_build_tree(g, K, T, qref, tree, dev_status, stream=None):
     _check("zha_build_tree", _lib.load().zha_build_tree(
-        ctypes.byref(g.c()), _ptr(K), T, _ptr(qref), _buf(tree), _ptr(dev_status), _stream(stream)))
+        ctypes.byref(g.c()), _ptr(K), T, _qref(g, qref), _buf(tree), _ptr(dev_status), _stream(stream)))
 
 
 def zha_append(g, K, V, k_new, v_new, t_old, qref, tree, dev_status, stream=None):
     _check("zha_append", _lib.load().zha_append(
         ctypes.byref(g.c()), _ptr(K), _ptr(V), _ptr(k_new), _ptr(v_new), t_old, k_new.shape[1],
-        _ptr(qref), _buf(tree), _ptr(dev_status), _stream(stream)))
+        _qref(g, qref), _buf(tree), _ptr(dev_status), _stream(stream)))
 
 
 def zha_route(g, Q, q_pos, p, tree, leaf_ids, leaf_cnt, ws, dev_status, level_cnt=None, level_ids=None,
@@ -153,7 +175,7 @@ def zha_sparse_attn_noalloc(g, Q, K, V, q_pos, leaf_ids, leaf_cnt, O, dev_status
 def zha_decode(g, q, k_new, v_new, K, V, T, qref, p, tree, leaf_ids, leaf_cnt, O, ws, dev_status,
                stream=None):
     _check("zha_decode", _lib.load().zha_decode(
-        ctypes.byref(g.c()), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(K), _ptr(V), T, _ptr(qref), float(p),
+        ctypes.byref(g.c()), _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(K), _ptr(V), T, _qref(g, qref), float(p),
         _buf(tree), _ptr(leaf_ids), _ptr(leaf_cnt), leaf_ids.shape[-1], _ptr(O), _buf(ws), _ptr(dev_status),
         _stream(stream)))
 

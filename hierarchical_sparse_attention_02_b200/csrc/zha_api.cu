@@ -51,7 +51,7 @@ zha_status zha_check_geom(const zha_geom* g) {
   if (g->B < 1 || g->Hq < 1 || g->Hkv < 1 || g->R < 1 || g->depth < 1 || g->t_cap < 1)
     return ZHA_ERR_INVALID_ARG;
   if (g->Hq % g->Hkv != 0) return ZHA_ERR_INVALID_ARG;
-  if (g->reserved != 0) return ZHA_ERR_INVALID_ARG;
+  if (g->rope_pairs < 0 || g->rope_pairs > g->d / 2) return ZHA_ERR_INVALID_ARG;
   if (g->d != kD || g->leaf != kLeaf) return ZHA_ERR_UNSUPPORTED;
   if (g->Hq / g->Hkv > kMaxG || g->R > kMaxR || g->depth > kMaxDepth) return ZHA_ERR_UNSUPPORTED;
   if (g->R & (g->R - 1)) return ZHA_ERR_UNSUPPORTED;     // R in {1, 2, 4, 8, 16}

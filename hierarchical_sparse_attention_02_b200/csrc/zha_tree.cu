@@ -5,6 +5,11 @@
 //   k_hat_r = sum_j a_rj k_j,  b_hat_r = F_r - q_hat_r . k_hat_r / sqrt(d).
 // Parent merge (§III-B; App. D-B2, per-reference stable-state merge, no re-anchoring):
 //   F_P = LSE_c F_c,  k_hat_P = sum_c exp(F_c - F_P) k_hat_c,  b_hat_P as above.
+// Rotary positions (§III-B, models with RoPE; geometry rope_pairs = h > 0, the h rotary
+// frequencies f_i stored after the reference queries): a node's references are rotated to
+// its last key position P, dims (i, i + h) by the angle P * f_i, and before a merge each
+// child's log mass moves to the parent's rotated reference along its tangent plane,
+//   F_c += <k_hat_c, q_hat_P - q_hat_c> / sqrt(d).
 // All arithmetic is fp64 with fixed-order reductions, so a summary is bit-identical
 // from run to run and agrees with an exact evaluation to ~1e-15 before it is stored
 // (merge state fp32, routing k_hat in the KV dtype, b_hat fp32).  The kernels are
@@ -12,6 +17,24 @@
 #include "zha_internal.cuh"
 
 namespace zha {
+
+// Element `dim` of reference row q (fp32, d values) rotated by the angles whose cosines and
+// sines are cs[i], sn[i] (i < h): dims i < h take x_i cos - x_{i+h} sin, dims h <= i < 2h
+// take x_i cos + x_{i-h} sin, the rest pass through.  Each product and the sum are rounded
+// separately (no fused multiply-add), the order of the plain formula.
+// rope_one: the same for one element, given the cosine and sine of its pair's angle.
+__device__ __forceinline__ double rope_one(const float* q, int dim, int h, double c, double s) {
+  const double x = (double)q[dim];
+  if (dim < h) return __dsub_rn(__dmul_rn(x, c), __dmul_rn((double)q[dim + h], s));
+  if (dim < 2 * h) return __dadd_rn(__dmul_rn(x, c), __dmul_rn((double)q[dim - h], s));
+  return x;
+}
+
+__device__ __forceinline__ double rope_elem(const float* q, int dim, int h, const double* cs,
+                                            const double* sn) {
+  const int j = dim < h ? dim : dim - h;             // the pair of dim (unused past 2h)
+  return dim < 2 * h ? rope_one(q, dim, h, cs[j], sn[j]) : (double)q[dim];
+}
 
 struct LevelPtrs {
   void* k_route;
@@ -50,10 +73,10 @@ struct alignas(16) LeafTcSmem {
   double red[4][R];                                  // per-warp q_hat . k_hat partials
 };
 
-template <typename KT, int R>
+template <typename KT, int R, bool ROPE>
 __global__ void __launch_bounds__(128) leaf_summarize_tc_kernel(
     const KT* __restrict__ K, const float* __restrict__ qref, int Hkv, int64_t t_cap,
-    int64_t leaf_lo, int64_t nleaf, LevelPtrs out, double scale) {
+    int64_t leaf_lo, int64_t nleaf, LevelPtrs out, double scale, int rope_pairs) {
   using Sm = LeafTcSmem<KT, R>;
   constexpr int NT = Sm::NT;
   extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -63,10 +86,24 @@ __global__ void __launch_bounds__(128) leaf_summarize_tc_kernel(
   const int64_t leaf = leaf_lo + blockIdx.x % nleaf;
   const int h = (int)(unit % Hkv);
   const float* q = qref + (int64_t)h * R * kD;
-  for (int i = tid; i < NT * 32 * 32; i += 128) {
-    const int nt = i / 1024, s = (i / 32) % 32, L = i % 32;
-    const int r = nt * 8 + (L >> 2);
-    sm.qf[nt][s][L] = r < R ? (double)q[r * kD + 32 * (L & 3) + s] : 0.0;
+  if constexpr (ROPE) {
+    // the references rotated to the leaf's last key
+    __shared__ double cs[kD / 2], sn[kD / 2];
+    const float* freq = qref + (int64_t)Hkv * R * kD;
+    const double pos = (double)((leaf + 1) * kLeaf - 1);
+    if (tid < rope_pairs) sincos(pos * (double)freq[tid], &sn[tid], &cs[tid]);
+    __syncthreads();
+    for (int i = tid; i < NT * 32 * 32; i += 128) {
+      const int nt = i / 1024, s = (i / 32) % 32, L = i % 32;
+      const int r = nt * 8 + (L >> 2);
+      sm.qf[nt][s][L] = r < R ? rope_elem(q + r * kD, 32 * (L & 3) + s, rope_pairs, cs, sn) : 0.0;
+    }
+  } else {
+    for (int i = tid; i < NT * 32 * 32; i += 128) {
+      const int nt = i / 1024, s = (i / 32) % 32, L = i % 32;
+      const int r = nt * 8 + (L >> 2);
+      sm.qf[nt][s][L] = r < R ? (double)q[r * kD + 32 * (L & 3) + s] : 0.0;
+    }
   }
   __syncthreads();
 
@@ -199,10 +236,10 @@ __global__ void __launch_bounds__(128) leaf_summarize_tc_kernel(
 
 constexpr int kMaxBranch = 64;
 
-template <typename KT, int R>
+template <typename KT, int R, bool ROPE>
 __global__ void __launch_bounds__(128) parent_merge_kernel(
     const float* __restrict__ qref, int Hkv, int branch, int64_t lo, int64_t n,
-    LevelPtrs child, LevelPtrs out, double scale) {
+    LevelPtrs child, LevelPtrs out, double scale, int rope_pairs, int64_t span_c) {
   __shared__ double Fc[kMaxBranch][R];
   __shared__ double w[kMaxBranch][R];
   __shared__ double Fp[R];
@@ -212,9 +249,40 @@ __global__ void __launch_bounds__(128) parent_merge_kernel(
   const int64_t node = lo + blockIdx.x % n;
   const int h = (int)(unit % Hkv);
   const int64_t c0 = unit * child.n_cap + node * branch;   // first child entry
+  const float* qh = qref + (int64_t)h * R * kD;
   for (int i = tid; i < branch * R; i += 128) {
     const int c = i / R, r = i % R;
     Fc[c][r] = (double)child.F[(c0 + c) * R + r];
+  }
+  // with rotation: this thread's element (dim = tid) of every rotated parent reference
+  double qp[ROPE ? R : 1];
+  if constexpr (ROPE) {
+    __shared__ double cr[2][4][R];                         // per-warp partials, double-buffered
+    const float* freq = qref + (int64_t)Hkv * R * kD;
+    const int j = tid < rope_pairs ? tid : (tid < 2 * rope_pairs ? tid - rope_pairs : -1);
+    const double f = j >= 0 ? (double)freq[j] : 0.0;
+    double c = 1.0, sv = 0.0;
+    if (j >= 0) sincos((double)((node + 1) * span_c * branch - 1) * f, &sv, &c);
+#pragma unroll
+    for (int r = 0; r < R; ++r) qp[r] = rope_one(qh + r * kD, tid, rope_pairs, c, sv);
+    __syncthreads();                                       // Fc is loaded
+    // re-anchor each child: F_c += scale * <k_hat_c, q_hat_P - q_hat_c>
+    for (int ci = 0; ci < branch; ++ci) {
+      double cc = 1.0, sc = 0.0;
+      if (j >= 0) sincos((double)((node * branch + ci + 1) * span_c - 1) * f, &sc, &cc);
+      const float* ks = child.k_state + (c0 + ci) * R * kD;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const double diff = j >= 0 ? qp[r] - rope_one(qh + r * kD, tid, rope_pairs, cc, sc) : 0.0;
+        double v = j >= 0 ? (double)ks[r * kD + tid] * diff : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) v += shfl_xor_f64(v, o);
+        if (lane == 0) cr[ci & 1][warp][r] = v;
+      }
+      __syncthreads();
+      if (tid < R)
+        Fc[ci][tid] += scale * ((cr[ci & 1][0][tid] + cr[ci & 1][1][tid]) + (cr[ci & 1][2][tid] + cr[ci & 1][3][tid]));
+    }
   }
   __syncthreads();
   // F_P = LSE_c F_c (one thread per reference, children in order)
@@ -242,7 +310,7 @@ __global__ void __launch_bounds__(128) parent_merge_kernel(
   }
 #pragma unroll
   for (int r = 0; r < R; ++r) {
-    double v = (double)qref[((int64_t)h * R + r) * kD + tid] * acc[r];
+    double v = (ROPE ? qp[ROPE ? r : 0] : (double)qh[r * kD + tid]) * acc[r];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += shfl_xor_f64(v, o);
     if (lane == 0) red[warp][r] = v;
@@ -288,56 +356,64 @@ __global__ void append_kv_kernel(uint4* __restrict__ K, uint4* __restrict__ V,
 // host drivers
 // ---------------------------------------------------------------------------
 
-template <typename KT, int R>
+template <typename KT, int R, bool ROPE>
 static cudaError_t launch_leaves(const zha_geom& g, const TreeLayout& L, const void* K,
                                  const float* qref, void* tree, int64_t lo, int64_t hi,
                                  cudaStream_t s) {
   const int64_t n = hi - lo;
   const int64_t blocks = (int64_t)g.B * g.Hkv * n;
   const size_t smem = sizeof(LeafTcSmem<KT, R>);
-  cudaFuncSetAttribute(leaf_summarize_tc_kernel<KT, R>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaFuncSetAttribute(leaf_summarize_tc_kernel<KT, R, ROPE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                        (int)smem);
-  leaf_summarize_tc_kernel<KT, R><<<(unsigned)blocks, 128, smem, s>>>(
-      (const KT*)K, qref, g.Hkv, g.t_cap, lo, n, level_ptrs(g, L, tree, 1), 1.0 / sqrt((double)g.d));
+  leaf_summarize_tc_kernel<KT, R, ROPE><<<(unsigned)blocks, 128, smem, s>>>(
+      (const KT*)K, qref, g.Hkv, g.t_cap, lo, n, level_ptrs(g, L, tree, 1), 1.0 / sqrt((double)g.d),
+      g.rope_pairs);
   count_launch();
   return launch_status("leaf_summarize_tc_kernel");
 }
 
-template <typename KT, int R>
+template <typename KT, int R, bool ROPE>
 static cudaError_t launch_merge(const zha_geom& g, const TreeLayout& L, const float* qref,
                                 void* tree, int level, int64_t lo, int64_t hi, cudaStream_t s) {
   const int64_t n = hi - lo;
   const int64_t blocks = (int64_t)g.B * g.Hkv * n;
-  parent_merge_kernel<KT, R><<<(unsigned)blocks, 128, 0, s>>>(
+  parent_merge_kernel<KT, R, ROPE><<<(unsigned)blocks, 128, 0, s>>>(
       qref, g.Hkv, g.branch, lo, n, level_ptrs(g, L, tree, level - 1), level_ptrs(g, L, tree, level),
-      1.0 / sqrt((double)g.d));
+      1.0 / sqrt((double)g.d), g.rope_pairs, span_of(g, level - 1));
   count_launch();
   return launch_status("parent_merge_kernel");
 }
 
-template <typename KT, int R>
+template <typename KT, int R, bool ROPE>
 static cudaError_t extend_t(const zha_geom& g, const TreeLayout& L, const void* K, const float* qref,
                             void* tree, int64_t t_old, int64_t t_new, cudaStream_t s) {
   for (int l = 1; l <= g.depth; ++l) {
     const int64_t span = span_of(g, l);
     const int64_t lo = t_old / span, hi = t_new / span;
     if (hi <= lo) break;   // nothing completes at this level, nor above
-    const cudaError_t e = l == 1 ? launch_leaves<KT, R>(g, L, K, qref, tree, lo, hi, s)
-                                 : launch_merge<KT, R>(g, L, qref, tree, l, lo, hi, s);
+    const cudaError_t e = l == 1 ? launch_leaves<KT, R, ROPE>(g, L, K, qref, tree, lo, hi, s)
+                                 : launch_merge<KT, R, ROPE>(g, L, qref, tree, l, lo, hi, s);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+template <typename KT, int R>
+static cudaError_t extend_rope(const zha_geom& g, const TreeLayout& L, const void* K, const float* qref,
+                               void* tree, int64_t t_old, int64_t t_new, cudaStream_t s) {
+  return g.rope_pairs > 0 ? extend_t<KT, R, true>(g, L, K, qref, tree, t_old, t_new, s)
+                          : extend_t<KT, R, false>(g, L, K, qref, tree, t_old, t_new, s);
 }
 
 template <typename KT>
 static cudaError_t extend_r(const zha_geom& g, const TreeLayout& L, const void* K, const float* qref,
                             void* tree, int64_t t_old, int64_t t_new, cudaStream_t s) {
   switch (g.R) {
-    case 1: return extend_t<KT, 1>(g, L, K, qref, tree, t_old, t_new, s);
-    case 2: return extend_t<KT, 2>(g, L, K, qref, tree, t_old, t_new, s);
-    case 4: return extend_t<KT, 4>(g, L, K, qref, tree, t_old, t_new, s);
-    case 8: return extend_t<KT, 8>(g, L, K, qref, tree, t_old, t_new, s);
-    case 16: return extend_t<KT, 16>(g, L, K, qref, tree, t_old, t_new, s);
+    case 1: return extend_rope<KT, 1>(g, L, K, qref, tree, t_old, t_new, s);
+    case 2: return extend_rope<KT, 2>(g, L, K, qref, tree, t_old, t_new, s);
+    case 4: return extend_rope<KT, 4>(g, L, K, qref, tree, t_old, t_new, s);
+    case 8: return extend_rope<KT, 8>(g, L, K, qref, tree, t_old, t_new, s);
+    case 16: return extend_rope<KT, 16>(g, L, K, qref, tree, t_old, t_new, s);
     default: return cudaErrorInvalidValue;   // zha_check_geom admits powers of two only
   }
 }

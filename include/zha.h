@@ -19,7 +19,9 @@
  *      Q, O      [B, nq, Hq, d]      dtype
  *      q_pos     [B, nq]             int64  absolute position t of each query (its own key
  *                                           is already in the cache at position t)
- *      qref      [Hkv, R, d]         fp32   reference queries, shared by all nodes and levels
+ *      qref      [Hkv, R, d]         fp32   reference queries, shared by all nodes and levels;
+ *                                           with g->rope_pairs = h > 0 followed by h fp32 rotary
+ *                                           frequencies f_0..f_{h-1} (the model's RoPE table)
  *      leaf_ids  [B, nq, Hq, leaf_cap] int32 selected leaf-chunk ids, ascending
  *      leaf_cnt  [B, nq, Hq]         int32
  *      k_new, v_new [B, n_new, Hkv, d] dtype
@@ -69,6 +71,7 @@ typedef enum zha_op {
 
 /* Geometry of one attention layer and its tree (host struct).
  * d must be 128; leaf must be 64; 2 <= branch <= 64; 1 <= depth <= 8; R in {1, 2, 4, 8, 16};
+ * 0 <= rope_pairs <= d / 2;
  * Hq % Hkv == 0 and Hq / Hkv <= 8; t_cap % leaf == 0; dtype a zha_dtype;
  * B * Hkv * t_cap * d * 4 <= 2^48 (bytes of the cache counted at 4 bytes per element),
  * else ZHA_ERR_UNSUPPORTED, so that no byte count the library forms can overflow. */
@@ -80,7 +83,8 @@ typedef struct zha_geom {
   int32_t R;        /* reference queries per KV head                       */
   int64_t t_cap;    /* cache capacity per sequence, in tokens              */
   int32_t dtype;    /* zha_dtype                                           */
-  int32_t reserved; /* must be 0                                           */
+  int32_t rope_pairs; /* 0: no rotary positions; h in 1..d/2: reference queries are
+                         rotated to each node's last position (see qref below)   */
 } zha_geom;
 
 /* A caller-owned device buffer. */
@@ -130,10 +134,15 @@ int64_t zha_leaf_cap(const zha_geom* g);
  *   k_hat_r = sum_j a_j k_j,   b_hat_r = F_r - q_hat_r . k_hat_r / sqrt(d).
  * Parents (§III-B, App. D-B2, stable-state merge without re-anchoring): per reference,
  *   F_P = LSE_c F_c,  k_hat_P = sum_c exp(F_c - F_P) k_hat_c,  b_hat_P = F_P - q_hat . k_hat_P / sqrt(d).
+ * Rotary positions (§III-B, models with RoPE), when g->rope_pairs = h > 0: the references
+ * of a node are rotated to its last key position P (dims i and i + h, i < h, by the angle
+ * P * f_i; dims >= 2h unrotated), and before a merge each child's log mass is moved to the
+ * parent's rotated reference along its tangent plane, F_c += <k_hat_c, q_hat_P - q_hat_c> / sqrt(d).
+ * The keys in the cache are taken as stored (already rotated by the model).
  * One launch for the leaves and one per parent level.  Arithmetic is fp64; the merge
  * state is stored as fp32, the routing k_hat in dtype, b_hat in fp32.
  *   K     [B, Hkv, t_cap, d] dtype; keys [0, T) are read.   0 <= T <= t_cap.
- *   qref  [Hkv, R, d] fp32.
+ *   qref  [Hkv, R, d] fp32 (+ g->rope_pairs fp32 frequencies).
  *   tree  at least zha_tree_bytes(g) bytes; nodes beyond T are left untouched.
  */
 zha_status zha_build_tree(const zha_geom* g, const void* K, int64_t T, const float* qref,

@@ -33,7 +33,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def geom(**kw):
-    base = dict(B=2, Hq=16, Hkv=2, d=128, leaf=64, branch=16, depth=3, R=4, t_cap=65536, dtype=1, reserved=0)
+    base = dict(B=2, Hq=16, Hkv=2, d=128, leaf=64, branch=16, depth=3, R=4, t_cap=65536, dtype=1, rope_pairs=0)
     base.update(kw)
     return _lib.Geom(**base)
 
@@ -47,7 +47,8 @@ def test_status_strings(lib):
 @pytest.mark.parametrize("kw,code", [
     ({}, 0), ({"d": 64}, 2), ({"leaf": 32}, 2), ({"Hq": 15}, 1), ({"Hq": 64, "Hkv": 2}, 2),
     ({"R": 17}, 2), ({"R": 0}, 1), ({"R": 3}, 2), ({"R": 16}, 0), ({"R": 1}, 0), ({"depth": 9}, 2), ({"branch": 1}, 2), ({"t_cap": 1000}, 1),
-    ({"dtype": 7}, 2), ({"reserved": 1}, 1), ({"B": 0}, 1),
+    ({"dtype": 7}, 2), ({"rope_pairs": 65}, 1), ({"rope_pairs": -1}, 1), ({"rope_pairs": 64}, 0),
+    ({"rope_pairs": 16}, 0), ({"B": 0}, 1),
     # a cache whose byte count (at 4 bytes per element) passes 2^48: 2^20 * 2 * 2^28 * 512 = 2^58
     ({"B": 1 << 20, "t_cap": 1 << 28}, 2),
     # the largest cache of the decode workloads (16M keys) is well inside the bound
@@ -148,3 +149,24 @@ def test_route_schedule_rejections(lib):
     assert lib.zha_route_schedule(ctypes.byref(g), fake, fake, 1, good, buf, fake, fake, 8, None, None,
                                   _lib.Buf(0x1000, 16), fake, None) == 3
     assert lib.zha_launch_count() == n0
+
+
+def test_reference_block_layout_and_size_check():
+    """The tree calls read Hkv*R*d reference values plus rope_pairs frequencies: the binding
+    builds that block and refuses a tensor of another size before calling the library."""
+    import torch
+    import hierarchical_sparse_attention_02_b200 as Z
+    qref = torch.randn(2, 4, 128)
+    f = torch.tensor([1.0, 0.5, 0.25])
+    qb = Z.reference_block(qref, f)
+    assert qb.shape == (2 * 4 * 128 + 3,) and qb.dtype == torch.float32
+    assert torch.equal(qb[:-3].view(2, 4, 128), qref) and torch.equal(qb[-3:], f)
+    assert torch.equal(Z.reference_block(qref), qref.reshape(-1))
+    g = Z.Geometry(B=1, Hq=8, Hkv=2, t_cap=4096, depth=2, R=4, rope_pairs=3)
+    n0 = Z.launch_count()
+    with pytest.raises(ValueError, match="qref"):
+        Z.zha_build_tree(g, None, 0, qref.reshape(-1), None, None)          # frequencies missing
+    with pytest.raises(ValueError, match="qref"):
+        Z.zha_decode(g, None, None, None, None, None, 0, qref.double(), 0.9, None, None, None, None, None,
+                     None)                                                   # fp64, not fp32
+    assert Z.launch_count() == n0

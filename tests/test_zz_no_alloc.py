@@ -22,7 +22,7 @@ def test_noalloc_rejects_oversize_before_any_launch():
     zbuild.build()
     lib = _lib.load()
     g = _lib.Geom(B=64, Hq=64, Hkv=8, d=128, leaf=64, branch=16, depth=3, R=4, t_cap=1 << 20, dtype=1,
-                  reserved=0)
+                  rope_pairs=0)
     fake = ctypes.c_void_p(0x1000)
     n0 = lib.zha_launch_count()
     assert lib.zha_sparse_attn_noalloc(ctypes.byref(g), fake, fake, fake, fake, 1, fake, fake, 8, fake, None,
