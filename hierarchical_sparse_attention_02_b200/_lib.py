@@ -17,7 +17,7 @@ ZHA_OP_ROUTE, ZHA_OP_ATTN, ZHA_OP_DECODE, ZHA_OP_DENSE, ZHA_OP_FLAT = 1, 2, 3, 4
 # every symbol include/zha.h declares, in declaration order
 EXPORTS = [
     "zha_status_str", "zha_check_geom", "zha_tree_bytes", "zha_tree_level", "zha_workspace_bytes",
-    "zha_leaf_cap", "zha_build_tree", "zha_append", "zha_route", "zha_route_schedule", "zha_sparse_attn",
+    "zha_leaf_cap", "zha_build_tree", "zha_append", "zha_route", "zha_route_schedule", "zha_route_topk", "zha_sparse_attn",
     "zha_decode",
     "zha_dense_decode", "zha_flat_index", "zha_sparse_attn_noalloc", "zha_launch_count",
     "zha_last_error", "zha_trace", "zha_trace_count",
@@ -57,6 +57,7 @@ _SIGS = {
     "zha_append": (_I32, [_G, _P, _P, _P, _P, _I64, _I32, _P, Buf, _P, _P]),
     "zha_route": (_I32, [_G, _P, _P, _I32, _F64, Buf, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_route_schedule": (_I32, [_G, _P, _P, _I32, _P, Buf, _P, _P, _I32, _P, _P, Buf, _P, _P]),
+    "zha_route_topk": (_I32, [_G, _P, _P, _I32, _P, Buf, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_sparse_attn": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_decode": (_I32, [_G, _P, _P, _P, _P, _P, _I64, _P, _F64, Buf, _P, _P, _I32, _P, Buf, _P, _P]),
     "zha_dense_decode": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, Buf, _P, _P]),

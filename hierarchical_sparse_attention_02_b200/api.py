@@ -159,6 +159,18 @@ def zha_route_schedule(g, Q, q_pos, p_levels, tree, leaf_ids, leaf_cnt, ws, dev_
         _stream(stream)))
 
 
+def zha_route_topk(g, Q, q_pos, k_levels, tree, leaf_ids, leaf_cnt, ws, dev_status, level_cnt=None,
+                   level_ids=None, stream=None):
+    """The tree walk with a fixed-count selector: level l keeps its k_levels[l-1] best candidates."""
+    if len(k_levels) != g.depth:
+        raise ValueError(f"k_levels holds {len(k_levels)} counts for {g.depth} levels")
+    arr = (ctypes.c_int32 * g.depth)(*[int(x) for x in k_levels])
+    _check("zha_route_topk", _lib.load().zha_route_topk(
+        ctypes.byref(g.c()), _ptr(Q), _ptr(q_pos), Q.shape[1], arr, _buf(tree), _ptr(leaf_ids),
+        _ptr(leaf_cnt), leaf_ids.shape[-1], _ptr(level_cnt), _ptr(level_ids), _buf(ws), _ptr(dev_status),
+        _stream(stream)))
+
+
 def zha_sparse_attn(g, Q, K, V, q_pos, leaf_ids, leaf_cnt, O, ws, dev_status, lse=None, stream=None):
     _check("zha_sparse_attn", _lib.load().zha_sparse_attn(
         ctypes.byref(g.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_pos), Q.shape[1], _ptr(leaf_ids),

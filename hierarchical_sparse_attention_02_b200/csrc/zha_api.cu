@@ -171,6 +171,25 @@ zha_status zha_route_schedule(const zha_geom* g, const void* Q, const int64_t* q
   return from_cuda(route_all(c));
 }
 
+zha_status zha_route_topk(const zha_geom* g, const void* Q, const int64_t* q_pos, int32_t nq,
+                          const int32_t* k_levels, zha_buf tree, int32_t* leaf_ids, int32_t* leaf_cnt,
+                          int32_t leaf_cap, int32_t* level_cnt, int32_t* level_ids, zha_buf ws,
+                          int32_t* dev_status, void* stream) {
+  zha_status s = zha_check_geom(g);
+  if (s != ZHA_OK) return s;
+  if (!k_levels) return ZHA_ERR_INVALID_ARG;
+  for (int l = 0; l < g->depth; ++l)
+    if (k_levels[l] < 1) return ZHA_ERR_INVALID_ARG;
+  if (!Q || !q_pos || nq < 1 || !tree.base || !leaf_ids || !leaf_cnt || leaf_cap < 1 || !ws.base ||
+      !dev_status)
+    return ZHA_ERR_INVALID_ARG;
+  if (tree.bytes < zha_tree_bytes(g)) return ZHA_ERR_CAPACITY;
+  if ((s = check_ws(g, nq, ZHA_OP_ROUTE, ws)) != ZHA_OK) return s;
+  RouteCall c{g, nq, Q, q_pos, 0, 1.0, tree.base, leaf_ids, leaf_cnt, leaf_cap, level_cnt, level_ids,
+              (char*)ws.base, dev_status, (cudaStream_t)stream, nullptr, k_levels};
+  return from_cuda(route_all(c));
+}
+
 zha_status zha_sparse_attn(const zha_geom* g, const void* Q, const void* K, const void* V,
                            const int64_t* q_pos, int32_t nq, const int32_t* leaf_ids,
                            const int32_t* leaf_cnt, int32_t leaf_cap, void* O, float* lse,

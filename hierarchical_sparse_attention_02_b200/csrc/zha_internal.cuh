@@ -282,6 +282,7 @@ struct RouteCall {
   int32_t* dev_status;
   cudaStream_t stream;
   const double* p_levels = nullptr;  // host [depth]: level l selects with p_levels[l-1]; null: p
+  const int32_t* k_levels = nullptr; // host [depth]: level l keeps its k_levels[l-1] best (top-K)
 };
 
 struct AttnCall {

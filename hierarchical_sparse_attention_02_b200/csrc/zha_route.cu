@@ -346,6 +346,7 @@ struct SelectArgs {
   int level;
   int flat;                      // 1: a single level over all visible leaves
   double p;
+  int64_t topk;                  // > 0: the fixed-count selector keeps the topk best; 0: top-p
   int mass_shift;                // fixed-point scale 2^mass_shift
   const int* cand_ids;
   const double* cand_score;
@@ -585,6 +586,21 @@ __device__ __forceinline__ unsigned long long mass_of(double s, double M, int sh
   return __double2ull_rn(ldexp(exp(s - M), shift));
 }
 
+// The selector's weights and target.  Top-p weighs a candidate by its fixed-point mass and
+// targets ceil(p Z); the fixed-count selector (topk > 0) runs the same cutoff with a weight
+// of 1 per candidate and the target topk, which keeps the topk first candidates in the same
+// (score desc, id asc) order.
+__device__ __forceinline__ unsigned long long sel_mass(const SelectArgs& a, double s, double M) {
+  return a.topk > 0 ? 1ull : mass_of(s, M, a.mass_shift);
+}
+__device__ __forceinline__ bool sel_keeps_all(const SelectArgs& a, int64_t n) {
+  return n == 0 || (a.topk > 0 ? a.topk >= n : a.p >= 1.0);
+}
+__device__ __forceinline__ unsigned long long sel_target(const SelectArgs& a, unsigned long long Z) {
+  if (a.topk > 0) return (unsigned long long)a.topk < Z ? (unsigned long long)a.topk : Z;
+  return target_of(a.p, Z);
+}
+
 // Writes the kept candidate `i` (id ids[i]) at output position pos.
 __device__ __forceinline__ void emit_kept(const SelectArgs& a, int64_t qh, const int* ids, int i,
                                           unsigned int pos, bool& overflow) {
@@ -642,7 +658,7 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
     unsigned long long z = 0;
     for (int i = lane; i < n; i += 32) {
       const double v = sc[i];
-      const unsigned long long e = mass_of(v, mx, a.mass_shift);
+      const unsigned long long e = sel_mass(a, v, mx);
       z += e;
       const int d = lb.digit(v);
       atomicAdd(&hcnt[d], 1u);
@@ -652,10 +668,10 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
     __syncwarp();
     // 3. the cutoff
     Cutoff c{};
-    c.keep_all = a.p >= 1.0 || n == 0;
+    c.keep_all = sel_keeps_all(a, n);
     c.shift = 64;
     if (!c.keep_all) {
-      const unsigned long long tgt = target_of(a.p, Z);
+      const unsigned long long tgt = sel_target(a, Z);
       unsigned long long above = 0;
       c.d1 = warp_boundary(hmass, above, tgt);
       unsigned int cnt_b = hcnt[c.d1];
@@ -672,7 +688,7 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
             const unsigned int slot = m + __popc(mb & lt);
             sm.m_pos[wid][slot] = i;
             sm.m_key[wid][slot] = order_key(sc[i]);
-            sm.m_mass[wid][slot] = mass_of(sc[i], mx, a.mass_shift);
+            sm.m_mass[wid][slot] = sel_mass(a, sc[i], mx);
           }
           m += __popc(mb);
         }
@@ -718,7 +734,7 @@ __global__ void __launch_bounds__(kWarpSelWarps * 32) route_select_warp_kernel(S
               if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
                 const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
                 atomicAdd(&hcnt[bkt], 1u);
-                atomicAdd(&hmass[bkt], mass_of(v, mx, a.mass_shift));
+                atomicAdd(&hmass[bkt], sel_mass(a, v, mx));
               }
             }
             __syncwarp();
@@ -985,7 +1001,7 @@ __global__ void __launch_bounds__(T) route_select_block_kernel(SelectArgs a) {
     unsigned long long z = 0;
     for (int i = tid; i < len; i += T) {
       const double v = sc[i];
-      const unsigned long long e = mass_of(v, M, a.mass_shift);
+      const unsigned long long e = sel_mass(a, v, M);
       z += e;
       const int d = lb.digit(v);
       atomicAdd(&sm.cnt[d], 1u);
@@ -999,10 +1015,10 @@ __global__ void __launch_bounds__(T) route_select_block_kernel(SelectArgs a) {
 
     // 3. the cutoff, with identical decisions in every CTA
     Cutoff c{};
-    c.keep_all = a.p >= 1.0 || n == 0;
+    c.keep_all = sel_keeps_all(a, n);
     c.shift = 64;
     if (!c.keep_all) {
-      const unsigned long long tgt = target_of(a.p, Z);
+      const unsigned long long tgt = sel_target(a, Z);
       unsigned long long above = 0, mass_b = 0;
       unsigned int cnt_b = 0;
       c.d1 = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
@@ -1014,7 +1030,7 @@ __global__ void __launch_bounds__(T) route_select_block_kernel(SelectArgs a) {
             const unsigned int slot = atomicAdd(&lead->m_cnt, 1u);
             lead->m_pos[slot] = r0 + i;
             lead->m_key[slot] = order_key(v);
-            lead->m_mass[slot] = mass_of(v, M, a.mass_shift);
+            lead->m_mass[slot] = sel_mass(a, v, M);
           }
         }
         csync<CL>();                                     // every member is in rank 0's list
@@ -1072,7 +1088,7 @@ __global__ void __launch_bounds__(T) route_select_block_kernel(SelectArgs a) {
               if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
                 const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
                 atomicAdd(&sm.cnt[bkt], 1u);
-                atomicAdd(&sm.mass[bkt], mass_of(v, M, a.mass_shift));
+                atomicAdd(&sm.mass[bkt], sel_mass(a, v, M));
               }
             }
             const int bstar = cl_boundary<T, CLK>(sm, CS, cr, above, tgt, cnt_b, mass_b);
@@ -1302,7 +1318,7 @@ __global__ void __launch_bounds__(kWideThreads) wide_hist_kernel(SelectArgs a, i
 #pragma unroll 4
   for (int i = i0 + threadIdx.x; i < i1; i += kWideThreads) {
     const double v = s[i];
-    const unsigned long long e = mass_of(v, M, a.mass_shift);
+    const unsigned long long e = sel_mass(a, v, M);
     z += e;
     const int d = lb.digit(v);
     atomicAdd(&cnt[d], 1u);
@@ -1324,12 +1340,12 @@ __global__ void __launch_bounds__(1024) wide_boundary_kernel(SelectArgs a) {
   const int64_t qh = blockIdx.x;
   WideHead* h = wide_head(a, qh);
   if (h->mode == kWideSkip) return;
-  if (a.p >= 1.0 || h->n == 0) {
+  if (sel_keeps_all(a, h->n)) {
     if (threadIdx.x == 0) h->mode = kWideAll;
     return;
   }
   for (int i = threadIdx.x; i < kBuckets; i += 1024) { sm.cnt[i] = h->cnt[i]; sm.mass[i] = h->mass[i]; }
-  const unsigned long long tgt = target_of(a.p, h->Z);
+  const unsigned long long tgt = sel_target(a, h->Z);
   unsigned long long above = 0ull, mass_b = 0ull;
   unsigned int cnt_b = 0u;
   const int d1 = cl_boundary<1024, false>(sm, 1, 0, above, tgt, cnt_b, mass_b);   // syncs first
@@ -1361,7 +1377,7 @@ __global__ void __launch_bounds__(kWideThreads) wide_gather_kernel(SelectArgs a,
     if (slot >= (unsigned)kWideMembers) continue;          // (the histogram counted them all)
     h->m_pos[slot] = i;
     h->m_key[slot] = order_key(v);
-    h->m_mass[slot] = mass_of(v, lb.M, a.mass_shift);
+    h->m_mass[slot] = sel_mass(a, v, lb.M);
   }
 }
 
@@ -1494,7 +1510,7 @@ __global__ void __launch_bounds__(1024) wide_resolve_kernel(SelectArgs a) {
         if ((hi == 63 ? 0ull : (key >> (hi + 1))) == pfx) {
           const unsigned int bkt = (unsigned int)((key >> lo) & ((1ull << width) - 1));
           atomicAdd(&sm.cnt[bkt], 1u);
-          atomicAdd(&sm.mass[bkt], mass_of(v, lb.M, a.mass_shift));
+          atomicAdd(&sm.mass[bkt], sel_mass(a, v, lb.M));
         }
       }
       const int bstar = cl_boundary<1024, false>(sm, 1, 0, above, tgt, cnt_b, mass_b);
@@ -1808,6 +1824,7 @@ static cudaError_t route_levels(const RouteCall& c) {
 
     SelectArgs se{};
     se.g = rg; se.level = l; se.flat = 0; se.p = c.p_levels ? c.p_levels[l - 1] : c.p;
+    se.topk = c.k_levels ? c.k_levels[l - 1] : 0;
     se.mass_shift = mass_shift_for(w.C1);
     se.cand_ids = sa.cand_ids; se.cand_score = sa.cand_score;
     se.cand_mass = (unsigned long long*)(c.ws + w.cand_mass);

@@ -202,6 +202,20 @@ zha_status zha_route_schedule(const zha_geom* g, const void* Q, const int64_t* q
                               int32_t* level_ids, zha_buf ws, int32_t* dev_status, void* stream);
 
 /*
+ * zha_route_topk - the tree walk of zha_route with a fixed-count selector: level l keeps
+ * its k_levels[l-1] best candidates in the same (score desc, node id asc) order, or all of
+ * them when there are fewer (the fixed selection budget K of arXiv 2610.42112 App. D,
+ * Table VI, which §III-C contrasts with top-p).  Candidates, expansion and outputs are
+ * those of zha_route.
+ *   k_levels  HOST array of g->depth int32 counts, each >= 1; read before the call returns.
+ *   Other arguments as zha_route.
+ */
+zha_status zha_route_topk(const zha_geom* g, const void* Q, const int64_t* q_pos, int32_t nq,
+                          const int32_t* k_levels, zha_buf tree, int32_t* leaf_ids, int32_t* leaf_cnt,
+                          int32_t leaf_cap, int32_t* level_cnt, int32_t* level_ids, zha_buf ws,
+                          int32_t* dev_status, void* stream);
+
+/*
  * zha_sparse_attn - exact softmax attention over the index set
  * ("ZHA summary" page, Routing):  I(q) = {0} u (keys of the chunks in S_1(q)) u C_cur(q),
  * C_cur(q) = [V(t), t],   o(q) = sum_{j in I} softmax_j(q . k_j / sqrt(d)) v_j.

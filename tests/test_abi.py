@@ -26,7 +26,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(lib):
     decl = declared_symbols()
-    assert len(decl) == 19
+    assert len(decl) == 20
     assert sorted(decl) == sorted(_lib.EXPORTS)
     for name in decl:
         assert hasattr(lib, name), name
@@ -170,3 +170,20 @@ def test_reference_block_layout_and_size_check():
         Z.zha_decode(g, None, None, None, None, None, 0, qref.double(), 0.9, None, None, None, None, None,
                      None)                                                   # fp64, not fp32
     assert Z.launch_count() == n0
+
+
+def test_route_topk_rejections(lib):
+    """Per-level counts: a null array or a count below 1 is rejected before any launch."""
+    g = geom()                                  # depth 3
+    fake = ctypes.c_void_p(0x1000)
+    buf = _lib.Buf(0x1000, 1 << 40)
+    n0 = lib.zha_launch_count()
+    arr = lambda *v: (ctypes.c_int32 * len(v))(*v)  # noqa: E731
+    for bad in (arr(4, 0, 4), arr(-1, 4, 4), arr(4, 4, -7)):
+        assert lib.zha_route_topk(ctypes.byref(g), fake, fake, 1, bad, buf, fake, fake, 8, None, None, buf,
+                                  fake, None) == 1
+    assert lib.zha_route_topk(ctypes.byref(g), fake, fake, 1, None, buf, fake, fake, 8, None, None, buf,
+                              fake, None) == 1
+    assert lib.zha_route_topk(ctypes.byref(g), fake, fake, 1, arr(1, 2, 3, 0), buf, fake, fake, 8, None, None,
+                              _lib.Buf(0x1000, 16), fake, None) == 3
+    assert lib.zha_launch_count() == n0

@@ -12,6 +12,7 @@ It does not run the kernels; the GPU parity tests do.
 from __future__ import annotations
 
 import math
+import zlib
 
 import numpy as np
 import pytest
@@ -43,12 +44,13 @@ def boundary(mass, above, tgt):
     raise AssertionError("no boundary bucket")
 
 
-def model_select(s, E, p, nb=2048, wd=11, members=32):
+def model_select(s, E, p, nb=2048, wd=11, members=32, k=None):
+    """With k (the fixed-count selector) every candidate weighs 1 and the target is k."""
     n = len(s)
-    if p >= 1.0 or n == 0:
+    if n == 0 or (p >= 1.0 if k is None else k >= n):
         return np.arange(n)
     Z = int(sum(int(e) for e in E))
-    tgt = max(1, min(Z, math.ceil(p * Z)))
+    tgt = max(1, min(Z, math.ceil(p * Z))) if k is None else k
     d = digits(s, s.max(), s.min(), nb)
     mass = [0] * nb
     cnt = np.bincount(d, minlength=nb)
@@ -144,7 +146,7 @@ def reference(s, E, p):
 @pytest.mark.parametrize("kind", ["normal", "narrow", "quartered", "outlier", "constant", "wide_range"])
 @pytest.mark.parametrize("nb,wd", [(256, 8), (2048, 11)])
 def test_bucket_select_equals_sorted_cutoff(kind, nb, wd):
-    rng = np.random.default_rng(hash((kind, nb)) % 2**32)
+    rng = np.random.default_rng(zlib.crc32(f"{kind}/{nb}".encode()))
     for trial in range(60):
         n = int(rng.integers(1, 700))
         if kind == "normal":
@@ -179,3 +181,30 @@ def test_reference_matches_oracle_top_p_on_distinct_scores():
         if sel.margin < 1e-9:
             continue
         assert np.array_equal(np.sort(sel.ids), reference(s, fixed_masses(s), p))
+
+
+@pytest.mark.parametrize("kind", ["normal", "quartered", "outlier", "constant", "wide_range"])
+@pytest.mark.parametrize("nb,wd", [(256, 8), (2048, 11)])
+def test_bucket_select_with_unit_masses_is_top_k(kind, nb, wd):
+    """The fixed-count selector runs the same procedure with a mass of 1 per candidate and
+    the target k: it must keep the oracle's top-k set (ties broken by position)."""
+    rng = np.random.default_rng(zlib.crc32(f"{kind}/{nb}/k".encode()))
+    for trial in range(60):
+        n = int(rng.integers(1, 700))
+        if kind == "normal":
+            s = rng.normal(size=n)
+        elif kind == "quartered":
+            s = np.round(rng.normal(size=n) * 4) / 4
+        elif kind == "outlier":
+            s = np.concatenate([rng.normal(size=n - 1) * 1e-9, [30.0]])
+        elif kind == "constant":
+            s = np.full(n, 1.25)
+        else:
+            s = rng.exponential(size=n) * rng.choice([1, -1], size=n) * 10.0 ** rng.integers(-8, 3, size=n)
+        s = s.astype(np.float64)
+        s[s == 0] = 0.0            # one zero: the order key tells -0.0 below +0.0, a sort does not
+        k = int(rng.integers(1, n + 3))
+        want = zo.top_k(s, np.arange(n, dtype=np.int64), k).ids
+        for members in (0, 32):
+            got = model_select(s, [1] * n, None, nb, wd, members, k=k)
+            assert np.array_equal(got, want), (kind, trial, n, k, members)

@@ -1,11 +1,14 @@
-"""GPU parity of zha_route_schedule (one top-p threshold per level, arXiv 2610.42112 §VII
-"Asymptotic length scaling") against the oracle's route with the same per-level thresholds.
+"""GPU parity of the selector variants against the oracle's route with the same parameters:
+zha_route_schedule (one top-p threshold per level, arXiv 2610.42112 §VII "Asymptotic length
+scaling") and zha_route_topk (a fixed count per level, the budget K of App. D, Table VI).
 
 The kept node sets of every level and the leaf lists must be identical, except at and below
-a level whose oracle cutoff margin is under 1e-4 (counted).  A constant schedule must give
-exactly the lists of zha_route / zha_decode with that p.
+a level whose oracle cutoff margin (top-p) or boundary gap (top-K) is under the near-cutoff
+threshold (counted).  A constant schedule must give exactly the lists of zha_route with that p.
 """
 from __future__ import annotations
+
+import dataclasses
 
 import numpy as np
 import pytest
@@ -14,6 +17,8 @@ import torch
 import zha_synth as S
 from oracle import zha_oracle as zo
 from tests.zha_cases import RouteCompare, compare_route, geometry, route_storage
+
+NEAR = 1e-12            # top-K: a softmax gap this small at the boundary is a near-tie
 
 pytestmark = pytest.mark.gpu
 
@@ -54,7 +59,7 @@ def _setup(w):
     return g, K, qref, q, tree, st
 
 
-def _route(g, w, q, tree, st, ps):
+def _route(g, w, q, tree, st, ps, ks=None):
     nst = sum(Z.tree_level(g, l).n_cap for l in range(2, w.depth + 1))
     level_cnt = torch.zeros(w.B, 1, w.Hq, w.depth, 2, dtype=torch.int32, device=DEV)
     level_ids = torch.full((w.B, 1, w.Hq, max(nst, 1)), -1, dtype=torch.int32, device=DEV)
@@ -62,7 +67,9 @@ def _route(g, w, q, tree, st, ps):
     cnt = torch.zeros(w.B, 1, w.Hq, dtype=torch.int32, device=DEV)
     pos = torch.full((w.B, 1), w.T, dtype=torch.int64, device=DEV)
     ws = Z.empty_workspace(g, 1, Z.ZHA_OP_ROUTE)
-    if isinstance(ps, float):
+    if ks is not None:
+        Z.zha_route_topk(g, q, pos, ks, tree, ids, cnt, ws, st, level_cnt, level_ids)
+    elif isinstance(ps, float):
         Z.zha_route(g, q, pos, ps, tree, ids, cnt, ws, st, level_cnt, level_ids)
     else:
         Z.zha_route_schedule(g, q, pos, ps, tree, ids, cnt, ws, st, level_cnt, level_ids)
@@ -114,3 +121,54 @@ def test_constant_schedule_is_zha_route():
     b = _route(g, w, q, tree, st, [p] * w.depth)
     for x, y in zip(a, b):
         assert np.array_equal(x, y)
+
+
+def _workload(spec, T, B):
+    base, _, ll = spec.partition("@L")
+    w = S.scaled(S.workload(base), T=T, B=B, n_centres=min(S.workload(base).n_centres, 1024))
+    return dataclasses.replace(w, depth=int(ll)) if ll else w
+
+
+@pytest.mark.parametrize("spec,T,B,ks", [
+    ("batched-decode-128k", 20000 + 7, 2, [64, 16, 4]),       # depth 3, a budget per level
+    ("batched-decode-128k", 20000 + 7, 1, [100, 100, 100]),   # budgets above n at the upper levels
+    ("tiny-decode-f32", 8192, None, [20, 3]),                  # fp32 cache, depth 2
+    ("deep-tree-16m@L1", 1200000 + 5, None, [5000]),           # ~18.7K candidates: a cluster select
+    ("deep-tree-16m@L1", 8700000 + 5, None, [20000]),          # ~136K candidates: the grid-wide chain
+])
+def test_route_topk_parity(spec, T, B, ks):
+    w = _workload(spec, T, B)
+    g, K, qref, q, tree, st = _setup(w)
+    ids, cnt, lc, lids = _route(g, w, q, tree, st, None, ks)
+    Kc = K.cpu()
+    qr = qref.double().cpu().numpy()
+    qc = q.double().cpu().numpy()
+    exact = near = heads = 0
+    units = [(b, h) for b in range(w.B) for h in range(w.Hkv)][:3]
+    for (b, hk) in units:
+        otree = zo.build_tree(Kc[b, hk], w.T + 1, qr[hk], w.depth, route_storage=route_storage(w))
+        for h in range(hk * w.G, (hk + 1) * w.G):
+            r = zo.route(qc[b, 0, h], w.T, otree, 0.5, k=ks)
+            heads += 1
+            ok = True
+            for l in range(r.top, 0, -1):
+                if l == 1:
+                    got = ids[b, 0, h, :int(cnt[b, 0, h])].astype(np.int64)
+                else:
+                    o = sum(Z.tree_level(g, j).n_cap for j in range(2, l))
+                    got = lids[b, 0, h, o:o + int(lc[b, 0, h, l - 1, 1])].astype(np.int64)
+                sel = r.sel[l]
+                assert int(lc[b, 0, h, l - 1, 1]) == sel.m or l == 1, (l, sel.m)
+                if np.array_equal(got, sel.ids):
+                    continue
+                # two candidates within rounding of each other at the boundary may swap
+                assert sel.gap < NEAR, (f"b{b} h{h} level {l}: oracle kept {sel.m} of {sel.n}, "
+                                        f"gpu {len(got)}, sym diff {len(np.setxor1d(got, sel.ids))}")
+                near += 1
+                ok = False
+                break
+            exact += ok
+            if ok:
+                assert int(cnt[b, 0, h]) == min(ks[0], len(r.cand[1]))
+    assert exact > 0
+    print(f"{w.name} top-K {ks}: {exact} exact, {near} near-ties of {heads}")
