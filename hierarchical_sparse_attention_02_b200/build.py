@@ -1,6 +1,6 @@
 """Builds libzha.so (CUDA sm_100a) in-tree with nvcc.
 
-Usage: python -m hierarchical_sparse_attention_02_b200.build [--checked]
+Usage: python -m hierarchical_sparse_attention_02_b200.build [-v]
 """
 from __future__ import annotations
 
@@ -35,14 +35,12 @@ def needs_build(out: str = LIB) -> bool:
     return any(os.path.getmtime(p) > t for p in deps if os.path.exists(p))
 
 
-def build(out: str = LIB, checked: bool = False, verbose: bool = False, force: bool = False) -> str:
+def build(out: str = LIB, verbose: bool = False, force: bool = False) -> str:
     if not force and not needs_build(out):
         return out
     cmd = [nvcc_path(), "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
            "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"), "-I", CSRC,
            "-Xptxas", "-v" if verbose else "-O3", "-o", out + ".tmp"] + sources()
-    if checked:
-        cmd.insert(1, "-DZHA_CHECKED=1")
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError("nvcc failed:\n" + r.stdout + r.stderr)
@@ -53,5 +51,5 @@ def build(out: str = LIB, checked: bool = False, verbose: bool = False, force: b
 
 
 if __name__ == "__main__":
-    build(checked="--checked" in sys.argv, verbose="-v" in sys.argv, force=True)
+    build(verbose="-v" in sys.argv, force=True)
     print(LIB)
