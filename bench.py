@@ -51,6 +51,9 @@ def parse():
     ap.add_argument("--segment", type=int, default=0,
                     help="structured keys: runs of this many positions share a cluster centre "
                          "(a variant of the generator, not one of the five workloads)")
+    ap.add_argument("--rope", type=int, default=0, metavar="H",
+                    help="rotary tree: reference queries rotated with H RoPE frequencies (base 10000 "
+                         "over 2H dims; the keys stay as generated)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat"],
@@ -376,14 +379,15 @@ def candidate_unions(level_cnt: np.ndarray, level_ids: np.ndarray, n_cap: dict, 
     return out
 
 
-def oracle_rate(w: S.Workload, p: float, seconds: float, device: str, routes: list = None):
+def oracle_rate(w: S.Workload, p: float, seconds: float, device: str, routes: list = None, inv_freq=None):
     """Query-heads/s of the CPU oracle on a bounded sample of the decode step.
 
     The sample: whole KV groups (G query heads of one (sequence, KV head) unit) of the
     same seeded workload, routed and attended by the oracle one head at a time until
     ``seconds`` of CPU time have been spent (at least one group).  The oracle's tree of
     each sampled unit is built first, untimed (it is the decode step's prior state).
-    With ``routes`` (a list) the oracle's route of every sampled head is appended to it.
+    With ``routes`` (a list) the oracle's route of every sampled head is appended to it;
+    ``inv_freq`` builds the oracle's rotary tree.
     """
     from oracle import zha_oracle as zo
     try:
@@ -404,7 +408,7 @@ def oracle_rate(w: S.Workload, p: float, seconds: float, device: str, routes: li
     heads, spent = 0, 0.0
     for hk in range(w.Hkv):
         tree = zo.build_tree(Kc[0, hk], w.T + 1, qr[hk], w.depth,
-                             route_storage="bf16" if w.dtype == "bf16" else "f32")
+                             route_storage="bf16" if w.dtype == "bf16" else "f32", inv_freq=inv_freq)
         t0 = time.process_time()
         for h in range(hk * w.G, (hk + 1) * w.G):
             r, _, _ = zo.decode_head(qc[0, 0, h], Kc[0, hk], Vc[0, hk], w.T, tree, p)
@@ -468,9 +472,11 @@ def run_reference(args, w, p, ws, rank):
     K, W = args.steps, args.warmup
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     per_step = max(1.0, 150.0 / max(1, K + W))
+    freq = (10000.0 ** (-np.arange(args.rope, dtype=np.float64) / args.rope)).astype(np.float32).astype(
+        np.float64) if args.rope else None
     rates = []
     for i in range(W + K):
-        r, heads, spent = oracle_rate(w, p, min(per_step, args.cpu_seconds), dev)
+        r, heads, spent = oracle_rate(w, p, min(per_step, args.cpu_seconds), dev, inv_freq=freq)
         if i >= W:
             rates.append((r, heads, spent))
     value = statistics.median(r[0] for r in rates)
@@ -479,7 +485,7 @@ def run_reference(args, w, p, ws, rank):
         "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": 1,
         "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(w, p), "impl": "reference",
+        "config": {**config_of(w, p), **({"rope_pairs": args.rope} if args.rope else {})}, "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
                          "sample": f"{rates[0][1]} query heads (whole KV groups) per step, fp64 numpy, 1 thread"},
         "e2e": {"value": value, "unit": "query-heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -605,9 +611,13 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     wr = S.Workload(**{**w.__dict__, "seed": w.seed + 1000 * rank}) if rank else w
     g = Z.Geometry(B=w.B, Hq=w.Hq, Hkv=w.Hkv, t_cap=w.t_cap, depth=w.depth, R=w.R, d=w.d,
-                   dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32)
+                   dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32, rope_pairs=args.rope)
     C, K, V = S.clustered_kv(wr, dev)
     qref = S.reference_queries(wr, dev)
+    freq = None
+    if args.rope:                     # the tree calls read the frequencies after the references
+        freq = (10000.0 ** (-torch.arange(args.rope, dtype=torch.float64) / args.rope)).float()
+        qref = Z.reference_block(qref, freq)
     k_new, v_new = S.new_tokens(wr, C, 1, dev)
     q = S.queries(wr, C, 1, dev)
     del C
@@ -793,7 +803,8 @@ def main():
     near = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         routes = []
-        r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda", routes)
+        r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda", routes,
+                                      freq.double().numpy() if freq is not None else None)
         cpu = {"value": r, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
                "sample": f"{heads} query heads (whole KV groups of sequence 0) of {w.name}, "
                          f"route + attention, fp64 numpy, 1 thread, {spent:.1f} s CPU"}
@@ -803,7 +814,7 @@ def main():
         "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": ws,
         "steps": Ksteps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {**config_of(w, p), "path": args.path},
+        "config": {**config_of(w, p), "path": args.path, **({"rope_pairs": args.rope} if args.rope else {})},
         "roofline": {"bound": "hbm", "kernel": dom_name,
                      "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
