@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--rope", type=int, default=0, metavar="H",
                     help="rotary tree: reference queries rotated with H RoPE frequencies (base 10000 "
                          "over 2H dims; the keys stay as generated)")
+    ap.add_argument("--graph", action="store_true",
+                    help="capture the step once in a CUDA graph and replay it in the timed loop "
+                         "(the dominant kernel's duration then comes from traced, uncaptured steps)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
     ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat"],
@@ -677,27 +680,51 @@ def main():
     torch.cuda.synchronize()
     # the dominant kernel is traced live: the attention, or the chunk scores of the flat path
     dom = _lib.ZHA_TRACE_ROUTE_SCORE if args.path == "flat" and w.dtype == "bf16" else _lib.ZHA_TRACE_ATTN
-    lib.zha_trace(dom, arr_s, arr_e, n_ev)
+    graph = None
+    if args.graph:
+        # the whole step captured once; the timed loop replays it (no host launches)
+        graph = torch.cuda.CUDAGraph()
+        n_g0 = Z.launch_count()
+        with torch.cuda.graph(graph):
+            step()
+        graph_launches = Z.launch_count() - n_g0
+        graph.replay()
+        torch.cuda.synchronize()
+    else:
+        lib.zha_trace(dom, arr_s, arr_e, n_ev)
     n_launch0 = Z.launch_count()
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks.mark_start()
     t_start.record(stream)
     for _ in range(Ksteps):
-        step()
+        if graph is not None:
+            graph.replay()
+        else:
+            step()
     t_end.record(stream)
     torch.cuda.synchronize()
     clocks.mark_end()
     barrier(ws)
-    launches = Z.launch_count() - n_launch0
-    traced = lib.zha_trace_count(dom)
-    lib.zha_trace(dom, None, None, 0)
+    if graph is None:
+        launches = Z.launch_count() - n_launch0
+        traced = lib.zha_trace_count(dom)
+        lib.zha_trace(dom, None, None, 0)
     ms_local = t_start.elapsed_time(t_end) / Ksteps
-    dom_launches = traced / Ksteps                         # launches of the traced kernel per step
-    dom_ms = sum(a.elapsed_time(b) for a, b in zip(starts[:traced], stops[:traced])) / max(1, traced)
+    if graph is None:
+        dom_launches = traced / Ksteps                     # launches of the traced kernel per step
+        dom_ms = sum(a.elapsed_time(b) for a, b in zip(starts[:traced], stops[:traced])) / max(1, traced)
     if st.item() != 0:
         raise RuntimeError(f"device status {st.item()} in the timed region")
     ms, value = whole_job_rate(w.B * w.Hq, ms_local, ws)
     stages = stage_breakdown(lib, step, stream, min(Ksteps, 20), ms_local)
+    if graph is not None:
+        # replays launch what the capture launched; the dominant kernel is timed on the
+        # traced (uncaptured) steps of the stage breakdown
+        launches = graph_launches * Ksteps
+        dom_name_stage = "route_score" if dom == _lib.ZHA_TRACE_ROUTE_SCORE else "attention"
+        per = stages.get(dom_name_stage + "_per_launch")
+        dom_launches = float(len(per)) if per else 1.0
+        dom_ms = stages[dom_name_stage] / dom_launches
 
     # end to end through the public API with host buffers
     pin = lambda t: torch.empty(t.shape, dtype=t.dtype, pin_memory=True)  # noqa: E731
@@ -814,7 +841,8 @@ def main():
         "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": ws,
         "steps": Ksteps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": {**config_of(w, p), "path": args.path, **({"rope_pairs": args.rope} if args.rope else {})},
+        "config": {**config_of(w, p), "path": args.path, **({"rope_pairs": args.rope} if args.rope else {}),
+                   **({"cuda_graph": True} if args.graph else {})},
         "roofline": {"bound": "hbm", "kernel": dom_name,
                      "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
