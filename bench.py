@@ -516,7 +516,8 @@ SWEEP_T = (16384, 32768, 65536, 131072, 262144, 524288, 1048576, 2097152)
 def run_sweep(args):
     """Crossover sweep: ms per decode step of zha_decode at every depth L = 1..6, of the
     dense kernel and of the flat indexer, for T in SWEEP_T at the long-decode head geometry (B=4, Hq=32, Hkv=4),
-    on the same seeded inputs per T.  One JSON line per (T, path, depth)."""
+    on the same seeded inputs per T (with --segment, the structured variant of the generator).
+    One JSON line per (T, path, depth)."""
     import dataclasses
     import hierarchical_sparse_attention_02_b200 as Z
     torch.cuda.set_device(0)
@@ -525,6 +526,9 @@ def run_sweep(args):
     p = args.p if args.p is not None else base.p[0]
     for T in SWEEP_T:
         w = S.scaled(base, T=T)
+        if args.segment > 0:          # the structured variant of the generator
+            w = dataclasses.replace(w, segment=args.segment)
+        tag = {"segment": args.segment} if args.segment > 0 else {}
         C, K, V = S.clustered_kv(w, dev)
         qref = S.reference_queries(w, dev)
         k_new, v_new = S.new_tokens(w, C, 1, dev)
@@ -559,7 +563,7 @@ def run_sweep(args):
             ms = timed(lambda: Z.zha_decode(g, q, k_new, v_new, K, V, w.T, qref, p, tree, ids, cnt, O, wsb, st))
             touched = float((cnt.double() * 64 + 1).mean().item()) / (w.T + 1)
             print(json.dumps({"sweep": "crossover", "T": T, "path": "zha", "depth": L, "p": p,
-                              "ms_per_step": ms, "kv_touched_approx": touched}), flush=True)
+                              "ms_per_step": ms, "kv_touched_approx": touched, **tag}), flush=True)
             best = min(best, ms) if best is not None else ms
             del tree, wsb, ids, cnt
         g = Z.Geometry(B=w.B, Hq=w.Hq, Hkv=w.Hkv, t_cap=w.t_cap, depth=1, R=w.R)
@@ -567,14 +571,14 @@ def run_sweep(args):
         pos = torch.full((w.B, 1), w.T, dtype=torch.int64, device=dev)
         ms_dense = timed(lambda: Z.zha_dense_decode(g, q, K, V, pos, O, wsd, st))
         print(json.dumps({"sweep": "crossover", "T": T, "path": "dense", "ms_per_step": ms_dense,
-                          "zha_best_ms": best, "zha_faster": best < ms_dense}), flush=True)
+                          "zha_best_ms": best, "zha_faster": best < ms_dense, **tag}), flush=True)
         wsf = Z.empty_workspace(g, 1, Z.ZHA_OP_FLAT, dev)
         ids = torch.empty(w.B, 1, w.Hq, Z.leaf_cap(g), dtype=torch.int32, device=dev)
         cnt = torch.empty(w.B, 1, w.Hq, dtype=torch.int32, device=dev)
         ms_flat = timed(lambda: Z.zha_flat_index(g, q, K, V, pos, p, ids, cnt, O, wsf, st))
         touched = float((cnt.double() * 64 + 1).mean().item()) / (w.T + 1)
         print(json.dumps({"sweep": "crossover", "T": T, "path": "flat", "ms_per_step": ms_flat,
-                          "kv_touched_approx": touched}), flush=True)
+                          "kv_touched_approx": touched, **tag}), flush=True)
         del K, V, wsd, wsf, ids, cnt
         torch.cuda.empty_cache()
 
