@@ -187,3 +187,40 @@ def test_route_topk_rejections(lib):
     assert lib.zha_route_topk(ctypes.byref(g), fake, fake, 1, arr(1, 2, 3, 0), buf, fake, fake, 8, None, None,
                               _lib.Buf(0x1000, 16), fake, None) == 3
     assert lib.zha_launch_count() == n0
+
+
+def _prototypes():
+    """name -> (return type, [parameter types]) of every prototype in include/zha.h."""
+    src = open(os.path.join(ROOT, "include", "zha.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"^\s*((?:const\s+)?[a-z_0-9]+\s*\*?)\s*(zha_[a-z_]+)\s*\(([^)]*)\)\s*;", src, flags=re.M):
+        params = [p.strip() for p in m.group(3).replace("\n", " ").split(",") if p.strip() and p.strip() != "void"]
+        types = [re.sub(r"\s*\b[a-z_A-Z0-9]+$", "", p).strip() if not p.endswith("*") else p for p in params]
+        out[m.group(2)] = (m.group(1).replace(" ", ""), [t.replace(" ", "") for t in types])
+    return out
+
+
+_C_TO_CTYPES = {
+    "int32_t": ctypes.c_int32, "int64_t": ctypes.c_int64, "double": ctypes.c_double, "size_t": ctypes.c_size_t,
+    "zha_status": ctypes.c_int32, "zha_buf": "Buf", "constchar*": ctypes.c_char_p, "void": None,
+}
+
+
+def test_ctypes_signatures_match_the_header():
+    """Every entry point's ctypes signature has the header's parameter count and, parameter by
+    parameter, the same kind (pointer, 32/64-bit integer, double, buffer struct): a mismatch
+    would pass garbage through the ABI on a GPU."""
+    protos = _prototypes()
+    assert sorted(protos) == sorted(_lib._SIGS)
+    for name, (ret, params) in protos.items():
+        cret, cargs = _lib._SIGS[name]
+        assert len(cargs) == len(params), (name, params)
+        want_ret = _C_TO_CTYPES.get(ret)
+        assert cret == want_ret, (name, ret, cret)
+        for i, (p, c) in enumerate(zip(params, cargs)):
+            if p.endswith("*"):                       # any pointer
+                assert c is ctypes.c_void_p or issubclass(c, ctypes._Pointer), (name, i, p, c)
+            else:
+                want = _C_TO_CTYPES[p]
+                assert (c is _lib.Buf) if want == "Buf" else (c is want), (name, i, p, c)
