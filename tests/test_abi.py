@@ -224,3 +224,34 @@ def test_ctypes_signatures_match_the_header():
             else:
                 want = _C_TO_CTYPES[p]
                 assert (c is _lib.Buf) if want == "Buf" else (c is want), (name, i, p, c)
+
+
+def test_struct_layouts_match_the_header(tmp_path):
+    """zha_geom, zha_buf and zha_level_layout as the C compiler lays them out (sizes and field
+    offsets, from a program compiled against include/zha.h) equal the ctypes structures."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    fields = {"zha_geom": [f for f, _ in _lib.Geom._fields_],
+              "zha_buf": [f for f, _ in _lib.Buf._fields_],
+              "zha_level_layout": [f for f, _ in _lib.LevelLayout._fields_]}
+    lines = ['#include <stdio.h>', '#include <stddef.h>', '#include "zha.h"', "int main(void) {"]
+    for s, fs in fields.items():
+        lines.append(f'  printf("{s} size %zu\\n", sizeof({s}));')
+        for f in fs:
+            lines.append(f'  printf("{s} {f} %zu\\n", offsetof({s}, {f}));')
+    lines += ["  return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    subprocess.run([cc, "-std=c99", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = {}
+    for line in subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.splitlines():
+        s, f, v = line.split()
+        got[(s, f)] = int(v)
+    for s, cls in (("zha_geom", _lib.Geom), ("zha_buf", _lib.Buf), ("zha_level_layout", _lib.LevelLayout)):
+        assert got[(s, "size")] == ctypes.sizeof(cls), s
+        for f in fields[s]:
+            assert got[(s, f)] == getattr(cls, f).offset, (s, f)
