@@ -22,7 +22,7 @@ Plain numpy in float64, written step by step from the method's definitions:
 * "ZHA summary" page, Methodology -> Routing: m_l(q), the final index set
   I(q) = {0} u (union of selected leaf chunks) u C_cur(q), o(q) = Attn(q, K_I, V_I).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
   * Tree nodes are stateless functions of the keys: a level-l node i spans
     keys [i*S_l, (i+1)*S_l), S_l = leaf * branch**(l-1); it exists once all its
     keys are in the cache.
