@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(kMaxG * 32) combine_cta_blocks_kernel(AttnGeom
 }
 
 // ---------------------------------------------------------------------------
-// host driver
+// host side: the launches of one attention call
 // ---------------------------------------------------------------------------
 
 

@@ -1756,7 +1756,7 @@ static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap
 }
 
 // ---------------------------------------------------------------------------
-// host driver
+// host side: the launches of one routing call
 // ---------------------------------------------------------------------------
 
 

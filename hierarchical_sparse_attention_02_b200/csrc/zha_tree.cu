@@ -353,7 +353,7 @@ __global__ void append_kv_kernel(uint4* __restrict__ K, uint4* __restrict__ V,
 }
 
 // ---------------------------------------------------------------------------
-// host drivers
+// host side: the launches of a tree extension
 // ---------------------------------------------------------------------------
 
 template <typename KT, int R, bool ROPE>
