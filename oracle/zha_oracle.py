@@ -235,6 +235,46 @@ def rows_f64(K, a: int, b: int) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
+def leaf_level(Kc: np.ndarray, qn: np.ndarray, scale: float):
+    """``leaf_summary`` of n chunks at once, the formula unchanged.
+
+    Kc: [n, C, d] keys of n chunks; qn: [n, R, d] the reference queries of each
+    chunk (rotated per chunk) or [1, R, d] (one set for every chunk).
+      s[n, r, c] = q_hat_{n,r} . k_{n,c} * scale,   F[n, r] = LSE_c s[n, r, c],
+      a = exp(s - F),   k_hat[n, r] = sum_c a[n, r, c] k_{n,c},
+      b_hat[n, r] = F[n, r] - q_hat_{n,r} . k_hat[n, r] * scale.
+    Returns (k_hat [n, R, d], F [n, R], b_hat [n, R]).
+    """
+    if qn.shape[0] == 1:   # one q_hat for every chunk: a single matrix product, then a reshape
+        n, C, d = Kc.shape
+        s = np.swapaxes((Kc.reshape(-1, d) @ qn[0].T).reshape(n, C, -1), 1, 2) * scale
+    else:
+        s = np.matmul(qn, np.swapaxes(Kc, 1, 2)) * scale
+    F = lse(s, axis=-1)
+    a = np.exp(s - F[..., None])
+    k_hat = np.matmul(a, Kc)                                # [n, r, d] = a[n, r, c] . K[n, c, d]
+    b_hat = F - np.sum(qn * k_hat, axis=-1) * scale
+    return k_hat, F, b_hat
+
+
+def merge_level(F_c: np.ndarray, k_hat_c: np.ndarray, qP: np.ndarray, scale: float):
+    """``merge_summaries`` of n parents at once, the formula unchanged.
+
+    F_c: [n, C, R] and k_hat_c: [n, C, R, d], the (already re-anchored, with
+    rotary positions) state of each parent's C children; qP: [n, R, d] the
+    parents' reference queries or [1, R, d].
+      F[n, r] = LSE_c F_c[n, c, r],   w = exp(F_c - F),
+      k_hat[n, r] = sum_c w[n, c, r] k_hat_c[n, c, r],
+      b_hat[n, r] = F[n, r] - q_hat_{n,r} . k_hat[n, r] * scale.
+    Returns (k_hat [n, R, d], F [n, R], b_hat [n, R]).
+    """
+    F = lse(F_c, axis=1)                                     # [n, R]
+    w = np.exp(F_c - F[:, None, :])                          # [n, C, R]
+    k_hat = np.einsum("ncr,ncrd->nrd", w, k_hat_c)
+    b_hat = F - np.sum(qP * k_hat, axis=-1) * scale
+    return k_hat, F, b_hat
+
+
 def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
                branch: int = 16, route_storage: str = "bf16", state_storage: str = "f32",
                block: int = 4096, inv_freq=None) -> Tree:
@@ -242,15 +282,16 @@ def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
 
     K: [>=T, d] keys (float64 values of the stored keys, or a CPU torch tensor
     read block by block), qref: [R, d].
-    Level 1 summarises raw keys (``leaf_summary``); level l >= 2 merges the
-    stored state of ``branch`` consecutive level-(l-1) nodes (``merge_summaries``).
+    Level 1 summarises raw keys (``leaf_level``: ``leaf_summary`` per chunk);
+    level l >= 2 merges the stored state of ``branch`` consecutive level-(l-1)
+    nodes (``merge_level``: ``merge_summaries`` per parent).
     ``block`` only bounds the temporary memory of the vectorised leaf pass.
 
     ``inv_freq`` (rotary frequencies, see ``rope``; None or empty: no rotation)
     gives the RoPE variant of paper §III-B: node i of level l summarises at the
     reference queries rotated to its last position, q_hat_{r,i} =
     rope(q_hat_r, (i + 1) * span_l - 1), and a parent moves each child's log
-    mass to its own rotated reference before the merge (``merge_summaries``).
+    mass to its own rotated reference before the merge (``reanchor``).
     The keys are the cache's keys as stored (already rotated by the model).
     """
     rot = inv_freq is not None and len(inv_freq) > 0
@@ -273,17 +314,7 @@ def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
     for i0 in range(0, n1, block):
         i1 = min(n1, i0 + block)
         Kc = rows_f64(K, i0 * leaf, i1 * leaf).reshape(i1 - i0, leaf, d)
-        qn = rotated(1, i0, i1)                                 # [n or 1, R, d]
-        if rot:   # s[n, r, c] = q_hat_{r,n} . k_{n,c} * scale
-            s = np.matmul(qn, np.swapaxes(Kc, 1, 2)) * scale
-        else:     # the same with one q_hat for every node: a matrix product, then a reshape
-            s = np.swapaxes((Kc.reshape(-1, d) @ qref.T).reshape(i1 - i0, leaf, -1), 1, 2) * scale
-        F = lse(s, axis=-1)
-        a = np.exp(s - F[..., None])
-        kh = np.matmul(a, Kc)                                   # [n, r, d] = a[n, r, c] . K[n, c, d]
-        k1[i0:i1] = kh
-        F1[i0:i1] = F
-        b1[i0:i1] = F - (np.sum(qn * kh, axis=-1) if rot else np.einsum("rd,nrd->nr", qref, kh)) * scale
+        k1[i0:i1], F1[i0:i1], b1[i0:i1] = leaf_level(Kc, rotated(1, i0, i1), scale)
     tree.levels.append(_store_level(leaf, k1, F1, b1, route_storage, state_storage))
     for lvl in range(2, depth + 1):
         child = tree.levels[-1]
@@ -294,10 +325,7 @@ def build_tree(K, T: int, qref: np.ndarray, depth: int, leaf: int = 64,
         if rot:                                                 # each child's log mass at the parent's q_hat
             qc = rotated(lvl - 1, 0, n * branch).reshape(n, branch, R, d)
             Fc = reanchor(Fc, kc, qP[:, None], qc, scale)
-        F = lse(Fc, axis=1)                                     # [n, R]
-        w = np.exp(Fc - F[:, None, :])                          # [n, C, R]
-        kh = np.einsum("ncr,ncrd->nrd", w, kc)
-        bh = F - (np.sum(qP * kh, axis=-1) if rot else np.einsum("rd,nrd->nr", qref, kh)) * scale
+        kh, F, bh = merge_level(Fc, kc, qP, scale)
         tree.levels.append(_store_level(tree.span(lvl), kh, F, bh, route_storage, state_storage))
     return tree
 

@@ -186,6 +186,51 @@ def test_merged_tree_equals_leaf_formula_over_span(d):
             np.testing.assert_allclose(L.b_hat[i], b_hat, rtol=0, atol=1e-11)
 
 
+TREE_FREQ = [1.0, 0.37, 0.05]     # partial rotary frequencies for the rotated-tree cases
+
+
+@pytest.mark.parametrize("d", [8, 128])
+@pytest.mark.parametrize("rotary", [False, True])
+def test_build_tree_nodes_equal_the_per_node_formulas(d, rotary):
+    """Every node of build_tree (its batched level passes) equals the one-node formulas:
+    a level-1 node is ``leaf_summary`` over its own keys at its own reference queries, a
+    level-l node ``merge_summaries`` over its stored children.  The batched passes are
+    pinned to the one-node functions, which the closed forms and identities pin."""
+    leaf, branch, depth = 8, 4, 3
+    T = leaf * branch ** 2 * 3 + leaf * 5 + 3              # ragged: orphan leaves and a partial chunk
+    _, K, _ = _clustered(T, d, 12, 31 + d)
+    rng = np.random.default_rng(32)
+    qref = 3 * rng.standard_normal((4, d)) / math.sqrt(d)
+    scale = 1 / math.sqrt(d)
+    freq = TREE_FREQ if rotary else None
+    tree = zo.build_tree(K, T, qref, depth, leaf=leaf, branch=branch, route_storage="f64",
+                         state_storage="f64", block=7, inv_freq=freq)
+    assert [lv.n for lv in tree.levels] == [T // leaf, T // (leaf * branch), T // (leaf * branch ** 2)]
+
+    def refs(level, i):
+        if not rotary:
+            return qref
+        return zo.rope(qref, zo.node_anchor(i, tree.span(level)), freq)
+
+    L1 = tree.levels[0]
+    for i in range(L1.n):
+        k_hat, F, b_hat = zo.leaf_summary(K[i * leaf:(i + 1) * leaf], refs(1, i), scale)
+        np.testing.assert_allclose(L1.F[i], F, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L1.k_state[i], k_hat, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L1.k_route[i], k_hat, rtol=0, atol=1e-13)
+        np.testing.assert_allclose(L1.b_hat[i], b_hat, rtol=0, atol=1e-12)
+    for lvl in range(2, depth + 1):
+        child, lv = tree.levels[lvl - 2], tree.levels[lvl - 1]
+        for i in range(lv.n):
+            ids = np.arange(i * branch, (i + 1) * branch)
+            q_c = np.stack([refs(lvl - 1, c) for c in ids]) if rotary else None
+            k_hat, F, b_hat = zo.merge_summaries(child.F[ids], child.k_state[ids], refs(lvl, i), scale,
+                                                 q_child=q_c)
+            np.testing.assert_allclose(lv.F[i], F, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(lv.k_state[i], k_hat, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(lv.b_hat[i], b_hat, rtol=0, atol=1e-12)
+
+
 def test_merge_entropy_chain_rule():
     d = 32
     _, K, _ = _clustered(64 * 16, d, 16, 9)

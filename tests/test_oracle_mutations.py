@@ -58,6 +58,34 @@ def merge_max_instead_of_lse(F_c, k_hat_c, qref, scale):
     return k_hat, F, F - np.sum(qref * k_hat, axis=-1) * scale
 
 
+def leaf_level_bias_sign(Kc, qn, scale):
+    k_hat, F, b_hat = _orig["leaf_level"](Kc, qn, scale)
+    return k_hat, F, F + np.sum(qn * k_hat, axis=-1) * scale
+
+
+def leaf_level_unnormalised(Kc, qn, scale):
+    s = np.matmul(np.broadcast_to(qn, (Kc.shape[0],) + qn.shape[1:]), np.swapaxes(Kc, 1, 2)) * scale
+    F = zo.lse(s, axis=-1)
+    k_hat = np.matmul(np.exp(s), Kc)                   # missing - F in the weights
+    return k_hat, F, F - np.sum(qn * k_hat, axis=-1) * scale
+
+
+def leaf_level_transposed(Kc, qn, scale):
+    k_hat, F, b_hat = _orig["leaf_level"](Kc, qn, scale)
+    return k_hat[:, ::-1], F, b_hat                    # references' k_hat swapped
+
+
+def merge_level_bias_sign(F_c, k_hat_c, qP, scale):
+    k_hat, F, b_hat = _orig["merge_level"](F_c, k_hat_c, qP, scale)
+    return k_hat, F, F + np.sum(qP * k_hat, axis=-1) * scale
+
+
+def merge_level_unnormalised(F_c, k_hat_c, qP, scale):
+    F = zo.lse(F_c, axis=1)
+    k_hat = np.einsum("ncr,ncrd->nrd", np.exp(F_c), k_hat_c)   # missing - F_P
+    return k_hat, F, F - np.sum(qP * k_hat, axis=-1) * scale
+
+
 def top_p_one_too_many(scores, ids, p):
     sel = _orig["top_p"](scores, ids, p)
     if sel.m < sel.n:
@@ -162,7 +190,14 @@ def rope_clockwise(x, pos, inv_freq):
     return _orig["rope"](x, -np.asarray(pos), inv_freq)  # the opposite sense of rotation
 
 
-_orig = {"leaf_summary": zo.leaf_summary, "top_p": zo.top_p, "top_k": zo.top_k, "rope": zo.rope}
+_orig = {"leaf_summary": zo.leaf_summary, "top_p": zo.top_p, "top_k": zo.top_k, "rope": zo.rope,
+         "leaf_level": zo.leaf_level, "merge_level": zo.merge_level}
+
+
+def _tree_pass_pins():
+    for d in (8, 128):
+        for rotary in (False, True):
+            pins.test_build_tree_nodes_equal_the_per_node_formulas(d, rotary)
 
 
 def _rope_tree_pins():
@@ -187,6 +222,11 @@ CASES = [
     ("merge_summaries", merge_unnormalised, lambda: pins.test_merge_closed_form(_golden())),
     ("merge_summaries", merge_max_instead_of_lse,
      lambda: (pins.test_merge_closed_form(_golden()), pins.test_merge_entropy_chain_rule())),
+    ("leaf_level", leaf_level_bias_sign, _tree_pass_pins),
+    ("leaf_level", leaf_level_unnormalised, _tree_pass_pins),
+    ("leaf_level", leaf_level_transposed, _tree_pass_pins),
+    ("merge_level", merge_level_bias_sign, _tree_pass_pins),
+    ("merge_level", merge_level_unnormalised, _tree_pass_pins),
     ("top_p", top_p_one_too_many, lambda: [pins.test_top_p_is_minimal_by_brute_force(s) for s in range(25)]),
     ("top_p", top_p_ties_descending, lambda: pins.test_top_p_closed_form_with_ties(_golden(), "top_p_ties")),
     ("top_p", top_p_strict, lambda: pins.test_top_p_closed_form_with_ties(_golden(), "top_p_exact_boundary")),
