@@ -420,9 +420,10 @@ class Route:
     cand: Dict[int, np.ndarray]               # level -> candidate ids (ascending)
     sel: Dict[int, Selection]                 # level -> selection
     leaves: np.ndarray                        # S_1(q), ascending chunk ids
+    kept: Dict[int, np.ndarray] = field(default_factory=dict)   # level -> the ids expanded
 
 
-def route(q: np.ndarray, t: int, tree: Tree, p, k=None) -> Route:
+def route(q: np.ndarray, t: int, tree: Tree, p, k=None, impose: Optional[Dict[int, np.ndarray]] = None) -> Route:
     """Top-down top-p routing of one query head at position ``t``.
 
     The top level is the highest level with a visible node; all its visible
@@ -433,6 +434,11 @@ def route(q: np.ndarray, t: int, tree: Tree, p, k=None) -> Route:
     per-level schedule (index l-1 = level l, e.g. ``p_root_schedule``).  With
     ``k`` (a count, or a per-level sequence of counts) each level keeps the
     k best candidates instead (``top_k``) and ``p`` is ignored.
+
+    ``impose`` (for comparisons only: level -> ids) replaces the kept set of those
+    levels by the given ids, which must be candidates of that level; the levels
+    below are then routed from them.  ``sel[l]`` still holds the oracle's own
+    selection of level l and ``kept[l]`` the set the expansion used.
     """
     d = q.shape[0]
     scale = 1.0 / math.sqrt(d)
@@ -451,11 +457,17 @@ def route(q: np.ndarray, t: int, tree: Tree, p, k=None) -> Route:
         sel = top_p(s, cand, _at_level(p, l)) if k is None else top_k(s, cand, _at_level(k, l))
         out.cand[l] = cand
         out.sel[l] = sel
+        kept = sel.ids
+        if impose is not None and l in impose:
+            kept = np.sort(np.asarray(impose[l], dtype=np.int64))
+            if len(np.unique(kept)) != len(kept) or not np.all(np.isin(kept, cand)):
+                raise ValueError(f"level {l}: imposed ids are not distinct candidates")
+        out.kept[l] = kept
         if l > 1:
-            children = (sel.ids[:, None] * tree.branch + np.arange(tree.branch)[None, :]).ravel()
+            children = (kept[:, None] * tree.branch + np.arange(tree.branch)[None, :]).ravel()
             orphans = np.arange(nvis[l] * tree.branch, nvis[l - 1], dtype=np.int64)
             cand = np.concatenate([children, orphans]).astype(np.int64)
-    out.leaves = out.sel[1].ids
+    out.leaves = out.kept[1]
     return out
 
 
