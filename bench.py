@@ -35,7 +35,7 @@ import torch  # noqa: E402
 
 import zha_synth as S  # noqa: E402
 
-DEFAULT_WORKLOAD = "batched-decode-128k"
+DEFAULT_WORKLOAD = "long-decode-1m"
 
 
 def parse():
@@ -47,7 +47,10 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(S.WORKLOADS))
     ap.add_argument("--p", type=float, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="CPU budget of one sampled oracle step, per worker process")
+    ap.add_argument("--cpu-workers", type=int, default=0,
+                    help="oracle worker processes (0: one per host core, at most one per query head)")
     ap.add_argument("--segment", type=int, default=0,
                     help="structured keys: runs of this many positions share a cluster centre "
                          "(a variant of the generator, not one of the five workloads)")
@@ -189,9 +192,8 @@ class ClockSampler:
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the attention
-# gather kernel, from the ncu capture summarised in
-# profiles/attn_tc_kernel.batched-decode-128k.md (batch 4, i.e. 16 of the 128 KV units),
-# valid while the kernel source is the one that was captured.
+# gather kernel, from an ncu capture of the batched 128K decode at batch 4 (16 of its 128 KV
+# units), valid while the kernel source is the one that was captured.
 PROFILED_TRAFFIC = {
     "batched-decode-128k": {"bytes": 1.075072e9 + 11.166976e6, "units": 16,
                             "source": "hierarchical_sparse_attention_02_b200/csrc/zha_attn_tc.cu",
@@ -235,12 +237,14 @@ def near_cutoff_count(routes) -> dict:
     mass at the cutoff lies within NEAR_CUTOFF of p, or whose two candidates at the
     boundary differ by less than NEAR_CUTOFF in softmax mass.  There a one-ulp difference
     in a score may legitimately change the kept set."""
-    levels = near = 0
-    for r in routes:
-        for sel in r.sel.values():
-            levels += 1
-            near += int(min(sel.margin, sel.gap) < NEAR_CUTOFF)
-    return {"heads": len(routes), "levels": levels, "near_cutoff": near, "threshold": NEAR_CUTOFF}
+    return near_cutoff_from_flags([[min(s.margin, s.gap) for s in r.sel.values()] for r in routes])
+
+
+def near_cutoff_from_flags(flags) -> dict:
+    """The same from per-head lists of min(margin, gap), one entry per routed level."""
+    levels = sum(len(f) for f in flags)
+    near = sum(int(x < NEAR_CUTOFF) for f in flags for x in f)
+    return {"heads": len(flags), "levels": levels, "near_cutoff": near, "threshold": NEAR_CUTOFF}
 
 
 def frontier_stats(level_cnt: np.ndarray) -> list:
@@ -382,48 +386,179 @@ def candidate_unions(level_cnt: np.ndarray, level_ids: np.ndarray, n_cap: dict, 
     return out
 
 
-def oracle_rate(w: S.Workload, p: float, seconds: float, device: str, routes: list = None, inv_freq=None):
-    """Query-heads/s of the CPU oracle on a bounded sample of the decode step.
+class _Bf16Rows:
+    """A [t_cap, d] bf16 array held as its raw 16-bit patterns, read row by row as float32
+    (exact: a bf16 value is the upper half of the fp32 with the same value).  It gives the
+    oracle's row readers (slices and index arrays) float values without a full fp32 copy."""
 
-    The sample: whole KV groups (G query heads of one (sequence, KV head) unit) of the
-    same seeded workload, routed and attended by the oracle one head at a time until
-    ``seconds`` of CPU time have been spent (at least one group).  The oracle's tree of
-    each sampled unit is built first, untimed (it is the decode step's prior state).
-    With ``routes`` (a list) the oracle's route of every sampled head is appended to it;
-    ``inv_freq`` builds the oracle's rotary tree.
-    """
-    from oracle import zha_oracle as zo
+    def __init__(self, bits: np.ndarray):
+        self.bits = bits
+        self.shape = bits.shape
+
+    def __getitem__(self, idx):
+        return (np.asarray(self.bits[idx]).astype(np.uint32) << 16).view(np.float32)
+
+
+def _oracle_worker(conn, spec):
+    """One process of the CPU-oracle pool (spawned: it never touches CUDA).
+
+    It attaches the shared K / V of sequence 0, builds the oracle's tree of every KV unit
+    its heads belong to (untimed: the step's prior state), then on each "step" message
+    routes and attends its query heads one at a time (zo.decode_head) until the step's
+    CPU budget is spent, and answers with the heads done and the seconds taken.  A
+    "check" message compares the GPU's leaf lists and outputs of its heads with the
+    oracle's results of the last step."""
+    from multiprocessing import shared_memory
     try:
         from threadpoolctl import threadpool_limits
-        limiter = threadpool_limits(1)
+        threadpool_limits(1)
     except Exception:  # pragma: no cover
-        limiter = None
-    one = S.scaled(w, T=w.T, B=1)
-    C, K, V = S.clustered_kv(one, device)
-    qref = S.reference_queries(one, device)
-    kn, vn = S.new_tokens(one, C, 1, device)
-    q = S.queries(one, C, 1, device)
-    K[:, :, w.T] = kn[:, 0]
-    V[:, :, w.T] = vn[:, 0]
-    Kc, Vc = K.cpu(), V.cpu()
-    qc = q.double().cpu().numpy()
-    qr = qref.double().cpu().numpy()
-    heads, spent = 0, 0.0
-    for hk in range(w.Hkv):
-        tree = zo.build_tree(Kc[0, hk], w.T + 1, qr[hk], w.depth,
-                             route_storage="bf16" if w.dtype == "bf16" else "f32", inv_freq=inv_freq)
-        t0 = time.process_time()
-        for h in range(hk * w.G, (hk + 1) * w.G):
-            r, _, _ = zo.decode_head(qc[0, 0, h], Kc[0, hk], Vc[0, hk], w.T, tree, p)
-            heads += 1
-            if routes is not None:
-                routes.append(r)
-        spent += time.process_time() - t0
-        if spent >= seconds:
+        pass
+    from oracle import zha_oracle as zo
+    shms = [shared_memory.SharedMemory(name=n) for n in (spec["k_name"], spec["v_name"])]
+    dt = np.uint16 if spec["dtype"] == "bf16" else np.float32
+    arrs = [np.ndarray(spec["shape"], dtype=dt, buffer=m.buf) for m in shms]
+    rows = (lambda a: _Bf16Rows(a)) if spec["dtype"] == "bf16" else (lambda a: a)
+    K = {hk: rows(arrs[0][hk]) for hk in spec["units"]}
+    V = {hk: rows(arrs[1][hk]) for hk in spec["units"]}
+    T, G = spec["T"], spec["G"]
+    t0 = time.perf_counter()
+    trees = {hk: zo.build_tree(K[hk], T + 1, spec["qref"][hk], spec["depth"], route_storage=spec["route_storage"],
+                               inv_freq=spec["inv_freq"]) for hk in spec["units"]}
+    conn.send(("ready", time.perf_counter() - t0))
+    last = {}
+    while True:
+        msg = conn.recv()
+        if msg[0] == "stop":
             break
-    if limiter is not None:
-        limiter.unregister() if hasattr(limiter, "unregister") else None
-    return heads / spent, heads, spent
+        if msg[0] == "step":
+            budget = msg[1]
+            last = {}
+            t0 = time.perf_counter()
+            for h in spec["heads"]:
+                r, o, _ = zo.decode_head(spec["q"][h], K[h // G], V[h // G], T, trees[h // G], spec["p"])
+                last[h] = (r, o)
+                if time.perf_counter() - t0 >= budget:
+                    break
+            conn.send(("done", len(last), time.perf_counter() - t0,
+                       [[(min(s.margin, s.gap)) for s in r.sel.values()] for r, _ in last.values()]))
+        if msg[0] == "check":
+            gpu = msg[1]                                 # h -> (leaf ids, output row)
+            out = []
+            for h, (r, o) in last.items():
+                leaves, og = gpu[h]
+                near = any(min(s.margin, s.gap) < NEAR_CUTOFF for s in r.sel.values())
+                same = np.array_equal(np.asarray(leaves, np.int64), r.leaves)
+                if not same:                             # the oracle's attention over the GPU's list
+                    o, _ = zo.attention(spec["q"][h], K[h // G], V[h // G], zo.index_set(leaves, T))
+                out.append((h, same, near, float(np.abs(np.asarray(og, np.float64) - o).max())))
+            conn.send(("checked", out))
+    for m in shms:
+        m.close()
+
+
+class OraclePool:
+    """The CPU oracle on the host cores: spawned worker processes, one BLAS thread each,
+    over the query heads of sequence 0 of a workload (contiguous blocks of heads, so a
+    worker builds the trees of one or two KV units).  The sample's K / V sit in shared
+    memory; nothing is copied per step."""
+
+    def __init__(self, w: S.Workload, p: float, K0, V0, q0, qref, inv_freq=None, workers: int = 0):
+        """K0, V0: [Hkv, t_cap, d] of sequence 0 with the step's new token at position T;
+        q0: [Hq, d] its queries; qref: [Hkv, R, d] (torch tensors on any device)."""
+        import multiprocessing as mp
+        from multiprocessing import shared_memory
+        bf16 = w.dtype == "bf16"
+        self.w, self.p = w, p
+        self.shms = []
+        names = []
+        for X in (K0, V0):
+            x = X.cpu()
+            a = (x.view(torch.int16).numpy().view(np.uint16) if bf16 else x.numpy())
+            m = shared_memory.SharedMemory(create=True, size=a.nbytes)
+            np.ndarray(a.shape, dtype=a.dtype, buffer=m.buf)[...] = a
+            self.shms.append(m)
+            names.append(m.name)
+            shape = a.shape
+        cpus = os.cpu_count() or 1
+        cap = max(1, int(32 * (1 << 20) // max(1, w.T)))      # bounds the trees held per unit
+        self.n = workers or max(1, min(cpus, w.Hq, cap))
+        self.cpus = cpus
+        qc = q0.double().cpu().numpy()
+        qr = qref.double().cpu().numpy()
+        ctx = mp.get_context("spawn")
+        self.conns, self.procs = [], []
+        per = [list(range(i * w.Hq // self.n, (i + 1) * w.Hq // self.n)) for i in range(self.n)]
+        for heads in per:
+            units = sorted({h // w.G for h in heads})
+            spec = {"k_name": names[0], "v_name": names[1], "shape": shape, "dtype": w.dtype, "units": units,
+                    "heads": heads, "q": {h: qc[h] for h in heads}, "qref": {u: qr[u] for u in units},
+                    "T": w.T, "G": w.G, "depth": w.depth, "p": p,
+                    "route_storage": "bf16" if bf16 else "f32", "inv_freq": inv_freq}
+            a, b = ctx.Pipe()
+            pr = ctx.Process(target=_oracle_worker, args=(b, spec), daemon=True)
+            pr.start()
+            self.conns.append(a)
+            self.procs.append(pr)
+        self.build_s = max(c.recv()[1] for c in self.conns)
+
+    @classmethod
+    def from_workload(cls, w: S.Workload, p: float, device: str, inv_freq=None, workers: int = 0):
+        """A pool over sequence 0 of the workload drawn afresh by the seeded generator."""
+        one = S.scaled(w, T=w.T, B=1)
+        C, K, V = S.clustered_kv(one, device)
+        qref = S.reference_queries(one, device)
+        kn, vn = S.new_tokens(one, C, 1, device)
+        q = S.queries(one, C, 1, device)
+        K[:, :, w.T] = kn[:, 0]
+        V[:, :, w.T] = vn[:, 0]
+        return cls(w, p, K[0], V[0], q[0, 0], qref, inv_freq=inv_freq, workers=workers)
+
+    def step(self, budget: float):
+        """One sampled step: every worker routes and attends its heads for at most `budget`
+        seconds (at least one head each).  Returns (heads done, wall seconds, near flags)."""
+        t0 = time.perf_counter()
+        for c in self.conns:
+            c.send(("step", budget))
+        res = [c.recv() for c in self.conns]
+        wall = time.perf_counter() - t0
+        return sum(r[1] for r in res), wall, [m for r in res for m in r[3]]
+
+    def check(self, leaves: dict, outputs: dict):
+        """Compare the GPU's leaf lists and outputs (dicts over heads of sequence 0) with the
+        oracle's results of the last step: a parity summary."""
+        for c, pr_heads in zip(self.conns, self._heads()):
+            c.send(("check", {h: (leaves[h], outputs[h]) for h in pr_heads}))
+        rows = [x for c in self.conns for x in c.recv()[1]]
+        return {"heads": len(rows), "exact": sum(1 for r in rows if r[1]),
+                "near_cutoff_mismatch": sum(1 for r in rows if not r[1] and r[2]),
+                "failed": sum(1 for r in rows if not r[1] and not r[2]),
+                "max_abs_err": max((r[3] for r in rows), default=None),
+                "rule": "leaf lists equal to the oracle's, or differing only for a head with a level whose "
+                        f"cutoff margin or boundary gap is under {NEAR_CUTOFF}; the output against the oracle's "
+                        "attention over the GPU's own list"}
+
+    def _heads(self):
+        w = self.w
+        return [list(range(i * w.Hq // self.n, (i + 1) * w.Hq // self.n)) for i in range(self.n)]
+
+    def close(self):
+        for c in self.conns:
+            try:
+                c.send(("stop",))
+            except Exception:  # noqa: BLE001
+                pass
+        for pr in self.procs:
+            pr.join(timeout=30)
+        for m in self.shms:
+            m.close()
+            m.unlink()
+
+
+def oracle_sample(pool: OraclePool, seconds: float) -> dict:
+    """Query-heads/s of the CPU oracle over one sampled step of the pool."""
+    heads, wall, flags = pool.step(seconds)
+    return {"value": heads / wall, "heads": heads, "wall_s": wall, "flags": flags}
 
 
 def stage_breakdown(lib, step, stream, nb, ms_step):
@@ -470,27 +605,41 @@ def stage_breakdown(lib, step, stream, nb, ms_step):
 
 
 def run_reference(args, w, p, ws, rank):
+    """The reference arm: the CPU oracle as it stands, on the host cores (a pool of
+    spawned worker processes, one BLAS thread each), on sampled steps of the workload:
+    each step routes and attends the query heads of sequence 0 (at most `cpu_seconds`
+    of CPU per worker).  value = query heads per second of that sample; ms_per_step is
+    the measured wall time of one sampled step."""
     if rank != 0:
         return
     K, W = args.steps, args.warmup
     dev = "cuda" if torch.cuda.is_available() else "cpu"
-    per_step = max(1.0, 150.0 / max(1, K + W))
+    per_step = max(0.5, 150.0 / max(1, K + W))
     freq = (10000.0 ** (-np.arange(args.rope, dtype=np.float64) / args.rope)).astype(np.float32).astype(
         np.float64) if args.rope else None
-    rates = []
-    for i in range(W + K):
-        r, heads, spent = oracle_rate(w, p, min(per_step, args.cpu_seconds), dev, inv_freq=freq)
-        if i >= W:
-            rates.append((r, heads, spent))
-    value = statistics.median(r[0] for r in rates)
-    ms = 1e3 * w.B * w.Hq / value
+    pool = OraclePool.from_workload(w, p, dev, inv_freq=freq, workers=args.cpu_workers)
+    try:
+        rates = []
+        for i in range(W + K):
+            r = oracle_sample(pool, min(per_step, args.cpu_seconds))
+            if i >= W:
+                rates.append(r)
+    finally:
+        pool.close()
+    value = statistics.median(r["value"] for r in rates)
+    ms = 1e3 * statistics.median(r["wall_s"] for r in rates)
+    heads = rates[0]["heads"]
     line = {
         "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": 1,
         "steps": K, "warmup": W, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {**config_of(w, p), **({"rope_pairs": args.rope} if args.rope else {})}, "impl": "reference",
-        "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
-                         "sample": f"{rates[0][1]} query heads (whole KV groups) per step, fp64 numpy, 1 thread"},
+        "step_sample": f"{heads} of the {w.B * w.Hq} query heads of a full step (sequence 0); "
+                       "ms_per_step is the measured wall time of that sample",
+        "cpu_baseline": {"value": value, "unit": "query-heads/s", "cores": pool.n, "host_cpus": pool.cpus,
+                         "kind": "oracle",
+                         "sample": f"{heads} query heads of sequence 0 per step, fp64 numpy, {pool.n} worker "
+                                   f"processes x 1 thread (tree built untimed, {pool.build_s:.1f} s)"},
         "e2e": {"value": value, "unit": "query-heads/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -621,6 +770,7 @@ def main():
                    dtype=torch.bfloat16 if w.dtype == "bf16" else torch.float32, rope_pairs=args.rope)
     C, K, V = S.clustered_kv(wr, dev)
     qref = S.reference_queries(wr, dev)
+    qref_plain = qref
     freq = None
     if args.rope:                     # the tree calls read the frequencies after the references
         freq = (10000.0 ** (-torch.arange(args.rope, dtype=torch.float64) / args.rope)).float()
@@ -832,15 +982,27 @@ def main():
             frontier = {"error": repr(e)}
     cpu = None
     near = None
+    parity = None
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        routes = []
-        r, heads, spent = oracle_rate(w, p, args.cpu_seconds, "cuda", routes,
-                                      freq.double().numpy() if freq is not None else None)
-        cpu = {"value": r, "unit": "query-heads/s", "cores": 1, "kind": "oracle",
-               "sample": f"{heads} query heads (whole KV groups of sequence 0) of {w.name}, "
-                         f"route + attention, fp64 numpy, 1 thread, {spent:.1f} s CPU"}
-        if args.path == "zha":
-            near = {**near_cutoff_count(routes), "sample": "the oracle's routes of the cpu_baseline sample"}
+        # the decode step's own inputs of sequence 0 (the cache holds the new token at T)
+        pool = OraclePool(w, p, K[0], V[0], q[0, 0], qref_plain,
+                          inv_freq=freq.double().numpy() if freq is not None else None, workers=args.cpu_workers)
+        try:
+            r = oracle_sample(pool, args.cpu_seconds)
+            cpu = {"value": r["value"], "unit": "query-heads/s", "cores": pool.n, "host_cpus": pool.cpus,
+                   "kind": "oracle",
+                   "sample": f"{r['heads']} query heads of sequence 0 of {w.name}, route + attention, fp64 "
+                             f"numpy, {pool.n} worker processes x 1 thread, {r['wall_s']:.1f} s wall "
+                             f"(trees built untimed, {pool.build_s:.1f} s)"}
+            if args.path == "zha":
+                near = {**near_cutoff_from_flags(r["flags"]), "sample": "the oracle's routes of the cpu_baseline sample"}
+                Oc = O.float().cpu().numpy()
+                leaves = {h: ids_c[0, 0, h, :cnt_c[0, 0, h]] for h in range(w.Hq)}
+                outs = {h: Oc[0, 0, h] for h in range(w.Hq)}
+                parity = {**pool.check(leaves, outs), "sample": "the heads of the cpu_baseline sample, "
+                          "against the decode step's leaf lists and outputs"}
+        finally:
+            pool.close()
     line = {
         "metric": "ZHA decode query-heads/s", "value": value, "unit": "query-heads/s", "n_gpus": ws,
         "steps": Ksteps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -861,6 +1023,7 @@ def main():
         "stages_ms": stages,
         "frontier": frontier,
         "near_cutoff": near,
+        "parity": parity,
         "tree_build": {"ms": build_ms, "gbs": k_bytes / (build_ms * 1e-3) / 1e9},
         "e2e": {"value": ws * w.B * w.Hq / (e2e_ms * 1e-3), "unit": "query-heads/s",
                 "h2d_bytes_per_step": (q.numel() + k_new.numel() + v_new.numel()) * es,

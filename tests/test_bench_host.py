@@ -129,3 +129,38 @@ def test_paper_model_terms():
     # launch overhead: the gaps between kernels plus the launches of the empty level 3
     assert m["launch_gaps_ms"] == pytest.approx(0.005 + 0.004 + 0.003) and m["launches_per_step"] == 8
     assert rows["route L3 (empty)"]["measured_ms"] == pytest.approx(0.007)
+
+
+def test_oracle_pool_parity_check_on_cpu():
+    """The bench's CPU-oracle pool: a step on spawned workers, then the parity summary of
+    GPU-shaped results made up on the host (the oracle's own lists and outputs: all exact;
+    one list with a far-off chunk: a failure)."""
+    import zha_synth as S
+    w = S.scaled(S.workload("batched-decode-128k"), T=4096 + 70, B=1, n_centres=64)
+    pool = bench.OraclePool.from_workload(w, 0.9, "cpu", workers=3)
+    try:
+        r = bench.oracle_sample(pool, 30.0)
+        assert r["heads"] == w.Hq and r["value"] > 0 and len(r["flags"]) == w.Hq
+        one = S.scaled(w, T=w.T, B=1)
+        C, K, V = S.clustered_kv(one, "cpu")
+        kn, vn = S.new_tokens(one, C, 1, "cpu")
+        q = S.queries(one, C, 1, "cpu")[0, 0].double().numpy()
+        K[:, :, w.T], V[:, :, w.T] = kn[:, 0], vn[:, 0]
+        qref = S.reference_queries(one, "cpu").double().numpy()
+        leaves, outs = {}, {}
+        for hk in range(w.Hkv):
+            tree = zo.build_tree(K[0, hk], w.T + 1, qref[hk], w.depth)
+            for h in range(hk * w.G, (hk + 1) * w.G):
+                rt, o, _ = zo.decode_head(q[h], K[0, hk], V[0, hk], w.T, tree, 0.9)
+                leaves[h], outs[h] = rt.leaves, o
+        got = pool.check(leaves, outs)
+        assert got["heads"] == w.Hq and got["exact"] == w.Hq and got["failed"] == 0
+        assert got["max_abs_err"] < 1e-12
+        bad = dict(leaves)
+        bad[3] = np.union1d(leaves[3], [w.T // 64 - 1])[-len(leaves[3]) - 1:]
+        if len(leaves[3]) == w.T // 64:
+            bad[3] = leaves[3][1:]
+        got = pool.check(bad, outs)
+        assert got["exact"] == w.Hq - 1 and got["failed"] + got["near_cutoff_mismatch"] == 1
+    finally:
+        pool.close()
