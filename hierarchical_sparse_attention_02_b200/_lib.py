@@ -19,7 +19,7 @@ EXPORTS = [
     "zha_status_str", "zha_check_geom", "zha_tree_bytes", "zha_tree_level", "zha_workspace_bytes",
     "zha_leaf_cap", "zha_build_tree", "zha_append", "zha_route", "zha_route_schedule", "zha_route_topk", "zha_sparse_attn",
     "zha_decode",
-    "zha_dense_decode", "zha_flat_index", "zha_sparse_attn_noalloc", "zha_launch_count",
+    "zha_dense_decode", "zha_flat_index", "zha_sparse_attn_noalloc", "zha_check_bounded_wait", "zha_launch_count",
     "zha_last_error", "zha_trace", "zha_trace_count",
 ]
 ZHA_NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -63,6 +63,7 @@ _SIGS = {
     "zha_dense_decode": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_flat_index": (_I32, [_G, _P, _P, _P, _P, _I32, _F64, _P, _P, _I32, _P, Buf, _P, _P]),
     "zha_sparse_attn_noalloc": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _P, _P, _P]),
+    "zha_check_bounded_wait": (_I32, [_I64, _P, _P, _P]),
     "zha_launch_count": (_I64, []),
     "zha_last_error": (ctypes.c_char_p, []),
     "zha_trace": (None, [_I32, ctypes.POINTER(ctypes.c_void_p), ctypes.POINTER(ctypes.c_void_p), _I32]),

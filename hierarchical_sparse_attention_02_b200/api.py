@@ -202,3 +202,9 @@ def zha_flat_index(g, Q, K, V, q_pos, p, leaf_ids, leaf_cnt, O, ws, dev_status, 
     _check("zha_flat_index", _lib.load().zha_flat_index(
         ctypes.byref(g.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_pos), Q.shape[1], float(p), _ptr(leaf_ids),
         _ptr(leaf_cnt), leaf_ids.shape[-1], _ptr(O), _buf(ws), _ptr(dev_status), _stream(stream)))
+
+
+def zha_check_bounded_wait(polls: int, dev_status, out, stream=None):
+    """The failure-detection check of the bounded device waits (out: int64 [4] on the device)."""
+    _check("zha_check_bounded_wait", _lib.load().zha_check_bounded_wait(
+        int(polls), _ptr(dev_status), _ptr(out), _stream(stream)))

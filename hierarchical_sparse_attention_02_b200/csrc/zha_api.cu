@@ -229,6 +229,13 @@ zha_status zha_decode(const zha_geom* g, const void* q, const void* k_new, const
   return from_cuda(attention(ac));
 }
 
+zha_status zha_check_bounded_wait(int64_t polls, int32_t* dev_status, int64_t* out, void* stream) {
+  if (polls < 1 || polls > ((int64_t)1 << 32) || !dev_status || !out) return ZHA_ERR_INVALID_ARG;
+  wait_check_launch((long long)polls, dev_status, (long long*)out, (cudaStream_t)stream);
+  count_launch();
+  return from_cuda(launch_status("wait_check_kernel"));
+}
+
 zha_status zha_dense_decode(const zha_geom* g, const void* Q, const void* K, const void* V,
                             const int64_t* q_pos, int32_t nq, void* O, float* lse, zha_buf ws,
                             int32_t* dev_status, void* stream) {

@@ -73,10 +73,11 @@ __device__ __forceinline__ bool mbar_try(unsigned long long* b, uint32_t parity)
   return ok != 0;
 }
 
-// Bounded wait: false after kSpinLimit polls, or at once when another thread of the CTA
+// Bounded wait: false after `limit` polls, or at once when another thread of the CTA
 // has given up (`abort` set); the caller then reports and stops waiting for anything.
-__device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity, const int* abort) {
-  for (long long i = 0; i < kSpinLimit; ++i) {
+__device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity, const int* abort,
+                                          long long limit = kSpinLimit) {
+  for (long long i = 0; i < limit; ++i) {
     if ((i & 255) == 0 && *(volatile const int*)abort) return false;
     if (mbar_try(b, parity)) return true;
   }
@@ -556,7 +557,45 @@ flat_tc_kernel(const __grid_constant__ CUtensorMap kmap, FlatTcArgs a) {
   }
 }
 
+// ---------------------------------------------------------------------------
+// Check of the bounded waits: warp 0 waits on an mbarrier that nothing ever completes, with
+// the rings' own wait and `polls` as its limit; when it gives up it reports ZHA_ERR_DEVICE
+// and raises `abort` as the ring kernels do.  Warp 1 waits on a second such barrier with a
+// limit 64 times larger; it stops early, through `abort`, once warp 0 has given up.
+// out[0], out[1] = the clock cycles each warp spent waiting, out[2] = 1 if warp 0 gave
+// up, out[3] = 1 if warp 1 returned without its barrier completing.  No copy is in flight
+// and nothing faults: the kernel ends normally.
+// ---------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(64) wait_check_kernel(long long polls, int32_t* st, long long* out) {
+  __shared__ unsigned long long bar[2];
+  __shared__ int abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    abort = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  if (lane != 0) return;
+  const long long t0 = clock64();
+  const bool ok = mbar_wait(&bar[warp], 0u, &abort, warp == 0 ? polls : polls * 64);
+  const long long dt = clock64() - t0;
+  if (!ok && warp == 0) {
+    set_status(st, ZHA_ERR_DEVICE);
+    atomicExch(&abort, 1);
+  }
+  out[warp] = dt;
+  out[2 + warp] = ok ? 0 : 1;
+}
+
 }  // namespace tc
+
+cudaError_t wait_check_launch(long long polls, int32_t* dev_status, long long* out, cudaStream_t stream) {
+  tc::wait_check_kernel<<<1, 64, 0, stream>>>(polls, dev_status, out);
+  return cudaSuccess;
+}
 
 // ---------------------------------------------------------------------------
 // host side: tensor maps and launch

@@ -318,6 +318,8 @@ cudaError_t attention(const AttnCall& c);
 cudaError_t flat_tc_launch(const zha_geom& g, int nq, const void* Q, const void* K, const int64_t* q_pos,
                           int64_t pos_uniform, int64_t C1, int* cand_ids, double* cand_score, int* cand_cnt,
                           int32_t* dev_status, cudaStream_t stream);
+// The bounded-wait check (zha_check_bounded_wait).
+cudaError_t wait_check_launch(long long polls, int32_t* dev_status, long long* out, cudaStream_t stream);
 cudaError_t attn_tc_launch(const AttnCall& c, const AttnWs& w, const int* stage_ids,
                            const unsigned int* stage_mask, const int* stage_cnt, const int* pair_off,
                            float* partials);

@@ -295,6 +295,23 @@ zha_status zha_sparse_attn_noalloc(const zha_geom* g, const void* Q, const void*
                                    const int32_t* leaf_cnt, int32_t leaf_cap, void* O, float* lse,
                                    int32_t* dev_status, void* stream);
 
+/*
+ * zha_check_bounded_wait - failure-detection check of the bounded device waits.
+ * The paper has no counterpart: this call exercises the error path of the shared-memory
+ * barrier waits that the TMA rings of the attention and flat-index kernels rely on.  It
+ * launches one CTA whose first warp waits, with the rings' own bounded wait, on an
+ * mbarrier that nothing ever completes and gives up after `polls` polls; it then sets
+ * *dev_status = ZHA_ERR_DEVICE (the first error wins) and raises the CTA's abort flag,
+ * as a ring kernel does.  A second warp waits on another never-completed barrier with a
+ * 64 times larger limit and must stop early, on that flag.  The kernel ends normally:
+ * no copy is in flight, nothing faults, and the context stays usable.
+ *   polls       in [1, 2^32].
+ *   out         device int64 [4]: the clock cycles each warp waited (warp 0, warp 1),
+ *               then 1 / 0 for each warp: it returned without its barrier completing.
+ *   dev_status  device int32 the caller zeroes.
+ */
+zha_status zha_check_bounded_wait(int64_t polls, int32_t* dev_status, int64_t* out, void* stream);
+
 /* Number of kernels this library has enqueued since it was loaded (host counter). */
 int64_t zha_launch_count(void);
 

@@ -26,7 +26,7 @@ def declared_symbols():
 
 def test_exports_every_declared_symbol(lib):
     decl = declared_symbols()
-    assert len(decl) == 20
+    assert len(decl) == 21
     assert sorted(decl) == sorted(_lib.EXPORTS)
     for name in decl:
         assert hasattr(lib, name), name
@@ -86,6 +86,9 @@ def test_host_side_rejections_enqueue_nothing(lib):
     buf = _lib.Buf(0x1000, 1 << 40)
     small = _lib.Buf(0x1000, 16)
     n0 = lib.zha_launch_count()
+    # the bounded-wait check: polls outside [1, 2^32], null pointers
+    for polls, st, out in ((0, fake, fake), (1 << 33, fake, fake), (100, None, fake), (100, fake, None)):
+        assert lib.zha_check_bounded_wait(polls, st, out, None) == 1
     # p outside (0, 1]
     for p in (0.0, -0.5, 1.5, float("nan")):
         assert lib.zha_route(ctypes.byref(g), fake, fake, 1, p, buf, fake, fake, 8, None, None, buf, fake, None) == 1
