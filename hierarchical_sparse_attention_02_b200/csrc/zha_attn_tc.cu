@@ -18,6 +18,7 @@
 #include <mutex>
 
 #include "zha_internal.cuh"
+#include "zha_ptx.cuh"
 
 namespace zha {
 
@@ -32,7 +33,7 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 constexpr int kBoxBytes = 64 * 128;              // 64 rows x 64 bf16, one swizzled box
 constexpr int kStageBytes = 4 * kBoxBytes;       // K lo/hi, V lo/hi
 constexpr uint32_t kTxBytes = kStageBytes;
-constexpr long long kSpinLimit = 1ll << 22;      // mbarrier polls before giving up
+using namespace ptx;
 
 struct Smem {
   unsigned char stage[kStages][kStageBytes];     // 1024-byte aligned (swizzle atoms)
@@ -44,83 +45,6 @@ struct Smem {
   int abort;                                     // set once any wait of the CTA gave up
   int zero;                                      // always 0
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-
-__device__ __forceinline__ void mbar_init(unsigned long long* b, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(b)), "r"(count));
-}
-
-__device__ __forceinline__ void mbar_arrive_tx(unsigned long long* b, uint32_t tx) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(b)), "r"(tx)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(unsigned long long* b) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(b)) : "memory");
-}
-
-__device__ __forceinline__ bool mbar_try(unsigned long long* b, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
-      " selp.u32 %0, 1, 0, p;\n}\n"
-      : "=r"(ok)
-      : "r"(smem_u32(b)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait: false after `limit` polls, or at once when another thread of the CTA
-// has given up (`abort` set); the caller then reports and stops waiting for anything.
-__device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity, const int* abort,
-                                          long long limit = kSpinLimit) {
-  for (long long i = 0; i < limit; ++i) {
-    if ((i & 255) == 0 && *(volatile const int*)abort) return false;
-    if (mbar_try(b, parity)) return true;
-  }
-  return false;
-}
-
-__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, int x, int y, int z,
-                                            unsigned long long* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-      "l"((unsigned long long)map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
-      : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
-               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
-                                         uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9},"
-      " {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-// Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a 128B-swizzled box.
-__device__ __forceinline__ uint32_t swz(int row, int chunk) {
-  return (uint32_t)(row * 128 + ((chunk ^ (row & 7)) << 4));
-}
 
 struct Args {
   int B, nq, Hq, Hkv, G;
@@ -601,7 +525,7 @@ cudaError_t wait_check_launch(long long polls, int32_t* dev_status, long long* o
 // host side: tensor maps and launch
 // ---------------------------------------------------------------------------
 
-static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
   std::call_once(once, [] {
@@ -615,7 +539,7 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // [units, t_cap, 128] bf16 cache as a 3-D tensor map with 64 x 64 boxes, 128B swizzle.
-static bool make_kv_map(CUtensorMap* map, const void* base, int64_t units, int64_t t_cap) {
+bool make_kv_map(CUtensorMap* map, const void* base, int64_t units, int64_t t_cap) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)t_cap, (cuuint64_t)units};
@@ -627,7 +551,7 @@ static bool make_kv_map(CUtensorMap* map, const void* base, int64_t units, int64
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-static int sm_count() {
+int sm_count() {
   int dev = 0, n = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
   return n;

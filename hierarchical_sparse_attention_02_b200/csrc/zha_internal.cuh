@@ -2,6 +2,7 @@
 // exact number conversions, block reductions and the device status word.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -140,6 +141,19 @@ inline AttnWs attn_ws(const zha_geom& g, int nq, size_t base = 0, int64_t cps = 
   w.bytes = off;
   return w;
 }
+
+// Query-tile attention for prefill (zha_prefill_attn): tiles of Qt = kPrefillRows / G
+// consecutive queries x the G heads of one KV head; per (tile, range of kRange chunk ids)
+// the union entries (chunk id, 128-bit mask of the rows that selected it) and a count.
+constexpr int kPrefillRows = 128;
+
+struct PrefillWs {
+  size_t ent_ids, ent_mask, ent_cnt, bytes;
+  int Qt;
+  int64_t nqt, tiles, nr;
+};
+
+PrefillWs prefill_ws(const zha_geom& g, int nq, size_t base = 0);
 
 // Host-side launch counter (exported as zha_launch_count).
 extern std::atomic<int64_t> g_launches;
@@ -305,6 +319,24 @@ struct AttnCall {
   int64_t cps = 0;               // chunks per work item; 0: the default of attn_ws
 };
 
+struct PrefillCall {
+  const zha_geom* g;
+  int nq;
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int64_t* q_pos;
+  const int* leaf_ids;
+  const int* leaf_cnt;
+  int leaf_cap;
+  void* O;
+  float* lse;
+  char* ws;                      // workspace base, layout prefill_ws(g, nq, 0)
+  int32_t* dev_status;
+  cudaStream_t stream;
+};
+
+cudaError_t prefill_attention(const PrefillCall& c);
 cudaError_t tree_extend(const zha_geom& g, const void* K, const float* qref, void* tree,
                         int64_t t_old, int64_t t_new, cudaStream_t s);
 cudaError_t append_tokens(const zha_geom& g, void* K, void* V, const void* k_new,
@@ -318,6 +350,10 @@ cudaError_t attention(const AttnCall& c);
 cudaError_t flat_tc_launch(const zha_geom& g, int nq, const void* Q, const void* K, const int64_t* q_pos,
                           int64_t pos_uniform, int64_t C1, int* cand_ids, double* cand_score, int* cand_cnt,
                           int32_t* dev_status, cudaStream_t stream);
+// Tensor maps and device facts shared by the TMA-fed kernels (zha_attn_tc.cu).
+// make_kv_map: a [units, t_cap, 128] bf16 cache as a 3-D map of 64 x 64 boxes, 128B swizzle.
+bool make_kv_map(CUtensorMap* map, const void* base, int64_t units, int64_t t_cap);
+int sm_count();
 // The bounded-wait check (zha_check_bounded_wait).
 cudaError_t wait_check_launch(long long polls, int32_t* dev_status, long long* out, cudaStream_t stream);
 cudaError_t attn_tc_launch(const AttnCall& c, const AttnWs& w, const int* stage_ids,
