@@ -62,8 +62,9 @@ def parse():
                          "(the dominant kernel's duration then comes from traced, uncaptured steps)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
-    ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat"],
-                    help="zha: the hot path (default); dense / flat: the baselines on the same inputs")
+    ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat", "prefill"],
+                    help="zha: the hot path (default); dense / flat: the baselines on the same inputs; "
+                         "prefill: the query-tile attention of the chunked-prefill workload")
     ap.add_argument("--sweep", action="store_true",
                     help="crossover sweep over T and depth against the dense kernel (one JSON line each)")
     ap.add_argument("--model", metavar="FILE", default=None,
@@ -732,6 +733,135 @@ def run_sweep(args):
         torch.cuda.empty_cache()
 
 
+def tile_unions(ids: np.ndarray, cnt: np.ndarray, pos: np.ndarray, Hkv: int, G: int) -> np.ndarray:
+    """Chunks each query tile gathers: the union over its Qt = 128 // G queries x G heads
+    of their leaf lists, plus chunk 0 and every query's own chunk (the tiles of
+    zha_prefill_attn).  ids [B, nq, Hq, cap], cnt [B, nq, Hq], pos [B, nq].  Returns the
+    entry count of every tile, in (sequence, KV head, tile) order."""
+    B, nq, Hq, _ = ids.shape
+    qt = 128 // G
+    out = []
+    for b in range(B):
+        for hk in range(Hkv):
+            for q0 in range(0, nq, qt):
+                qs = range(q0, min(nq, q0 + qt))
+                parts = [np.array([0]), np.asarray(pos[b, list(qs)]) // 64]
+                for qi in qs:
+                    for h in range(hk * G, (hk + 1) * G):
+                        parts.append(ids[b, qi, h, :cnt[b, qi, h]])
+                out.append(len(np.unique(np.concatenate(parts))))
+    return np.asarray(out, np.int64)
+
+
+def run_prefill(args):
+    """Chunked-prefill attention: the workload's n_new appended causal queries, routed once
+    (untimed), then attended by the query-tile tensor-core path (zha_prefill_attn, timed
+    over --steps calls) and by the per-query gather path (zha_sparse_attn) on the same
+    leaf lists.  One JSON line; the roofline is the tile kernel's tensor-pipe rate."""
+    import hierarchical_sparse_attention_02_b200 as Z
+    from hierarchical_sparse_attention_02_b200 import _lib
+    Z.load_library()
+    torch.cuda.set_device(0)
+    dev = torch.device("cuda", 0)
+    w = S.workload("prefill-append-256k")
+    if args.batch is not None:
+        w = S.scaled(w, T=w.T, B=args.batch)
+    p = args.p if args.p is not None else w.p[0]
+    g = Z.Geometry(B=w.B, Hq=w.Hq, Hkv=w.Hkv, t_cap=w.t_cap, depth=w.depth, R=w.R)
+    C, K, V = S.clustered_kv(w, dev)
+    qref = S.reference_queries(w, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    tree = Z.empty_tree(g, dev)
+    Z.zha_build_tree(g, K, w.T, qref, tree, st)
+    kn, vn = S.new_tokens(w, C, w.n_new, dev)
+    Z.zha_append(g, K, V, kn, vn, w.T, qref, tree, st)
+    Q = S.queries(w, C, w.n_new, dev)
+    del C
+    nq = w.n_new
+    pos = (w.T + torch.arange(nq, device=dev, dtype=torch.int64)).view(1, -1).repeat(w.B, 1).contiguous()
+    ids = torch.empty(w.B, nq, w.Hq, Z.leaf_cap(g), dtype=torch.int32, device=dev)
+    cnt = torch.empty(w.B, nq, w.Hq, dtype=torch.int32, device=dev)
+    wr = Z.empty_workspace(g, nq, Z.ZHA_OP_ROUTE, dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    Z.zha_route(g, Q, pos, p, tree, ids, cnt, wr, st)
+    torch.cuda.synchronize()
+    e0.record(); Z.zha_route(g, Q, pos, p, tree, ids, cnt, wr, st); e1.record()
+    torch.cuda.synchronize()
+    route_ms = e0.elapsed_time(e1)
+    del wr
+    O1 = torch.empty(w.B, nq, w.Hq, w.d, dtype=torch.bfloat16, device=dev)
+    O2 = torch.empty_like(O1)
+    wp = Z.empty_workspace(g, nq, Z.ZHA_OP_PREFILL, dev)
+    wa = Z.empty_workspace(g, nq, Z.ZHA_OP_ATTN, dev)
+    lib = _lib.load()
+
+    def timed(fn, steps, warm):
+        for _ in range(warm):
+            fn()
+        torch.cuda.synchronize()
+        n_ev = steps
+        a = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+        b = [torch.cuda.Event(enable_timing=True) for _ in range(n_ev)]
+        for x in a + b:
+            x.record()
+        torch.cuda.synchronize()
+        arr_s = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(x.cuda_event) for x in a])
+        arr_e = (ctypes.c_void_p * n_ev)(*[ctypes.c_void_p(x.cuda_event) for x in b])
+        lib.zha_trace(_lib.ZHA_TRACE_ATTN, arr_s, arr_e, n_ev)
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for _ in range(steps):
+            fn()
+        t1.record()
+        torch.cuda.synchronize()
+        k = lib.zha_trace_count(_lib.ZHA_TRACE_ATTN)
+        lib.zha_trace(_lib.ZHA_TRACE_ATTN, None, None, 0)
+        if st.item() != 0:
+            raise RuntimeError(f"device status {st.item()}")
+        kern = sum(x.elapsed_time(y) for x, y in zip(a[:k], b[:k])) / max(1, k)
+        return t0.elapsed_time(t1) / steps, kern
+
+    clocks = ClockSampler(0)
+    time.sleep(0.3)
+    clocks.mark_start()
+    tile_ms, tile_kern = timed(lambda: Z.zha_prefill_attn(g, Q, K, V, pos, ids, cnt, O2, wp, st),
+                               args.steps, args.warmup)
+    clocks.mark_end()
+    clk = clocks.stop()
+    q_ms, q_kern = timed(lambda: Z.zha_sparse_attn(g, Q, K, V, pos, ids, cnt, O1, wa, st),
+                         max(1, min(args.steps, 3)), 1)
+    diff = (O1.float() - O2.float()).abs()
+    ent = tile_unions(ids.cpu().numpy(), cnt.cpu().numpy(), pos.cpu().numpy(), w.Hkv, w.G)
+    flops_exec = float(ent.sum()) * 4.0 * 128 * 64 * 128          # S and P.V on 128 rows per chunk
+    kept = cnt.cpu().numpy().astype(np.float64)
+    useful = float((kept * 64).sum() + w.B * nq * w.Hq) * 4.0 * 128   # rows x their own keys (approx.)
+    peaks = {"bf16_tflops": 1590.0, "kind": "fallback"}
+    try:
+        mp = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        peaks = {"bf16_tflops": float(mp["bf16_tflops"]), "kind": "measured (burst)"}
+    except (OSError, ValueError, KeyError):
+        pass
+    achieved = flops_exec / (tile_kern * 1e-3) / 1e12
+    qh = w.B * nq * w.Hq
+    line = {
+        "metric": "ZHA prefill attention query-heads/s", "value": qh / (tile_ms * 1e-3), "unit": "query-heads/s",
+        "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": tile_ms, "higher_is_better": True,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {**config_of(w, p), "path": "prefill", "n_new": nq, "tile_queries": 128 // w.G},
+        "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel", "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+                     "peak_kind": peaks["kind"], "flops_per_launch": flops_exec, "kernel_ms": tile_kern,
+                     "useful_flops_fraction": useful / flops_exec},
+        "tiles": {"count": int(len(ent)), "entries_mean": float(ent.mean()), "entries_max": int(ent.max()),
+                  "kv_bytes_per_launch": float(ent.sum()) * 2 * 64 * 128 * 2},
+        "per_query_path": {"ms": q_ms, "kernel_ms": q_kern, "speedup_of_tiles": q_ms / tile_ms},
+        "route_ms": route_ms,
+        "max_abs_diff_vs_per_query_path": float(diff.max().item()),
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.model:
@@ -747,6 +877,9 @@ def main():
         return
     if args.sweep:
         run_sweep(args)
+        return
+    if args.path == "prefill":
+        run_prefill(args)
         return
     w = S.workload(args.workload)
     if args.batch is not None:

@@ -12,13 +12,13 @@ LIB_PATH = os.path.join(HERE, "libzha.so")
 
 ZHA_OK, ZHA_ERR_INVALID_ARG, ZHA_ERR_UNSUPPORTED, ZHA_ERR_CAPACITY, ZHA_ERR_CUDA, ZHA_ERR_DEVICE = range(6)
 ZHA_F32, ZHA_BF16 = 0, 1
-ZHA_OP_ROUTE, ZHA_OP_ATTN, ZHA_OP_DECODE, ZHA_OP_DENSE, ZHA_OP_FLAT = 1, 2, 3, 4, 5
+ZHA_OP_ROUTE, ZHA_OP_ATTN, ZHA_OP_DECODE, ZHA_OP_DENSE, ZHA_OP_FLAT, ZHA_OP_PREFILL = 1, 2, 3, 4, 5, 6
 
 # every symbol include/zha.h declares, in declaration order
 EXPORTS = [
     "zha_status_str", "zha_check_geom", "zha_tree_bytes", "zha_tree_level", "zha_workspace_bytes",
     "zha_leaf_cap", "zha_build_tree", "zha_append", "zha_route", "zha_route_schedule", "zha_route_topk", "zha_sparse_attn",
-    "zha_decode",
+    "zha_prefill_attn", "zha_decode",
     "zha_dense_decode", "zha_flat_index", "zha_sparse_attn_noalloc", "zha_check_bounded_wait", "zha_launch_count",
     "zha_last_error", "zha_trace", "zha_trace_count",
 ]
@@ -59,6 +59,7 @@ _SIGS = {
     "zha_route_schedule": (_I32, [_G, _P, _P, _I32, _P, Buf, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_route_topk": (_I32, [_G, _P, _P, _I32, _P, Buf, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_sparse_attn": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _P, Buf, _P, _P]),
+    "zha_prefill_attn": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_decode": (_I32, [_G, _P, _P, _P, _P, _P, _I64, _P, _F64, Buf, _P, _P, _I32, _P, Buf, _P, _P]),
     "zha_dense_decode": (_I32, [_G, _P, _P, _P, _P, _I32, _P, _P, Buf, _P, _P]),
     "zha_flat_index": (_I32, [_G, _P, _P, _P, _P, _I32, _F64, _P, _P, _I32, _P, Buf, _P, _P]),

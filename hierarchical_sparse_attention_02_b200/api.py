@@ -177,6 +177,13 @@ def zha_sparse_attn(g, Q, K, V, q_pos, leaf_ids, leaf_cnt, O, ws, dev_status, ls
         _ptr(leaf_cnt), leaf_ids.shape[-1], _ptr(O), _ptr(lse), _buf(ws), _ptr(dev_status), _stream(stream)))
 
 
+def zha_prefill_attn(g, Q, K, V, q_pos, leaf_ids, leaf_cnt, O, ws, dev_status, lse=None, stream=None):
+    """zha_sparse_attn for many queries per sequence, one tensor-core tile of queries at a time."""
+    _check("zha_prefill_attn", _lib.load().zha_prefill_attn(
+        ctypes.byref(g.c()), _ptr(Q), _ptr(K), _ptr(V), _ptr(q_pos), Q.shape[1], _ptr(leaf_ids),
+        _ptr(leaf_cnt), leaf_ids.shape[-1], _ptr(O), _ptr(lse), _buf(ws), _ptr(dev_status), _stream(stream)))
+
+
 def zha_sparse_attn_noalloc(g, Q, K, V, q_pos, leaf_ids, leaf_cnt, O, dev_status, lse=None, stream=None):
     """zha_sparse_attn with the library's own fixed device scratch instead of a workspace."""
     _check("zha_sparse_attn_noalloc", _lib.load().zha_sparse_attn_noalloc(

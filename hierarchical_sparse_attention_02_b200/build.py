@@ -13,7 +13,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libzha.so")
-SOURCES = ["zha_api.cu", "zha_tree.cu", "zha_route.cu", "zha_attn.cu", "zha_attn_tc.cu", "zha_noalloc.cu"]
+SOURCES = ["zha_api.cu", "zha_tree.cu", "zha_route.cu", "zha_attn.cu", "zha_attn_tc.cu", "zha_prefill_tc.cu", "zha_noalloc.cu"]
 
 
 def nvcc_path() -> str:

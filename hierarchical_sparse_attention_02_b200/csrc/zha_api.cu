@@ -87,6 +87,7 @@ size_t zha_workspace_bytes(const zha_geom* g, int32_t nq, int32_t op) {
     case ZHA_OP_ROUTE: return route_ws(*g, nq).bytes;
     case ZHA_OP_ATTN:
     case ZHA_OP_DENSE: return attn_ws(*g, nq).bytes;
+    case ZHA_OP_PREFILL: return prefill_ws(*g, nq).bytes;
     case ZHA_OP_DECODE:
     case ZHA_OP_FLAT: {
       const size_t r = route_ws(*g, nq).bytes;
@@ -227,6 +228,22 @@ zha_status zha_decode(const zha_geom* g, const void* q, const void* k_new, const
   AttnCall ac{g, 1, q, K, V, nullptr, T, 0, leaf_ids, leaf_cnt, leaf_cap, O, nullptr,
               (char*)ws.base, dev_status, st};
   return from_cuda(attention(ac));
+}
+
+zha_status zha_prefill_attn(const zha_geom* g, const void* Q, const void* K, const void* V,
+                            const int64_t* q_pos, int32_t nq, const int32_t* leaf_ids,
+                            const int32_t* leaf_cnt, int32_t leaf_cap, void* O, float* lse,
+                            zha_buf ws, int32_t* dev_status, void* stream) {
+  zha_status s = zha_check_geom(g);
+  if (s != ZHA_OK) return s;
+  if (g->dtype != ZHA_BF16) return ZHA_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !q_pos || nq < 1 || !leaf_ids || !leaf_cnt || leaf_cap < 1 || !O ||
+      !ws.base || !dev_status)
+    return ZHA_ERR_INVALID_ARG;
+  if ((s = check_ws(g, nq, ZHA_OP_PREFILL, ws)) != ZHA_OK) return s;
+  PrefillCall c{g, nq, Q, K, V, q_pos, leaf_ids, leaf_cnt, leaf_cap, O, lse, (char*)ws.base, dev_status,
+                (cudaStream_t)stream};
+  return from_cuda(prefill_attention(c));
 }
 
 zha_status zha_check_bounded_wait(int64_t polls, int32_t* dev_status, int64_t* out, void* stream) {

@@ -1,0 +1,572 @@
+// Query-tile sparse attention for chunked prefill on the 5th-generation tensor cores.
+//
+// arXiv 2610.42112, App. A-B (Table I) counts the KV footprint of a tile of Q consecutive
+// queries as the union of the leaf lists of its Q queries x G heads, while every query
+// keeps its own output o(q) = Attn(q, K_I(q), V_I(q)) ("ZHA summary" page, Routing):
+//   I(q) = {0} u (keys of the chunks in S_1(q)) u C_cur(q),   C_cur(q) = [V(t), t].
+// Here a tile is Qt = floor(128 / G) consecutive queries of one sequence and the G query
+// heads of one KV head: M = Qt * G <= 128 rows (row r = query r / G, head r % G), the M of
+// one tcgen05 MMA.  For every 64-key chunk of the tile's union the kernel computes
+//     S[128 x 64]  = Q_tile . K_chunk^T     (tcgen05.mma kind::f16, bf16 in, fp32 in TMEM)
+//     P            = exp2(S * log2(e)/sqrt(d) - m)  per row, masked to the row's own keys
+//     O[128 x 128] += P . V_chunk           (tcgen05.mma, P from shared memory, O in TMEM)
+// with an online softmax per row whose running maximum is raised lazily (O in TMEM is
+// rescaled only when a row's maximum grows by more than 2^8).  A row sees key j of chunk c
+// iff c is in its S_1, or j = 0, or c is its own chunk and j <= t.
+//
+// Roles in one CTA of 192 threads, one tile after another (a persistent grid):
+//   warps 0-3  softmax and epilogue, thread r <-> row r <-> TMEM lane r;
+//   warp 4     producer: TMA loads of the Q tile (4-D map) and of each chunk's K and V
+//              (3-D maps, 128-byte swizzle) into a 3-stage ring; this GPU's memory only,
+//              no multicast;
+//   warp 5     TMEM allocation; lane 0 issues the MMAs and their commits.
+// Every wait is bounded; a wait that gives up reports ZHA_ERR_DEVICE, the CTA stops, waits
+// (bounded) for its copies and MMAs in flight, frees its TMEM and returns.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include "zha_internal.cuh"
+#include "zha_ptx.cuh"
+
+namespace zha {
+
+namespace qt {
+
+using namespace ptx;
+
+constexpr int kRows = 128;                       // MMA M
+constexpr int kStages = 3;                       // K/V ring depth
+constexpr int kBox = 64 * 128;                   // 64 rows x 128 bytes
+constexpr int kKVBytes = 4 * kBox;               // K dims 0-63 | 64-127, V dims 0-63 | 64-127
+constexpr int kQHalf = kRows * 128;              // 128 rows x 64 dims of Q
+constexpr int kPBytes = kRows * 128;             // 128 rows x 64 keys of P (bf16)
+constexpr uint32_t kTmemCols = 256;              // S0 [0,64), S1 [64,128), O [128,256)
+constexpr uint32_t kColO = 128;
+constexpr int kThreads = 192;
+constexpr float kLazy = 8.0f;                    // rescale O when a row max grows by > 2^8
+constexpr uint32_t kIdescS = idesc_bf16(128, 64, 0);   // S = Q . K^T, both K-major
+constexpr uint32_t kIdescPV = idesc_bf16(128, 128, 1); // O += P . V, V MN-major
+
+struct alignas(1024) Smem {
+  unsigned char q[2][kQHalf];                    // two 128B-swizzled boxes [128 rows][64 dims]
+  unsigned char kv[kStages][kKVBytes];
+  unsigned char p[2][kPBytes];                   // [128 rows][64 keys], 128B swizzle
+  uint4 meta_mask[kStages];                      // rows of the tile that selected the chunk
+  int meta_id[kStages];                          // chunk id of each stage
+  unsigned long long full[kStages], empty[kStages];
+  unsigned long long q_full, q_empty;
+  unsigned long long s_full[2], s_free[2], p_full[2], pv_done[2];
+  unsigned long long o_free, drain;
+  uint32_t tmem_base;
+  int abort, zero;
+};
+
+struct Args {
+  int B, nq, Hq, Hkv, G, Qt, nqt;
+  int64_t t_cap, nr, tiles;
+  const int64_t* q_pos;
+  const int* ent_ids;                            // [tiles, nr, kRange]
+  const uint4* ent_mask;                         // [tiles, nr, kRange] 128-bit row masks
+  const int* ent_cnt;                            // [tiles, nr]
+  __nv_bfloat16* O;
+  float* lse;
+  int32_t* dev_status;
+};
+
+struct Tile {
+  int b, hk, q0;
+  int64_t unit;                                  // b * Hkv + hk (K/V map z coordinate)
+};
+
+__device__ __forceinline__ Tile tile_of(const Args& a, int64_t tile) {
+  Tile t;
+  t.unit = tile / a.nqt;                          // tiles of one KV unit are consecutive
+  t.q0 = (int)(tile % a.nqt) * a.Qt;
+  t.b = (int)(t.unit / a.Hkv);
+  t.hk = (int)(t.unit % a.Hkv);
+  return t;
+}
+
+__device__ __forceinline__ int tile_entries(const Args& a, int64_t tile) {
+  int n = 0;
+  for (int64_t r = 0; r < a.nr; ++r) n += a.ent_cnt[tile * a.nr + r];
+  return n;
+}
+
+// The e-th entry of a tile (ranges in order): its slot in the entry arrays.
+struct EntryWalk {
+  int64_t base, r, e, cnt;
+  __device__ void start(const Args& a, int64_t tile) {
+    base = tile * a.nr;
+    r = 0;
+    e = 0;
+    cnt = a.ent_cnt[base];
+    while (cnt == 0 && r + 1 < a.nr) { ++r; cnt = a.ent_cnt[base + r]; }
+  }
+  __device__ int64_t slot() const { return (base + r) * kRange + e; }
+  __device__ void next(const Args& a) {
+    if (++e >= cnt) {
+      e = 0;
+      do { ++r; cnt = r < a.nr ? a.ent_cnt[base + r] : 0; } while (cnt == 0 && r + 1 < a.nr);
+    }
+  }
+};
+
+__device__ __forceinline__ bool warp_wait(unsigned long long* b, uint32_t parity, int* abort) {
+  const bool ok = __all_sync(0xffffffffu, mbar_wait(b, parity, abort));
+  return ok;
+}
+
+__device__ __forceinline__ void give_up(Smem& sm, int32_t* st) {
+  set_status(st, ZHA_ERR_DEVICE);
+  atomicExch(&sm.abort, 1);
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
+                  const __grid_constant__ CUtensorMap vmap, Args a) {
+  extern __shared__ unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sm.s_full[i], 1);
+      mbar_init(&sm.s_free[i], 4);
+      mbar_init(&sm.p_full[i], 4);
+      mbar_init(&sm.pv_done[i], 1);
+    }
+    mbar_init(&sm.o_free, 4);
+    mbar_init(&sm.drain, 1);
+    sm.abort = 0;
+    sm.zero = 0;
+    mbar_init_fence();
+  }
+  if (warp == 5) tmem_alloc(&sm.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      prefetch_tensormap(&qmap);
+      prefetch_tensormap(&kmap);
+      prefetch_tensormap(&vmap);
+      const uint32_t q_tx = (uint32_t)(2 * 128 * a.G * a.Qt);
+      long long it = 0, nq_loads = 0;
+      long long issued[kStages] = {};
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
+        const Tile t = tile_of(a, tile);
+        if (nq_loads > 0 && !mbar_wait(&sm.q_empty, (uint32_t)((nq_loads - 1) & 1), &sm.abort)) {
+          give_up(sm, a.dev_status);
+          break;
+        }
+        mbar_arrive_tx(&sm.q_full, q_tx);
+        tma_load_4d(sm.q[0], &qmap, 0, t.hk * a.G, t.q0, t.b, &sm.q_full);
+        tma_load_4d(sm.q[1], &qmap, 64, t.hk * a.G, t.q0, t.b, &sm.q_full);
+        ++nq_loads;
+        const int n = tile_entries(a, tile);
+        EntryWalk w;
+        w.start(a, tile);
+        for (int i = 0; i < n; ++i, ++it, w.next(a)) {
+          const int s = (int)(it % kStages);
+          if (it >= kStages && !mbar_wait(&sm.empty[s], (uint32_t)(((it / kStages) - 1) & 1), &sm.abort)) {
+            give_up(sm, a.dev_status);
+            ok = false;
+            break;
+          }
+          const int64_t slot = w.slot();
+          const int c = a.ent_ids[slot];
+          sm.meta_id[s] = c;
+          sm.meta_mask[s] = a.ent_mask[slot];
+          mbar_arrive_tx(&sm.full[s], (uint32_t)kKVBytes);
+          unsigned char* st = sm.kv[s];
+          const int z = (int)t.unit;
+          tma_load_3d(st + 0 * kBox, &kmap, 0, c * kLeaf, z, &sm.full[s]);
+          tma_load_3d(st + 1 * kBox, &kmap, 64, c * kLeaf, z, &sm.full[s]);
+          tma_load_3d(st + 2 * kBox, &vmap, 0, c * kLeaf, z, &sm.full[s]);
+          tma_load_3d(st + 3 * kBox, &vmap, 64, c * kLeaf, z, &sm.full[s]);
+          ++issued[s];
+        }
+      }
+      // drain: no copy may land after the CTA exits (bounded, independent of `abort`)
+      for (int s = 0; s < kStages; ++s)
+        if (issued[s] > 0 && !mbar_wait(&sm.full[s], (uint32_t)((issued[s] - 1) & 1), &sm.zero))
+          set_status(a.dev_status, ZHA_ERR_DEVICE);
+      if (nq_loads > 0 && !mbar_wait(&sm.q_full, (uint32_t)((nq_loads - 1) & 1), &sm.zero))
+        set_status(a.dev_status, ZHA_ERR_DEVICE);
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t qa = smem_u32(sm.q[0]);
+      long long j = 0, tl = 0;                   // entries and tiles of this CTA so far
+      bool ok = true;
+      auto issue_pv = [&](long long e, bool first_of_tile) -> bool {
+        if (!mbar_wait(&sm.p_full[e & 1], (uint32_t)((e >> 1) & 1), &sm.abort)) return false;
+        if (first_of_tile && tl > 0 && !mbar_wait(&sm.o_free, (uint32_t)((tl - 1) & 1), &sm.abort)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sm.p[e & 1]);
+        const uint32_t va = smem_u32(sm.kv[e % kStages] + 2 * kBox);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          umma_bf16(tmem + kColO, sw128_desc(pa + kk * 32, 16, 1024), sw128_desc(va + kk * 2048, kBox, 1024),
+                    kIdescPV, (first_of_tile && kk == 0) ? 0u : 1u);
+        umma_commit(&sm.pv_done[e & 1]);
+        umma_commit(&sm.empty[e % kStages]);
+        return true;
+      };
+      for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tl) {
+        const int n = tile_entries(a, tile);
+        if (!mbar_wait(&sm.q_full, (uint32_t)(tl & 1), &sm.abort)) { ok = false; break; }
+        tc_fence_after();
+        for (int i = 0; i < n; ++i, ++j) {
+          const int s = (int)(j % kStages);
+          if (!mbar_wait(&sm.full[s], (uint32_t)((j / kStages) & 1), &sm.abort)) { ok = false; break; }
+          if (j >= 2 && !mbar_wait(&sm.s_free[j & 1], (uint32_t)(((j >> 1) - 1) & 1), &sm.abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ka = smem_u32(sm.kv[s]);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            umma_bf16(tmem + (uint32_t)(j & 1) * 64, sw128_desc(qa + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024),
+                      sw128_desc(ka + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+          umma_commit(&sm.s_full[j & 1]);
+          if (i >= 1 && !issue_pv(j - 1, i == 1)) { ok = false; break; }
+        }
+        if (!ok) break;
+        if (n >= 1 && !issue_pv(j - 1, n == 1)) { ok = false; break; }
+        umma_commit(&sm.q_empty);                  // Q is free once this tile's MMAs are done
+      }
+      if (!ok) give_up(sm, a.dev_status);
+      // drain: every MMA this thread issued has completed before TMEM is freed
+      umma_commit(&sm.drain);
+      if (!mbar_wait(&sm.drain, 0u, &sm.zero)) set_status(a.dev_status, ZHA_ERR_DEVICE);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax + epilogue
+    const int r = threadIdx.x;                   // row = TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
+    long long j = 0, tl = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tl) {
+      const Tile t = tile_of(a, tile);
+      const int n = tile_entries(a, tile);
+      // this row's query
+      const int qi = t.q0 + r / a.G;
+      const int h = t.hk * a.G + r % a.G;
+      bool valid = r < a.Qt * a.G && qi < a.nq;
+      int64_t pos = 0;
+      if (valid) {
+        pos = a.q_pos[(int64_t)t.b * a.nq + qi];
+        if (pos < 0 || pos >= a.t_cap) valid = false;   // reported by the union kernel
+      }
+      const int64_t cur = valid ? pos / kLeaf : -1;    // the row's own chunk = n_vis(t)
+      const uint32_t mword = (uint32_t)(r >> 5), mbit = 1u << (r & 31);
+      float m = -INFINITY, l = 0.f;
+      for (int i = 0; i < n; ++i, ++j) {
+        const int s = (int)(j % kStages);
+        if (!warp_wait(&sm.full[s], (uint32_t)((j / kStages) & 1), &sm.abort)) { ok = false; break; }
+        const int c = sm.meta_id[s];
+        const uint4 mk = sm.meta_mask[s];
+        if (!warp_wait(&sm.s_full[j & 1], (uint32_t)((j >> 1) & 1), &sm.abort)) { ok = false; break; }
+        tc_fence_after();
+        float x[64];
+        {
+          float v[32];
+          tmem_ld32(lane_addr + (uint32_t)(j & 1) * 64, v);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) x[k] = v[k];
+          tmem_ld32(lane_addr + (uint32_t)(j & 1) * 64 + 32, v);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) x[32 + k] = v[k];
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.s_free[j & 1]);
+        // visibility of the chunk's keys for this row
+        const uint32_t wsel = mword == 0 ? mk.x : mword == 1 ? mk.y : mword == 2 ? mk.z : mk.w;
+        const bool sel = valid && (wsel & mbit) && c < cur;
+        const bool own = valid && c == cur;
+        const int lim = own ? (int)(pos - (int64_t)c * kLeaf) : (sel ? 63 : -1);   // keys 0..lim
+        const bool sink = valid && c == 0;                                           // key 0
+        float mx = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          const bool vis = (sel || k <= lim) || (sink && k == 0);
+          x[k] = vis ? x[k] * sl2 : -INFINITY;
+          mx = fmaxf(mx, x[k]);
+        }
+        // lazy rescale: only when the row maximum grows by more than 2^kLazy (warp-wide)
+        const bool grow = m != -INFINITY && mx > m + kLazy;
+        if (__any_sync(0xffffffffu, grow)) {
+          if (i >= 1 && !warp_wait(&sm.pv_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float alpha = grow ? exp2f(m - mx) : 1.f;
+#pragma unroll 1
+          for (int cc = 0; cc < 4; ++cc) {
+            float v[32];
+            tmem_ld32(lane_addr + kColO + cc * 32, v);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) v[k] *= alpha;
+            tmem_st32(lane_addr + kColO + cc * 32, v);
+          }
+          tmem_wait_st();
+          if (grow) { l *= alpha; m = mx; }
+        }
+        if (m == -INFINITY) m = mx;                // first visible key of the row (O is zero)
+        const float mu = m == -INFINITY ? 0.f : m;
+        // P buffer j & 1 is free once PV of entry j - 2 has completed
+        if (j >= 2 && !warp_wait(&sm.pv_done[j & 1], (uint32_t)(((j - 2) >> 1) & 1), &sm.abort)) { ok = false; break; }
+        unsigned char* prow = sm.p[j & 1] + r * 128;
+        float psum = 0.f;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const float p0 = exp2f(x[ch * 8 + 2 * u] - mu), p1 = exp2f(x[ch * 8 + 2 * u + 1] - mu);
+            w4[u] = pack_bf16(p0, p1);
+            psum += p0 + p1;                       // the log-sum-exp from the unrounded weights
+          }
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        l += psum;
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[j & 1]);
+      }
+      if (!ok) break;
+      // epilogue: O / l of each valid row
+      if (n >= 1 && !warp_wait(&sm.pv_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) { ok = false; break; }
+      tc_fence_after();
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = a.O + (((int64_t)t.b * a.nq + qi) * a.Hq + h) * kD;
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        float v[32];
+        if (n >= 1) {
+          tmem_ld32(lane_addr + kColO + cc * 32, v);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) v[k] = 0.f;
+        }
+        if (valid) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            uint4 o4;
+            o4.x = pack_bf16(v[u * 8 + 0] * inv, v[u * 8 + 1] * inv);
+            o4.y = pack_bf16(v[u * 8 + 2] * inv, v[u * 8 + 3] * inv);
+            o4.z = pack_bf16(v[u * 8 + 4] * inv, v[u * 8 + 5] * inv);
+            o4.w = pack_bf16(v[u * 8 + 6] * inv, v[u * 8 + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + cc * 32 + u * 8) = o4;
+          }
+        }
+      }
+      if (valid && a.lse) a.lse[((int64_t)t.b * a.nq + qi) * a.Hq + h] =
+          l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.o_free);
+    }
+    if (!ok) give_up(sm, a.dev_status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) {
+    __syncwarp();
+    tmem_free(tmem, kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// union of a tile's leaf lists, one CTA per (tile, range of kRange chunk ids):
+// every chunk some row selected (with the 128-bit mask of those rows), chunk 0 (the first
+// key) and each row's own chunk, in ascending id order
+// ---------------------------------------------------------------------------
+
+struct UnionArgs {
+  int B, nq, Hq, Hkv, G, Qt, nqt;
+  int64_t t_cap, nr;
+  const int64_t* q_pos;
+  const int* leaf_ids;
+  const int* leaf_cnt;
+  int leaf_cap;
+  int* ent_ids;
+  uint4* ent_mask;
+  int* ent_cnt;
+  int32_t* dev_status;
+};
+
+__global__ void __launch_bounds__(256) prefill_union_kernel(UnionArgs a) {
+  __shared__ uint32_t mask[4][kRange];
+  __shared__ uint32_t present[kRange / 32];
+  __shared__ unsigned int wtot[8];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t tile = blockIdx.x / a.nr, rg = blockIdx.x % a.nr;
+  const int64_t unit = tile / a.nqt;
+  const int q0 = (int)(tile % a.nqt) * a.Qt;
+  const int b = (int)(unit / a.Hkv), hk = (int)(unit % a.Hkv);
+  const int64_t lo = rg * kRange, hi = lo + kRange;
+  const int rows = a.Qt * a.G;
+  for (int i = tid; i < kRange; i += 256) mask[0][i] = mask[1][i] = mask[2][i] = mask[3][i] = 0u;
+  if (tid < kRange / 32) present[tid] = 0u;
+  __syncthreads();
+  // chunk 0 and each valid row's own chunk
+  for (int r = tid; r < rows; r += 256) {
+    const int qi = q0 + r / a.G;
+    if (qi >= a.nq) continue;
+    const int64_t t = a.q_pos[(int64_t)b * a.nq + qi];
+    if (t < 0 || t >= a.t_cap) {
+      if (rg == 0) set_status(a.dev_status, ZHA_ERR_INVALID_ARG);
+      continue;
+    }
+    const int64_t cur = t / kLeaf;
+    if (cur >= lo && cur < hi) atomicOr(&present[(cur - lo) >> 5], 1u << ((cur - lo) & 31));
+    if (lo == 0) atomicOr(&present[0], 1u);
+  }
+  // selected chunks: warp w takes rows w, w + 8, ...
+  for (int r = warp; r < rows; r += 8) {
+    const int qi = q0 + r / a.G;
+    if (qi >= a.nq) continue;
+    const int64_t t = a.q_pos[(int64_t)b * a.nq + qi];
+    if (t < 0 || t >= a.t_cap) continue;
+    const int64_t nvis = t / kLeaf;
+    const int64_t qh = ((int64_t)b * a.nq + qi) * a.Hq + hk * a.G + r % a.G;
+    const int* lst = a.leaf_ids + qh * a.leaf_cap;
+    int cnt = a.leaf_cnt[qh];
+    cnt = cnt < 0 ? 0 : (cnt > a.leaf_cap ? a.leaf_cap : cnt);
+    const int x0 = warp_lower_bound(lst, cnt, lo);
+    const int x1 = warp_lower_bound(lst, cnt, hi);
+    for (int x = x0 + lane; x < x1; x += 32) {
+      const int id = lst[x];
+      // ids outside [lo, hi) mean an unsorted list; beyond n_vis an invisible chunk
+      if (id < lo || id >= hi || id >= nvis) { set_status(a.dev_status, ZHA_ERR_INVALID_ARG); continue; }
+      atomicOr(&mask[r >> 5][id - lo], 1u << (r & 31));
+    }
+  }
+  __syncthreads();
+  // ordered compaction: thread tid owns ids [4 tid, 4 tid + 4)
+  constexpr int kPer = kRange / 256;
+  unsigned int cntl = 0;
+  bool on[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int i = tid * kPer + q;
+    on[q] = ((present[i >> 5] >> (i & 31)) & 1u) || (mask[0][i] | mask[1][i] | mask[2][i] | mask[3][i]);
+    cntl += on[q];
+  }
+  unsigned int x = cntl;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wtot[warp] = x;
+  __syncthreads();
+  unsigned int before = 0, total = 0;
+  for (int w = 0; w < 8; ++w) { if (w < warp) before += wtot[w]; total += wtot[w]; }
+  before += x - cntl;
+  const int64_t base = blockIdx.x * (int64_t)kRange;
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    if (!on[q]) continue;
+    const int i = tid * kPer + q;
+    a.ent_ids[base + before] = (int)(lo + i);
+    a.ent_mask[base + before] = make_uint4(mask[0][i], mask[1][i], mask[2][i], mask[3][i]);
+    ++before;
+  }
+  if (tid == 0) a.ent_cnt[blockIdx.x] = (int)total;
+}
+
+}  // namespace qt
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn();
+
+// Q [B, nq, Hq, 128] bf16 as a 4-D map with boxes of 64 dims x G heads x Qt queries x 1.
+static bool make_q_map(CUtensorMap* map, const void* Q, int B, int nq, int Hq, int G, int Qt) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)Hq, (cuuint64_t)nq, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)kD * 2, (cuuint64_t)Hq * kD * 2, (cuuint64_t)nq * Hq * kD * 2};
+  const cuuint32_t box[4] = {64, (cuuint32_t)G, (cuuint32_t)Qt, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(Q), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+PrefillWs prefill_ws(const zha_geom& g, int nq, size_t base) {
+  PrefillWs w{};
+  const int G = g.Hq / g.Hkv;
+  w.Qt = kPrefillRows / G;
+  w.nqt = (nq + w.Qt - 1) / w.Qt;
+  w.tiles = (int64_t)g.B * g.Hkv * w.nqt;
+  w.nr = (ncap_of(g, 1) + 1 + kRange - 1) / kRange;
+  const size_t slots = (size_t)w.tiles * w.nr * kRange;
+  size_t off = base;
+  w.ent_ids = off;  off = align_up(off + slots * 4);
+  w.ent_mask = off; off = align_up(off + slots * 16);
+  w.ent_cnt = off;  off = align_up(off + (size_t)w.tiles * w.nr * 4);
+  w.bytes = off;
+  return w;
+}
+
+cudaError_t prefill_attention(const PrefillCall& c) {
+  const zha_geom& g = *c.g;
+  const PrefillWs w = prefill_ws(g, c.nq, 0);
+  const int G = g.Hq / g.Hkv;
+  qt::UnionArgs ua{};
+  ua.B = g.B; ua.nq = c.nq; ua.Hq = g.Hq; ua.Hkv = g.Hkv; ua.G = G; ua.Qt = w.Qt; ua.nqt = (int)w.nqt;
+  ua.t_cap = g.t_cap; ua.nr = w.nr; ua.q_pos = c.q_pos;
+  ua.leaf_ids = c.leaf_ids; ua.leaf_cnt = c.leaf_cnt; ua.leaf_cap = c.leaf_cap;
+  ua.ent_ids = (int*)(c.ws + w.ent_ids);
+  ua.ent_mask = (uint4*)(c.ws + w.ent_mask);
+  ua.ent_cnt = (int*)(c.ws + w.ent_cnt);
+  ua.dev_status = c.dev_status;
+  qt::prefill_union_kernel<<<(unsigned)(w.tiles * w.nr), 256, 0, c.stream>>>(ua);
+  count_launch();
+  cudaError_t e = launch_status("prefill_union_kernel");
+  if (e != cudaSuccess) return e;
+
+  CUtensorMap qm, km, vm;
+  const int64_t units_kv = (int64_t)g.B * g.Hkv;
+  if (!make_q_map(&qm, c.Q, g.B, c.nq, g.Hq, G, w.Qt) || !make_kv_map(&km, c.K, units_kv, g.t_cap) ||
+      !make_kv_map(&vm, c.V, units_kv, g.t_cap)) {
+    note_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled");
+    return cudaErrorInvalidValue;
+  }
+  qt::Args a{};
+  a.B = g.B; a.nq = c.nq; a.Hq = g.Hq; a.Hkv = g.Hkv; a.G = G; a.Qt = w.Qt; a.nqt = (int)w.nqt;
+  a.t_cap = g.t_cap; a.nr = w.nr; a.tiles = w.tiles; a.q_pos = c.q_pos;
+  a.ent_ids = ua.ent_ids; a.ent_mask = ua.ent_mask; a.ent_cnt = ua.ent_cnt;
+  a.O = (__nv_bfloat16*)c.O; a.lse = c.lse; a.dev_status = c.dev_status;
+  const size_t smem = sizeof(qt::Smem) + 1024;
+  cudaFuncSetAttribute(qt::prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const int64_t grid = w.tiles < sm_count() ? w.tiles : sm_count();
+  trace_begin(ZHA_TRACE_ATTN, c.stream);
+  qt::prefill_tc_kernel<<<(unsigned)grid, qt::kThreads, smem, c.stream>>>(qm, km, vm, a);
+  trace_end(ZHA_TRACE_ATTN, c.stream);
+  count_launch();
+  return launch_status("prefill_tc_kernel");
+}
+
+}  // namespace zha

@@ -66,7 +66,8 @@ typedef enum zha_op {
   ZHA_OP_ATTN = 2,    /* zha_sparse_attn                            */
   ZHA_OP_DECODE = 3,  /* zha_decode (route + attention, nq = 1)     */
   ZHA_OP_DENSE = 4,   /* zha_dense_decode                           */
-  ZHA_OP_FLAT = 5     /* zha_flat_index (scores + select + attention) */
+  ZHA_OP_FLAT = 5,    /* zha_flat_index (scores + select + attention) */
+  ZHA_OP_PREFILL = 6  /* zha_prefill_attn (query tiles)             */
 } zha_op;
 
 /* Geometry of one attention layer and its tree (host struct).
@@ -230,6 +231,27 @@ zha_status zha_sparse_attn(const zha_geom* g, const void* Q, const void* K, cons
                            const int64_t* q_pos, int32_t nq, const int32_t* leaf_ids,
                            const int32_t* leaf_cnt, int32_t leaf_cap, void* O, float* lse,
                            zha_buf ws, int32_t* dev_status, void* stream);
+
+/*
+ * zha_prefill_attn - zha_sparse_attn for many queries per sequence (chunked prefill),
+ * computed per query tile on the 5th-generation tensor cores.
+ * Outputs are those of zha_sparse_attn: every query attends over its own index set
+ * I(q) = {0} u (keys of the chunks in S_1(q)) u C_cur(q) ("ZHA summary" page, Routing).
+ * arXiv 2610.42112, App. A-B (Table I) counts a tile of Q consecutive queries by the union
+ * of the leaf lists of its Q queries x G heads; here a tile holds Qt = floor(128 / G)
+ * consecutive queries of one sequence and the G heads of one KV head (Qt * G <= 128 rows
+ * of one tcgen05 MMA), the tile's union is gathered once, and each row is masked to its
+ * own chunks, the first key and its causal limit inside its own chunk.
+ *   bf16 caches only (ZHA_ERR_UNSUPPORTED for fp32).
+ *   Q, O [B, nq, Hq, d]; q_pos [B, nq] (required); leaf_ids / leaf_cnt as zha_route wrote them.
+ *   lse  nullable [B, nq, Hq] fp32 (natural log).
+ *   ws   at least zha_workspace_bytes(g, nq, ZHA_OP_PREFILL) bytes.
+ * Softmax in fp32 (base 2, P rounded to bf16 for the second product), accumulation in fp32.
+ */
+zha_status zha_prefill_attn(const zha_geom* g, const void* Q, const void* K, const void* V,
+                            const int64_t* q_pos, int32_t nq, const int32_t* leaf_ids,
+                            const int32_t* leaf_cnt, int32_t leaf_cap, void* O, float* lse,
+                            zha_buf ws, int32_t* dev_status, void* stream);
 
 /*
  * zha_decode - one decode step for every sequence: append the new token at position T
