@@ -142,9 +142,10 @@ inline AttnWs attn_ws(const zha_geom& g, int nq, size_t base = 0, int64_t cps = 
   return w;
 }
 
-// Query-tile attention for prefill (zha_prefill_attn): tiles of Qt = kPrefillRows / G
-// consecutive queries x the G heads of one KV head; per (tile, range of kRange chunk ids)
-// the union entries (chunk id, 128-bit mask of the rows that selected it) and a count.
+// Query-tile attention for prefill (zha_prefill_attn): sub-tiles of Qt = kPrefillRows / G
+// consecutive queries x the G heads of one KV head, two per tile; per (tile, range of
+// kRange chunk ids) the union entries (chunk id, a 128-bit mask per sub-tile of the rows
+// that selected it) and a count.
 constexpr int kPrefillRows = 128;
 
 struct PrefillWs {

@@ -20,7 +20,8 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[ZHA_NOALLOC_SCR
 
 // Device address of the scratch array, resolved once per device.  In host code the
 // array's name is only a host-side stand-in for the symbol, so the address must come from
-// cudaGetSymbolAddress with that device current.
+// cudaGetSymbolAddress with that device current.  The address is kept per device index
+// for the life of the process: after a cudaDeviceReset the library must be reloaded.
 constexpr int kMaxDevices = 64;
 static void* g_scratch_ptr[kMaxDevices] = {};
 static std::mutex g_scratch_mu;
@@ -34,7 +35,10 @@ static cudaError_t scratch_on_current_device(void** out) {
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
+    if (e != cudaSuccess) {
+      cudaGetLastError();          // clear it, so that the next launch check reports its own error
+      return e;
+    }
     g_scratch_ptr[dev] = p;
   }
   *out = g_scratch_ptr[dev];

@@ -4,9 +4,12 @@
 // queries as the union of the leaf lists of its Q queries x G heads, while every query
 // keeps its own output o(q) = Attn(q, K_I(q), V_I(q)) ("ZHA summary" page, Routing):
 //   I(q) = {0} u (keys of the chunks in S_1(q)) u C_cur(q),   C_cur(q) = [V(t), t].
-// Here a tile is Qt = floor(128 / G) consecutive queries of one sequence and the G query
-// heads of one KV head: M = Qt * G <= 128 rows (row r = query r / G, head r % G), the M of
-// one tcgen05 MMA.  For every 64-key chunk of the tile's union the kernel computes
+// Here a sub-tile is Qt = floor(128 / G) consecutive queries of one sequence and the G
+// query heads of one KV head: M = Qt * G <= 128 rows (row r = query r / G, head r % G), the
+// M of one tcgen05 MMA.  A CTA takes two consecutive sub-tiles at a time (a tile of 2 Qt
+// queries): both share every K / V chunk load and run their softmax on separate warps, so
+// the MMAs of one overlap the softmax of the other.  For every 64-key chunk of the tile's
+// union the kernel computes, for each sub-tile,
 //     S[128 x 64]  = Q_tile . K_chunk^T     (tcgen05.mma kind::f16, bf16 in, fp32 in TMEM)
 //     P            = exp2(S * log2(e)/sqrt(d) - m)  per row, masked to the row's own keys
 //     O[128 x 128] += P . V_chunk           (tcgen05.mma, P from shared memory, O in TMEM)
@@ -14,12 +17,13 @@
 // rescaled only when a row's maximum grows by more than 2^8).  A row sees key j of chunk c
 // iff c is in its S_1, or j = 0, or c is its own chunk and j <= t.
 //
-// Roles in one CTA of 192 threads, one tile after another (a persistent grid):
-//   warps 0-3  softmax and epilogue, thread r <-> row r <-> TMEM lane r;
-//   warp 4     producer: TMA loads of the Q tile (4-D map) and of each chunk's K and V
+// Roles in one CTA of 320 threads, one tile after another (a persistent grid):
+//   warps 0-3, 4-7  softmax and epilogue of sub-tile 0, 1: thread r <-> row r <-> TMEM lane r
+//              (sub-tile u owns TMEM columns [256 u, 256 u + 256));
+//   warp 8     producer: TMA loads of the Q sub-tiles (4-D map) and of each chunk's K and V
 //              (3-D maps, 128-byte swizzle) into a 3-stage ring; this GPU's memory only,
 //              no multicast;
-//   warp 5     TMEM allocation; lane 0 issues the MMAs and their commits.
+//   warp 9     TMEM allocation; lane 0 issues the MMAs and their commits.
 // Every wait is bounded; a wait that gives up reports ZHA_ERR_DEVICE, the CTA stops, waits
 // (bounded) for its copies and MMAs in flight, frees its TMEM and returns.
 #include <cuda.h>
@@ -34,39 +38,44 @@ namespace qt {
 
 using namespace ptx;
 
-constexpr int kRows = 128;                       // MMA M
+constexpr int kRows = 128;                       // MMA M: rows of a sub-tile
+constexpr int kSub = 2;                          // sub-tiles per tile
 constexpr int kStages = 3;                       // K/V ring depth
 constexpr int kBox = 64 * 128;                   // 64 rows x 128 bytes
 constexpr int kKVBytes = 4 * kBox;               // K dims 0-63 | 64-127, V dims 0-63 | 64-127
 constexpr int kQHalf = kRows * 128;              // 128 rows x 64 dims of Q
 constexpr int kPBytes = kRows * 128;             // 128 rows x 64 keys of P (bf16)
-constexpr uint32_t kTmemCols = 256;              // S0 [0,64), S1 [64,128), O [128,256)
+constexpr uint32_t kTmemCols = 512;              // per sub-tile: S0, S1 (64 each), O (128)
+constexpr uint32_t kSubCols = 256;
 constexpr uint32_t kColO = 128;
-constexpr int kThreads = 192;
+constexpr int kSoftWarps = 4 * kSub;
+constexpr int kProducerWarp = kSoftWarps, kMmaWarp = kSoftWarps + 1;
+constexpr int kThreads = (kSoftWarps + 2) * 32;
 constexpr float kLazy = 8.0f;                    // rescale O when a row max grows by > 2^8
 constexpr uint32_t kIdescS = idesc_bf16(128, 64, 0);   // S = Q . K^T, both K-major
 constexpr uint32_t kIdescPV = idesc_bf16(128, 128, 1); // O += P . V, V MN-major
 
 struct alignas(1024) Smem {
-  unsigned char q[2][kQHalf];                    // two 128B-swizzled boxes [128 rows][64 dims]
+  unsigned char q[kSub][2][kQHalf];              // per sub-tile two 128B-swizzled boxes [128 rows][64 dims]
   unsigned char kv[kStages][kKVBytes];
-  unsigned char p[2][kPBytes];                   // [128 rows][64 keys], 128B swizzle
-  uint4 meta_mask[kStages];                      // rows of the tile that selected the chunk
+  unsigned char p[kSub][2][kPBytes];             // [128 rows][64 keys], 128B swizzle
+  uint4 meta_mask[kStages][kSub];                // rows of each sub-tile that selected the chunk
   int meta_id[kStages];                          // chunk id of each stage
   unsigned long long full[kStages], empty[kStages];
   unsigned long long q_full, q_empty;
-  unsigned long long s_full[2], s_free[2], p_full[2], pv_done[2];
-  unsigned long long o_free, drain;
+  unsigned long long s_full[kSub][2], s_free[kSub][2], p_full[kSub][2], pv_done[kSub][2];
+  unsigned long long o_free[kSub], drain;
   uint32_t tmem_base;
   int abort, zero;
 };
+static_assert(sizeof(Smem) + 1024 <= 232448, "shared memory of the prefill kernel");
 
 struct Args {
-  int B, nq, Hq, Hkv, G, Qt, nqt;
+  int B, nq, Hq, Hkv, G, Qt, nqt;                // nqt: tiles of 2 Qt queries per KV unit
   int64_t t_cap, nr, tiles;
   const int64_t* q_pos;
   const int* ent_ids;                            // [tiles, nr, kRange]
-  const uint4* ent_mask;                         // [tiles, nr, kRange] 128-bit row masks
+  const uint4* ent_mask;                         // [tiles, nr, kRange, kSub] 128-bit row masks
   const int* ent_cnt;                            // [tiles, nr]
   __nv_bfloat16* O;
   float* lse;
@@ -81,7 +90,7 @@ struct Tile {
 __device__ __forceinline__ Tile tile_of(const Args& a, int64_t tile) {
   Tile t;
   t.unit = tile / a.nqt;                          // tiles of one KV unit are consecutive
-  t.q0 = (int)(tile % a.nqt) * a.Qt;
+  t.q0 = (int)(tile % a.nqt) * kSub * a.Qt;
   t.b = (int)(t.unit / a.Hkv);
   t.hk = (int)(t.unit % a.Hkv);
   return t;
@@ -122,6 +131,13 @@ __device__ __forceinline__ void give_up(Smem& sm, int32_t* st) {
   atomicExch(&sm.abort, 1);
 }
 
+// 2^x on the SFU (approximate, flushes subnormal results to zero; 2^-inf = 0).
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constant__ CUtensorMap kmap,
                   const __grid_constant__ CUtensorMap vmap, Args a) {
@@ -133,31 +149,33 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     for (int s = 0; s < kStages; ++s) { mbar_init(&sm.full[s], 1); mbar_init(&sm.empty[s], 1); }
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_empty, 1);
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.s_full[i], 1);
-      mbar_init(&sm.s_free[i], 4);
-      mbar_init(&sm.p_full[i], 4);
-      mbar_init(&sm.pv_done[i], 1);
+    for (int u = 0; u < kSub; ++u) {
+      for (int i = 0; i < 2; ++i) {
+        mbar_init(&sm.s_full[u][i], 1);
+        mbar_init(&sm.s_free[u][i], 4);
+        mbar_init(&sm.p_full[u][i], 4);
+        mbar_init(&sm.pv_done[u][i], 1);
+      }
+      mbar_init(&sm.o_free[u], 4);
     }
-    mbar_init(&sm.o_free, 4);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     sm.zero = 0;
     mbar_init_fence();
   }
-  if (warp == 5) tmem_alloc(&sm.tmem_base, kTmemCols);
+  if (warp == kMmaWarp) tmem_alloc(&sm.tmem_base, kTmemCols);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
-      const uint32_t q_tx = (uint32_t)(2 * 128 * a.G * a.Qt);
+      const uint32_t q_tx = (uint32_t)(kSub * 2 * 128 * a.G * a.Qt);
       long long it = 0, nq_loads = 0;
       long long issued[kStages] = {};
       bool ok = true;
@@ -168,8 +186,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           break;
         }
         mbar_arrive_tx(&sm.q_full, q_tx);
-        tma_load_4d(sm.q[0], &qmap, 0, t.hk * a.G, t.q0, t.b, &sm.q_full);
-        tma_load_4d(sm.q[1], &qmap, 64, t.hk * a.G, t.q0, t.b, &sm.q_full);
+        for (int u = 0; u < kSub; ++u) {           // a sub-tile past nq reads the fill value (0)
+          tma_load_4d(sm.q[u][0], &qmap, 0, t.hk * a.G, t.q0 + u * a.Qt, t.b, &sm.q_full);
+          tma_load_4d(sm.q[u][1], &qmap, 64, t.hk * a.G, t.q0 + u * a.Qt, t.b, &sm.q_full);
+        }
         ++nq_loads;
         const int n = tile_entries(a, tile);
         EntryWalk w;
@@ -184,7 +204,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           const int64_t slot = w.slot();
           const int c = a.ent_ids[slot];
           sm.meta_id[s] = c;
-          sm.meta_mask[s] = a.ent_mask[slot];
+#pragma unroll
+          for (int u = 0; u < kSub; ++u) sm.meta_mask[s][u] = a.ent_mask[slot * kSub + u];
           mbar_arrive_tx(&sm.full[s], (uint32_t)kKVBytes);
           unsigned char* st = sm.kv[s];
           const int z = (int)t.unit;
@@ -202,24 +223,35 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (nq_loads > 0 && !mbar_wait(&sm.q_full, (uint32_t)((nq_loads - 1) & 1), &sm.zero))
         set_status(a.dev_status, ZHA_ERR_DEVICE);
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      const uint32_t qa = smem_u32(sm.q[0]);
       long long j = 0, tl = 0;                   // entries and tiles of this CTA so far
       bool ok = true;
-      auto issue_pv = [&](long long e, bool first_of_tile) -> bool {
-        if (!mbar_wait(&sm.p_full[e & 1], (uint32_t)((e >> 1) & 1), &sm.abort)) return false;
-        if (first_of_tile && tl > 0 && !mbar_wait(&sm.o_free, (uint32_t)((tl - 1) & 1), &sm.abort)) return false;
+      auto issue_s = [&](int u, long long e) -> bool {
+        if (e >= 2 && !mbar_wait(&sm.s_free[u][e & 1], (uint32_t)(((e >> 1) - 1) & 1), &sm.abort)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sm.p[e & 1]);
+        const uint32_t qa = smem_u32(sm.q[u][0]);
+        const uint32_t ka = smem_u32(sm.kv[e % kStages]);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_bf16(tmem + u * kSubCols + (uint32_t)(e & 1) * 64,
+                    sw128_desc(qa + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024),
+                    sw128_desc(ka + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        umma_commit(&sm.s_full[u][e & 1]);
+        return true;
+      };
+      auto issue_pv = [&](int u, long long e, bool first_of_tile) -> bool {
+        if (!mbar_wait(&sm.p_full[u][e & 1], (uint32_t)((e >> 1) & 1), &sm.abort)) return false;
+        if (first_of_tile && tl > 0 && !mbar_wait(&sm.o_free[u], (uint32_t)((tl - 1) & 1), &sm.abort)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sm.p[u][e & 1]);
         const uint32_t va = smem_u32(sm.kv[e % kStages] + 2 * kBox);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tmem + kColO, sw128_desc(pa + kk * 32, 16, 1024), sw128_desc(va + kk * 2048, kBox, 1024),
-                    kIdescPV, (first_of_tile && kk == 0) ? 0u : 1u);
-        umma_commit(&sm.pv_done[e & 1]);
-        umma_commit(&sm.empty[e % kStages]);
+          umma_bf16(tmem + u * kSubCols + kColO, sw128_desc(pa + kk * 32, 16, 1024),
+                    sw128_desc(va + kk * 2048, kBox, 1024), kIdescPV, (first_of_tile && kk == 0) ? 0u : 1u);
+        umma_commit(&sm.pv_done[u][e & 1]);
         return true;
       };
       for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tl) {
@@ -229,18 +261,17 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         for (int i = 0; i < n; ++i, ++j) {
           const int s = (int)(j % kStages);
           if (!mbar_wait(&sm.full[s], (uint32_t)((j / kStages) & 1), &sm.abort)) { ok = false; break; }
-          if (j >= 2 && !mbar_wait(&sm.s_free[j & 1], (uint32_t)(((j >> 1) - 1) & 1), &sm.abort)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t ka = smem_u32(sm.kv[s]);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            umma_bf16(tmem + (uint32_t)(j & 1) * 64, sw128_desc(qa + (kk >> 2) * kQHalf + (kk & 3) * 32, 16, 1024),
-                      sw128_desc(ka + (kk >> 2) * kBox + (kk & 3) * 32, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
-          umma_commit(&sm.s_full[j & 1]);
-          if (i >= 1 && !issue_pv(j - 1, i == 1)) { ok = false; break; }
+          if (!issue_s(0, j) || !issue_s(1, j)) { ok = false; break; }
+          if (i >= 1) {
+            if (!issue_pv(0, j - 1, i == 1) || !issue_pv(1, j - 1, i == 1)) { ok = false; break; }
+            umma_commit(&sm.empty[(j - 1) % kStages]);
+          }
         }
         if (!ok) break;
-        if (n >= 1 && !issue_pv(j - 1, n == 1)) { ok = false; break; }
+        if (n >= 1) {
+          if (!issue_pv(0, j - 1, n == 1) || !issue_pv(1, j - 1, n == 1)) { ok = false; break; }
+          umma_commit(&sm.empty[(j - 1) % kStages]);
+        }
         umma_commit(&sm.q_empty);                  // Q is free once this tile's MMAs are done
       }
       if (!ok) give_up(sm, a.dev_status);
@@ -250,8 +281,9 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int r = threadIdx.x;                   // row = TMEM lane
-    const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+    const int u = warp >> 2;                     // sub-tile of this warpgroup
+    const int r = threadIdx.x & 127;             // row = TMEM lane
+    const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + u * kSubCols;
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
     long long j = 0, tl = 0;
     bool ok = true;
@@ -259,7 +291,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       const Tile t = tile_of(a, tile);
       const int n = tile_entries(a, tile);
       // this row's query
-      const int qi = t.q0 + r / a.G;
+      const int qi = t.q0 + u * a.Qt + r / a.G;
       const int h = t.hk * a.G + r % a.G;
       bool valid = r < a.Qt * a.G && qi < a.nq;
       int64_t pos = 0;
@@ -274,8 +306,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const int s = (int)(j % kStages);
         if (!warp_wait(&sm.full[s], (uint32_t)((j / kStages) & 1), &sm.abort)) { ok = false; break; }
         const int c = sm.meta_id[s];
-        const uint4 mk = sm.meta_mask[s];
-        if (!warp_wait(&sm.s_full[j & 1], (uint32_t)((j >> 1) & 1), &sm.abort)) { ok = false; break; }
+        const uint4 mk = sm.meta_mask[s][u];
+        if (!warp_wait(&sm.s_full[u][j & 1], (uint32_t)((j >> 1) & 1), &sm.abort)) { ok = false; break; }
         tc_fence_after();
         float x[64];
         {
@@ -290,29 +322,35 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_free[j & 1]);
-        // visibility of the chunk's keys for this row
+        if (lane == 0) mbar_arrive(&sm.s_free[u][j & 1]);
+        // visibility of the chunk's keys for this row: all of them (a selected chunk), the
+        // keys up to t (its own chunk), key 0 (chunk 0), or none
         const uint32_t wsel = mword == 0 ? mk.x : mword == 1 ? mk.y : mword == 2 ? mk.z : mk.w;
         const bool sel = valid && (wsel & mbit) && c < cur;
         const bool own = valid && c == cur;
-        const int lim = own ? (int)(pos - (int64_t)c * kLeaf) : (sel ? 63 : -1);   // keys 0..lim
-        const bool sink = valid && c == 0;                                           // key 0
-        float mx = -INFINITY;
+        const int lim = sel ? 63 : (own ? (int)(pos - (int64_t)c * kLeaf) : (valid && c == 0 ? 0 : -1));
+        float mx;
+        {
+          float m8[8];                             // eight independent max chains
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
-          const bool vis = (sel || k <= lim) || (sink && k == 0);
-          x[k] = vis ? x[k] * sl2 : -INFINITY;
-          mx = fmaxf(mx, x[k]);
+          for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
+#pragma unroll
+          for (int k = 0; k < 64; ++k) {
+            x[k] = k <= lim ? x[k] : -INFINITY;
+            m8[k & 7] = fmaxf(m8[k & 7], x[k]);
+          }
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          mx *= sl2;                               // the row maximum in log2 units (-inf stays)
         }
         // lazy rescale: only when the row maximum grows by more than 2^kLazy (warp-wide)
         const bool grow = m != -INFINITY && mx > m + kLazy;
         if (__any_sync(0xffffffffu, grow)) {
-          if (i >= 1 && !warp_wait(&sm.pv_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
+          if (i >= 1 && !warp_wait(&sm.pv_done[u][(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const float alpha = grow ? exp2f(m - mx) : 1.f;
+          const float alpha = grow ? ex2(m - mx) : 1.f;
 #pragma unroll 1
           for (int cc = 0; cc < 4; ++cc) {
             float v[32];
@@ -328,29 +366,37 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (m == -INFINITY) m = mx;                // first visible key of the row (O is zero)
         const float mu = m == -INFINITY ? 0.f : m;
         // P buffer j & 1 is free once PV of entry j - 2 has completed
-        if (j >= 2 && !warp_wait(&sm.pv_done[j & 1], (uint32_t)(((j - 2) >> 1) & 1), &sm.abort)) { ok = false; break; }
-        unsigned char* prow = sm.p[j & 1] + r * 128;
-        float psum = 0.f;
+        if (j >= 2 && !warp_wait(&sm.pv_done[u][j & 1], (uint32_t)(((j - 2) >> 1) & 1), &sm.abort)) {
+          ok = false;
+          break;
+        }
+        unsigned char* prow = sm.p[u][j & 1] + r * 128;
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};        // four independent sum chains
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           uint32_t w4[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const float p0 = exp2f(x[ch * 8 + 2 * u] - mu), p1 = exp2f(x[ch * 8 + 2 * u + 1] - mu);
-            w4[u] = pack_bf16(p0, p1);
-            psum += p0 + p1;                       // the log-sum-exp from the unrounded weights
+          for (int q = 0; q < 4; ++q) {
+            // 2^(x * log2(e)/sqrt(d) - mu); a masked key (-inf) gives 0
+            const float p0 = ex2(fmaf(x[ch * 8 + 2 * q], sl2, -mu));
+            const float p1 = ex2(fmaf(x[ch * 8 + 2 * q + 1], sl2, -mu));
+            w4[q] = pack_bf16(p0, p1);
+            ps[q] += p0 + p1;                      // the log-sum-exp from the unrounded weights
           }
           *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
-        l += psum;
+        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[j & 1]);
+        if (lane == 0) mbar_arrive(&sm.p_full[u][j & 1]);
       }
       if (!ok) break;
       // epilogue: O / l of each valid row
-      if (n >= 1 && !warp_wait(&sm.pv_done[(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) { ok = false; break; }
+      if (n >= 1 && !warp_wait(&sm.pv_done[u][(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
       const float inv = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = a.O + (((int64_t)t.b * a.nq + qi) * a.Hq + h) * kD;
@@ -366,13 +412,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
         if (valid) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
+          for (int q = 0; q < 4; ++q) {
             uint4 o4;
-            o4.x = pack_bf16(v[u * 8 + 0] * inv, v[u * 8 + 1] * inv);
-            o4.y = pack_bf16(v[u * 8 + 2] * inv, v[u * 8 + 3] * inv);
-            o4.z = pack_bf16(v[u * 8 + 4] * inv, v[u * 8 + 5] * inv);
-            o4.w = pack_bf16(v[u * 8 + 6] * inv, v[u * 8 + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + cc * 32 + u * 8) = o4;
+            o4.x = pack_bf16(v[q * 8 + 0] * inv, v[q * 8 + 1] * inv);
+            o4.y = pack_bf16(v[q * 8 + 2] * inv, v[q * 8 + 3] * inv);
+            o4.z = pack_bf16(v[q * 8 + 4] * inv, v[q * 8 + 5] * inv);
+            o4.w = pack_bf16(v[q * 8 + 6] * inv, v[q * 8 + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + cc * 32 + q * 8) = o4;
           }
         }
       }
@@ -380,14 +426,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.o_free);
+      if (lane == 0) mbar_arrive(&sm.o_free[u]);
     }
     if (!ok) give_up(sm, a.dev_status);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     __syncwarp();
     tmem_free(tmem, kTmemCols);
   }
@@ -395,8 +441,8 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
 // ---------------------------------------------------------------------------
 // union of a tile's leaf lists, one CTA per (tile, range of kRange chunk ids):
-// every chunk some row selected (with the 128-bit mask of those rows), chunk 0 (the first
-// key) and each row's own chunk, in ascending id order
+// every chunk some row selected (with the masks of those rows, 128 bits per sub-tile),
+// chunk 0 (the first key) and each row's own chunk, in ascending id order
 // ---------------------------------------------------------------------------
 
 struct UnionArgs {
@@ -412,24 +458,37 @@ struct UnionArgs {
   int32_t* dev_status;
 };
 
+constexpr int kMaskWords = 4 * kSub;             // 32-bit words of a tile's row mask
+
 __global__ void __launch_bounds__(256) prefill_union_kernel(UnionArgs a) {
-  __shared__ uint32_t mask[4][kRange];
+  __shared__ uint32_t mask[kMaskWords][kRange];
   __shared__ uint32_t present[kRange / 32];
   __shared__ unsigned int wtot[8];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t tile = blockIdx.x / a.nr, rg = blockIdx.x % a.nr;
   const int64_t unit = tile / a.nqt;
-  const int q0 = (int)(tile % a.nqt) * a.Qt;
+  const int q0 = (int)(tile % a.nqt) * kSub * a.Qt;
   const int b = (int)(unit / a.Hkv), hk = (int)(unit % a.Hkv);
   const int64_t lo = rg * kRange, hi = lo + kRange;
-  const int rows = a.Qt * a.G;
-  for (int i = tid; i < kRange; i += 256) mask[0][i] = mask[1][i] = mask[2][i] = mask[3][i] = 0u;
+  const int sub_rows = a.Qt * a.G;
+  for (int i = tid; i < kRange; i += 256) {
+#pragma unroll
+    for (int w = 0; w < kMaskWords; ++w) mask[w][i] = 0u;
+  }
   if (tid < kRange / 32) present[tid] = 0u;
   __syncthreads();
+  // row R of the tile: sub-tile R / 128, row R % 128 of it (query (R % 128) / G, head (R % 128) % G)
+  auto row_query = [&](int R, int& qi, int& hh) -> bool {
+    const int u = R >> 7, rr = R & 127;
+    if (rr >= sub_rows) return false;
+    qi = q0 + u * a.Qt + rr / a.G;
+    hh = hk * a.G + rr % a.G;
+    return qi < a.nq;
+  };
   // chunk 0 and each valid row's own chunk
-  for (int r = tid; r < rows; r += 256) {
-    const int qi = q0 + r / a.G;
-    if (qi >= a.nq) continue;
+  for (int R = tid; R < kSub * 128; R += 256) {
+    int qi, hh;
+    if (!row_query(R, qi, hh)) continue;
     const int64_t t = a.q_pos[(int64_t)b * a.nq + qi];
     if (t < 0 || t >= a.t_cap) {
       if (rg == 0) set_status(a.dev_status, ZHA_ERR_INVALID_ARG);
@@ -440,13 +499,13 @@ __global__ void __launch_bounds__(256) prefill_union_kernel(UnionArgs a) {
     if (lo == 0) atomicOr(&present[0], 1u);
   }
   // selected chunks: warp w takes rows w, w + 8, ...
-  for (int r = warp; r < rows; r += 8) {
-    const int qi = q0 + r / a.G;
-    if (qi >= a.nq) continue;
+  for (int R = warp; R < kSub * 128; R += 8) {
+    int qi, hh;
+    if (!row_query(R, qi, hh)) continue;
     const int64_t t = a.q_pos[(int64_t)b * a.nq + qi];
     if (t < 0 || t >= a.t_cap) continue;
     const int64_t nvis = t / kLeaf;
-    const int64_t qh = ((int64_t)b * a.nq + qi) * a.Hq + hk * a.G + r % a.G;
+    const int64_t qh = ((int64_t)b * a.nq + qi) * a.Hq + hh;
     const int* lst = a.leaf_ids + qh * a.leaf_cap;
     int cnt = a.leaf_cnt[qh];
     cnt = cnt < 0 ? 0 : (cnt > a.leaf_cap ? a.leaf_cap : cnt);
@@ -456,7 +515,7 @@ __global__ void __launch_bounds__(256) prefill_union_kernel(UnionArgs a) {
       const int id = lst[x];
       // ids outside [lo, hi) mean an unsorted list; beyond n_vis an invisible chunk
       if (id < lo || id >= hi || id >= nvis) { set_status(a.dev_status, ZHA_ERR_INVALID_ARG); continue; }
-      atomicOr(&mask[r >> 5][id - lo], 1u << (r & 31));
+      atomicOr(&mask[R >> 5][id - lo], 1u << (R & 31));
     }
   }
   __syncthreads();
@@ -467,7 +526,10 @@ __global__ void __launch_bounds__(256) prefill_union_kernel(UnionArgs a) {
 #pragma unroll
   for (int q = 0; q < kPer; ++q) {
     const int i = tid * kPer + q;
-    on[q] = ((present[i >> 5] >> (i & 31)) & 1u) || (mask[0][i] | mask[1][i] | mask[2][i] | mask[3][i]);
+    uint32_t any = (present[i >> 5] >> (i & 31)) & 1u;
+#pragma unroll
+    for (int w = 0; w < kMaskWords; ++w) any |= mask[w][i];
+    on[q] = any != 0u;
     cntl += on[q];
   }
   unsigned int x = cntl;
@@ -487,7 +549,10 @@ __global__ void __launch_bounds__(256) prefill_union_kernel(UnionArgs a) {
     if (!on[q]) continue;
     const int i = tid * kPer + q;
     a.ent_ids[base + before] = (int)(lo + i);
-    a.ent_mask[base + before] = make_uint4(mask[0][i], mask[1][i], mask[2][i], mask[3][i]);
+#pragma unroll
+    for (int u = 0; u < kSub; ++u)
+      a.ent_mask[(base + before) * kSub + u] = make_uint4(mask[4 * u][i], mask[4 * u + 1][i], mask[4 * u + 2][i],
+                                                          mask[4 * u + 3][i]);
     ++before;
   }
   if (tid == 0) a.ent_cnt[blockIdx.x] = (int)total;
@@ -518,13 +583,13 @@ PrefillWs prefill_ws(const zha_geom& g, int nq, size_t base) {
   PrefillWs w{};
   const int G = g.Hq / g.Hkv;
   w.Qt = kPrefillRows / G;
-  w.nqt = (nq + w.Qt - 1) / w.Qt;
+  w.nqt = (nq + qt::kSub * w.Qt - 1) / (qt::kSub * w.Qt);
   w.tiles = (int64_t)g.B * g.Hkv * w.nqt;
   w.nr = (ncap_of(g, 1) + 1 + kRange - 1) / kRange;
   const size_t slots = (size_t)w.tiles * w.nr * kRange;
   size_t off = base;
   w.ent_ids = off;  off = align_up(off + slots * 4);
-  w.ent_mask = off; off = align_up(off + slots * 16);
+  w.ent_mask = off; off = align_up(off + slots * 16 * qt::kSub);
   w.ent_cnt = off;  off = align_up(off + (size_t)w.tiles * w.nr * 4);
   w.bytes = off;
   return w;

@@ -301,11 +301,16 @@ zha_status zha_flat_index(const zha_geom* g, const void* Q, const void* K, const
  *   Arguments and result as zha_sparse_attn (same kernels; the split size is enlarged
  *   until the scratch fits, so values agree with zha_sparse_attn to fp32 rounding).
  *   Sizes whose scratch cannot fit even with the largest split return
- *   ZHA_ERR_CAPACITY before anything is enqueued: the array holds about 400
- *   (sequence, query, KV head) units while t_cap < 256K tokens, and proportionally
- *   fewer for longer caches (about 32 KiB of union lists per unit and 4096 leaf chunks).
+ *   ZHA_ERR_CAPACITY before anything is enqueued.  At the largest split (1026 chunk ids per
+ *   work item) a (sequence, query, KV head) unit needs about
+ *     nr * (8216 + 528 G) + 528 G * ceil((t_cap/64 + 2) / 1026) bytes,
+ *   nr = ceil((t_cap/64 + 1) / 1024), G = Hq / Hkv (the union lists of each block of 1024
+ *   chunk ids, and one split partial of d + 4 floats per head and work item): with G = 8,
+ *   366 units fit at t_cap = 128K, 255 at 240K and 60 at 1M; with G = 1, 614 at 128K.
  *   The first call on a device resolves the array's device address (cudaGetSymbolAddress
- *   with that device current); make that first call before any stream capture.
+ *   with that device current); make that first call before any stream capture.  The
+ *   address is kept per device index until the process exits: after cudaDeviceReset the
+ *   library must be reloaded.
  *   Every call shares the array, and it keeps the previous call's contents (nothing in
  *   it needs to start at zero: every value read is written earlier in the same call).
  *   Calls that overlap on the GPU race on the array: issue them on one stream, or order
