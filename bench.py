@@ -62,6 +62,8 @@ def parse():
                          "(the dominant kernel's duration then comes from traced, uncaptured steps)")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling)")
+    ap.add_argument("--n-new", type=int, default=None,
+                    help="prefill path: appended queries (default: the workload's 4096)")
     ap.add_argument("--path", default="zha", choices=["zha", "dense", "flat", "prefill"],
                     help="zha: the hot path (default); dense / flat: the baselines on the same inputs; "
                          "prefill: the query-tile attention of the chunked-prefill workload")
@@ -764,8 +766,8 @@ def run_prefill(args):
     torch.cuda.set_device(0)
     dev = torch.device("cuda", 0)
     w = S.workload("prefill-append-256k")
-    if args.batch is not None:
-        w = S.scaled(w, T=w.T, B=args.batch)
+    if args.batch is not None or args.n_new is not None:
+        w = S.scaled(w, T=w.T, B=args.batch, n_new=args.n_new)
     p = args.p if args.p is not None else w.p[0]
     g = Z.Geometry(B=w.B, Hq=w.Hq, Hkv=w.Hkv, t_cap=w.t_cap, depth=w.depth, R=w.R)
     C, K, V = S.clustered_kv(w, dev)

@@ -116,3 +116,5 @@ def test_near_cutoff_valid_rules():
     assert near_cutoff_valid(s, c, np.array([0, 2]), None, k=2) != ""
     tie = np.array([1.0, 1.0 + NEAR_CUTOFF / 2, 0.0])
     assert near_cutoff_valid(tie, np.arange(3), np.array([0]), None, k=1) == ""   # a near tie may swap
+    far = np.array([1.0, 1.01, 0.0])                                              # mass gap ~ 3.5e-3
+    assert near_cutoff_valid(far, np.arange(3), np.array([0]), None, k=1) != ""

@@ -56,7 +56,6 @@ def f32_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     return np.abs(ordinal(a) - ordinal(b))
 
 
-NEAR_TIE = 1e-4         # score gap (natural-log units) below which two candidates are a near tie
 MAX_EXCUSED = 1 / 32    # fraction of the compared heads that may differ at a near cutoff (at least 1)
 
 
@@ -103,9 +102,10 @@ def near_cutoff_valid(scores: np.ndarray, cand: np.ndarray, got: np.ndarray, p, 
     ``scores``) up to the rounding the cutoff tolerance allows; '' if so, else why not.
 
     Top-p (threshold p): the set's softmax mass reaches p - NEAR_CUTOFF, dropping its
-    smallest member leaves less than p + NEAR_CUTOFF, and no candidate left out scores
-    more than NEAR_TIE above a kept one.  Top-K: |got| = min(K, n) and the same order
-    condition.  p >= 1 keeps everything: no tolerance."""
+    smallest member leaves less than p + NEAR_CUTOFF, and no candidate left out has more
+    softmax mass than a kept one by NEAR_CUTOFF or more (the boundary gap of the near-cutoff
+    reading).  Top-K: |got| = min(K, n) and the same order condition.  p >= 1 keeps
+    everything: no tolerance."""
     if len(np.unique(got)) != len(got) or not np.all(np.isin(got, cand)):
         return "kept ids are not distinct candidates"
     inside = np.isin(cand, got)
@@ -123,8 +123,9 @@ def near_cutoff_valid(scores: np.ndarray, cand: np.ndarray, got: np.ndarray, p, 
             return f"not minimal: mass without the smallest kept {mass - pi[inside].min():.6g}"
     elif inside.sum() != min(int(k), len(cand)):
         return f"kept {int(inside.sum())} of {len(cand)}, K = {k}"
-    if (~inside).any() and scores[~inside].max() > scores[inside].min() + NEAR_TIE:
-        return f"a dropped candidate outscores a kept one by {scores[~inside].max() - scores[inside].min():.3g}"
+    if (~inside).any() and pi[~inside].max() - pi[inside].min() >= NEAR_CUTOFF:
+        return (f"a dropped candidate has {pi[~inside].max() - pi[inside].min():.3g} more mass than a kept one "
+                f"(scores {scores[~inside].max():.6g} > {scores[inside].min():.6g})")
     return ""
 
 
