@@ -305,10 +305,12 @@ def paper_model(line: dict, peaks: dict) -> dict:
     st = line["stages_ms"]
     levels = line["frontier"]["levels"]               # top level first
     depth = cfg["depth"]
-    # one score and one select launch per level, from level `depth` down (empty levels too)
-    score_ms = lambda l: st["route_score_per_launch"][depth - l]     # noqa: E731
-    select_ms = lambda l: st["route_select_per_launch"][depth - l]   # noqa: E731
     top = levels[0]["level"]
+    # one score and one select launch per level, top level first; lines that also timed the
+    # (empty) levels above the top start at level `depth`
+    first = depth if len(st["route_score_per_launch"]) == depth else top
+    score_ms = lambda l: st["route_score_per_launch"][first - l]     # noqa: E731
+    select_ms = lambda l: st["route_select_per_launch"][first - l]   # noqa: E731
     tau = {"score": score_ms(top), "select": select_ms(top)}
 
     def row(stage, kind, flops, byts, peak, unit, measured):
@@ -340,7 +342,7 @@ def paper_model(line: dict, peaks: dict) -> dict:
     # levels above the top one have no visible node: their score and select launches are
     # launch overhead only (the lambda_l of the model), with the gaps between kernels
     empty = 0.0
-    for l in range(depth, top, -1):
+    for l in range(first, top, -1):
         t = score_ms(l) + select_ms(l)
         empty += t
         rows.append({"stage": f"route L{l} (empty)", "flops": 0.0, "bytes": 0.0, "flops_ms": 0.0,

@@ -17,13 +17,16 @@
 // rescaled only when a row's maximum grows by more than 2^8).  A row sees key j of chunk c
 // iff c is in its S_1, or j = 0, or c is its own chunk and j <= t.
 //
-// Roles in one CTA of 320 threads, one tile after another (a persistent grid):
-//   warps 0-3, 4-7  softmax and epilogue of sub-tile 0, 1: thread r <-> row r <-> TMEM lane r
-//              (sub-tile u owns TMEM columns [256 u, 256 u + 256));
-//   warp 8     producer: TMA loads of the Q sub-tiles (4-D map) and of each chunk's K and V
+// Roles in one CTA of 576 threads, one tile after another (a persistent grid):
+//   warps 0-15 softmax and epilogue: warp w serves sub-tile w / 8, the keys [32 h, 32 h + 32)
+//              of each chunk and the output dims [64 h, 64 h + 64) for h = (w / 4) % 2, and
+//              the rows 32 (w % 4) + lane (= its TMEM lanes); the two threads of a row share
+//              their maxima through shared memory and a named barrier (sub-tile u owns TMEM
+//              columns [256 u, 256 u + 256));
+//   warp 16    producer: TMA loads of the Q sub-tiles (4-D map) and of each chunk's K and V
 //              (3-D maps, 128-byte swizzle) into a 3-stage ring; this GPU's memory only,
 //              no multicast;
-//   warp 9     TMEM allocation; lane 0 issues the MMAs and their commits.
+//   warp 17    TMEM allocation; lane 0 issues the MMAs and their commits.
 // Every wait is bounded; a wait that gives up reports ZHA_ERR_DEVICE, the CTA stops, waits
 // (bounded) for its copies and MMAs in flight, frees its TMEM and returns.
 #include <cuda.h>
@@ -48,7 +51,8 @@ constexpr int kPBytes = kRows * 128;             // 128 rows x 64 keys of P (bf1
 constexpr uint32_t kTmemCols = 512;              // per sub-tile: S0, S1 (64 each), O (128)
 constexpr uint32_t kSubCols = 256;
 constexpr uint32_t kColO = 128;
-constexpr int kSoftWarps = 4 * kSub;
+constexpr int kHalves = 2;                      // softmax threads per row (32 of its 64 keys each)
+constexpr int kSoftWarps = 4 * kHalves * kSub;
 constexpr int kProducerWarp = kSoftWarps, kMmaWarp = kSoftWarps + 1;
 constexpr int kThreads = (kSoftWarps + 2) * 32;
 constexpr float kLazy = 8.0f;                    // rescale O when a row max grows by > 2^8
@@ -58,13 +62,15 @@ constexpr uint32_t kIdescPV = idesc_bf16(128, 128, 1); // O += P . V, V MN-major
 struct alignas(1024) Smem {
   unsigned char q[kSub][2][kQHalf];              // per sub-tile two 128B-swizzled boxes [128 rows][64 dims]
   unsigned char kv[kStages][kKVBytes];
-  unsigned char p[kSub][2][kPBytes];             // [128 rows][64 keys], 128B swizzle
+  unsigned char p[kSub][kPBytes];                // [128 rows][64 keys], 128B swizzle
   uint4 meta_mask[kStages][kSub];                // rows of each sub-tile that selected the chunk
   int meta_id[kStages];                          // chunk id of each stage
   unsigned long long full[kStages], empty[kStages];
   unsigned long long q_full, q_empty;
   unsigned long long s_full[kSub][2], s_free[kSub][2], p_full[kSub][2], pv_done[kSub][2];
   unsigned long long o_free[kSub], drain;
+  float xmax[2][kSub][kHalves][kRows];           // row maxima (per entry) and sums (epilogue) of the
+                                                 // two halves of a row, by entry parity
   uint32_t tmem_base;
   int abort, zero;
 };
@@ -122,7 +128,7 @@ struct EntryWalk {
 };
 
 __device__ __forceinline__ bool warp_wait(unsigned long long* b, uint32_t parity, int* abort) {
-  const bool ok = __all_sync(0xffffffffu, mbar_wait(b, parity, abort));
+  const bool ok = __all_sync(0xffffffffu, mbar_wait_sleep(b, parity, abort));
   return ok;
 }
 
@@ -152,11 +158,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     for (int u = 0; u < kSub; ++u) {
       for (int i = 0; i < 2; ++i) {
         mbar_init(&sm.s_full[u][i], 1);
-        mbar_init(&sm.s_free[u][i], 4);
-        mbar_init(&sm.p_full[u][i], 4);
+        mbar_init(&sm.s_free[u][i], 4 * kHalves);
+        mbar_init(&sm.p_full[u][i], 4 * kHalves);
         mbar_init(&sm.pv_done[u][i], 1);
       }
-      mbar_init(&sm.o_free[u], 4);
+      mbar_init(&sm.o_free[u], 4 * kHalves);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -181,7 +187,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       bool ok = true;
       for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
         const Tile t = tile_of(a, tile);
-        if (nq_loads > 0 && !mbar_wait(&sm.q_empty, (uint32_t)((nq_loads - 1) & 1), &sm.abort)) {
+        if (nq_loads > 0 && !mbar_wait_sleep(&sm.q_empty, (uint32_t)((nq_loads - 1) & 1), &sm.abort)) {
           give_up(sm, a.dev_status);
           break;
         }
@@ -196,7 +202,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         w.start(a, tile);
         for (int i = 0; i < n; ++i, ++it, w.next(a)) {
           const int s = (int)(it % kStages);
-          if (it >= kStages && !mbar_wait(&sm.empty[s], (uint32_t)(((it / kStages) - 1) & 1), &sm.abort)) {
+          if (it >= kStages && !mbar_wait_sleep(&sm.empty[s], (uint32_t)(((it / kStages) - 1) & 1), &sm.abort)) {
             give_up(sm, a.dev_status);
             ok = false;
             break;
@@ -229,7 +235,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       long long j = 0, tl = 0;                   // entries and tiles of this CTA so far
       bool ok = true;
       auto issue_s = [&](int u, long long e) -> bool {
-        if (e >= 2 && !mbar_wait(&sm.s_free[u][e & 1], (uint32_t)(((e >> 1) - 1) & 1), &sm.abort)) return false;
+        if (e >= 2 && !mbar_wait_sleep(&sm.s_free[u][e & 1], (uint32_t)(((e >> 1) - 1) & 1), &sm.abort)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(sm.q[u][0]);
         const uint32_t ka = smem_u32(sm.kv[e % kStages]);
@@ -242,10 +248,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         return true;
       };
       auto issue_pv = [&](int u, long long e, bool first_of_tile) -> bool {
-        if (!mbar_wait(&sm.p_full[u][e & 1], (uint32_t)((e >> 1) & 1), &sm.abort)) return false;
-        if (first_of_tile && tl > 0 && !mbar_wait(&sm.o_free[u], (uint32_t)((tl - 1) & 1), &sm.abort)) return false;
+        if (!mbar_wait_sleep(&sm.p_full[u][e & 1], (uint32_t)((e >> 1) & 1), &sm.abort)) return false;
+        if (first_of_tile && tl > 0 && !mbar_wait_sleep(&sm.o_free[u], (uint32_t)((tl - 1) & 1), &sm.abort)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sm.p[u][e & 1]);
+        const uint32_t pa = smem_u32(sm.p[u]);
         const uint32_t va = smem_u32(sm.kv[e % kStages] + 2 * kBox);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
@@ -256,11 +262,11 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       };
       for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tl) {
         const int n = tile_entries(a, tile);
-        if (!mbar_wait(&sm.q_full, (uint32_t)(tl & 1), &sm.abort)) { ok = false; break; }
+        if (!mbar_wait_sleep(&sm.q_full, (uint32_t)(tl & 1), &sm.abort)) { ok = false; break; }
         tc_fence_after();
         for (int i = 0; i < n; ++i, ++j) {
           const int s = (int)(j % kStages);
-          if (!mbar_wait(&sm.full[s], (uint32_t)((j / kStages) & 1), &sm.abort)) { ok = false; break; }
+          if (!mbar_wait_sleep(&sm.full[s], (uint32_t)((j / kStages) & 1), &sm.abort)) { ok = false; break; }
           if (!issue_s(0, j) || !issue_s(1, j)) { ok = false; break; }
           if (i >= 1) {
             if (!issue_pv(0, j - 1, i == 1) || !issue_pv(1, j - 1, i == 1)) { ok = false; break; }
@@ -281,9 +287,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     }
   } else {
     // ------------------------------------------------------------------ softmax + epilogue
-    const int u = warp >> 2;                     // sub-tile of this warpgroup
-    const int r = threadIdx.x & 127;             // row = TMEM lane
+    const int u = warp >> 3;                     // sub-tile of this warp
+    const int hf = (warp >> 2) & 1;              // half of the row: keys 32 hf.., dims 64 hf..
+    const int r = (warp & 3) * 32 + lane;        // row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + u * kSubCols;
+    const uint32_t s_col = (uint32_t)hf * 32, o_col = kColO + (uint32_t)hf * 64;
+    const int bar_id = 1 + u * 4 + (warp & 3);   // named barrier of the row group's two warps
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
     long long j = 0, tl = 0;
     bool ok = true;
@@ -309,40 +318,35 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const uint4 mk = sm.meta_mask[s][u];
         if (!warp_wait(&sm.s_full[u][j & 1], (uint32_t)((j >> 1) & 1), &sm.abort)) { ok = false; break; }
         tc_fence_after();
-        float x[64];
-        {
-          float v[32];
-          tmem_ld32(lane_addr + (uint32_t)(j & 1) * 64, v);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) x[k] = v[k];
-          tmem_ld32(lane_addr + (uint32_t)(j & 1) * 64 + 32, v);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) x[32 + k] = v[k];
-        }
+        float x[32];
+        tmem_ld32(lane_addr + (uint32_t)(j & 1) * 64 + s_col, x);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.s_free[u][j & 1]);
         // visibility of the chunk's keys for this row: all of them (a selected chunk), the
-        // keys up to t (its own chunk), key 0 (chunk 0), or none
+        // keys up to t (its own chunk), key 0 (chunk 0), or none; this thread holds keys
+        // 32 hf + k
         const uint32_t wsel = mword == 0 ? mk.x : mword == 1 ? mk.y : mword == 2 ? mk.z : mk.w;
         const bool sel = valid && (wsel & mbit) && c < cur;
         const bool own = valid && c == cur;
-        const int lim = sel ? 63 : (own ? (int)(pos - (int64_t)c * kLeaf) : (valid && c == 0 ? 0 : -1));
+        const int lim = (sel ? 63 : (own ? (int)(pos - (int64_t)c * kLeaf) : (valid && c == 0 ? 0 : -1))) - 32 * hf;
         float mx;
         {
-          float m8[8];                             // eight independent max chains
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent max chains
 #pragma unroll
-          for (int q = 0; q < 8; ++q) m8[q] = -INFINITY;
-#pragma unroll
-          for (int k = 0; k < 64; ++k) {
+          for (int k = 0; k < 32; ++k) {
             x[k] = k <= lim ? x[k] : -INFINITY;
-            m8[k & 7] = fmaxf(m8[k & 7], x[k]);
+            m4[k & 3] = fmaxf(m4[k & 3], x[k]);
           }
-          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-          mx *= sl2;                               // the row maximum in log2 units (-inf stays)
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;   // log2 units (-inf stays)
         }
-        // lazy rescale: only when the row maximum grows by more than 2^kLazy (warp-wide)
+        // the row maximum over both halves
+        sm.xmax[j & 1][u][hf][r] = mx;
+        asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+        mx = fmaxf(mx, sm.xmax[j & 1][u][hf ^ 1][r]);
+        // lazy rescale: only when the row maximum grows by more than 2^kLazy (the same
+        // decision in both halves: same m, same maximum)
         const bool grow = m != -INFINITY && mx > m + kLazy;
         if (__any_sync(0xffffffffu, grow)) {
           if (i >= 1 && !warp_wait(&sm.pv_done[u][(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
@@ -352,59 +356,64 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           tc_fence_after();
           const float alpha = grow ? ex2(m - mx) : 1.f;
 #pragma unroll 1
-          for (int cc = 0; cc < 4; ++cc) {
+          for (int cc = 0; cc < 2; ++cc) {
             float v[32];
-            tmem_ld32(lane_addr + kColO + cc * 32, v);
+            tmem_ld32(lane_addr + o_col + cc * 32, v);
             tmem_wait_ld();
 #pragma unroll
             for (int k = 0; k < 32; ++k) v[k] *= alpha;
-            tmem_st32(lane_addr + kColO + cc * 32, v);
+            tmem_st32(lane_addr + o_col + cc * 32, v);
           }
           tmem_wait_st();
           if (grow) { l *= alpha; m = mx; }
         }
         if (m == -INFINITY) m = mx;                // first visible key of the row (O is zero)
         const float mu = m == -INFINITY ? 0.f : m;
-        // P buffer j & 1 is free once PV of entry j - 2 has completed
-        if (j >= 2 && !warp_wait(&sm.pv_done[u][j & 1], (uint32_t)(((j - 2) >> 1) & 1), &sm.abort)) {
+        uint32_t pw[16];                           // P (bf16 pairs) of this thread's 32 keys
+        float ps[4] = {0.f, 0.f, 0.f, 0.f};        // four independent sum chains
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          // 2^(x * log2(e)/sqrt(d) - mu); a masked key (-inf) gives 0
+          const float p0 = ex2(fmaf(x[2 * q], sl2, -mu)), p1 = ex2(fmaf(x[2 * q + 1], sl2, -mu));
+          pw[q] = pack_bf16(p0, p1);
+          ps[q & 3] += p0 + p1;                    // the log-sum-exp from the unrounded weights
+        }
+        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
+        // the P buffer of this sub-tile is free once PV of entry j - 1 has completed
+        if (j >= 1 && !warp_wait(&sm.pv_done[u][(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
           ok = false;
           break;
         }
-        unsigned char* prow = sm.p[u][j & 1] + r * 128;
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};        // four independent sum chains
+        unsigned char* prow = sm.p[u] + r * 128;
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            // 2^(x * log2(e)/sqrt(d) - mu); a masked key (-inf) gives 0
-            const float p0 = ex2(fmaf(x[ch * 8 + 2 * q], sl2, -mu));
-            const float p1 = ex2(fmaf(x[ch * 8 + 2 * q + 1], sl2, -mu));
-            w4[q] = pack_bf16(p0, p1);
-            ps[q] += p0 + p1;                      // the log-sum-exp from the unrounded weights
-          }
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        for (int ch = 0; ch < 4; ++ch) {
+          const int chunk = hf * 4 + ch;           // 16-byte chunk of the row (8 keys)
+          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) =
+              make_uint4(pw[4 * ch], pw[4 * ch + 1], pw[4 * ch + 2], pw[4 * ch + 3]);
         }
-        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
         fence_proxy_async_smem();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.p_full[u][j & 1]);
       }
       if (!ok) break;
-      // epilogue: O / l of each valid row
+      // epilogue: O / l of each valid row, the row sum from both halves (in the maxima slot
+      // of the next entry's parity: both halves have read the last entry's maxima)
+      sm.xmax[j & 1][u][hf][r] = l;
+      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+      const float lr = sm.xmax[j & 1][u][0][r] + sm.xmax[j & 1][u][1][r];
       if (n >= 1 && !warp_wait(&sm.pv_done[u][(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = a.O + (((int64_t)t.b * a.nq + qi) * a.Hq + h) * kD;
+      const float inv = lr > 0.f ? 1.f / lr : 0.f;
+      __nv_bfloat16* orow = a.O + (((int64_t)t.b * a.nq + qi) * a.Hq + h) * kD + hf * 64;
 #pragma unroll 1
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int cc = 0; cc < 2; ++cc) {
         float v[32];
         if (n >= 1) {
-          tmem_ld32(lane_addr + kColO + cc * 32, v);
+          tmem_ld32(lane_addr + o_col + cc * 32, v);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -422,8 +431,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           }
         }
       }
-      if (valid && a.lse) a.lse[((int64_t)t.b * a.nq + qi) * a.Hq + h] =
-          l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (valid && hf == 0 && a.lse) a.lse[((int64_t)t.b * a.nq + qi) * a.Hq + h] =
+          lr > 0.f ? (m + log2f(lr)) * 0.6931471805599453f : -INFINITY;
+      // the sums of this tile are read before the next tile's epilogue writes them
+      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[u]);

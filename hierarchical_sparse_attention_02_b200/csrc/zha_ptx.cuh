@@ -60,6 +60,39 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long* b, uint32_t parity
   return false;
 }
 
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// One poll that may suspend the thread until the phase completes or about `hint_ns` pass.
+__device__ __forceinline__ bool mbar_try_sleep(unsigned long long* b, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
+      " selp.u32 %0, 1, 0, p;\n}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(b)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for long waits of many threads: each poll may suspend the thread (so waiting
+// warps take few issue slots), and the wait gives up after `limit_ns` of wall time (global
+// timer) or at once when another thread of the CTA has given up (`abort` set).
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
+__device__ __forceinline__ bool mbar_wait_sleep(unsigned long long* b, uint32_t parity, const int* abort,
+                                                unsigned long long limit_ns = kWaitLimitNs) {
+  if (mbar_try(b, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (;;) {
+    if (mbar_try_sleep(b, parity, 20000u)) return true;
+    if (*(volatile const int*)abort) return false;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // TMA (this GPU's memory only; no multicast)
 // ---------------------------------------------------------------------------

@@ -1790,7 +1790,20 @@ static cudaError_t route_levels(const RouteCall& c) {
   int64_t level_ids_stride = 0;
   for (int l = 2; l <= g.depth; ++l) level_ids_stride += ncap_of(g, l);
   int64_t level_off = level_ids_stride;
-  for (int l = g.depth; l >= 1; --l) {
+  // One position for every query (a decode step) and no level counts requested: the levels
+  // above the query's top level hold no visible node, so their launches are skipped (they
+  // would only record empty selections).  Level 1 always runs: it writes the leaf counts.
+  int lmax = g.depth;
+  if (!c.q_pos && !c.level_cnt && !c.level_ids && c.pos_uniform >= 0 && c.pos_uniform < g.t_cap) {
+    const int64_t vis = (c.pos_uniform / kLeaf) * kLeaf;
+    int top = 0;
+    for (int l = g.depth; l >= 1 && top == 0; --l)
+      if (vis / span_of(g, l) >= 1) top = l;
+    lmax = top < 1 ? 1 : top;
+  }
+  for (int l = g.depth; l > lmax; --l)
+    if (l >= 2) level_off -= ncap_of(g, l);
+  for (int l = lmax; l >= 1; --l) {
     const int cur = l & 1, prev = (l + 1) & 1;
     ScoreArgs sa{};
     sa.g = rg; sa.level = l; sa.Q = c.Q;
