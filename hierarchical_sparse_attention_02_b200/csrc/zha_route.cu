@@ -1709,6 +1709,10 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
   return cudaLaunchKernelEx(&cfg, kernel, se);
 }
 
+#ifndef ZHA_WARP_SELECT_MAX
+#define ZHA_WARP_SELECT_MAX 256
+#endif
+
 // One select launch per level.  Kernels, by the frontier capacity ncap they hold:
 //   warp     a warp per head (scores in shared memory)            ncap <= 1024
 //   cta256   a CTA of 256 threads per head (30 or 48 KiB)         ncap <= 2560 or 4096
@@ -1721,7 +1725,8 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
 static cudaError_t launch_select(const SelectArgs& se, int64_t nqh, int64_t ncap, cudaStream_t s) {
   const int64_t res256 = 148ll * 3, res1024 = 148;
   int kind;                                            // 0 warp, 1 cta256, 2 cta1024, 3 cluster, 4 wide
-  if (ncap <= kCta1024Cap && nqh <= res1024) kind = 2;
+  if (ncap <= ZHA_WARP_SELECT_MAX) kind = 0;           // small frontiers: a warp per head is the quickest
+  else if (ncap <= kCta1024Cap && nqh <= res1024) kind = 2;
   else if (ncap <= 4096 && nqh <= res256) kind = 1;
   else if (ncap <= kWarpCap) kind = 0;
   else if (ncap <= 4096) kind = 1;
