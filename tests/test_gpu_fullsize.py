@@ -128,8 +128,15 @@ def test_prefill_append_256k_full(Z):
     O = torch.empty(1, w.n_new, w.Hq, w.d, dtype=g.dtype, device=DEV)
     wa = Z.empty_workspace(g, w.n_new, Z.ZHA_OP_ATTN, DEV)
     Z.zha_sparse_attn(g, Q, K, V, pos, ids, cnt, O, wa, st)
+    del wa
+    # the same attention per query tile on the tensor cores (the launch bench.py times)
+    Ot = torch.empty_like(O)
+    wp = Z.empty_workspace(g, w.n_new, Z.ZHA_OP_PREFILL, DEV)
+    Z.zha_prefill_attn(g, Q, K, V, pos, ids, cnt, Ot, wp, st)
     torch.cuda.synchronize()
     assert st.item() == 0
+    d = (Ot.float() - O.float()).abs()
+    assert d.max().item() <= 2e-2 and d.mean().item() <= 2e-3, (d.max().item(), d.mean().item())
     qc = Q.double().cpu().numpy()
     qr = qref.double().cpu().numpy()
     Kc = [K[0, hk].cpu() for hk in range(w.Hkv)]
@@ -151,6 +158,7 @@ def test_prefill_append_256k_full(Z):
             leaves = compare_route(qc[0, qi, h], t, trees[hk], w.p[0], lv, got, cmp, f"q{qi} h{h}")
             o, _ = zo.attention(qc[0, qi, h], Kc[hk], Vc[hk], zo.index_set(leaves, t))
             errs.append(np.abs(O[0, qi, h].float().cpu().numpy() - o))
+            errs.append(np.abs(Ot[0, qi, h].float().cpu().numpy() - o))
     assert cmp.ok(), cmp.problems()
     e = np.stack(errs)
     assert e.max() <= 2e-2 and e.mean() <= 2e-3, (e.max(), e.mean())
