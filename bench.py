@@ -306,12 +306,18 @@ def paper_model(line: dict, peaks: dict) -> dict:
     levels = line["frontier"]["levels"]               # top level first
     depth = cfg["depth"]
     top = levels[0]["level"]
-    # one score and one select launch per level, top level first; lines that also timed the
-    # (empty) levels above the top start at level `depth`
-    first = depth if len(st["route_score_per_launch"]) == depth else top
-    score_ms = lambda l: st["route_score_per_launch"][first - l]     # noqa: E731
-    select_ms = lambda l: st["route_select_per_launch"][first - l]   # noqa: E731
-    tau = {"score": score_ms(top), "select": select_ms(top)}
+    # one score and one select launch per level launched on its own, top level first (lines
+    # that also timed the empty levels above the top start at level `depth`); the small top
+    # levels may instead share one fused launch (route_fused), above the per-level ones
+    per_s = st.get("route_score_per_launch") or ([st["route_score"]] if st.get("route_score") else [])
+    per_x = st.get("route_select_per_launch") or ([st["route_select"]] if st.get("route_select") else [])
+    n_sep = len(per_s)                                # levels n_sep .. 1 launched on their own
+    first = depth if n_sep == depth else n_sep
+    fused_ms = st.get("route_fused", 0.0) or 0.0
+    score_ms = lambda l: per_s[first - l] if l <= first else None      # noqa: E731
+    select_ms = lambda l: per_x[first - l] if l <= first else None     # noqa: E731
+    sep_top = min(top, first)
+    tau = {"score": score_ms(sep_top), "select": select_ms(sep_top)}
 
     def row(stage, kind, flops, byts, peak, unit, measured):
         t_f, t_b = 1e3 * flops / peak, 1e3 * byts / bw
@@ -322,14 +328,24 @@ def paper_model(line: dict, peaks: dict) -> dict:
                 "waves_ms": t_w, "model_ms": model, "bound": bound, "measured_ms": measured}
 
     rows = []
+    fused = []
     for f in levels:
         l = f["level"]
         k_head = f["candidates_mean"]
         k_grp = f.get("candidates_group_union", f["candidates_max"])
-        rows.append(row(f"route score L{l}", "score", 2.0 * B * Hq * R * d * k_head,
-                        R * (s * d + 4) * B * Hkv * k_grp + s * d * B * Hq, p64, "fp64 tensor", score_ms(l)))
-        rows.append(row(f"route select L{l}", "select", 0.0, 12.0 * B * Hq * k_head, p64, "alu",
-                        select_ms(l)))
+        r_s = row(f"route score L{l}", "score", 2.0 * B * Hq * R * d * k_head,
+                  R * (s * d + 4) * B * Hkv * k_grp + s * d * B * Hq, p64, "fp64 tensor", score_ms(l))
+        r_x = row(f"route select L{l}", "select", 0.0, 12.0 * B * Hq * k_head, p64, "alu", select_ms(l))
+        if l > first:                                 # inside the fused launch
+            fused += [r_s, r_x]
+        else:
+            rows += [r_s, r_x]
+    if fused:
+        rows.insert(0, {"stage": f"route fused L{top}..L{first + 1}", "flops": sum(r["flops"] for r in fused),
+                        "bytes": sum(r["bytes"] for r in fused), "flops_ms": sum(r["flops_ms"] for r in fused),
+                        "bytes_ms": sum(r["bytes_ms"] for r in fused), "waves_ms": 0.0,
+                        "model_ms": max(r["model_ms"] for r in fused), "bound": "latency (one wave)",
+                        "measured_ms": fused_ms})
     T1 = cfg["T"] + 1
     k0 = line["kv_touched"]["mean"] * T1
     byts = line["roofline"]["algorithmic_bytes_per_launch"] * line["roofline"]["launches_per_step"]
@@ -343,6 +359,8 @@ def paper_model(line: dict, peaks: dict) -> dict:
     # launch overhead only (the lambda_l of the model), with the gaps between kernels
     empty = 0.0
     for l in range(first, top, -1):
+        if score_ms(l) is None:
+            continue
         t = score_ms(l) + select_ms(l)
         empty += t
         rows.append({"stage": f"route L{l} (empty)", "flops": 0.0, "bytes": 0.0, "flops_ms": 0.0,
@@ -572,8 +590,8 @@ def stage_breakdown(lib, step, stream, nb, ms_step):
     With a chunked decode the routing of later chunks runs concurrently with attention,
     so the stage sum exceeds the step time by the overlap."""
     from hierarchical_sparse_attention_02_b200 import _lib
-    kinds = {"route_score": _lib.ZHA_TRACE_ROUTE_SCORE, "route_select": _lib.ZHA_TRACE_ROUTE_SELECT,
-             "attention": _lib.ZHA_TRACE_ATTN}
+    kinds = {"route_fused": _lib.ZHA_TRACE_ROUTE_FUSED, "route_score": _lib.ZHA_TRACE_ROUTE_SCORE,
+             "route_select": _lib.ZHA_TRACE_ROUTE_SELECT, "attention": _lib.ZHA_TRACE_ATTN}
     cap = nb * 64                     # <= 8 chunks x 8 levels per step
     ev = {}
     for name, kid in kinds.items():
@@ -601,8 +619,7 @@ def stage_breakdown(lib, step, stream, nb, ms_step):
         t = [x.elapsed_time(y) for x, y in zip(a[:n], b[:n])]
         out[name] = sum(t) / nb
         per = n // nb                 # launches per step, in launch order (top level first)
-        if per > 1:
-            out[name + "_per_launch"] = [round(sum(t[j::per]) / nb, 4) for j in range(per)]
+        out[name + "_per_launch"] = [round(sum(t[j::per]) / nb, 4) for j in range(per)]
     out["stage_sum"] = sum(out[k] for k in kinds)
     out["step"] = ms_step
     out["steps"] = nb

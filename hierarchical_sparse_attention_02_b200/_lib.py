@@ -23,7 +23,7 @@ EXPORTS = [
     "zha_last_error", "zha_trace", "zha_trace_count",
 ]
 ZHA_NOALLOC_SCRATCH_BYTES = 16 << 20
-ZHA_TRACE_ATTN, ZHA_TRACE_ROUTE_SCORE, ZHA_TRACE_ROUTE_SELECT = 1, 2, 3
+ZHA_TRACE_ATTN, ZHA_TRACE_ROUTE_SCORE, ZHA_TRACE_ROUTE_SELECT, ZHA_TRACE_ROUTE_FUSED = 1, 2, 3, 4
 
 
 class Geom(ctypes.Structure):

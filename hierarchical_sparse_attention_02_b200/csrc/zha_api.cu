@@ -8,7 +8,7 @@
 namespace zha {
 
 std::atomic<int64_t> g_launches{0};
-Tracer g_trace[4];
+Tracer g_trace[5];
 
 static char g_last_error[256] = "no error";
 
@@ -103,7 +103,7 @@ int64_t zha_launch_count(void) { return g_launches.load(); }
 const char* zha_last_error(void) { return g_last_error; }
 
 void zha_trace(int32_t which, void* const* start, void* const* stop, int32_t n) {
-  if (which < 1 || which > 3) return;
+  if (which < 1 || which > 4) return;
   Tracer& t = g_trace[which];
   t.start = start;
   t.stop = stop;
@@ -111,7 +111,7 @@ void zha_trace(int32_t which, void* const* start, void* const* stop, int32_t n) 
   t.done = 0;
 }
 
-int32_t zha_trace_count(int32_t which) { return (which >= 1 && which <= 3) ? g_trace[which].done : 0; }
+int32_t zha_trace_count(int32_t which) { return (which >= 1 && which <= 4) ? g_trace[which].done : 0; }
 
 zha_status zha_build_tree(const zha_geom* g, const void* K, int64_t T, const float* qref,
                           zha_buf tree, int32_t* dev_status, void* stream) {

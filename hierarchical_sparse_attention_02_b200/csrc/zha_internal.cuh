@@ -174,7 +174,7 @@ struct Tracer {
   void* const* stop = nullptr;
   int n = 0, done = 0;
 };
-extern Tracer g_trace[4];
+extern Tracer g_trace[5];
 inline void trace_begin(int which, cudaStream_t s) {
   Tracer& t = g_trace[which];
   if (t.done < t.n) cudaEventRecord((cudaEvent_t)t.start[t.done], s);

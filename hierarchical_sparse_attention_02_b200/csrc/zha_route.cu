@@ -1709,6 +1709,232 @@ static cudaError_t launch_cluster(K kernel, const SelectArgs& se, int64_t cluste
   return cudaLaunchKernelEx(&cfg, kernel, se);
 }
 
+// ---------------------------------------------------------------------------
+// The small top levels in one launch.  Levels whose frontier capacity is at most
+// kSmallCap nodes (the top of the tree) are scored and selected by one CTA per (sequence,
+// query, KV head) unit, level after level: the scores with the arithmetic of
+// route_score_kernel (the same fp64 tensor-core products, in the same order), the cutoff
+// with the rule of the select kernels (fixed-point masses, target ceil(p Z), order score
+// desc then id asc: a candidate is kept iff the mass of the candidates before it is below
+// the target), so the kept sets are those of the per-level launches.
+// ---------------------------------------------------------------------------
+
+#ifndef ZHA_SMALL_CAP
+#define ZHA_SMALL_CAP 64
+#endif
+constexpr int kSmallCap = ZHA_SMALL_CAP;        // frontier capacity of a fused level
+constexpr int kSmallThreads = 256;
+
+struct SmallArgs {
+  RouteGeom g;
+  int l_lo, l_hi;                                // fused levels: l_hi down to l_lo (>= 2)
+  const void* Q;
+  const void* k_route[kMaxDepth + 1];            // per level
+  const float* b_hat[kMaxDepth + 1];
+  double p[kMaxDepth + 1];
+  int64_t topk[kMaxDepth + 1];
+  int mass_shift;
+  int* out_ids;                                  // kept ids of level l_lo, [nqh, out_stride]
+  int* out_cnt;
+  int64_t out_stride;
+  int* level_cnt;                                // nullable [nqh, depth, 2]
+  int* level_ids;                                // nullable [nqh, level_ids_stride]
+  int64_t level_ids_stride;
+  int64_t level_ids_off[kMaxDepth + 1];
+  int32_t* dev_status;
+};
+
+template <typename KT>
+__global__ void __launch_bounds__(kSmallThreads, 2) route_small_kernel(SmallArgs a) {
+  __shared__ __align__(16) double qfs[32][32];
+  __shared__ double sc[kMaxG][kSmallCap];            // scores of the union's nodes, per head
+  __shared__ unsigned long long ms[kMaxG][kSmallCap]; // their fixed-point masses
+  __shared__ int uid[kSmallCap];                     // the union of the heads' candidates (ascending)
+  __shared__ unsigned int umask[kSmallCap];          // heads that have the union's node as candidate
+  __shared__ unsigned int hm[kSmallCap];             // head bits per node id (building the union)
+  __shared__ int kept[kMaxG][kSmallCap];             // each head's kept ids (ascending)
+  __shared__ int kcnt[kMaxG];
+  __shared__ unsigned int wtot[kSmallThreads / 32];
+  __shared__ int nu;
+  const RouteGeom& g = a.g;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const double scale = 1.0 / sqrt((double)kD);
+  const int64_t units = (int64_t)g.B * g.nq * g.Hkv;
+  const unsigned int all = (g.G >= 32) ? 0xffffffffu : ((1u << g.G) - 1u);
+  const int R = g.R;
+  constexpr int kVec = 16 / sizeof(KT);
+  constexpr int kNv = 32 / kVec;
+  for (int64_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const int64_t bq = u / g.Hkv;
+    const int hk = (int)(u % g.Hkv);
+    const int64_t b = bq / g.nq;
+    const int64_t qh0 = bq * g.Hq + (int64_t)hk * g.G;
+    const int64_t t = query_pos(g.q_pos, g.pos_uniform, bq);
+    const int top = pos_ok(g, t) ? top_level(g, t) : 0;
+    __syncthreads();                                     // shared memory of the previous unit
+    if (!pos_ok(g, t) && tid == 0) set_status(a.dev_status, ZHA_ERR_INVALID_ARG);
+    // fused levels above the query's top level: empty selections
+    if (a.level_cnt && tid < g.G)
+      for (int l = a.l_hi; l >= a.l_lo && l > top; --l) {
+        int* lc = a.level_cnt + ((qh0 + tid) * g.depth + (l - 1)) * 2;
+        lc[0] = 0;
+        lc[1] = 0;
+      }
+    if (top < a.l_lo) continue;                          // the per-level launches start at its top
+    for (int i = tid; i < 32 * 32; i += kSmallThreads) {
+      const int s2 = i / 32, L = i % 32, h = L >> 2;
+      const KT* q = reinterpret_cast<const KT*>(a.Q) + qh0 * kD;
+      qfs[s2][L] = h < g.G ? to_f64(q[h * kD + 32 * (L & 3) + s2]) : 0.0;
+    }
+    for (int l = top < a.l_hi ? top : a.l_hi; l >= a.l_lo; --l) {
+      const int64_t nvis = visible_nodes(t, g.span[l]);  // <= n_cap(l) <= kSmallCap
+      const bool at_top = l == top;
+      const int64_t orph_lo = at_top ? 0 : visible_nodes(t, g.span[l + 1]) * g.branch;
+      // ---- the union of the heads' candidates with their head bits
+      for (int i = tid; i < kSmallCap; i += kSmallThreads) hm[i] = 0u;
+      __syncthreads();
+      if (at_top) {
+        for (int i = tid; i < nvis; i += kSmallThreads) hm[i] = all;
+      } else {
+        for (int h = warp; h < g.G; h += kSmallThreads / 32)
+          for (int k = lane; k < kcnt[h] * g.branch; k += 32) {
+            const int id = kept[h][k / g.branch] * g.branch + k % g.branch;
+            if (id < kSmallCap) atomicOr(&hm[id], 1u << h);
+          }
+        for (int64_t i = orph_lo + tid; i < nvis; i += kSmallThreads) hm[i] = all;
+      }
+      __syncthreads();
+      {
+        const bool on = tid < kSmallCap && hm[tid] != 0u;
+        const unsigned int bal = __ballot_sync(0xffffffffu, on);
+        if (lane == 0) wtot[warp] = __popc(bal);
+        __syncthreads();
+        unsigned int before = __popc(bal & ((1u << lane) - 1u));
+        for (int w = 0; w < warp; ++w) before += wtot[w];
+        if (on) { uid[before] = tid; umask[before] = hm[tid]; }
+        if (tid == 0) {
+          unsigned int tot = 0;
+          for (int w = 0; w < kSmallThreads / 32; ++w) tot += wtot[w];
+          nu = (int)tot;
+        }
+      }
+      __syncthreads();
+      // ---- scores: groups of 8 union nodes x 8 heads on the fp64 tensor cores
+      const int64_t node0 = (b * g.Hkv + hk) * g.ncap[l];
+      const int h0 = 2 * (lane & 3), h1 = h0 + 1;
+      for (int grp = warp; grp * 8 < nu; grp += kSmallThreads / 32) {
+        const int pos = grp * 8 + (lane >> 2);
+        const bool has = pos < nu;
+        const int id = has ? uid[pos] : 0;
+        const unsigned int m = has ? umask[pos] : 0u;
+        double best0 = -INFINITY, best1 = -INFINITY;
+        for (int r0 = 0; r0 < R; r0 += 4) {
+          // the rows of up to four references load together (one memory latency per four)
+          constexpr int kRb = 4;
+          uint4 v[kRb][kNv];
+          float bh[kRb];
+#pragma unroll
+          for (int rr = 0; rr < kRb; ++rr) {
+            const bool on = m && r0 + rr < R;
+            const uint4* src = reinterpret_cast<const uint4*>(
+                reinterpret_cast<const KT*>(a.k_route[l]) + ((node0 + id) * R + r0 + rr) * kD + 32 * (lane & 3));
+#pragma unroll
+            for (int i = 0; i < kNv; ++i) v[rr][i] = on ? __ldg(src + i) : make_uint4(0, 0, 0, 0);
+            bh[rr] = on ? __ldg(a.b_hat[l] + (node0 + id) * R + r0 + rr) : 0.f;
+          }
+#pragma unroll
+          for (int rr = 0; rr < kRb; ++rr) {
+            if (r0 + rr >= R) break;
+            double c0[4] = {0.0, 0.0, 0.0, 0.0}, c1[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll
+            for (int s2 = 0; s2 < 32; ++s2) {
+              const double av = (double)u4_elem<KT>(v[rr][s2 / kVec], s2 % kVec);
+              mma_f64(c0[s2 & 3], c1[s2 & 3], av, qfs[s2][lane]);
+            }
+            const double bb = (double)bh[rr];
+            best0 = fmax(best0, fma((c0[0] + c0[1]) + (c0[2] + c0[3]), scale, bb));
+            best1 = fmax(best1, fma((c1[0] + c1[1]) + (c1[2] + c1[3]), scale, bb));
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+          const int h = q ? h1 : h0;
+          if (h < g.G && ((m >> h) & 1u)) {
+            double s = q ? best1 : best0;
+            if (s == 0.0) s = 0.0;                       // one zero (no -0.0) for the key order
+            sc[h][pos] = s;
+          }
+        }
+      }
+      __syncthreads();
+      // ---- the cutoff of each head (warp h)
+      if (warp < g.G) {
+        const int h = warp;
+        const int64_t qh = qh0 + h;
+        const unsigned int hb = 1u << h;
+        int n_h = 0;
+        double M = -INFINITY;
+        for (int i = lane; i < nu; i += 32)
+          if (umask[i] & hb) { ++n_h; M = fmax(M, sc[h][i]); }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          n_h += __shfl_xor_sync(0xffffffffu, n_h, o);
+          M = fmax(M, __shfl_xor_sync(0xffffffffu, M, o));
+        }
+        unsigned long long Z = 0;
+        for (int i = lane; i < nu; i += 32)
+          if (umask[i] & hb) {
+            const unsigned long long e = a.topk[l] > 0 ? 1ull : mass_of(sc[h][i], M, a.mass_shift);
+            ms[h][i] = e;
+            Z += e;
+          }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+        __syncwarp();
+        const bool keep_all = n_h == 0 || (a.topk[l] > 0 ? a.topk[l] >= n_h : a.p[l] >= 1.0);
+        unsigned long long tgt = 0;
+        if (!keep_all)
+          tgt = a.topk[l] > 0 ? ((unsigned long long)a.topk[l] < Z ? (unsigned long long)a.topk[l] : Z)
+                              : target_of(a.p[l], Z);
+        int kc = 0;
+        for (int base = 0; base < nu; base += 32) {
+          const int i = base + lane;
+          bool keep = false;
+          if (i < nu && (umask[i] & hb)) {
+            keep = keep_all;
+            if (!keep) {
+              const double si = sc[h][i];
+              unsigned long long before = 0;             // mass of the candidates ordered before i
+              for (int j = 0; j < nu; ++j)
+                if ((umask[j] & hb) && (sc[h][j] > si || (sc[h][j] == si && j < i))) before += ms[h][j];
+              keep = before < tgt;
+            }
+          }
+          const unsigned int bal = __ballot_sync(0xffffffffu, keep);
+          if (keep) {
+            const int at = kc + __popc(bal & ((1u << lane) - 1u));
+            const int id = uid[i];
+            kept[h][at] = id;
+            if (a.level_ids) a.level_ids[qh * a.level_ids_stride + a.level_ids_off[l] + at] = id;
+            if (l == a.l_lo) a.out_ids[qh * a.out_stride + at] = id;
+          }
+          kc += __popc(bal);
+        }
+        if (lane == 0) {
+          kcnt[h] = kc;
+          if (a.level_cnt) {
+            int* lc = a.level_cnt + (qh * g.depth + (l - 1)) * 2;
+            lc[0] = n_h;
+            lc[1] = kc;
+          }
+          if (l == a.l_lo) a.out_cnt[qh] = kc;
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
 #ifndef ZHA_WARP_SELECT_MAX
 #define ZHA_WARP_SELECT_MAX 256
 #endif
@@ -1808,6 +2034,34 @@ static cudaError_t route_levels(const RouteCall& c) {
   }
   for (int l = g.depth; l > lmax; --l)
     if (l >= 2) level_off -= ncap_of(g, l);
+  // the top levels whose frontier capacity is at most kSmallCap: one fused launch
+  int l_lo = lmax + 1;
+  for (int l = lmax; l >= 2 && ncap_of(g, l) <= kSmallCap; --l) l_lo = l;
+  if (l_lo <= lmax) {
+    SmallArgs sm{};
+    sm.g = rg; sm.l_lo = l_lo; sm.l_hi = lmax; sm.Q = c.Q;
+    int64_t off = 0;
+    for (int l = 2; l <= g.depth; ++l) { sm.level_ids_off[l] = off; off += ncap_of(g, l); }
+    for (int l = l_lo; l <= lmax; ++l) {
+      sm.k_route[l] = (char*)c.tree + L.lv[l].k_route_off;
+      sm.b_hat[l] = (const float*)((char*)c.tree + L.lv[l].b_hat_off);
+      sm.p[l] = c.p_levels ? c.p_levels[l - 1] : c.p;
+      sm.topk[l] = c.k_levels ? c.k_levels[l - 1] : 0;
+    }
+    sm.mass_shift = mass_shift_for(w.C1);
+    sm.out_ids = selbuf[l_lo & 1]; sm.out_cnt = selcnt[l_lo & 1]; sm.out_stride = w.C2;
+    sm.level_cnt = c.level_cnt; sm.level_ids = c.level_ids; sm.level_ids_stride = level_ids_stride;
+    sm.dev_status = c.dev_status;
+    const int64_t units = (int64_t)g.B * c.nq * g.Hkv;
+    trace_begin(ZHA_TRACE_ROUTE_FUSED, c.stream);
+    route_small_kernel<KT><<<grid_for(units, 4), kSmallThreads, 0, c.stream>>>(sm);
+    trace_end(ZHA_TRACE_ROUTE_FUSED, c.stream);
+    count_launch();
+    cudaError_t e = launch_status("route_small_kernel");
+    if (e != cudaSuccess) return e;
+    for (int l = lmax; l >= l_lo; --l) level_off -= ncap_of(g, l);
+    lmax = l_lo - 1;
+  }
   for (int l = lmax; l >= 1; --l) {
     const int cur = l & 1, prev = (l + 1) & 1;
     ScoreArgs sa{};

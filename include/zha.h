@@ -349,9 +349,11 @@ const char* zha_last_error(void);
 /* Measurement hook.  Kernel ids for zha_trace. */
 typedef enum zha_trace_kernel {
   ZHA_TRACE_ATTN = 1,        /* the split-KV gather kernel of the sparse / dense attention */
-  ZHA_TRACE_ROUTE_SCORE = 2, /* the routing score kernel (every level); the flat indexer's
-                                chunk scores                                                */
-  ZHA_TRACE_ROUTE_SELECT = 3 /* the routing top-p select kernels (every level; both kinds)  */
+  ZHA_TRACE_ROUTE_SCORE = 2, /* the routing score kernel (every level launched on its own);
+                                the flat indexer's chunk scores                             */
+  ZHA_TRACE_ROUTE_SELECT = 3, /* the routing top-p select kernels (every level; both kinds) */
+  ZHA_TRACE_ROUTE_FUSED = 4   /* the fused score + select of the small top levels of the tree
+                                 (levels of at most 64 nodes per (b, h_kv)), one launch      */
 } zha_trace_kernel;
 
 /* Until n launches of kernel `which` have been traced, record start[i] just before and

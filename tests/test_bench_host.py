@@ -164,3 +164,28 @@ def test_oracle_pool_parity_check_on_cpu():
         assert got["exact"] == w.Hq - 1 and got["failed"] + got["near_cutoff_mismatch"] == 1
     finally:
         pool.close()
+
+
+def test_paper_model_with_the_fused_top_levels():
+    """Lines whose small top levels share one fused launch: the per-level lists start at the
+    first level launched on its own, and the fused levels form one row."""
+    line = {"dtype": "bf16", "steps": 10, "gpu_launches": 80,
+            "config": {"workload": "w", "B": 4, "Hq": 32, "Hkv": 4, "d": 128, "R": 4, "T": 1 << 20,
+                       "leaf": 64, "branch": 16, "depth": 5},
+            "frontier": {"levels": [
+                {"level": 4, "candidates_mean": 4.0, "candidates_max": 4},
+                {"level": 3, "candidates_mean": 64.0, "candidates_max": 64},
+                {"level": 2, "candidates_mean": 976.0, "candidates_max": 976},
+                {"level": 1, "candidates_mean": 14700.0, "candidates_max": 14750}]},
+            "stages_ms": {"route_fused": 0.01, "route_fused_per_launch": [0.01],
+                          "route_score_per_launch": [0.02, 0.15], "route_select_per_launch": [0.015, 0.04],
+                          "attention": 1.2, "step": 1.5, "stage_sum": 1.435},
+            "kv_touched": {"mean": 0.8}, "tree_build": {"ms": 3.6},
+            "roofline": {"algorithmic_bytes_per_launch": 8e9, "launches_per_step": 1.0}}
+    m = bench.paper_model(line, {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0})
+    rows = {r["stage"]: r for r in m["rows"]}
+    assert rows["route fused L4..L3"]["measured_ms"] == 0.01
+    assert rows["route score L2"]["measured_ms"] == 0.02 and rows["route score L1"]["measured_ms"] == 0.15
+    assert rows["route select L1"]["measured_ms"] == 0.04
+    assert "route score L4" not in rows and "route score L3" not in rows
+    assert m["launch_gaps_ms"] == pytest.approx(1.5 - 1.435)
