@@ -198,9 +198,9 @@ class ClockSampler:
 # gather kernel, from an ncu capture of the batched 128K decode at batch 4 (16 of its 128 KV
 # units), valid while the kernel source is the one that was captured.
 PROFILED_TRAFFIC = {
-    "batched-decode-128k": {"bytes": 1.075072e9 + 11.166976e6, "units": 16,
+    "batched-decode-128k": {"bytes": 1.075083776e9 + 11.032576e6, "units": 16,
                             "source": "hierarchical_sparse_attention_02_b200/csrc/zha_attn_tc.cu",
-                            "sha1": "7cd49e01f798c1e4020732017f021f6d675035d1"},
+                            "sha1": "66fb0e96b0d9ccbdee5e0bc5c25088c89c77ee09"},
 }
 
 
