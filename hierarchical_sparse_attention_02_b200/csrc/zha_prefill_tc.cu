@@ -12,7 +12,7 @@
 // union the kernel computes, for each sub-tile,
 //     S[128 x 64]  = Q_tile . K_chunk^T     (tcgen05.mma kind::f16, bf16 in, fp32 in TMEM)
 //     P            = exp2(S * log2(e)/sqrt(d) - m)  per row, masked to the row's own keys
-//     O[128 x 128] += P . V_chunk           (tcgen05.mma, P from shared memory, O in TMEM)
+//     O[128 x 128] += P . V_chunk           (tcgen05.mma, P from TMEM, O in TMEM)
 // with an online softmax per row whose running maximum is raised lazily (O in TMEM is
 // rescaled only when a row's maximum grows by more than 2^8).  A row sees key j of chunk c
 // iff c is in its S_1, or j = 0, or c is its own chunk and j <= t.
@@ -22,9 +22,11 @@
 //              of each chunk and the output dims [64 h, 64 h + 64) for h = (w / 4) % 2, and
 //              the rows 32 (w % 4) + lane (= its TMEM lanes); the two threads of a row share
 //              their maxima through shared memory and a named barrier (sub-tile u owns TMEM
-//              columns [256 u, 256 u + 256));
+//              columns [256 u, 256 u + 256)); each thread writes its 32 weights of P as
+//              bf16 pairs over the first 16 of the 32 S columns it has just read, where the
+//              P . V MMA reads them as its A operand;
 //   warp 16    producer: TMA loads of the Q sub-tiles (4-D map) and of each chunk's K and V
-//              (3-D maps, 128-byte swizzle) into a 3-stage ring; this GPU's memory only,
+//              (3-D maps, 128-byte swizzle) into a 4-stage ring; this GPU's memory only,
 //              no multicast;
 //   warp 17    TMEM allocation; lane 0 issues the MMAs and their commits.
 // Every wait is bounded; a wait that gives up reports ZHA_ERR_DEVICE, the CTA stops, waits
@@ -43,12 +45,11 @@ using namespace ptx;
 
 constexpr int kRows = 128;                       // MMA M: rows of a sub-tile
 constexpr int kSub = 2;                          // sub-tiles per tile
-constexpr int kStages = 3;                       // K/V ring depth
+constexpr int kStages = 4;                       // K/V ring depth
 constexpr int kBox = 64 * 128;                   // 64 rows x 128 bytes
 constexpr int kKVBytes = 4 * kBox;               // K dims 0-63 | 64-127, V dims 0-63 | 64-127
 constexpr int kQHalf = kRows * 128;              // 128 rows x 64 dims of Q
-constexpr int kPBytes = kRows * 128;             // 128 rows x 64 keys of P (bf16)
-constexpr uint32_t kTmemCols = 512;              // per sub-tile: S0, S1 (64 each), O (128)
+constexpr uint32_t kTmemCols = 512;              // per sub-tile: S0, S1 (64 each, P over them), O (128)
 constexpr uint32_t kSubCols = 256;
 constexpr uint32_t kColO = 128;
 constexpr int kHalves = 2;                      // softmax threads per row (32 of its 64 keys each)
@@ -62,12 +63,11 @@ constexpr uint32_t kIdescPV = idesc_bf16(128, 128, 1); // O += P . V, V MN-major
 struct alignas(1024) Smem {
   unsigned char q[kSub][2][kQHalf];              // per sub-tile two 128B-swizzled boxes [128 rows][64 dims]
   unsigned char kv[kStages][kKVBytes];
-  unsigned char p[kSub][kPBytes];                // [128 rows][64 keys], 128B swizzle
   uint4 meta_mask[kStages][kSub];                // rows of each sub-tile that selected the chunk
   int meta_id[kStages];                          // chunk id of each stage
   unsigned long long full[kStages], empty[kStages];
   unsigned long long q_full, q_empty;
-  unsigned long long s_full[kSub][2], s_free[kSub][2], p_full[kSub][2], pv_done[kSub][2];
+  unsigned long long s_full[kSub][2], p_full[kSub][2], pv_done[kSub][2];
   unsigned long long o_free[kSub], drain;
   float xmax[2][kSub][kHalves][kRows];           // row maxima (per entry) and sums (epilogue) of the
                                                  // two halves of a row, by entry parity
@@ -108,24 +108,45 @@ __device__ __forceinline__ int tile_entries(const Args& a, int64_t tile) {
   return n;
 }
 
-// The e-th entry of a tile (ranges in order): its slot in the entry arrays.
-struct EntryWalk {
-  int64_t base, r, e, cnt;
+// Up to 32 consecutive entries of one range of a tile, one per lane (nb = how many).
+struct Batch {
+  int c, nb;
+  uint4 m0, m1;
+};
+
+// Walks a tile's entries in batches of at most 32 within one range.
+struct BatchWalk {
+  int64_t base, r, e0, cnt;
   __device__ void start(const Args& a, int64_t tile) {
     base = tile * a.nr;
     r = 0;
-    e = 0;
+    e0 = 0;
     cnt = a.ent_cnt[base];
     while (cnt == 0 && r + 1 < a.nr) { ++r; cnt = a.ent_cnt[base + r]; }
   }
-  __device__ int64_t slot() const { return (base + r) * kRange + e; }
-  __device__ void next(const Args& a) {
-    if (++e >= cnt) {
-      e = 0;
-      do { ++r; cnt = r < a.nr ? a.ent_cnt[base + r] : 0; } while (cnt == 0 && r + 1 < a.nr);
+  // the next batch (nb = 0 once the tile's entries are exhausted); every lane calls it
+  __device__ Batch load(const Args& a, int lane) {
+    Batch b;
+    b.nb = e0 < cnt ? (int)(cnt - e0 < 32 ? cnt - e0 : 32) : 0;
+    b.c = 0;
+    b.m0 = b.m1 = make_uint4(0u, 0u, 0u, 0u);
+    if (lane < b.nb) {
+      const int64_t slot = (base + r) * kRange + e0 + lane;
+      b.c = a.ent_ids[slot];
+      b.m0 = a.ent_mask[slot * kSub];
+      b.m1 = a.ent_mask[slot * kSub + 1];
     }
+    if (b.nb > 0) {
+      e0 += 32;
+      if (e0 >= cnt) {
+        e0 = 0;
+        do { ++r; cnt = r < a.nr ? a.ent_cnt[base + r] : 0; } while (cnt == 0 && r + 1 < a.nr);
+      }
+    }
+    return b;
   }
 };
+static_assert(kSub == 2, "a batch carries the row masks of two sub-tiles");
 
 __device__ __forceinline__ bool warp_wait(unsigned long long* b, uint32_t parity, int* abort) {
   const bool ok = __all_sync(0xffffffffu, mbar_wait_sleep(b, parity, abort));
@@ -158,7 +179,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     for (int u = 0; u < kSub; ++u) {
       for (int i = 0; i < 2; ++i) {
         mbar_init(&sm.s_full[u][i], 1);
-        mbar_init(&sm.s_free[u][i], 4 * kHalves);
         mbar_init(&sm.p_full[u][i], 4 * kHalves);
         mbar_init(&sm.pv_done[u][i], 1);
       }
@@ -177,51 +197,69 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ producer
+    // The whole warp reads the entries' chunk ids and row masks 32 at a time (one coalesced
+    // load per lane, the next batch in flight while this one is issued); lane 0 waits for
+    // the ring slots and issues the TMA copies.
     if (lane == 0) {
       prefetch_tensormap(&qmap);
       prefetch_tensormap(&kmap);
       prefetch_tensormap(&vmap);
-      const uint32_t q_tx = (uint32_t)(kSub * 2 * 128 * a.G * a.Qt);
-      long long it = 0, nq_loads = 0;
-      long long issued[kStages] = {};
-      bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
-        const Tile t = tile_of(a, tile);
+    }
+    const uint32_t q_tx = (uint32_t)(kSub * 2 * 128 * a.G * a.Qt);
+    long long it = 0, nq_loads = 0;
+    long long issued[kStages] = {};
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x) {
+      const Tile t = tile_of(a, tile);
+      int okw = 1;
+      if (lane == 0) {
         if (nq_loads > 0 && !mbar_wait_sleep(&sm.q_empty, (uint32_t)((nq_loads - 1) & 1), &sm.abort)) {
-          give_up(sm, a.dev_status);
-          break;
-        }
-        mbar_arrive_tx(&sm.q_full, q_tx);
-        for (int u = 0; u < kSub; ++u) {           // a sub-tile past nq reads the fill value (0)
-          tma_load_4d(sm.q[u][0], &qmap, 0, t.hk * a.G, t.q0 + u * a.Qt, t.b, &sm.q_full);
-          tma_load_4d(sm.q[u][1], &qmap, 64, t.hk * a.G, t.q0 + u * a.Qt, t.b, &sm.q_full);
-        }
-        ++nq_loads;
-        const int n = tile_entries(a, tile);
-        EntryWalk w;
-        w.start(a, tile);
-        for (int i = 0; i < n; ++i, ++it, w.next(a)) {
-          const int s = (int)(it % kStages);
-          if (it >= kStages && !mbar_wait_sleep(&sm.empty[s], (uint32_t)(((it / kStages) - 1) & 1), &sm.abort)) {
-            give_up(sm, a.dev_status);
-            ok = false;
-            break;
+          okw = 0;
+        } else {
+          mbar_arrive_tx(&sm.q_full, q_tx);
+          for (int u = 0; u < kSub; ++u) {         // a sub-tile past nq reads the fill value (0)
+            tma_load_4d(sm.q[u][0], &qmap, 0, t.hk * a.G, t.q0 + u * a.Qt, t.b, &sm.q_full);
+            tma_load_4d(sm.q[u][1], &qmap, 64, t.hk * a.G, t.q0 + u * a.Qt, t.b, &sm.q_full);
           }
-          const int64_t slot = w.slot();
-          const int c = a.ent_ids[slot];
-          sm.meta_id[s] = c;
-#pragma unroll
-          for (int u = 0; u < kSub; ++u) sm.meta_mask[s][u] = a.ent_mask[slot * kSub + u];
-          mbar_arrive_tx(&sm.full[s], (uint32_t)kKVBytes);
-          unsigned char* st = sm.kv[s];
-          const int z = (int)t.unit;
-          tma_load_3d(st + 0 * kBox, &kmap, 0, c * kLeaf, z, &sm.full[s]);
-          tma_load_3d(st + 1 * kBox, &kmap, 64, c * kLeaf, z, &sm.full[s]);
-          tma_load_3d(st + 2 * kBox, &vmap, 0, c * kLeaf, z, &sm.full[s]);
-          tma_load_3d(st + 3 * kBox, &vmap, 64, c * kLeaf, z, &sm.full[s]);
-          ++issued[s];
         }
       }
+      if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
+      ++nq_loads;
+      BatchWalk w;
+      w.start(a, tile);
+      Batch cur = w.load(a, lane), nxt = w.load(a, lane);
+      while (cur.nb > 0 && ok) {
+        for (int k = 0; k < cur.nb; ++k, ++it) {
+          const int s = (int)(it % kStages);
+          okw = 1;
+          if (lane == 0 && it >= kStages &&
+              !mbar_wait_sleep(&sm.empty[s], (uint32_t)(((it / kStages) - 1) & 1), &sm.abort))
+            okw = 0;
+          if (!__shfl_sync(0xffffffffu, okw, 0)) { ok = false; break; }
+          if (lane == k) {                         // the entry's owner lane publishes its metadata
+            sm.meta_id[s] = cur.c;
+            sm.meta_mask[s][0] = cur.m0;
+            sm.meta_mask[s][1] = cur.m1;
+          }
+          const int c = __shfl_sync(0xffffffffu, cur.c, k);
+          __syncwarp();                            // the metadata is written before the arrival
+          if (lane == 0) {
+            mbar_arrive_tx(&sm.full[s], (uint32_t)kKVBytes);
+            unsigned char* st = sm.kv[s];
+            const int z = (int)t.unit;
+            tma_load_3d(st + 0 * kBox, &kmap, 0, c * kLeaf, z, &sm.full[s]);
+            tma_load_3d(st + 1 * kBox, &kmap, 64, c * kLeaf, z, &sm.full[s]);
+            tma_load_3d(st + 2 * kBox, &vmap, 0, c * kLeaf, z, &sm.full[s]);
+            tma_load_3d(st + 3 * kBox, &vmap, 64, c * kLeaf, z, &sm.full[s]);
+            ++issued[s];
+          }
+        }
+        cur = nxt;
+        nxt = w.load(a, lane);
+      }
+    }
+    if (lane == 0) {
+      if (!ok) give_up(sm, a.dev_status);
       // drain: no copy may land after the CTA exits (bounded, independent of `abort`)
       for (int s = 0; s < kStages; ++s)
         if (issued[s] > 0 && !mbar_wait(&sm.full[s], (uint32_t)((issued[s] - 1) & 1), &sm.zero))
@@ -234,8 +272,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     if (lane == 0) {
       long long j = 0, tl = 0;                   // entries and tiles of this CTA so far
       bool ok = true;
+      // S of entry e overwrites the columns that held S and then P of entry e - 2: it waits
+      // until the P . V MMA of e - 2 (issued after its P was written) has completed
       auto issue_s = [&](int u, long long e) -> bool {
-        if (e >= 2 && !mbar_wait_sleep(&sm.s_free[u][e & 1], (uint32_t)(((e >> 1) - 1) & 1), &sm.abort)) return false;
+        if (e >= 2 && !mbar_wait_sleep(&sm.pv_done[u][e & 1], (uint32_t)(((e >> 1) - 1) & 1), &sm.abort)) return false;
         tc_fence_after();
         const uint32_t qa = smem_u32(sm.q[u][0]);
         const uint32_t ka = smem_u32(sm.kv[e % kStages]);
@@ -251,12 +291,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         if (!mbar_wait_sleep(&sm.p_full[u][e & 1], (uint32_t)((e >> 1) & 1), &sm.abort)) return false;
         if (first_of_tile && tl > 0 && !mbar_wait_sleep(&sm.o_free[u], (uint32_t)((tl - 1) & 1), &sm.abort)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sm.p[u]);
+        // P of keys [16 kk, 16 kk + 16): columns 8 (kk % 2) of the S half 32 (kk / 2)
+        const uint32_t pa = tmem + u * kSubCols + (uint32_t)(e & 1) * 64;
         const uint32_t va = smem_u32(sm.kv[e % kStages] + 2 * kBox);
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-          umma_bf16(tmem + u * kSubCols + kColO, sw128_desc(pa + kk * 32, 16, 1024),
-                    sw128_desc(va + kk * 2048, kBox, 1024), kIdescPV, (first_of_tile && kk == 0) ? 0u : 1u);
+          umma_bf16_ts(tmem + u * kSubCols + kColO, pa + (uint32_t)((kk >> 1) * 32 + (kk & 1) * 8),
+                       sw128_desc(va + kk * 2048, kBox, 1024), kIdescPV, (first_of_tile && kk == 0) ? 0u : 1u);
         umma_commit(&sm.pv_done[u][e & 1]);
         return true;
       };
@@ -321,9 +362,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         float x[32];
         tmem_ld32(lane_addr + (uint32_t)(j & 1) * 64 + s_col, x);
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.s_free[u][j & 1]);
         // visibility of the chunk's keys for this row: all of them (a selected chunk), the
         // keys up to t (its own chunk), key 0 (chunk 0), or none; this thread holds keys
         // 32 hf + k
@@ -331,15 +369,22 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         const bool sel = valid && (wsel & mbit) && c < cur;
         const bool own = valid && c == cur;
         const int lim = (sel ? 63 : (own ? (int)(pos - (int64_t)c * kLeaf) : (valid && c == 0 ? 0 : -1))) - 32 * hf;
+        // A row sees all 32 of this thread's keys (lim >= 31) or none of them (lim < 0) on
+        // every entry but its own chunk and chunk 0; only those few entries mask key by key.
+        if (__any_sync(0xffffffffu, lim >= 0 && lim < 31)) {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) x[k] = k <= lim ? x[k] : -INFINITY;
+        }
         float mx;
         {
-          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // independent max chains
+          float m4[4];                                 // independent chains of 3-input maxima
 #pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            x[k] = k <= lim ? x[k] : -INFINITY;
-            m4[k & 3] = fmaxf(m4[k & 3], x[k]);
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const float* y = x + 8 * c4;
+            m4[c4] = fmax3(fmax3(y[0], y[1], y[2]), fmax3(y[3], y[4], y[5]), fmaxf(y[6], y[7]));
           }
-          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;   // log2 units (-inf stays)
+          mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]) * sl2;   // log2 units (-inf stays)
+          if (lim < 0) mx = -INFINITY;               // the row sees none of these keys
         }
         // the row maximum over both halves
         sm.xmax[j & 1][u][hf][r] = mx;
@@ -368,30 +413,30 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
           if (grow) { l *= alpha; m = mx; }
         }
         if (m == -INFINITY) m = mx;                // first visible key of the row (O is zero)
-        const float mu = m == -INFINITY ? 0.f : m;
+        // subtrahend of the exponents: the running maximum, or +inf where the row sees none
+        // of these keys (every weight 0)
+        const float mu = lim < 0 ? INFINITY : (m == -INFINITY ? 0.f : m);
         uint32_t pw[16];                           // P (bf16 pairs) of this thread's 32 keys
-        float ps[4] = {0.f, 0.f, 0.f, 0.f};        // four independent sum chains
+        const unsigned long long sl2x2 = f2_pack(sl2, sl2), nmu2 = f2_pack(-mu, -mu);
+        unsigned long long ps2[2] = {0ull, 0ull};  // two independent chains of packed sums
 #pragma unroll
         for (int q = 0; q < 16; ++q) {
-          // 2^(x * log2(e)/sqrt(d) - mu); a masked key (-inf) gives 0
-          const float p0 = ex2(fmaf(x[2 * q], sl2, -mu)), p1 = ex2(fmaf(x[2 * q + 1], sl2, -mu));
+          // 2^(x * log2(e)/sqrt(d) - mu) for a pair of keys; a masked key (-inf) gives 0
+          float e0, e1;
+          f2_unpack(f2_fma(f2_pack(x[2 * q], x[2 * q + 1]), sl2x2, nmu2), e0, e1);
+          const float p0 = ex2(e0), p1 = ex2(e1);
           pw[q] = pack_bf16(p0, p1);
-          ps[q & 3] += p0 + p1;                    // the log-sum-exp from the unrounded weights
+          ps2[q & 1] = f2_add(ps2[q & 1], f2_pack(p0, p1));   // the sums of the unrounded weights
         }
-        l += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-        // the P buffer of this sub-tile is free once PV of entry j - 1 has completed
-        if (j >= 1 && !warp_wait(&sm.pv_done[u][(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
-          ok = false;
-          break;
+        {
+          float a0, a1, b0, b1;
+          f2_unpack(ps2[0], a0, a1);
+          f2_unpack(ps2[1], b0, b1);
+          l += (a0 + b0) + (a1 + b1);
         }
-        unsigned char* prow = sm.p[u] + r * 128;
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int chunk = hf * 4 + ch;           // 16-byte chunk of the row (8 keys)
-          *reinterpret_cast<uint4*>(prow + ((chunk ^ (r & 7)) << 4)) =
-              make_uint4(pw[4 * ch], pw[4 * ch + 1], pw[4 * ch + 2], pw[4 * ch + 3]);
-        }
-        fence_proxy_async_smem();
+        // P over the first 16 of the 32 S columns this thread has read
+        tmem_st16(lane_addr + (uint32_t)(j & 1) * 64 + s_col, pw);
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.p_full[u][j & 1]);
