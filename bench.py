@@ -195,9 +195,13 @@ class ClockSampler:
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of the attention
-# gather kernel, from an ncu capture of the batched 128K decode at batch 4 (16 of its 128 KV
-# units), valid while the kernel source is the one that was captured.
+# gather kernel, from ncu captures of the 1M-token decode at batch 1 (4 of its 16 KV units)
+# and of the batched 128K decode at batch 4 (16 of its 128 KV units), each valid while the
+# kernel source is the one that was captured.
 PROFILED_TRAFFIC = {
+    "long-decode-1m": {"bytes": 2.149206784e9 + 18.750208e6, "units": 4,
+                       "source": "hierarchical_sparse_attention_02_b200/csrc/zha_attn_tc.cu",
+                       "sha1": "66fb0e96b0d9ccbdee5e0bc5c25088c89c77ee09"},
     "batched-decode-128k": {"bytes": 1.075083776e9 + 11.032576e6, "units": 16,
                             "source": "hierarchical_sparse_attention_02_b200/csrc/zha_attn_tc.cu",
                             "sha1": "66fb0e96b0d9ccbdee5e0bc5c25088c89c77ee09"},
