@@ -281,8 +281,12 @@ def paper_model(line: dict, peaks: dict) -> dict:
 
     Per stage x, Phi_x = max(FLOPs_x / P_x, bytes_x / BW, t_waves).  The worker-wave term
     needs a per-block latency tau_x; it is calibrated here as the measured time of the same
-    kernel's launch at the top level, whose few candidates fit in one wave (so tau is the
-    kernel's fixed latency and the wave count is taken as 1).  Counts follow App. D-B1
+    kernel's launch at the highest level launched on its own when that level is above the
+    leaves (its few candidates fit in one wave, so tau is the kernel's fixed latency and the
+    wave count is taken as 1).  The fused launch of the small top levels is its own one-wave
+    calibration.  A line whose only separately launched level is the leaf level has no
+    one-wave launch of the score and select kernels: their wave term is then left out
+    (t_waves = 0).  Counts follow App. D-B1
     with this implementation's element sizes:
       routing, level l:  FLOPs = 2 B Hq R d K_l (every head scores its own candidates, on the
                          fp64 tensor cores here); bytes = R (s d + 4) B Hkv K_l^grp + s d B Hq
@@ -321,7 +325,7 @@ def paper_model(line: dict, peaks: dict) -> dict:
     score_ms = lambda l: per_s[first - l] if l <= first else None      # noqa: E731
     select_ms = lambda l: per_x[first - l] if l <= first else None     # noqa: E731
     sep_top = min(top, first)
-    tau = {"score": score_ms(sep_top), "select": select_ms(sep_top)}
+    tau = {"score": score_ms(sep_top), "select": select_ms(sep_top)} if sep_top > 1 else {}
 
     def row(stage, kind, flops, byts, peak, unit, measured):
         t_f, t_b = 1e3 * flops / peak, 1e3 * byts / bw
@@ -347,9 +351,10 @@ def paper_model(line: dict, peaks: dict) -> dict:
     if fused:
         rows.insert(0, {"stage": f"route fused L{top}..L{first + 1}", "flops": sum(r["flops"] for r in fused),
                         "bytes": sum(r["bytes"] for r in fused), "flops_ms": sum(r["flops_ms"] for r in fused),
-                        "bytes_ms": sum(r["bytes_ms"] for r in fused), "waves_ms": 0.0,
-                        "model_ms": max(r["model_ms"] for r in fused), "bound": "latency (one wave)",
-                        "measured_ms": fused_ms})
+                        "bytes_ms": sum(r["bytes_ms"] for r in fused), "waves_ms": fused_ms,
+                        "model_ms": max(sum(r["flops_ms"] for r in fused), sum(r["bytes_ms"] for r in fused),
+                                        fused_ms),
+                        "bound": "latency (one wave)", "measured_ms": fused_ms})
     T1 = cfg["T"] + 1
     k0 = line["kv_touched"]["mean"] * T1
     byts = line["roofline"]["algorithmic_bytes_per_launch"] * line["roofline"]["launches_per_step"]
