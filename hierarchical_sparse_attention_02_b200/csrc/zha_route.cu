@@ -76,6 +76,7 @@ route_score_kernel(ScoreArgs a) {
   __shared__ __align__(16) double qfs[32][32];
   __shared__ int rank[kScoreSlots][kMaxG];       // per parent slot: rank in each head's list
   __shared__ int pcnt[kMaxG];
+  __shared__ int n_kept;                         // kept parents of this item, over all heads
   const RouteGeom& g = a.g;
   const int tid = threadIdx.x;
   const int64_t units = (int64_t)g.B * g.nq * g.Hkv;
@@ -116,12 +117,7 @@ route_score_kernel(ScoreArgs a) {
     }
     __syncthreads();                                     // smem reuse across items
     if (tid < g.G) pcnt[tid] = at_top ? 0 : a.parents_cnt[qh0 + tid];
-    // B fragments of the mma: qfs[s][L] = q[head L/4][32 * (L%4) + s] (0 for heads >= G)
-    for (int i = tid; i < 32 * 32; i += kThreads) {
-      const int s2 = i / 32, L = i % 32, h = L >> 2;
-      const KT* q = reinterpret_cast<const KT*>(a.Q) + qh0 * kD;
-      qfs[s2][L] = h < g.G ? to_f64(q[h * kD + 32 * (L & 3) + s2]) : 0.0;
-    }
+    if (tid == 0) n_kept = 0;
     __syncthreads();
     if (blk == 0 && tid < g.G)
       a.cand_cnt[qh0 + tid] = (int)(at_top ? nvis : (int64_t)pcnt[tid] * g.branch + (nvis - orph_lo));
@@ -138,15 +134,29 @@ route_score_kernel(ScoreArgs a) {
         const int* lst = a.parents + (qh0 + h) * a.C2;
         const int cnt = pcnt[h];
         const int x = warp_lower_bound(lst, cnt, p0);
+        int found = 0;
         for (int j = lane_; j < per_blk; j += 32) {
           if (x + j < cnt) {
             const int v = lst[x + j];
-            if (v < p0 + per_blk && v < npar) rank[v - p0][h] = x + j;
+            if (v < p0 + per_blk && v < npar) {
+              rank[v - p0][h] = x + j;
+              ++found;
+            }
           }
         }
+        if (found) atomicAdd(&n_kept, found);
       }
       __syncthreads();
+      // no head kept a parent of this item (sparse frontiers): nothing to score
+      if (n_kept == 0) continue;
     }
+    // B fragments of the mma: qfs[s][L] = q[head L/4][32 * (L%4) + s] (0 for heads >= G)
+    for (int i = tid; i < 32 * 32; i += kThreads) {
+      const int s2 = i / 32, L = i % 32, h = L >> 2;
+      const KT* q = reinterpret_cast<const KT*>(a.Q) + qh0 * kD;
+      qfs[s2][L] = h < g.G ? to_f64(q[h * kD + 32 * (L & 3) + s2]) : 0.0;
+    }
+    __syncthreads();
     // Scores on the fp64 tensor cores: each warp takes its 8*GPW slots as GPW groups of 8
     // nodes; D[8 nodes x 8 heads] += A[8 nodes x 4 dims] . B[4 dims x 8 heads] per
     // mma.m8n8k4.f64.  Lane L holds A[node L/4][dim 32*(L%4) + s] and B[dim][head L/4]
