@@ -189,3 +189,46 @@ def test_paper_model_with_the_fused_top_levels():
     assert rows["route select L1"]["measured_ms"] == 0.04
     assert "route score L4" not in rows and "route score L3" not in rows
     assert m["launch_gaps_ms"] == pytest.approx(1.5 - 1.435)
+
+
+def test_paper_model_wave_term_needs_a_one_wave_launch():
+    """The wave term of the score and select rows is calibrated from the highest level
+    launched on its own only when that level lies above the leaves.  When every level above
+    the leaves is fused, no launch of those kernels fits one wave: the level-1 rows keep only
+    their flop and byte terms.  The fused row takes its own launch as its wave term."""
+    line = {"dtype": "bf16", "steps": 10, "gpu_launches": 60,
+            "config": {"workload": "w", "B": 32, "Hq": 32, "Hkv": 4, "d": 128, "R": 4, "T": 1 << 17,
+                       "leaf": 64, "branch": 16, "depth": 3},
+            "frontier": {"levels": [
+                {"level": 3, "candidates_mean": 8.0, "candidates_max": 8},
+                {"level": 2, "candidates_mean": 128.0, "candidates_max": 128},
+                {"level": 1, "candidates_mean": 1936.0, "candidates_max": 1936,
+                 "candidates_group_union": 2048.0}]},
+            "stages_ms": {"route_fused": 0.06, "route_fused_per_launch": [0.06],
+                          "route_score_per_launch": [0.149], "route_select_per_launch": [0.045],
+                          "attention": 1.25, "step": 1.55, "stage_sum": 1.504},
+            "kv_touched": {"mean": 0.87}, "tree_build": {"ms": 3.6},
+            "roofline": {"algorithmic_bytes_per_launch": 8.6e9, "launches_per_step": 1.0}}
+    m = bench.paper_model(line, {"hbm_gbs": 6448.4, "bf16_tflops": 1725.8})
+    rows = {r["stage"]: r for r in m["rows"]}
+    fused = rows["route fused L3..L2"]
+    assert fused["waves_ms"] == 0.06 and fused["model_ms"] == pytest.approx(0.06)
+    score, select = rows["route score L1"], rows["route select L1"]
+    assert score["waves_ms"] == 0.0 and select["waves_ms"] == 0.0
+    # no wave term: the score row is its fp64 flops (2 B Hq R d K) over the fp64 tensor rate
+    flops = 2.0 * 32 * 32 * 4 * 128 * 1936.0
+    assert score["model_ms"] == pytest.approx(1e3 * flops / (bench.FP64_TENSOR_TFLOPS * 1e12))
+    assert score["bound"] == "fp64 tensor"
+    # the select row is its bytes (12 B Hq K) over the copy bandwidth
+    assert select["model_ms"] == pytest.approx(1e3 * 12.0 * 32 * 32 * 1936.0 / (6448.4e9))
+    assert select["bound"] == "hbm"
+    # a line whose highest separate level lies above the leaves does calibrate from it
+    line2 = dict(line)
+    line2["config"] = dict(line["config"], depth=3)
+    line2["stages_ms"] = dict(line["stages_ms"], route_fused=0.0, route_fused_per_launch=[],
+                              route_score_per_launch=[0.013, 0.02, 0.149],
+                              route_select_per_launch=[0.011, 0.013, 0.045])
+    m2 = bench.paper_model(line2, {"hbm_gbs": 6448.4, "bf16_tflops": 1725.8})
+    rows2 = {r["stage"]: r for r in m2["rows"]}
+    assert rows2["route score L1"]["waves_ms"] == 0.013 and rows2["route select L2"]["waves_ms"] == 0.011
+    assert rows2["route score L3"]["bound"] == "latency (one wave)"
