@@ -21,7 +21,7 @@
 //   warps 0-15 softmax and epilogue: warp w serves sub-tile w / 8, the keys [32 h, 32 h + 32)
 //              of each chunk and the output dims [64 h, 64 h + 64) for h = (w / 4) % 2, and
 //              the rows 32 (w % 4) + lane (= its TMEM lanes); the two threads of a row share
-//              their maxima through shared memory and a named barrier (sub-tile u owns TMEM
+//              their maxima through shared memory and an mbarrier (sub-tile u owns TMEM
 //              columns [256 u, 256 u + 256)); each thread writes its 32 weights of P as
 //              bf16 pairs over the first 16 of the 32 S columns it has just read, where the
 //              P . V MMA reads them as its A operand;
@@ -69,6 +69,7 @@ struct alignas(1024) Smem {
   unsigned long long q_full, q_empty;
   unsigned long long s_full[kSub][2], p_full[kSub][2], pv_done[kSub][2];
   unsigned long long o_free[kSub], drain;
+  unsigned long long pair[kSub][4];              // the two warps (halves) of each row group
   float xmax[2][kSub][kHalves][kRows];           // row maxima (per entry) and sums (epilogue) of the
                                                  // two halves of a row, by entry parity
   uint32_t tmem_base;
@@ -183,6 +184,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         mbar_init(&sm.pv_done[u][i], 1);
       }
       mbar_init(&sm.o_free[u], 4 * kHalves);
+      for (int g4 = 0; g4 < 4; ++g4) mbar_init(&sm.pair[u][g4], kHalves);
     }
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
@@ -333,10 +335,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
     const int r = (warp & 3) * 32 + lane;        // row = TMEM lane
     const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16) + u * kSubCols;
     const uint32_t s_col = (uint32_t)hf * 32, o_col = kColO + (uint32_t)hf * 64;
-    const int bar_id = 1 + u * 4 + (warp & 3);   // named barrier of the row group's two warps
+    long long npair = 0;                         // phases of this row group's pair barrier
     const float sl2 = 1.4426950408889634f * 0.08838834764831845f;   // log2(e) / sqrt(128)
     long long j = 0, tl = 0;
     bool ok = true;
+    // the two warps of this row group meet (bounded): shared-memory writes before it are seen
+    // after it
+    auto pair_sync = [&]() -> bool {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.pair[u][warp & 3]);
+      const bool k2 = warp_wait(&sm.pair[u][warp & 3], (uint32_t)(npair & 1), &sm.abort);
+      ++npair;
+      return k2;
+    };
     for (int64_t tile = blockIdx.x; tile < a.tiles && ok; tile += gridDim.x, ++tl) {
       const Tile t = tile_of(a, tile);
       const int n = tile_entries(a, tile);
@@ -388,7 +399,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
         }
         // the row maximum over both halves
         sm.xmax[j & 1][u][hf][r] = mx;
-        asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+        if (!pair_sync()) { ok = false; break; }
         mx = fmaxf(mx, sm.xmax[j & 1][u][hf ^ 1][r]);
         // lazy rescale: only when the row maximum grows by more than 2^kLazy (the same
         // decision in both halves: same m, same maximum)
@@ -445,7 +456,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       // epilogue: O / l of each valid row, the row sum from both halves (in the maxima slot
       // of the next entry's parity: both halves have read the last entry's maxima)
       sm.xmax[j & 1][u][hf][r] = l;
-      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+      if (!pair_sync()) { ok = false; break; }
       const float lr = sm.xmax[j & 1][u][0][r] + sm.xmax[j & 1][u][1][r];
       if (n >= 1 && !warp_wait(&sm.pv_done[u][(j - 1) & 1], (uint32_t)(((j - 1) >> 1) & 1), &sm.abort)) {
         ok = false;
@@ -479,7 +490,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap qmap, const __grid_constan
       if (valid && hf == 0 && a.lse) a.lse[((int64_t)t.b * a.nq + qi) * a.Hq + h] =
           lr > 0.f ? (m + log2f(lr)) * 0.6931471805599453f : -INFINITY;
       // the sums of this tile are read before the next tile's epilogue writes them
-      asm volatile("bar.sync %0, 64;" ::"r"(bar_id) : "memory");
+      if (!pair_sync()) { ok = false; break; }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.o_free[u]);
