@@ -185,21 +185,24 @@ route_score_kernel(ScoreArgs a) {
         if (id < nvis) mask = (1u << g.G) - 1u;
       }
     };
-    unsigned int any_mask = 0;
+    // this warp's groups that hold a candidate of some head (warp-uniform); the steps run
+    // over those groups only, so a sparse frontier costs fewer dependent steps
+    uint32_t gsel = 0;                                   // 4 bits per selected group
+    int ngrp = 0;
     for (int grp = 0; grp < GPW; ++grp) {
       int64_t id; unsigned int m; int jj, cc;
       slot_of(grp, id, m, jj, cc);
-      any_mask |= m;
+      if (__any_sync(0xffffffffu, m != 0)) gsel |= (uint32_t)grp << (4 * ngrp++);
     }
-    if (!__any_sync(0xffffffffu, any_mask != 0)) continue;   // warp-uniform
+    if (ngrp == 0) continue;                             // warp-uniform
     constexpr int kVec = 16 / sizeof(KT);
     constexpr int kNv = 32 / kVec;                       // 16-byte vectors of 32 dims
     const int R = g.R;
-    const int nsteps = GPW * R;
+    const int nsteps = ngrp * R;
     const int64_t node0 = (b * g.Hkv + hk) * g.ncap[a.level];
     // a step's row and its b_hat are loaded together, one step ahead of their use
     auto load_step = [&](uint4 (&v)[kNv], float& bh, int st) {
-      const int grp = st / R, r = st - grp * R;
+      const int gi = st / R, r = st - gi * R, grp = (int)((gsel >> (4 * gi)) & 15u);
       int64_t id; unsigned int m; int jj, cc;
       slot_of(grp, id, m, jj, cc);
       const uint4* src = reinterpret_cast<const uint4*>(
@@ -210,7 +213,7 @@ route_score_kernel(ScoreArgs a) {
     };
     double best0 = -INFINITY, best1 = -INFINITY;
     auto compute_step = [&](const uint4 (&v)[kNv], float bh, int st) {
-      const int grp = st / R, r = st - grp * R;
+      const int gi = st / R, r = st - gi * R, grp = (int)((gsel >> (4 * gi)) & 15u);
       double c0[4] = {0.0, 0.0, 0.0, 0.0}, c1[4] = {0.0, 0.0, 0.0, 0.0};   // 4 independent chains
 #pragma unroll
       for (int s2 = 0; s2 < 32; ++s2) {
