@@ -25,3 +25,25 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """The routing tallies of the GPU parity tests (heads whose kept sets equal the
+    oracle's at every level, heads that differ only at a near cutoff, mismatches), one line
+    per comparison and a total, so that they are visible in a quiet run."""
+    cases = sys.modules.get("zha_cases")
+    if cases is None:
+        return
+    reps = [(name, r) for name, r in cases.ROUTE_REPORTS if r.heads and "test_gpu" in name]
+    if not reps:
+        return
+    terminalreporter.section("routing against the oracle (GPU tests)")
+    for name, r in reps:
+        status = "" if r.ok() else "  FAILED: " + "; ".join(r.problems())
+        terminalreporter.write_line(f"{name}: {r.summary()}{status}")
+    heads = sum(r.heads for _, r in reps)
+    exact = sum(r.exact for _, r in reps)
+    near = sum(r.near_cutoff for _, r in reps)
+    bad = sum(len(r.mismatched) for _, r in reps)
+    terminalreporter.write_line(f"total: {exact} exact, {near} near-cutoff mismatches, {bad} mismatched "
+                                f"of {heads} heads in {len(reps)} comparisons")

@@ -3,8 +3,9 @@ through its C ABI, and the CPU oracle on the same bytes (copied to the host)."""
 from __future__ import annotations
 
 import math
+import os
 from dataclasses import dataclass, field
-from typing import Dict, List, Optional
+from typing import Dict, List, Optional, Tuple
 
 import numpy as np
 import torch
@@ -58,6 +59,10 @@ def f32_ulp_diff(a: np.ndarray, b: np.ndarray) -> np.ndarray:
 
 MAX_EXCUSED = 1 / 32    # fraction of the compared heads that may differ at a near cutoff (at least 1)
 
+# every RouteCompare of the session with the test that made it; the terminal summary
+# (tests/conftest.py) prints the GPU tests' tallies, so they show under `pytest -q`
+ROUTE_REPORTS: List[Tuple[str, "RouteCompare"]] = []
+
 
 @dataclass
 class RouteCompare:
@@ -78,6 +83,10 @@ class RouteCompare:
     near_levels: int = 0
     levels: int = 0
     mismatched: List[str] = field(default_factory=list)
+
+    def __post_init__(self):
+        test = os.environ.get("PYTEST_CURRENT_TEST", "").split(" (")[0]
+        ROUTE_REPORTS.append((test, self))
 
     def excused_limit(self) -> int:
         return max(1, int(self.heads * MAX_EXCUSED))
