@@ -31,10 +31,13 @@ def pytest_terminal_summary(terminalreporter, exitstatus, config):
     """The routing tallies of the GPU parity tests (heads whose kept sets equal the
     oracle's at every level, heads that differ only at a near cutoff, mismatches), one line
     per comparison and a total, so that they are visible in a quiet run."""
-    cases = sys.modules.get("zha_cases")
-    if cases is None:
-        return
-    reps = [(name, r) for name, r in cases.ROUTE_REPORTS if r.heads and "test_gpu" in name]
+    reps, seen = [], set()
+    for mod in ("tests.zha_cases", "zha_cases"):       # the tests import it as tests.zha_cases
+        cases = sys.modules.get(mod)
+        for name, r in (cases.ROUTE_REPORTS if cases is not None else []):
+            if id(r) not in seen and r.heads and "test_gpu" in name:
+                seen.add(id(r))
+                reps.append((name, r))
     if not reps:
         return
     terminalreporter.section("routing against the oracle (GPU tests)")
