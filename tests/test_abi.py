@@ -258,3 +258,31 @@ def test_struct_layouts_match_the_header(tmp_path):
         assert got[(s, "size")] == ctypes.sizeof(cls), s
         for f in fields[s]:
             assert got[(s, f)] == getattr(cls, f).offset, (s, f)
+
+
+def test_prefill_host_rejections_enqueue_nothing(lib):
+    """zha_prefill_attn serves bf16 caches only and checks its pointers, sizes and workspace
+    on the host, before anything is enqueued; its workspace grows with the query count."""
+    g = geom()
+    fake = ctypes.c_void_p(0x1000)
+    buf = _lib.Buf(0x1000, 1 << 40)
+    n0 = lib.zha_launch_count()
+    op = _lib.ZHA_OP_PREFILL
+    w16 = lib.zha_workspace_bytes(ctypes.byref(g), 16, op)
+    w64 = lib.zha_workspace_bytes(ctypes.byref(g), 64, op)
+    assert 0 < w16 < w64
+    small = _lib.Buf(0x1000, w16 - 1)
+
+    def call(gg, q_pos=fake, nq=16, ids=fake, cap=8, ws=buf, st=fake):
+        return lib.zha_prefill_attn(ctypes.byref(gg), fake, fake, fake, q_pos, nq, ids, fake, cap, fake, None,
+                                    ws, st, None)
+
+    assert call(geom(dtype=0)) == _lib.ZHA_ERR_UNSUPPORTED            # fp32 caches
+    assert call(geom(d=256)) == _lib.ZHA_ERR_UNSUPPORTED              # bad geometry
+    assert call(g, q_pos=None) == _lib.ZHA_ERR_INVALID_ARG            # positions are required
+    assert call(g, nq=0) == _lib.ZHA_ERR_INVALID_ARG
+    assert call(g, ids=None) == _lib.ZHA_ERR_INVALID_ARG
+    assert call(g, cap=0) == _lib.ZHA_ERR_INVALID_ARG
+    assert call(g, st=None) == _lib.ZHA_ERR_INVALID_ARG
+    assert call(g, ws=small) == _lib.ZHA_ERR_CAPACITY                 # workspace one byte short
+    assert lib.zha_launch_count() == n0
