@@ -7,7 +7,13 @@ seeded synthetic clustered keys; the KV cache (8 GiB for the default workload) i
 than L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl zha|reference]
-                    [--workload NAME] [--p P]
+                    [--workload NAME] [--p P] [--path zha|dense|flat|prefill]
+
+The default workload is the 1M-token decode (long-decode-1m).  `--path prefill` times the
+query-tile prefill attention (zha_prefill_attn) on the chunked-prefill workload against the
+per-query path over the same leaf lists.  `--sweep` runs the crossover sweep over T,
+`--segment N` the structured variant of the generator, and `--model FILE` the pages' roofline
+model over saved bench lines (no GPU work).
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own independent replica of
 the workload (the path shards over (sequence, KV head) units with no exchange), so the
